@@ -1,0 +1,272 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test fixes one function of oracle/calibatt_oracle.py to a library routine,
+a closed form, a brute-force enumeration or a value stated by the paper note
+"Accelerating Text-to-Video Generation with Calibrated Sparse Attention".
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import calibatt_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(seed, *shape, std=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * std
+
+
+# ---------------------------------------------------------------- attention
+
+@pytest.mark.parametrize("n,block,d", [(37, 8, 16), (64, 16, 8), (100, 32, 64)])
+def test_all_ones_mask_equals_sdpa(n, block, d):
+    q, k, v = (_rand(s, n, d) for s in (1, 2, 3))
+    nb = O.num_blocks(n, block)
+    o, lse = O.block_sparse_attention(q, k, v, np.ones((nb, nb), bool), block)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None])[0]
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+    ref_lse = torch.logsumexp(torch.from_numpy(q) @ torch.from_numpy(k).T / math.sqrt(d), dim=1)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
+
+
+def test_diagonal_only_mask_matches_bruteforce_loops():
+    n, block, d = 21, 8, 4          # ragged: last block has 5 tokens
+    q, k, v = (_rand(s, n, d) for s in (4, 5, 6))
+    nb = O.num_blocks(n, block)
+    o, _ = O.block_sparse_attention(q, k, v, np.eye(nb, dtype=bool), block, scale=0.7)
+    for i in range(n):
+        r = i // block
+        keys = [j for j in range(n) if j // block == r]
+        scores = []
+        for j in keys:
+            acc = 0.0
+            for t in range(d):
+                acc += q[i, t] * k[j, t]
+            scores.append(0.7 * acc)
+        mx = max(scores)
+        w = [math.exp(s - mx) for s in scores]
+        tot = sum(w)
+        for t in range(d):
+            expect = sum(w[a] * v[keys[a], t] for a in range(len(keys))) / tot
+            assert abs(o[i, t] - expect) < 1e-12
+
+
+def test_constant_keys_give_mean_of_retained_values():
+    n, block, d = 50, 16, 8
+    q = _rand(7, n, d, std=3.0)
+    k = np.tile(_rand(8, 1, d), (n, 1))
+    v = _rand(9, n, d)
+    nb = O.num_blocks(n, block)
+    mask = np.random.default_rng(10).random((nb, nb)) < 0.5
+    mask[np.arange(nb), np.arange(nb)] = True
+    o, _ = O.block_sparse_attention(q, k, v, mask, block)
+    for i in range(n):
+        keep = [j for j in range(n) if mask[i // block, j // block]]
+        np.testing.assert_allclose(o[i], v[keep].mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_one_query_two_keys_closed_form():
+    d = 4
+    q = np.array([[1.0, -2.0, 0.5, 3.0]])
+    k = np.array([[0.5, 1.0, -1.0, 2.0], [-1.0, 0.0, 2.0, 1.0]])
+    v = np.array([[1.0, 2.0, 3.0, 4.0], [-4.0, 0.0, 8.0, 1.0]])
+    s1 = (0.5 - 2.0 - 0.5 + 6.0) / 2.0     # q.k1 / sqrt(4)
+    s2 = (-1.0 + 0.0 + 1.0 + 3.0) / 2.0
+    w1 = 1.0 / (1.0 + math.exp(s2 - s1))
+    expect = w1 * v[0] + (1 - w1) * v[1]
+    o, lse = O.attention_rows(q, k, v, 2, 1.0 / math.sqrt(d))
+    np.testing.assert_allclose(o[0], expect, rtol=0, atol=1e-14)
+    assert abs(lse[0] - math.log(math.exp(s1) + math.exp(s2))) < 1e-14
+
+
+def test_empty_row_gives_zero_output_and_minus_inf_lse():
+    n, block, d = 32, 8, 4
+    q, k, v = (_rand(s, n, d) for s in (11, 12, 13))
+    mask = np.eye(4, dtype=bool)
+    mask[2, 2] = False
+    o, lse = O.block_sparse_attention(q, k, v, mask, block)
+    assert np.all(o[16:24] == 0.0)
+    assert np.all(np.isneginf(lse[16:24]))
+    assert np.all(np.isfinite(lse[:16]))
+
+
+def test_padding_rows_beyond_seq_len_are_never_read():
+    n, block, d = 40, 16, 8
+    q, k, v = (_rand(s, 48, d) for s in (14, 15, 16))
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for t in (q2, k2, v2):
+        t[n:] = np.nan
+    nb = O.num_blocks(n, block)
+    m = np.ones((nb, nb), bool)
+    o1, _ = O.block_sparse_attention(q, k, v, m, block, seq_len=n)
+    o2, _ = O.block_sparse_attention(q2, k2, v2, m, block, seq_len=n)
+    np.testing.assert_array_equal(o1, o2)
+
+
+def test_probability_rows_sum_to_one():
+    n, d = 77, 16
+    q, k = _rand(17, n, d, std=2.0), _rand(18, n, d, std=2.0)
+    p = O.attention_probabilities(q, k, n, 0.25)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(p >= 0)
+
+
+def test_bnhd_wrapper_indexes_heads_and_batches():
+    b, n, h, d, block = 2, 24, 3, 8, 8
+    q, k, v = (_rand(s, b, n, h, d) for s in (19, 20, 21))
+    rng = np.random.default_rng(22)
+    masks = [rng.random((3, 3)) < 0.6 for _ in range(h)]
+    for m in masks:
+        m[np.arange(3), np.arange(3)] = True
+    out, _ = O.block_sparse_attention_bnhd(q, k, v, masks, block)
+    for bi in range(b):
+        for hi in range(h):
+            ref, _ = O.block_sparse_attention(q[bi, :, hi], k[bi, :, hi], v[bi, :, hi],
+                                              masks[hi], block)
+            np.testing.assert_array_equal(out[bi, :, hi], ref)
+
+
+# ---------------------------------------------------------------- anchors
+
+def test_nearest_anchor_tables():
+    for t in _golden("nearest_anchor_tables.json")["tables"]:
+        got = O.nearest_anchor_rows(t["rows"], t["anchors"])
+        assert got.tolist() == t["nearest"]
+
+
+def test_anchor_query_reduction():
+    for c in _golden("anchor_query_reduction.json")["cases"]:
+        anchors = list(range(c["k"]))  # any k distinct rows
+        src = O.anchor_source_tokens(1, c["H"], c["W"], anchors)
+        assert len(np.unique(src)) == c["queries_after"]
+        assert c["H"] * c["W"] == c["queries_before"]
+        assert abs(1 - len(np.unique(src)) / c["queries_before"] - c["sparsity"]) < 1e-12
+
+
+def test_anchor_attention_rows():
+    frames, rows, cols, d = 2, 8, 5, 16
+    n = frames * rows * cols
+    q, k, v = (_rand(s, n, d) for s in (23, 24, 25))
+    anchors = [0, 4]
+    o, _ = O.anchor_attention(q, k, v, frames, rows, cols, anchors)
+    dense = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None])[0].numpy()
+    near = [0, 0, 0, 4, 4, 4, 4, 4]
+    for f in range(frames):
+        for rho in range(rows):
+            for w in range(cols):
+                i = (f * rows + rho) * cols + w
+                a = (f * rows + near[rho]) * cols + w
+                np.testing.assert_allclose(o[i], dense[a], rtol=0, atol=1e-12)
+                if rho in anchors:
+                    np.testing.assert_allclose(o[i], dense[i], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- energy
+
+def test_block_energy_rows_sum_to_one_ragged():
+    n, block, d = 45, 16, 8          # last block has 13 valid tokens
+    q, k = _rand(26, n, d, std=2.0), _rand(27, n, d, std=2.0)
+    e = O.block_energy(q, k, block)
+    assert e.shape == (3, 3)
+    np.testing.assert_allclose(e.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_block_energy_constant_keys_closed_form():
+    n, block, d = 45, 16, 8
+    q = _rand(28, n, d)
+    k = np.tile(_rand(29, 1, d), (n, 1))
+    e = O.block_energy(q, k, block)
+    sizes = np.array([16, 16, 13], float)
+    np.testing.assert_allclose(e, np.tile(sizes / n, (3, 1)), rtol=0, atol=1e-14)
+
+
+def test_block_energy_double_loop_bruteforce():
+    n, block, d = 11, 4, 3
+    q, k = _rand(30, n, d, std=1.5), _rand(31, n, d, std=1.5)
+    e = O.block_energy(q, k, block, scale=0.9)
+    for r in range(3):
+        rows = [i for i in range(n) if i // block == r]
+        for c in range(3):
+            tot = 0.0
+            for i in rows:
+                scores = [0.9 * sum(q[i, t] * k[j, t] for t in range(d)) for j in range(n)]
+                mx = max(scores)
+                z = sum(math.exp(s - mx) for s in scores)
+                tot += sum(math.exp(scores[j] - mx) / z for j in range(n) if j // block == c)
+            assert abs(e[r, c] - tot / len(rows)) < 1e-13
+
+
+# ---------------------------------------------------------------- selection
+
+def _bruteforce_min_size(row, tau):
+    """Smallest number of blocks of which SOME subset carries mass >= tau (exhaustive)."""
+    nk = len(row)
+    for size in range(1, nk + 1):
+        for subset in itertools.combinations(range(nk), size):
+            if math.fsum(row[list(subset)]) >= tau:
+                return size
+    return nk
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_select_blocks_minimal_and_canonical(seed):
+    rng = np.random.default_rng(100 + seed)
+    nk = 6
+    e = rng.dirichlet(np.full(nk, 0.4), size=5)
+    if seed % 3 == 0:                       # exact ties at the boundary
+        e[:, 1] = e[:, 2]
+        e /= e.sum(axis=1, keepdims=True)
+    for tau in (0.5, 0.9, 0.99):
+        sel = O.select_blocks(e, tau)
+        for r in range(e.shape[0]):
+            size = _bruteforce_min_size(e[r], tau)
+            chosen = tuple(np.flatnonzero(sel[r]))
+            assert len(chosen) == size
+            # the chosen set is the canonical (energy desc, index asc) prefix of that size
+            canonical = sorted(range(nk), key=lambda c: (-e[r, c], c))[:size]
+            assert chosen == tuple(sorted(canonical))
+            if math.fsum(e[r]) >= tau:
+                assert math.fsum(e[r, list(chosen)]) >= tau
+
+
+def test_select_blocks_keeps_all_when_mass_never_reaches_tau():
+    e = np.array([[0.25, 0.25, 0.25, 0.25 - 1e-9]])
+    assert O.select_blocks(e, 1.0).all()
+
+
+def test_select_blocks_single_dominant_block():
+    e = np.array([[0.01, 0.97, 0.01, 0.01]])
+    assert O.select_blocks(e, 0.95).tolist() == [[False, True, False, False]]
+    assert O.select_blocks(e, 0.99).sum() == 3
+
+
+# ---------------------------------------------------------------- aggregation
+
+def test_aggregation_worked_example():
+    g = _golden("aggregation_worked_example.json")
+    counts = np.array(g["kept_counts"] + g["dropped_counts"])
+    keep = O.aggregate_masks(counts, g["n_prompts"], g["rho"])
+    assert keep.tolist() == [True] * len(g["kept_counts"]) + [False] * len(g["dropped_counts"])
+
+
+def test_aggregation_from_stacked_masks_and_union():
+    rng = np.random.default_rng(33)
+    masks = rng.random((4, 3, 5)) < 0.3
+    union = O.aggregate_masks(masks, 4, 0.25)
+    np.testing.assert_array_equal(union, masks.any(axis=0))
+    inter = O.aggregate_masks(masks, 4, 1.0)
+    np.testing.assert_array_equal(inter, masks.all(axis=0))

@@ -1,0 +1,56 @@
+"""Checks of the seeded input generators (structure of the synthetic masks and layouts)."""
+
+import numpy as np
+
+import workloads as W
+
+
+def test_synthetic_mask_structure_720p():
+    wl = W.WORKLOADS["720p"]
+    nb = wl.num_blocks
+    assert nb == 591 and wl.seq_len == 75600
+    for target in (0.32, 0.35, 0.38):
+        m = W.synthetic_block_mask(7, nb, wl.block, wl.tokens_per_frame, target)
+        assert m.shape == (nb, nb)
+        assert m[np.arange(nb), np.arange(nb)].all()
+        first_frame_cols = np.flatnonzero(np.arange(nb) * wl.block < wl.tokens_per_frame)
+        assert m[:, first_frame_cols].all()
+        assert abs(m.sum() - round(target * nb * nb)) <= 0
+    # the structured band alone: w=2 -> ~26.6%, w=3 -> ~34.6%
+    assert abs(W.band_mask(nb, 128, 3600, 2).mean() - 0.266) < 0.005
+    assert abs(W.band_mask(nb, 128, 3600, 3).mean() - 0.346) < 0.005
+
+
+def test_masks_are_seeded_and_deterministic():
+    a = W.synthetic_block_mask(3, 64, 128, 3600, 0.35)
+    b = W.synthetic_block_mask(3, 64, 128, 3600, 0.35)
+    c = W.synthetic_block_mask(4, 64, 128, 3600, 0.35)
+    assert (a == b).all() and (a != c).any()
+
+
+def test_tiny_mask_density_and_diagonal():
+    m = W.tiny_block_mask(1, 4, 0.5)
+    assert m.sum() == 8 and m[np.arange(4), np.arange(4)].all()
+
+
+def test_anchor_placement_and_repetitive_heads():
+    assert W.equally_spaced_anchors(45, 5) == (4, 13, 22, 31, 40)
+    rep = W.repetitive_heads(5, 40, 12)
+    assert len(rep) == 12 and len(set(rep)) == 12 and all(0 <= h < 40 for h in rep)
+
+
+def test_mask_to_csr_roundtrip():
+    rng = np.random.default_rng(0)
+    m = rng.random((9, 7)) < 0.4
+    rp, ci = W.mask_to_csr(m)
+    back = np.zeros_like(m)
+    for r in range(9):
+        cols = ci[rp[r]:rp[r + 1]]
+        assert (np.diff(cols) > 0).all()
+        back[r, cols] = True
+    assert (back == m).all()
+
+
+def test_sweep_density_ramp():
+    assert abs(W.sweep_density(0, 50, 1) - 0.60) <= 0.03 + 1e-12
+    assert abs(W.sweep_density(49, 50, 1) - 0.20) <= 0.03 + 1e-12
