@@ -22,9 +22,9 @@ def test_synthetic_mask_structure_720p():
 
 
 def test_masks_are_seeded_and_deterministic():
-    a = W.synthetic_block_mask(3, 64, 128, 3600, 0.35)
-    b = W.synthetic_block_mask(3, 64, 128, 3600, 0.35)
-    c = W.synthetic_block_mask(4, 64, 128, 3600, 0.35)
+    a = W.synthetic_block_mask(3, 300, 128, 3600, 0.35)
+    b = W.synthetic_block_mask(3, 300, 128, 3600, 0.35)
+    c = W.synthetic_block_mask(4, 300, 128, 3600, 0.35)
     assert (a == b).all() and (a != c).any()
 
 
