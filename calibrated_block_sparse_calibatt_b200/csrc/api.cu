@@ -1,0 +1,818 @@
+// C ABI of libcalibatt.so (declared in include/calibatt.h): argument
+// validation, the mask dictionary with its longest-processing-time schedules,
+// TMA tensor-map encoding and kernel dispatch.  All host logic is here; the
+// kernels live in attn_tc.cu, attn_simt.cu and energy.cu.
+#include "calibatt.h"
+#include "internal.h"
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <functional>
+#include <mutex>
+#include <numeric>
+#include <queue>
+#include <string>
+#include <utility>
+#include <vector>
+
+using calibatt::AnchorGeom;
+using calibatt::LayerSchedule;
+using calibatt::SimtParams;
+using calibatt::TcParams;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_timeout_ns{4000000000ull};
+
+__device__ int32_t g_status_word;
+
+calibatt_status fail(calibatt_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+calibatt_status cuda_fail(cudaError_t e, const char* what) {
+  cudaGetLastError();  // clear the sticky-free error state
+  return fail(e == cudaErrorMemoryAllocation ? CALIBATT_ERR_OOM : CALIBATT_ERR_CUDA, "%s: %s", what,
+              cudaGetErrorString(e));
+}
+
+int32_t* status_word_ptr() {
+  static std::mutex mu;
+  static int32_t* ptrs[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<int32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+// ------------------------------------------------------------- schedule
+
+void lpt(int32_t n, const int64_t* cost, int32_t bins, int32_t* bin_ptr, int32_t* order,
+         int64_t* makespan) {
+  std::vector<int32_t> idx(n);
+  std::iota(idx.begin(), idx.end(), 0);
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) { return cost[a] > cost[b]; });
+  using Slot = std::pair<int64_t, int32_t>;  // (load, bin): least load, then lowest bin
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int32_t b = 0; b < bins; ++b) heap.push({0, b});
+  std::vector<std::vector<int32_t>> per_bin(bins);
+  for (int32_t i : idx) {
+    Slot s = heap.top();
+    heap.pop();
+    per_bin[s.second].push_back(i);
+    heap.push({s.first + cost[i], s.second});
+  }
+  int64_t mk = 0;
+  while (!heap.empty()) {
+    mk = std::max(mk, heap.top().first);
+    heap.pop();
+  }
+  int32_t pos = 0;
+  for (int32_t b = 0; b < bins; ++b) {
+    bin_ptr[b] = pos;
+    for (int32_t i : per_bin[b]) order[pos++] = i;
+  }
+  bin_ptr[bins] = pos;
+  if (makespan) *makespan = mk;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 4-D bf16 map {D, x1, x2, x3} with (x1, x2, x3) the N, H, batch dimensions in
+// increasing stride order; box {64, 128 rows of N, 1, 1}, 128-byte swizzle.
+// The N extent is seq_len, so rows past the valid tokens read as zeros.
+calibatt_status encode_qkv_map(CUtensorMap* map, const void* base, const calibatt_shape& s, int* pos_n,
+                               int* pos_h, int* pos_b) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(CALIBATT_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  struct Dim {
+    int64_t stride;
+    uint64_t size;
+    int which;  // 0 = N, 1 = H, 2 = batch
+  } d[3] = {{s.stride_n, static_cast<uint64_t>(s.seq_len), 0},
+            {s.stride_h, static_cast<uint64_t>(s.heads), 1},
+            {s.stride_b, static_cast<uint64_t>(s.batch), 2}};
+  std::stable_sort(d, d + 3, [](const Dim& a, const Dim& b) { return a.stride < b.stride; });
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(s.head_dim), d[0].size, d[1].size, d[2].size};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d[0].stride * 2), static_cast<cuuint64_t>(d[1].stride * 2),
+                           static_cast<cuuint64_t>(d[2].stride * 2)};
+  cuuint32_t box[4] = {64, d[0].which == 0 ? 128u : 1u, d[1].which == 0 ? 128u : 1u, d[2].which == 0 ? 128u : 1u};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  for (int i = 0; i < 3; ++i) {
+    if (d[i].which == 0) *pos_n = i + 1;
+    if (d[i].which == 1) *pos_h = i + 1;
+    if (d[i].which == 2) *pos_b = i + 1;
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CALIBATT_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return CALIBATT_OK;
+}
+
+// ------------------------------------------------------------ validation
+
+calibatt_status check_shape(const calibatt_shape* s) {
+  if (!s) return fail(CALIBATT_ERR_INVALID_ARG, "shape is NULL");
+  if (s->reserved != 0) return fail(CALIBATT_ERR_INVALID_ARG, "shape.reserved must be 0");
+  if (s->batch < 1 || s->seq_len < 1 || s->heads < 1)
+    return fail(CALIBATT_ERR_INVALID_ARG, "batch, seq_len and heads must be >= 1 (got %d, %d, %d)", s->batch,
+                s->seq_len, s->heads);
+  if (s->heads > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "heads must be <= 65535");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(CALIBATT_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
+  if (s->dtype != CALIBATT_DTYPE_BF16 && s->dtype != CALIBATT_DTYPE_FP32)
+    return fail(CALIBATT_ERR_UNSUPPORTED, "dtype %d not supported", s->dtype);
+  if (s->stride_b < 1 || s->stride_n < 1 || s->stride_h < 1)
+    return fail(CALIBATT_ERR_INVALID_ARG, "strides must be positive");
+  const int64_t align = s->dtype == CALIBATT_DTYPE_BF16 ? 8 : 4;
+  if (s->stride_b % align || s->stride_n % align || s->stride_h % align)
+    return fail(CALIBATT_ERR_INVALID_ARG, "strides must be multiples of %lld elements (16 bytes)", (long long)align);
+  if (s->stride_n < s->head_dim && s->stride_h < s->head_dim)
+    return fail(CALIBATT_ERR_INVALID_ARG, "rows of head_dim elements overlap (stride_n and stride_h < head_dim)");
+  return CALIBATT_OK;
+}
+
+calibatt_status check_ptrs(const void* q, const void* k, const void* v, const void* o) {
+  if (!q || !k || !v || !o) return fail(CALIBATT_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+  for (const void* p : {q, k, v, o})
+    if (reinterpret_cast<uintptr_t>(p) % 16)
+      return fail(CALIBATT_ERR_INVALID_ARG, "q, k, v and o must be 16-byte aligned");
+  return CALIBATT_OK;
+}
+
+calibatt_status check_block(int32_t block) {
+  if (block != 64 && block != 128) return fail(CALIBATT_ERR_UNSUPPORTED, "block %d not supported (64 or 128)", block);
+  return CALIBATT_OK;
+}
+
+calibatt_status validate_csr(int32_t nq, int32_t nk, const int32_t* row_ptr, const int32_t* col_idx,
+                             bool require_diag, const char* what) {
+  if (nq < 0 || nk < 1) return fail(CALIBATT_ERR_INVALID_ARG, "%s: nq must be >= 0 and nk >= 1", what);
+  if (!row_ptr) return fail(CALIBATT_ERR_INVALID_ARG, "%s: row_ptr is NULL", what);
+  if (row_ptr[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "%s: row_ptr[0] = %d, expected 0", what, row_ptr[0]);
+  for (int32_t r = 0; r < nq; ++r)
+    if (row_ptr[r + 1] < row_ptr[r])
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: row_ptr decreases at row %d", what, r);
+  if (row_ptr[nq] > 0 && !col_idx) return fail(CALIBATT_ERR_INVALID_ARG, "%s: col_idx is NULL", what);
+  if (require_diag && nq != nk)
+    return fail(CALIBATT_ERR_INVALID_ARG, "%s: diagonal requested but nq %d != nk %d", what, nq, nk);
+  for (int32_t r = 0; r < nq; ++r) {
+    bool diag = false;
+    for (int32_t i = row_ptr[r]; i < row_ptr[r + 1]; ++i) {
+      const int32_t c = col_idx[i];
+      if (c < 0 || c >= nk)
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: row %d column %d outside [0, %d)", what, r, c, nk);
+      if (i > row_ptr[r] && c <= col_idx[i - 1])
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: row %d columns not strictly ascending", what, r);
+      diag |= (c == r);
+    }
+    if (require_diag && !diag) return fail(CALIBATT_ERR_INVALID_ARG, "%s: row %d lacks its diagonal block", what, r);
+  }
+  return CALIBATT_OK;
+}
+
+// Rows of a frame served by each anchor: nearest anchor, distance ties to the lower one.
+void anchor_groups(int32_t rows, const int32_t* anchors, int32_t n, AnchorGeom& g) {
+  for (int a = 0; a < n; ++a) {
+    g.anchor_row[a] = static_cast<int16_t>(anchors[a]);
+    g.group_lo[a] = static_cast<int16_t>(rows);
+    g.group_hi[a] = -1;
+  }
+  for (int32_t rho = 0; rho < rows; ++rho) {
+    int best = 0;
+    for (int a = 1; a < n; ++a)
+      if (std::abs(rho - anchors[a]) < std::abs(rho - anchors[best])) best = a;
+    g.group_lo[best] = static_cast<int16_t>(std::min<int>(g.group_lo[best], rho));
+    g.group_hi[best] = static_cast<int16_t>(std::max<int>(g.group_hi[best], rho));
+  }
+}
+
+float scale_log2_of(float softmax_scale, int head_dim) {
+  const double sc = softmax_scale > 0.f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(head_dim));
+  return static_cast<float>(sc * 1.4426950408889634);
+}
+
+}  // namespace
+
+// ================================================================ dictionary
+
+struct calibatt_dict {
+  int32_t T = 0, L = 0, H = 0, nq = 0, nk = 0, block = 0, G = 0;
+  int32_t device = 0;
+  int64_t nnz_cap = 0, nnz_used = 0;
+  int32_t* d_row_ptr = nullptr;
+  int64_t* d_col_base = nullptr;
+  uint16_t* d_col = nullptr;
+  uint32_t* d_items = nullptr;
+  int32_t* d_cta_ptr = nullptr;
+  int64_t device_bytes = 0;
+  std::vector<uint8_t> layer_set;   // [T*L]
+  std::vector<uint8_t> rep;         // [T*L*H]
+  std::vector<int32_t> n_sparse;    // [T*L]
+  std::vector<int32_t> n_rep;       // [T*L]
+  std::vector<int64_t> retained;    // [T*L]
+
+  int64_t layer(int t, int l) const { return static_cast<int64_t>(t) * L + l; }
+
+  LayerSchedule schedule(int t, int l) const {
+    const int64_t ly = layer(t, l);
+    LayerSchedule s;
+    s.row_ptr = d_row_ptr + ly * H * (nq + 1);
+    s.col_base = d_col_base + ly * H;
+    s.col = d_col;
+    s.items = d_items + ly * H * nq;
+    s.cta_ptr = d_cta_ptr + ly * (G + 1);
+    s.nq = nq;
+    return s;
+  }
+
+  void release() {
+    cudaFree(d_row_ptr);
+    cudaFree(d_col_base);
+    cudaFree(d_col);
+    cudaFree(d_items);
+    cudaFree(d_cta_ptr);
+    d_row_ptr = nullptr;
+    d_col_base = nullptr;
+    d_col = nullptr;
+    d_items = nullptr;
+    d_cta_ptr = nullptr;
+  }
+};
+
+namespace {
+
+calibatt_status check_dict_layer(const calibatt_dict* d, int32_t t, int32_t l) {
+  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+  if (t < 0 || t >= d->T || l < 0 || l >= d->L)
+    return fail(CALIBATT_ERR_INVALID_ARG, "record (t=%d, l=%d) outside the dictionary (%d x %d)", t, l, d->T, d->L);
+  if (!d->layer_set[d->layer(t, l)]) return fail(CALIBATT_ERR_INVALID_ARG, "layer (t=%d, l=%d) was never set", t, l);
+  return CALIBATT_OK;
+}
+
+calibatt_status launch_sparse(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
+                              int32_t block, const calibatt_dict* d, int32_t t, int32_t l, float softmax_scale,
+                              float* lse, cudaStream_t stream) {
+  const int64_t ly = d->layer(t, l);
+  if (d->n_sparse[ly] == 0) return CALIBATT_OK;
+  const float sl2 = scale_log2_of(softmax_scale, s.head_dim);
+  const LayerSchedule sch = d->schedule(t, l);
+  if (s.dtype == CALIBATT_DTYPE_BF16 && block == 128) {
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    calibatt_status st;
+    if ((st = encode_qkv_map(&p.tm_q, q, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    if ((st = encode_qkv_map(&p.tm_k, k, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    if ((st = encode_qkv_map(&p.tm_v, v, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    p.q = static_cast<const uint16_t*>(q);
+    p.o = static_cast<uint16_t*>(o);
+    p.lse = lse;
+    p.sb = s.stride_b;
+    p.sn = s.stride_n;
+    p.sh = s.stride_h;
+    p.batch = s.batch;
+    p.seq_len = s.seq_len;
+    p.heads = s.heads;
+    p.nb = ceil_div(s.seq_len, 128);
+    p.scale_log2 = sl2;
+    p.sched = sch;
+    p.status = status_word_ptr();
+    p.timeout_ns = g_timeout_ns.load();
+    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, false, d->G, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "block-sparse tensor-core launch");
+    return CALIBATT_OK;
+  }
+  // CUDA-core path, heads in chunks of kMaxHeadsPerCall.
+  std::vector<int16_t> heads;
+  for (int h = 0; h < d->H; ++h)
+    if (!d->rep[ly * d->H + h]) heads.push_back(static_cast<int16_t>(h));
+  for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
+    SimtParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.lse = lse;
+    p.sb = s.stride_b;
+    p.sn = s.stride_n;
+    p.sh = s.stride_h;
+    p.batch = s.batch;
+    p.seq_len = s.seq_len;
+    p.heads = s.heads;
+    p.nb = ceil_div(s.seq_len, block);
+    p.scale_log2 = sl2;
+    p.sched = sch;
+    const size_t nh = std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0);
+    p.n_heads = static_cast<int32_t>(nh);
+    for (size_t i = 0; i < nh; ++i) p.head_ids[i] = heads[h0 + i];
+    const int64_t n_items = static_cast<int64_t>(s.batch) * nh * d->nq;
+    cudaError_t e = calibatt::launch_simt_attn(p, s.head_dim, block, s.dtype, false, static_cast<int>(n_items), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "block-sparse CUDA-core launch");
+  }
+  return CALIBATT_OK;
+}
+
+calibatt_status launch_anchor(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
+                              int32_t block, int32_t frames, int32_t rows, int32_t cols, const int32_t* anchors,
+                              int32_t n_anchors, const int32_t* head_ids, int32_t n_heads, float softmax_scale,
+                              cudaStream_t stream) {
+  if (frames < 1 || rows < 1 || cols < 1)
+    return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
+  if (static_cast<int64_t>(frames) * rows * cols != s.seq_len)
+    return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d",
+                (long long)frames * rows * cols, s.seq_len);
+  if (!anchors || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
+  for (int a = 0; a < n_anchors; ++a) {
+    if (anchors[a] < 0 || anchors[a] >= rows)
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchors[a], rows);
+    if (a > 0 && anchors[a] <= anchors[a - 1])
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
+  }
+  if (n_heads == 0) return CALIBATT_OK;
+  if (!head_ids || n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d] with a non-NULL list", calibatt::kMaxHeadsPerCall);
+  std::vector<uint8_t> seen(s.heads, 0);
+  for (int i = 0; i < n_heads; ++i) {
+    if (head_ids[i] < 0 || head_ids[i] >= s.heads)
+      return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", head_ids[i], s.heads);
+    if (seen[head_ids[i]]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", head_ids[i]);
+  }
+  AnchorGeom g;
+  std::memset(&g, 0, sizeof(g));
+  g.frames = frames;
+  g.rows = rows;
+  g.cols = cols;
+  g.n_anchors = n_anchors;
+  g.anchor_tokens = frames * n_anchors * cols;
+  g.n_heads = n_heads;
+  anchor_groups(rows, anchors, n_anchors, g);
+  for (int i = 0; i < n_heads; ++i) g.head_ids[i] = static_cast<int16_t>(head_ids[i]);
+  const float sl2 = scale_log2_of(softmax_scale, s.head_dim);
+  if (s.dtype == CALIBATT_DTYPE_BF16) {
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    calibatt_status st;
+    if ((st = encode_qkv_map(&p.tm_q, q, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    if ((st = encode_qkv_map(&p.tm_k, k, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    if ((st = encode_qkv_map(&p.tm_v, v, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+    p.q = static_cast<const uint16_t*>(q);
+    p.o = static_cast<uint16_t*>(o);
+    p.sb = s.stride_b;
+    p.sn = s.stride_n;
+    p.sh = s.stride_h;
+    p.batch = s.batch;
+    p.seq_len = s.seq_len;
+    p.heads = s.heads;
+    p.nb = ceil_div(s.seq_len, 128);
+    p.scale_log2 = sl2;
+    g.tiles_per_head = ceil_div(g.anchor_tokens, 128);
+    p.anc = g;
+    p.status = status_word_ptr();
+    p.timeout_ns = g_timeout_ns.load();
+    const int sms = device_sm_count();
+    if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    const int64_t items = static_cast<int64_t>(n_heads) * g.tiles_per_head;
+    const int grid = static_cast<int>(std::min<int64_t>(sms, items));
+    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, true, grid, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "anchor tensor-core launch");
+    return CALIBATT_OK;
+  }
+  SimtParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.sb = s.stride_b;
+  p.sn = s.stride_n;
+  p.sh = s.stride_h;
+  p.batch = s.batch;
+  p.seq_len = s.seq_len;
+  p.heads = s.heads;
+  p.nb = ceil_div(s.seq_len, block);
+  p.scale_log2 = sl2;
+  g.tiles_per_head = ceil_div(g.anchor_tokens, block);
+  p.anc = g;
+  const int64_t n_items = static_cast<int64_t>(s.batch) * n_heads * g.tiles_per_head;
+  cudaError_t e = calibatt::launch_simt_attn(p, s.head_dim, block, s.dtype, true, static_cast<int>(n_items), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "anchor CUDA-core launch");
+  return CALIBATT_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+
+extern "C" {
+
+const char* calibatt_status_string(calibatt_status status) {
+  switch (status) {
+    case CALIBATT_OK: return "ok";
+    case CALIBATT_ERR_INVALID_ARG: return "invalid argument";
+    case CALIBATT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CALIBATT_ERR_CUDA: return "CUDA error";
+    case CALIBATT_ERR_TIMEOUT: return "device wait timed out";
+    case CALIBATT_ERR_OOM: return "out of device memory";
+    default: return "unknown status";
+  }
+}
+
+const char* calibatt_last_error(void) { return g_last_error.c_str(); }
+
+int32_t calibatt_abi_version(void) { return 1; }
+
+calibatt_status calibatt_csr_validate(int32_t nq, int32_t nk, const int32_t* row_ptr, const int32_t* col_idx,
+                                      int32_t require_diagonal) {
+  return validate_csr(nq, nk, row_ptr, col_idx, require_diagonal != 0, "csr");
+}
+
+calibatt_status calibatt_csr_to_intervals(int32_t nq, const int32_t* row_ptr, const int32_t* col_idx,
+                                          int32_t* interval_ptr, int32_t* interval_start, int32_t* interval_len,
+                                          int64_t capacity, int64_t* n_intervals) {
+  if (nq < 0 || !row_ptr || !interval_ptr || !n_intervals) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+  if (row_ptr[nq] > 0 && !col_idx) return fail(CALIBATT_ERR_INVALID_ARG, "col_idx is NULL");
+  int64_t total = 0;
+  for (int32_t r = 0; r < nq; ++r) {
+    interval_ptr[r] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
+    for (int32_t i = row_ptr[r]; i < row_ptr[r + 1]; ++i) {
+      const bool starts = (i == row_ptr[r]) || (col_idx[i] != col_idx[i - 1] + 1);
+      if (starts) {
+        if (total < capacity && interval_start && interval_len) {
+          interval_start[total] = col_idx[i];
+          interval_len[total] = 1;
+        }
+        ++total;
+      } else if (total - 1 < capacity && interval_len) {
+        interval_len[total - 1] += 1;
+      }
+    }
+  }
+  interval_ptr[nq] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
+  *n_intervals = total;
+  if (total > capacity) return fail(CALIBATT_ERR_INVALID_ARG, "capacity %lld < %lld intervals", (long long)capacity, (long long)total);
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_lpt_schedule(int32_t n_items, const int64_t* cost, int32_t n_bins, int32_t* bin_ptr,
+                                      int32_t* item_order, int64_t* makespan) {
+  if (n_items < 0 || n_bins < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_items must be >= 0 and n_bins >= 1");
+  if (!bin_ptr || (n_items > 0 && (!cost || !item_order))) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+  for (int32_t i = 0; i < n_items; ++i)
+    if (cost[i] < 0) return fail(CALIBATT_ERR_INVALID_ARG, "negative cost at item %d", i);
+  lpt(n_items, cost, n_bins, bin_ptr, item_order, makespan);
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk, int32_t block,
+                                     int64_t nnz_capacity, int32_t num_ctas, calibatt_dict** out) {
+  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1 || nnz_capacity < 0)
+    return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1 and nnz_capacity >= 0");
+  if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
+  if (nq > 65535 || H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "nq and H must be <= 65535");
+  calibatt_status st = check_block(block);
+  if (st != CALIBATT_OK) return st;
+  int G = num_ctas;
+  if (G <= 0) G = device_sm_count();
+  if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+  auto* d = new calibatt_dict();
+  d->T = T;
+  d->L = L;
+  d->H = H;
+  d->nq = nq;
+  d->nk = nk;
+  d->block = block;
+  d->G = G;
+  cudaGetDevice(&d->device);
+  d->nnz_cap = nnz_capacity;
+  const int64_t layers = static_cast<int64_t>(T) * L;
+  const size_t b_rp = sizeof(int32_t) * layers * H * (nq + 1);
+  const size_t b_cb = sizeof(int64_t) * layers * H;
+  const size_t b_col = sizeof(uint16_t) * std::max<int64_t>(1, nnz_capacity);
+  const size_t b_it = sizeof(uint32_t) * layers * H * nq;
+  const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
+  cudaError_t e = cudaMalloc(&d->d_row_ptr, b_rp);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_col_base, b_cb);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_col, b_col);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+  if (e != cudaSuccess) {
+    d->release();
+    delete d;
+    return cuda_fail(e, "dictionary allocation");
+  }
+  d->device_bytes = static_cast<int64_t>(b_rp + b_cb + b_col + b_it + b_cta);
+  d->layer_set.assign(layers, 0);
+  d->rep.assign(layers * H, 0);
+  d->n_sparse.assign(layers, 0);
+  d->n_rep.assign(layers, 0);
+  d->retained.assign(layers, 0);
+  *out = d;
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, const int32_t* row_ptr,
+                                        const int32_t* col_idx, const uint8_t* repetitive) {
+  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+  if (t < 0 || t >= d->T || l < 0 || l >= d->L)
+    return fail(CALIBATT_ERR_INVALID_ARG, "record (t=%d, l=%d) outside the dictionary", t, l);
+  const int64_t ly = d->layer(t, l);
+  if (d->layer_set[ly]) return fail(CALIBATT_ERR_INVALID_ARG, "layer (t=%d, l=%d) is already set", t, l);
+  if (!row_ptr) return fail(CALIBATT_ERR_INVALID_ARG, "row_ptr is NULL");
+  const int H = d->H, nq = d->nq;
+  std::vector<int64_t> head_off(H + 1, 0);
+  char what[64];
+  for (int h = 0; h < H; ++h) {
+    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+    snprintf(what, sizeof(what), "layer (%d, %d) head %d", t, l, h);
+    calibatt_status st = validate_csr(nq, d->nk, rp, col_idx ? col_idx + head_off[h] : nullptr, false, what);
+    if (st != CALIBATT_OK) return st;
+    if (repetitive && repetitive[h] && rp[nq] != 0)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s is repetitive but has a non-empty skip list", what);
+    head_off[h + 1] = head_off[h] + rp[nq];
+  }
+  const int64_t nnz = head_off[H];
+  if (d->nnz_used + nnz > d->nnz_cap)
+    return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld)",
+                (long long)d->nnz_used, (long long)nnz, (long long)d->nnz_cap);
+  std::vector<uint16_t> col16(nnz);
+  for (int64_t i = 0; i < nnz; ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
+  std::vector<int64_t> col_base(H);
+  for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + head_off[h];
+  // Work items of the sparse heads and their LPT schedule over the grid.
+  std::vector<uint32_t> items;
+  std::vector<int64_t> cost;
+  int32_t n_sparse = 0, n_rep = 0;
+  int64_t retained = 0;
+  for (int h = 0; h < H; ++h) {
+    if (repetitive && repetitive[h]) {
+      ++n_rep;
+      continue;
+    }
+    ++n_sparse;
+    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+    for (int r = 0; r < nq; ++r) {
+      items.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
+      cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);  // +2: Q load and epilogue
+      retained += rp[r + 1] - rp[r];
+    }
+  }
+  std::vector<int32_t> cta_ptr(d->G + 1), order(items.size());
+  lpt(static_cast<int32_t>(items.size()), cost.data(), d->G, cta_ptr.data(), order.data(), nullptr);
+  std::vector<uint32_t> sched(items.size());
+  for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != d->device) cudaSetDevice(d->device);
+  cudaError_t e = cudaSuccess;
+  if (nnz > 0) e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !sched.empty())
+    e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(d->d_cta_ptr + ly * (d->G + 1), cta_ptr.data(), sizeof(int32_t) * (d->G + 1), cudaMemcpyHostToDevice);
+  if (prev != d->device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return cuda_fail(e, "dictionary upload");
+  d->nnz_used += nnz;
+  for (int h = 0; h < H; ++h) d->rep[ly * H + h] = (repetitive && repetitive[h]) ? 1 : 0;
+  d->n_sparse[ly] = n_sparse;
+  d->n_rep[ly] = n_rep;
+  d->retained[ly] = retained;
+  d->layer_set[ly] = 1;
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_info(const calibatt_dict* d, int64_t* device_bytes, int64_t* nnz_total,
+                                   int32_t* num_ctas) {
+  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+  if (device_bytes) *device_bytes = d->device_bytes;
+  if (nnz_total) *nnz_total = d->nnz_used;
+  if (num_ctas) *num_ctas = d->G;
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_layer_info(const calibatt_dict* d, int32_t t, int32_t l, int32_t* n_sparse_heads,
+                                         int32_t* n_repetitive_heads, int64_t* retained_tiles) {
+  calibatt_status st = check_dict_layer(d, t, l);
+  if (st != CALIBATT_OK) return st;
+  const int64_t ly = d->layer(t, l);
+  if (n_sparse_heads) *n_sparse_heads = d->n_sparse[ly];
+  if (n_repetitive_heads) *n_repetitive_heads = d->n_rep[ly];
+  if (retained_tiles) *retained_tiles = d->retained[ly];
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_destroy(calibatt_dict* d) {
+  if (!d) return CALIBATT_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != d->device) cudaSetDevice(d->device);
+  cudaDeviceSynchronize();
+  d->release();
+  if (prev != d->device) cudaSetDevice(prev);
+  delete d;
+  cudaGetLastError();
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                                           const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
+                                           int32_t t, int32_t l, float softmax_scale, float* lse, void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+  if ((st = check_block(block)) != CALIBATT_OK) return st;
+  if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
+  if (dict->H != shape->heads) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
+  if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
+  if (dict->nq != ceil_div(shape->seq_len, block))
+    return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq, shape->seq_len,
+                ceil_div(shape->seq_len, block));
+  if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  return launch_sparse(q, k, v, o, *shape, block, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
+}
+
+calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
+                                     const calibatt_shape* shape, int32_t block, int32_t frames, int32_t rows,
+                                     int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
+                                     const int32_t* head_ids, int32_t n_heads, float softmax_scale, void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+  if ((st = check_block(block)) != CALIBATT_OK) return st;
+  return launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, head_ids, n_heads,
+                       softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void* v, void* o,
+                                        const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
+                                        int32_t t, int32_t l, int32_t frames, int32_t rows, int32_t cols,
+                                        const int32_t* anchor_rows, int32_t n_anchors, float softmax_scale,
+                                        float* lse, void* stream) {
+  calibatt_status st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
+  if (st != CALIBATT_OK) return st;
+  const int64_t ly = dict->layer(t, l);
+  std::vector<int32_t> heads;
+  for (int h = 0; h < dict->H; ++h)
+    if (dict->rep[ly * dict->H + h]) heads.push_back(h);
+  if (heads.empty()) return CALIBATT_OK;
+  for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
+    const int32_t nh = static_cast<int32_t>(std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0));
+    st = launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, heads.data() + h0, nh,
+                       softmax_scale, static_cast<cudaStream_t>(stream));
+    if (st != CALIBATT_OK) return st;
+  }
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_block_energy_workspace_size(const calibatt_shape* shape, size_t* bytes) {
+  calibatt_status st = check_shape(shape);
+  if (st != CALIBATT_OK) return st;
+  if (!bytes) return fail(CALIBATT_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = sizeof(float) * static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len;
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_block_energy(const void* q, const void* k, const calibatt_shape* shape, int32_t block,
+                                      float softmax_scale, float* energy, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if ((st = check_block(block)) != CALIBATT_OK) return st;
+  if (!q || !k || !energy || !workspace) return fail(CALIBATT_ERR_INVALID_ARG, "q, k, energy and workspace must be non-NULL");
+  size_t need = 0;
+  calibatt_block_energy_workspace_size(shape, &need);
+  if (workspace_bytes < need)
+    return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+  const int nb = ceil_div(shape->seq_len, block);
+  if (nb > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
+  calibatt::EnergyParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.k = k;
+  p.energy = energy;
+  p.lse = static_cast<float*>(workspace);
+  p.sb = shape->stride_b;
+  p.sn = shape->stride_n;
+  p.sh = shape->stride_h;
+  p.batch = shape->batch;
+  p.seq_len = shape->seq_len;
+  p.heads = shape->heads;
+  p.nb = nb;
+  p.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
+  cudaError_t e = calibatt::launch_block_energy(p, shape->head_dim, block, shape->dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block energy launch");
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_select_blocks(const float* energy, int64_t n_rows, int32_t nk, float tau, uint8_t* mask,
+                                       int32_t* count_accum, void* stream) {
+  if (n_rows < 0 || nk < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_rows must be >= 0 and nk >= 1");
+  if (nk > 4096) return fail(CALIBATT_ERR_UNSUPPORTED, "nk %d > 4096", nk);
+  if (n_rows > 2147483647LL) return fail(CALIBATT_ERR_UNSUPPORTED, "too many rows");
+  if (n_rows > 0 && (!energy || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "energy and mask must be non-NULL");
+  if (!(tau == tau)) return fail(CALIBATT_ERR_INVALID_ARG, "tau is NaN");
+  cudaError_t e = calibatt::launch_select_blocks(energy, n_rows, nk, tau, mask, count_accum, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,
+                                         uint8_t* mask, void* stream) {
+  if (n < 0 || n_prompts < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0 and n_prompts >= 1");
+  if (n > 0 && (!counts || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "counts and mask must be non-NULL");
+  if (!(rho == rho)) return fail(CALIBATT_ERR_INVALID_ARG, "rho is NaN");
+  cudaError_t e = calibatt::launch_aggregate(counts, n, n_prompts, rho, mask, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "aggregate launch");
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear) {
+  if (!code) return fail(CALIBATT_ERR_INVALID_ARG, "code is NULL");
+  int32_t* p = status_word_ptr();
+  if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  e = cudaMemcpy(code, p, sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (clear) {
+    e = cudaMemset(p, 0, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  }
+  if (*code != 0) return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_set_wait_timeout_ms(int32_t ms) {
+  if (ms < 1) return fail(CALIBATT_ERR_INVALID_ARG, "timeout must be >= 1 ms");
+  g_timeout_ns.store(static_cast<unsigned long long>(ms) * 1000000ull);
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_device_sm_count(int32_t* out) {
+  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+  const int n = device_sm_count();
+  if (n < 1) {
+    cudaGetLastError();
+    return fail(CALIBATT_ERR_CUDA, "no CUDA device");
+  }
+  *out = n;
+  return CALIBATT_OK;
+}
+
+}  // extern "C"

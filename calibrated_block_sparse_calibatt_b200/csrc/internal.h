@@ -1,0 +1,97 @@
+// Internal declarations shared by the library's translation units: kernel
+// parameter blocks and the launch functions the C ABI layer calls.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace calibatt {
+
+constexpr int kMaxAnchors = 16;
+constexpr int kMaxHeadsPerCall = 128;
+
+// Skip lists and persistent schedule of one dictionary layer (t, l).
+// Work item = (head << 16) | query_block.
+struct LayerSchedule {
+  const int32_t* row_ptr;   // [H][nq + 1], per head, starting at 0
+  const int64_t* col_base;  // [H], offset of each head's list in `col`
+  const uint16_t* col;      // retained key-block indices
+  const uint32_t* items;    // work items grouped by CTA
+  const int32_t* cta_ptr;   // [grid + 1], CTA c runs items[cta_ptr[c] .. cta_ptr[c+1])
+  int32_t nq;
+};
+
+// Frame geometry of the anchor path.  Token = (f * rows + row) * cols + col.
+// Packed anchor query p (0 <= p < anchor_tokens) is
+//   f = p / (n_anchors * cols), a = (p / cols) % n_anchors, col = p % cols,
+// served rows of anchor a are [group_lo[a], group_hi[a]].
+struct AnchorGeom {
+  int32_t frames, rows, cols, n_anchors;
+  int32_t anchor_tokens;   // frames * n_anchors * cols
+  int32_t tiles_per_head;  // ceil(anchor_tokens / 128)
+  int32_t n_heads;
+  int16_t anchor_row[kMaxAnchors];
+  int16_t group_lo[kMaxAnchors];
+  int16_t group_hi[kMaxAnchors];
+  int16_t head_ids[kMaxHeadsPerCall];
+};
+
+// Tensor-core (tcgen05) attention kernel parameters, passed as __grid_constant__.
+struct TcParams {
+  CUtensorMap tm_q;  // bf16 Q/K/V, dims {D, x1, x2, x3}, box {64, 1|128, ...}
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  const uint16_t* q;  // raw Q (anchor-row gather)
+  uint16_t* o;
+  float* lse;  // nullable [batch, heads, seq_len]
+  int64_t sb, sn, sh;  // element strides shared by Q, K, V, O
+  int32_t batch, seq_len, heads, nb;
+  int32_t pos_n, pos_h, pos_b;  // which tensor-map dimension (1..3) holds N, H, batch
+  float scale_log2;             // softmax_scale * log2(e)
+  LayerSchedule sched;
+  AnchorGeom anc;
+  int32_t* status;
+  unsigned long long timeout_ns;
+};
+
+// CUDA-core attention kernel parameters (FP32 or BF16, any supported block).
+struct SimtParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int64_t sb, sn, sh;
+  int32_t batch, seq_len, heads, nb;
+  float scale_log2;
+  LayerSchedule sched;           // sparse mode: items unused, heads from head list
+  int32_t n_heads;               // sparse mode: number of heads in head_ids
+  int16_t head_ids[kMaxHeadsPerCall];
+  AnchorGeom anc;
+};
+
+struct EnergyParams {
+  const void* q;
+  const void* k;
+  float* energy;  // [batch, heads, nb, nb]
+  float* lse;     // workspace [batch, heads, seq_len]
+  int64_t sb, sn, sh;
+  int32_t batch, seq_len, heads, nb;
+  float scale_log2;
+};
+
+cudaError_t launch_tc_attn(const TcParams& p, int head_dim, bool anchor, int grid, cudaStream_t s);
+cudaError_t launch_simt_attn(const SimtParams& p, int head_dim, int block, int dtype, bool anchor,
+                             int n_items, cudaStream_t s);
+cudaError_t launch_block_energy(const EnergyParams& p, int head_dim, int block, int dtype,
+                                cudaStream_t s);
+cudaError_t launch_select_blocks(const float* energy, int64_t n_rows, int32_t nk, float tau,
+                                 uint8_t* mask, int32_t* count_accum, cudaStream_t s);
+cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,
+                             uint8_t* mask, cudaStream_t s);
+
+// Dynamic shared memory the tensor-core kernel needs for a head dimension.
+size_t tc_smem_bytes(int head_dim);
+
+}  // namespace calibatt

@@ -1,0 +1,267 @@
+/*
+ * calibatt.h - C ABI of the CalibAtt B200 library (libcalibatt.so).
+ *
+ * CalibAtt ("Accelerating Text-to-Video Generation with Calibrated Sparse
+ * Attention", paper note on papernotes.org, section "Method") runs video
+ * self-attention through one of two precompiled paths per (timestep, layer,
+ * head):
+ *   - block-sparse attention over a calibrated list of retained key blocks
+ *     per query block (Key Designs 1, 2 and 4);
+ *   - anchor-row attention with output broadcast for heads flagged spatially
+ *     repetitive (Key Designs 3 and 4).
+ * It also exposes the offline calibration steps: block energy (Eq. (5)),
+ * top-mass selection and cross-prompt aggregation (Eq. (8)-(9)).
+ *
+ * Conventions for every entry point:
+ *   - Every call returns a calibatt_status.  No C++ exception crosses the ABI.
+ *     On failure calibatt_last_error() returns a message for the calling thread.
+ *   - Device pointers are owned by the caller.  The library never allocates
+ *     device memory on the attention or calibration calls; the mask dictionary
+ *     is the one library-owned object and is allocated at creation.
+ *   - GPU work is enqueued asynchronously on the caller's stream (a
+ *     cudaStream_t passed as void*; NULL is the legacy default stream).
+ *     Nothing is synchronised except where a function says so.
+ *   - Activations are [batch, N_alloc, heads, head_dim] with the last dimension
+ *     contiguous; strides are in elements.  Tokens are ordered frame-major,
+ *     then spatial row, then column: token = f*R*C + row*C + col.  Only the
+ *     first seq_len tokens are read; padded rows of the output are not written.
+ *   - A block is B consecutive tokens; nb = ceil(seq_len / B) blocks, the last
+ *     one possibly partial.  Keys at index >= seq_len are excluded.
+ *   - softmax_scale <= 0 selects 1/sqrt(head_dim).
+ *   - Arguments are validated on the host before anything is enqueued:
+ *     CALIBATT_ERR_INVALID_ARG for null pointers, inconsistent sizes, strides or
+ *     misaligned bases; CALIBATT_ERR_UNSUPPORTED for head_dim, block or dtype
+ *     outside the supported set; CALIBATT_ERR_CUDA when a CUDA call or a launch
+ *     fails (the CUDA error is cleared and named in calibatt_last_error()).
+ */
+#ifndef CALIBATT_H_
+#define CALIBATT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t calibatt_status;
+
+#define CALIBATT_OK 0
+#define CALIBATT_ERR_INVALID_ARG 1
+#define CALIBATT_ERR_UNSUPPORTED 2
+#define CALIBATT_ERR_CUDA 3
+#define CALIBATT_ERR_TIMEOUT 4
+#define CALIBATT_ERR_OOM 5
+
+#define CALIBATT_DTYPE_BF16 0
+#define CALIBATT_DTYPE_FP32 1
+
+/* Shape of Q, K, V and O (all four share it).  head_dim in {64, 128};
+ * dtype CALIBATT_DTYPE_BF16 or CALIBATT_DTYPE_FP32.  Strides in elements;
+ * the head_dim dimension has stride 1.  For BF16 every stride must be a
+ * multiple of 8 elements and every base 16-byte aligned. */
+typedef struct calibatt_shape {
+  int32_t batch;
+  int32_t seq_len;   /* N: valid tokens */
+  int32_t heads;     /* H */
+  int32_t head_dim;  /* D */
+  int64_t stride_b;
+  int64_t stride_n;
+  int64_t stride_h;
+  int32_t dtype;
+  int32_t reserved;  /* must be 0 */
+} calibatt_shape;
+
+/* Opaque mask dictionary: per (timestep t, layer l, head h) either a skip
+ * list of retained key blocks for every query block, or the repetitive flag
+ * that routes the head to the anchor path (Key Designs 4: "the current
+ * timestep, layer, and head select the appropriate record"). */
+typedef struct calibatt_dict calibatt_dict;
+
+/* ---------------------------------------------------------------- status */
+
+/* Static text for a status code. */
+const char* calibatt_status_string(calibatt_status status);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* calibatt_last_error(void);
+
+/* ABI version of this header (incremented on incompatible change). */
+int32_t calibatt_abi_version(void);
+
+/* ------------------------------------------------- host-only utilities */
+
+/* Checks one skip list in CSR form (Key Designs 4: each binary mask becomes
+ * a read-only list of key blocks to compute for each query block).
+ *   row_ptr: host int32[nq + 1], row_ptr[0] == 0, non-decreasing;
+ *   col_idx: host int32[row_ptr[nq]], each row strictly ascending, in [0, nk);
+ *   require_diagonal != 0 additionally demands block r in row r (nq == nk).
+ * Returns CALIBATT_OK or CALIBATT_ERR_INVALID_ARG naming the first offence. */
+calibatt_status calibatt_csr_validate(int32_t nq, int32_t nk, const int32_t* row_ptr,
+                                      const int32_t* col_idx, int32_t require_diagonal);
+
+/* Re-encodes a validated CSR skip list as contiguous key-block intervals, the
+ * encoding the paper note describes (Key Designs 4).  Outputs (host):
+ *   interval_ptr int32[nq + 1]; interval_start, interval_len int32[capacity].
+ * *n_intervals receives the total.  CALIBATT_ERR_INVALID_ARG if capacity is
+ * too small (*n_intervals still receives the needed count). */
+calibatt_status calibatt_csr_to_intervals(int32_t nq, const int32_t* row_ptr,
+                                          const int32_t* col_idx, int32_t* interval_ptr,
+                                          int32_t* interval_start, int32_t* interval_len,
+                                          int64_t capacity, int64_t* n_intervals);
+
+/* Longest-processing-time list scheduling of n_items work items with the
+ * given costs onto n_bins bins: items in descending cost (ties by index) each
+ * go to the currently least-loaded bin (ties by lower bin).  Outputs (host):
+ *   bin_ptr int32[n_bins + 1]; item_order int32[n_items] lists the items of
+ *   bin b at item_order[bin_ptr[b] .. bin_ptr[b+1]) in assignment order;
+ *   *makespan (nullable) receives the largest bin load.
+ * The paper note does not describe a schedule; this balances the persistent
+ * attention kernel's query-block work by retained key-block count. */
+calibatt_status calibatt_lpt_schedule(int32_t n_items, const int64_t* cost, int32_t n_bins,
+                                      int32_t* bin_ptr, int32_t* item_order,
+                                      int64_t* makespan);
+
+/* --------------------------------------------------------- dictionary */
+
+/* Creates an empty dictionary for T timesteps x L layers x H heads with
+ * nq == nk == number of blocks of size `block` (64 or 128).  Device memory
+ * for up to nnz_capacity retained blocks in total (2 bytes each) plus
+ * per-record offsets and schedules is allocated now, on the current device.
+ * num_ctas <= 0 selects the device's SM count (the persistent grid size the
+ * schedules are built for).  CALIBATT_ERR_OOM if the allocation fails. */
+calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk,
+                                     int32_t block, int64_t nnz_capacity, int32_t num_ctas,
+                                     calibatt_dict** out);
+
+/* Fills the records of layer l at timestep t for all H heads (each layer
+ * may be set once).  Host inputs:
+ *   row_ptr int32[H][nq + 1]: each head's CSR row pointer, starting at 0;
+ *   col_idx int32[...]: the heads' column lists concatenated in head order;
+ *   repetitive uint8[H] (nullable = none): non-zero routes the head to the
+ *     anchor path (Key Designs 3); its CSR must then be empty (row_ptr all 0).
+ * Every CSR is validated as calibatt_csr_validate (no diagonal requirement),
+ * converted to 16-bit indices, copied to the device (synchronously), and a
+ * longest-processing-time schedule of the layer's (head, query block) work
+ * is built for the dictionary's num_ctas. */
+calibatt_status calibatt_dict_set_layer(calibatt_dict* dict, int32_t t, int32_t l,
+                                        const int32_t* row_ptr, const int32_t* col_idx,
+                                        const uint8_t* repetitive);
+
+/* Totals: device bytes held, retained blocks stored, persistent grid size. */
+calibatt_status calibatt_dict_info(const calibatt_dict* dict, int64_t* device_bytes,
+                                   int64_t* nnz_total, int32_t* num_ctas);
+
+/* Per-layer counts: heads on each path and retained (query, key) block tiles
+ * of its sparse heads.  CALIBATT_ERR_INVALID_ARG if the layer is not set. */
+calibatt_status calibatt_dict_layer_info(const calibatt_dict* dict, int32_t t, int32_t l,
+                                         int32_t* n_sparse_heads, int32_t* n_repetitive_heads,
+                                         int64_t* retained_tiles);
+
+/* Frees the dictionary's device and host memory (synchronises the device). */
+calibatt_status calibatt_dict_destroy(calibatt_dict* dict);
+
+/* ------------------------------------------------------- hot path */
+
+/* Block-sparse attention for every non-repetitive head of record (t, l)
+ * (Key Designs 4: non-repetitive heads skip unselected blocks and compute the
+ * retained connections from the current input).  For query i of head h:
+ *   O_i = softmax over keys j < N with M_h[floor(i/B), floor(j/B)] = 1 of
+ *         (scale * q_i . k_j), weighting v_j;
+ * a query block whose list is empty produces zeros.  q, k, v, o: device
+ * arrays of `shape` (the output shares the input strides and dtype); only
+ * heads routed to this path are written.  lse (nullable): device float32
+ * [batch, heads, seq_len], receives ln(sum_j exp(scale * q_i . k_j)) over the
+ * retained keys, -inf for empty lists.  shape->heads must equal the
+ * dictionary's H and block its block size.
+ * BF16 with block 128 runs the tensor-core kernel; other combinations run the
+ * CUDA-core kernel (FP32 keeps float32 products). */
+calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const void* v, void* o,
+                                           const calibatt_shape* shape, int32_t block,
+                                           const calibatt_dict* dict, int32_t t, int32_t l,
+                                           float softmax_scale, float* lse, void* stream);
+
+/* Anchor-row attention with broadcast for the given heads (Key Designs 3):
+ * only queries of the anchor rows of every frame attend, densely over all N
+ * keys and values; every token (f, row, col) takes the output of the anchor
+ * row nearest to `row` in the same frame and column (distance ties go to the
+ * lower anchor).  frames * rows * cols must equal shape->seq_len.
+ *   anchor_rows: host int32[n_anchors], strictly ascending in [0, rows),
+ *     1 <= n_anchors <= 16;
+ *   head_ids: host int32[n_heads], distinct heads in [0, heads), n_heads <= 128.
+ * Every token of the listed heads is written. */
+calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
+                                     const calibatt_shape* shape, int32_t block,
+                                     int32_t frames, int32_t rows, int32_t cols,
+                                     const int32_t* anchor_rows, int32_t n_anchors,
+                                     const int32_t* head_ids, int32_t n_heads,
+                                     float softmax_scale, void* stream);
+
+/* Both paths of record (t, l): the dictionary's repetitive heads through the
+ * anchor path and the rest through the block-sparse path, enqueued on one
+ * stream (Key Designs 4: the repetition flag selects one path per head; the
+ * paths are alternatives, never stacked).  Arguments as above; lse
+ * (nullable) is written for the sparse heads only. */
+calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void* v, void* o,
+                                        const calibatt_shape* shape, int32_t block,
+                                        const calibatt_dict* dict, int32_t t, int32_t l,
+                                        int32_t frames, int32_t rows, int32_t cols,
+                                        const int32_t* anchor_rows, int32_t n_anchors,
+                                        float softmax_scale, float* lse, void* stream);
+
+/* ------------------------------------------------ offline calibration */
+
+/* Device scratch bytes calibatt_block_energy needs for `shape`. */
+calibatt_status calibatt_block_energy_workspace_size(const calibatt_shape* shape,
+                                                     size_t* bytes);
+
+/* Block energies (Key Designs 1, Eq. (5)) of the dense, unmasked attention:
+ *   E[b, h, r, c] = (1/|I_r|) * sum_{i in I_r} sum_{j in J_c} P_ij
+ * with |I_r| the valid queries of block r (B for full blocks), so every row
+ * of E sums to one.  energy: device float32 [batch, heads, nb, nb].
+ * workspace: caller-owned device scratch of at least
+ * calibatt_block_energy_workspace_size() bytes (row log-sum-exp values).
+ * Computed on CUDA cores in float32 with a fixed summation order, so repeated
+ * calls give bitwise identical energies. */
+calibatt_status calibatt_block_energy(const void* q, const void* k,
+                                      const calibatt_shape* shape, int32_t block,
+                                      float softmax_scale, float* energy, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/* Top-mass selection (Key Designs 1, after Eq. (5)) for n_rows rows of nk
+ * energies (device float32 [n_rows, nk], nk <= 4096): order each row by
+ * energy descending, ties to the lower key block; keep the shortest prefix
+ * whose cumulative mass, summed in float64 in that order, is >= tau (as
+ * float64); keep every block if none is.  mask: device uint8 [n_rows, nk]
+ * (1 = kept).  count_accum (nullable): device int32 [n_rows, nk], incremented
+ * by the mask (for cross-prompt aggregation). */
+calibatt_status calibatt_select_blocks(const float* energy, int64_t n_rows, int32_t nk,
+                                       float tau, uint8_t* mask, int32_t* count_accum,
+                                       void* stream);
+
+/* Cross-prompt aggregation (Key Designs 2, Eq. (8)-(9)): mask[i] =
+ * (counts[i] / n_prompts >= rho), evaluated in float64 with rho widened from
+ * float.  counts: device int32[n]; mask: device uint8[n]. */
+calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32_t n_prompts,
+                                         float rho, uint8_t* mask, void* stream);
+
+/* ------------------------------------------------------- diagnostics */
+
+/* Synchronises `stream`, then reports the device status word that the
+ * kernels set when a bounded wait runs out (CALIBATT_ERR_TIMEOUT in the low
+ * byte, the waiting role and barrier above it) and optionally clears it.
+ * Returns CALIBATT_ERR_TIMEOUT when the word is non-zero. */
+calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);
+
+/* Time limit of every in-kernel barrier wait, in milliseconds (default 4000;
+ * applies to launches made after the call). */
+calibatt_status calibatt_set_wait_timeout_ms(int32_t ms);
+
+/* Number of SMs of the current device (the default persistent grid size). */
+calibatt_status calibatt_device_sm_count(int32_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CALIBATT_H_ */

@@ -1,0 +1,360 @@
+"""GPU parity of libcalibatt.so against the float64 CPU oracle.
+
+Every call goes through the C ABI (ctypes binding).  Tolerances: float32
+inputs max-abs <= 1e-4; bf16 inputs max-abs <= 2e-2 and mean-abs <= 2e-3;
+selected block sets bit-exact.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import calibatt_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX, BF16_MEAN, FP32_MAX = 2e-2, 2e-3, 1e-4
+
+
+@pytest.fixture(scope="module")
+def C(calibatt_lib):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    calibatt_lib.set_wait_timeout_ms(4000)
+    return calibatt_lib
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _check_status(C):
+    torch.cuda.synchronize()
+    assert C.device_status() == 0
+
+
+def _assert_close(got, ref, dtype):
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), "non-finite output"
+    if dtype == "fp32":
+        assert err.max() <= FP32_MAX, f"max-abs {err.max():.3e}"
+    else:
+        assert err.max() <= BF16_MAX, f"max-abs {err.max():.3e}"
+        assert err.mean() <= BF16_MEAN, f"mean-abs {err.mean():.3e}"
+    return float(err.max()), float(err.mean())
+
+
+def _run_sparse(C, q, k, v, masks, block, lse=False, num_ctas=0):
+    b, n, h, d = q.shape
+    nb = O.num_blocks(n, block)
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    out = torch.full_like(q, float("nan"))
+    lse_t = torch.full((b, h, n), float("nan"), device=q.device) if lse else None
+    with C.MaskDictionary(1, 1, h, nb, nb, block, max(1, ci.size), num_ctas) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_block_sparse_attn(q, k, v, out, dct, 0, 0, block, lse=lse_t)
+        _check_status(C)
+    return out, lse_t
+
+
+def _random_masks(seed, h, nb, density, empty_row_head=None):
+    rng = np.random.default_rng(seed)
+    masks = []
+    for hh in range(h):
+        m = rng.random((nb, nb)) < density
+        m[np.arange(nb), np.arange(nb)] = True
+        if hh == empty_row_head:
+            m[1, :] = False
+        masks.append(m)
+    return masks
+
+
+# ------------------------------------------------------------------ tiny config
+
+def _tiny_inputs(dtype):
+    wl = W.WORKLOADS["tiny"]
+    q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, dtype, wl.input_std, "cuda")
+    mask0 = W.tiny_block_mask(1, wl.num_blocks, 0.5)
+    return wl, q, k, v, mask0
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_tiny_dual_path(C, dtype):
+    wl, q, k, v, mask0 = _tiny_inputs(dtype)
+    nb = wl.num_blocks
+    rp, ci, rep = C.masks_to_layer_csr([mask0, None], wl.heads, nb)
+    out = torch.full_like(q, float("nan"))
+    with C.MaskDictionary(1, 1, wl.heads, nb, nb, wl.block, ci.size) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_dual_path_attn(q, k, v, out, dct, 0, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
+        _check_status(C)
+    qn, kn, vn = _np(q)[0], _np(k)[0], _np(v)[0]
+    ref0, _ = O.block_sparse_attention(qn[:, 0], kn[:, 0], vn[:, 0], mask0, wl.block)
+    ref1, _ = O.anchor_attention(qn[:, 1], kn[:, 1], vn[:, 1], wl.frames, wl.rows, wl.cols, wl.anchors)
+    got = _np(out)[0]
+    _assert_close(got[:, 0], ref0, dtype)
+    _assert_close(got[:, 1], ref1, dtype)
+
+
+# ------------------------------------------------------------ tensor-core sparse
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_tc_sparse_ragged_multi_batch(C, d):
+    b, n, h, block = 2, 1000, 3, 128            # 8 blocks, last holds 104 tokens
+    # allocations of 1024 rows whose padding rows are NaN; the library sees views of the n valid rows
+    qa, ka, va = W.make_qkv(11, b, n, h, d, "bf16", 1.0, "cuda", seq_alloc=1024)
+    q, k, v = qa[:, :n], ka[:, :n], va[:, :n]
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(5, h, nb, 0.5, empty_row_head=2)
+    out_alloc = torch.full_like(qa, float("nan"))
+    lse = torch.full((b, h, n), float("nan"), device="cuda")
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    with C.MaskDictionary(1, 1, h, nb, nb, block, ci.size) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_block_sparse_attn(q, k, v, out_alloc[:, :n], dct, 0, 0, block, lse=lse)
+        _check_status(C)
+    out = out_alloc[:, :n]
+    ref, ref_lse = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block, seq_len=n)
+    _assert_close(_np(out), ref, "bf16")
+    assert torch.isnan(out_alloc[:, n:]).all(), "padding rows of the output were written"
+    got_lse = lse.cpu().numpy().astype(np.float64)
+    finite = np.isfinite(ref_lse)
+    assert (np.isneginf(got_lse) == ~finite).all()
+    assert np.abs(got_lse[finite] - ref_lse[finite]).max() < 2e-2
+    # head 2 row-block 1 is empty -> zeros
+    assert (out[:, 128:256, 2].float() == 0).all()
+
+
+def test_tc_all_ones_mask_is_dense_attention(C):
+    b, n, h, d, block = 1, 777, 2, 128, 128
+    q, k, v = W.make_qkv(12, b, n, h, d, "bf16", 1.0, "cuda")
+    nb = O.num_blocks(n, block)
+    out, _ = _run_sparse(C, q, k, v, [np.ones((nb, nb), bool)] * h, block)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double().permute(0, 2, 1, 3).cpu(), k.double().permute(0, 2, 1, 3).cpu(),
+        v.double().permute(0, 2, 1, 3).cpu()).permute(0, 2, 1, 3).numpy()
+    _assert_close(_np(out), ref, "bf16")
+
+
+def test_tc_sparse_deterministic_and_schedule_independent(C):
+    b, n, h, d, block = 1, 2048, 4, 128, 128
+    q, k, v = W.make_qkv(13, b, n, h, d, "bf16", 128 ** -0.25, "cuda")
+    masks = _random_masks(6, h, 16, 0.35)
+    o1, _ = _run_sparse(C, q, k, v, masks, block)
+    o2, _ = _run_sparse(C, q, k, v, masks, block)
+    o3, _ = _run_sparse(C, q, k, v, masks, block, num_ctas=7)   # different persistent grid
+    assert torch.equal(o1, o2)
+    assert torch.equal(o1, o3)
+
+
+def test_tc_sparse_peaked_scores_rescale(C):
+    # large logits make the running maximum jump across blocks (rescale path)
+    b, n, h, d, block = 1, 1536, 2, 128, 128
+    q, k, v = W.make_qkv(14, b, n, h, d, "bf16", 1.0, "cuda")
+    q = (q.float() * 3.0).to(torch.bfloat16)
+    masks = _random_masks(7, h, 12, 0.6)
+    out, _ = _run_sparse(C, q, k, v, masks, block)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block)
+    _assert_close(_np(out), ref, "bf16")
+
+
+# ------------------------------------------------------------ tensor-core anchor
+
+def test_tc_anchor_broadcast(C):
+    frames, rows, cols, h, d = 3, 10, 24, 3, 128
+    n = frames * rows * cols
+    anchors = (1, 4, 8)
+    q, k, v = W.make_qkv(15, 1, n, h, d, "bf16", 1.0, "cuda")
+    out = torch.full_like(q, float("nan"))
+    C.calibatt_anchor_attn(q, k, v, out, frames, rows, cols, anchors, [0, 2])
+    _check_status(C)
+    ref = O.anchor_attention_bnhd(_np(q), _np(k), _np(v), frames, rows, cols, anchors, heads=[0, 2])
+    got = _np(out)
+    _assert_close(got[:, :, [0, 2]], ref, "bf16")
+    assert torch.isnan(out[:, :, 1]).all(), "a head not listed was written"
+    # every broadcast row is a bitwise copy of its anchor row
+    near = O.nearest_anchor_rows(rows, anchors)
+    o = out.view(1, frames, rows, cols, h, d)
+    for rho in range(rows):
+        assert torch.equal(o[:, :, rho, :, [0, 2]], o[:, :, near[rho], :, [0, 2]])
+
+
+def test_simt_anchor_fp32(C):
+    frames, rows, cols, h, d = 2, 9, 16, 2, 64
+    n = frames * rows * cols
+    anchors = (2, 6)
+    q, k, v = W.make_qkv(16, 1, n, h, d, "fp32", 1.0, "cuda")
+    out = torch.full_like(q, float("nan"))
+    C.calibatt_anchor_attn(q, k, v, out, frames, rows, cols, anchors, [1], block=64)
+    _check_status(C)
+    ref = O.anchor_attention_bnhd(_np(q), _np(k), _np(v), frames, rows, cols, anchors, heads=[1])
+    _assert_close(_np(out)[:, :, [1]], ref, "fp32")
+
+
+def test_simt_sparse_bf16_block64_and_fp32_block128(C):
+    for dtype, block, d in (("bf16", 64, 128), ("fp32", 128, 128)):
+        b, n, h = 1, 700, 2
+        q, k, v = W.make_qkv(17, b, n, h, d, dtype, 1.0, "cuda")
+        nb = O.num_blocks(n, block)
+        masks = _random_masks(8, h, nb, 0.5, empty_row_head=1)
+        out, lse = _run_sparse(C, q, k, v, masks, block, lse=True)
+        ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block)
+        _assert_close(_np(out), ref, dtype)
+
+
+# ------------------------------------------------------ full-size sampled parity
+
+def _sampled_blocks(rng, nb, k):
+    mid = rng.choice(np.arange(1, nb - 1), size=k - 2, replace=False)
+    return sorted({0, nb - 1, *mid.tolist()})
+
+
+@pytest.mark.parametrize("name", ["480p", "720p"])
+def test_full_size_sparse_sampled(C, name):
+    wl = W.WORKLOADS[name]
+    q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    masks, _ = W.workload_masks(wl)
+    masks = [masks[h] for h in range(wl.heads)]
+    out, _ = _run_sparse(C, q, k, v, masks, wl.block)
+    rng = np.random.default_rng(1)
+    errs = []
+    heads_deep = set(rng.choice(wl.heads, 3, replace=False).tolist())
+    for h in range(wl.heads):
+        blocks = _sampled_blocks(rng, wl.num_blocks, 8 if h in heads_deep else 3)
+        rows = np.concatenate([np.arange(r * 128, min(wl.seq_len, (r + 1) * 128)) for r in blocks])
+        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
+        ref, _ = O.block_sparse_attention(qh, kh, vh, masks[h], wl.block, rows=rows)
+        got = _np(out[0, torch.as_tensor(rows, device=q.device), h])
+        errs.append(np.abs(got - ref))
+    err = np.concatenate([e.ravel() for e in errs])
+    assert err.max() <= BF16_MAX and err.mean() <= BF16_MEAN, (err.max(), err.mean())
+
+
+def test_full_size_dual_path_sampled(C):
+    wl = W.WORKLOADS["720p_dual"]
+    q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    masks, rep_heads = W.workload_masks(wl)
+    assert len(rep_heads) == 12
+    rp, ci, rep = C.masks_to_layer_csr([masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks)
+    out = torch.full_like(q, float("nan"))
+    with C.MaskDictionary(1, 1, wl.heads, wl.num_blocks, wl.num_blocks, wl.block, ci.size) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_dual_path_attn(q, k, v, out, dct, 0, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
+        _check_status(C)
+    assert not torch.isnan(out).any()
+    rng = np.random.default_rng(2)
+    # anchor heads: rows of two frames, including the last frame's last row
+    f_rows = np.concatenate([np.arange(f * wl.tokens_per_frame, (f + 1) * wl.tokens_per_frame)
+                             for f in (int(rng.integers(0, wl.frames - 1)), wl.frames - 1)])
+    sample = f_rows[rng.choice(len(f_rows), 600, replace=False)]
+    for h in rep_heads[:4]:
+        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
+        ref, _ = O.anchor_attention(qh, kh, vh, wl.frames, wl.rows, wl.cols, wl.anchors, rows=sample)
+        got = _np(out[0, torch.as_tensor(sample, device=q.device), h])
+        _assert_close(got, ref, "bf16")
+    # broadcast rows are bitwise copies of their anchor rows, for every repetitive head
+    near = O.nearest_anchor_rows(wl.rows, wl.anchors)
+    o = out.view(1, wl.frames, wl.rows, wl.cols, wl.heads, wl.head_dim)[..., list(rep_heads), :]
+    for rho in range(wl.rows):
+        assert torch.equal(o[:, :, rho], o[:, :, near[rho]])
+    # sparse heads: three sampled q-blocks each for four heads
+    sparse_heads = [h for h in range(wl.heads) if h not in rep_heads][:4]
+    for h in sparse_heads:
+        blocks = _sampled_blocks(rng, wl.num_blocks, 3)
+        rows = np.concatenate([np.arange(r * 128, min(wl.seq_len, (r + 1) * 128)) for r in blocks])
+        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
+        ref, _ = O.block_sparse_attention(qh, kh, vh, masks[h], wl.block, rows=rows)
+        got = _np(out[0, torch.as_tensor(rows, device=q.device), h])
+        _assert_close(got, ref, "bf16")
+
+
+# --------------------------------------------------------- offline calibration
+
+def _energy(C, q, k, block):
+    b, n, h, _ = q.shape
+    nb = O.num_blocks(n, block)
+    e = torch.full((b, h, nb, nb), float("nan"), device=q.device)
+    ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, device=q.device)
+    C.calibatt_block_energy(q, k, e, ws, block)
+    _check_status(C)
+    return e
+
+
+@pytest.mark.parametrize("dtype,n,block,d,std", [("fp32", 256, 64, 64, 1.0), ("bf16", 300, 128, 128, 1.0),
+                                                  ("fp32", 500, 64, 128, 0.3)])
+def test_block_energy(C, dtype, n, block, d, std):
+    q, k, _ = W.make_qkv(20, 1, n, 2, d, dtype, std, "cuda")
+    e = _energy(C, q, k, block)
+    ref = O.block_energy_bnhd(_np(q), _np(k), block)
+    got = e.cpu().numpy().astype(np.float64)
+    assert np.abs(got - ref).max() < 2e-6
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-5)
+    e2 = _energy(C, q, k, block)
+    assert torch.equal(e, e2), "energies are not bitwise repeatable"
+
+
+def test_select_blocks_bit_exact_on_identical_energies(C):
+    rng = np.random.default_rng(21)
+    n_rows, nk = 300, 37
+    e = rng.dirichlet(np.full(nk, 0.3), size=n_rows).astype(np.float32)
+    e[::3, 5] = e[::3, 6]                          # exact ties
+    e[::7] = np.round(e[::7] * 64) / 64            # many ties
+    et = torch.from_numpy(e).cuda()
+    for tau in (0.5, 0.9, 0.99, 1.0):
+        mask = torch.zeros((n_rows, nk), dtype=torch.uint8, device="cuda")
+        cnt = torch.zeros((n_rows, nk), dtype=torch.int32, device="cuda")
+        C.calibatt_select_blocks(et, tau, mask, cnt)
+        _check_status(C)
+        ref = O.select_blocks(e.astype(np.float64), float(np.float32(tau)))
+        assert (mask.cpu().numpy().astype(bool) == ref).all()
+        assert (cnt.cpu().numpy() == ref.astype(np.int32)).all()
+
+
+def test_aggregate_worked_example(C):
+    counts = torch.tensor([32, 33, 63, 64, 0, 1, 30, 31], dtype=torch.int32, device="cuda")
+    mask = torch.zeros(8, dtype=torch.uint8, device="cuda")
+    C.calibatt_aggregate_masks(counts, 64, 0.5, mask)
+    _check_status(C)
+    assert mask.cpu().tolist() == [1, 1, 1, 1, 0, 0, 0, 0]
+
+
+def _margin_ok(e_ref, tau, margin=1e-5):
+    """Rows whose selection is decided with a float64 margin above `margin`."""
+    ok = []
+    for row in e_ref.reshape(-1, e_ref.shape[-1]):
+        srt = np.sort(row)[::-1]
+        cum = np.add.accumulate(srt)
+        gaps = np.abs(np.diff(srt)) if len(srt) > 1 else np.array([1.0])
+        ok.append(min(np.abs(cum - tau).min(), gaps.min() if gaps.size else 1.0) > margin)
+    return np.array(ok)
+
+
+@pytest.mark.parametrize("std,tau", [(1.0, 0.99), (4.0, 0.5), (4.0, 0.9)])
+def test_energy_select_union_tiny(C, std, tau):
+    """Tiny configuration: 4 seeded Q/K draws, selection at tau, masks unioned (rho = 1/4)."""
+    wl = W.WORKLOADS["tiny"]
+    nb = wl.num_blocks
+    cnt = torch.zeros((wl.batch * wl.heads * nb, nb), dtype=torch.int32, device="cuda")
+    ref_masks = []
+    decided = []
+    for s in (10, 11, 12, 13):
+        q, k, _ = W.make_qkv(s, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "fp32", std, "cuda")
+        e = _energy(C, q, k, wl.block)
+        mask = torch.zeros((wl.batch * wl.heads * nb, nb), dtype=torch.uint8, device="cuda")
+        C.calibatt_select_blocks(e.view(-1, nb), tau, mask, cnt)
+        e_ref = O.block_energy_bnhd(_np(q), _np(k), wl.block).reshape(-1, nb)
+        tau64 = float(np.float32(tau))
+        ref = O.select_blocks(e_ref, tau64)
+        ok = _margin_ok(e_ref, tau64)
+        decided.append(ok)
+        got = mask.cpu().numpy().astype(bool)
+        assert (got[ok] == ref[ok]).all()
+        ref_masks.append(ref)
+    union = torch.zeros_like(cnt, dtype=torch.uint8)
+    C.calibatt_aggregate_masks(cnt, 4, 0.25, union)
+    _check_status(C)
+    all_ok = np.logical_and.reduce(decided)
+    ref_union = O.aggregate_masks(np.stack(ref_masks), 4, 0.25)
+    assert (union.cpu().numpy().astype(bool)[all_ok] == ref_union[all_ok]).all()
+    assert all_ok.mean() > 0.5
