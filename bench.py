@@ -205,6 +205,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the dense / dual-path / e2e legs")
+    ap.add_argument("--heads", type=int, default=40,
+                    help="heads of the 720p layer (fewer heads = smaller case for profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -231,8 +233,9 @@ def main():
 
     pk = peaks()
     stream = torch.cuda.current_stream()
-    wl = W.WORKLOADS["720p"]
-    masks, _ = W.workload_masks(wl)
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
+    masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])
     q, k, v = W.make_qkv(wl.seed + 7919 * rank, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
     o = torch.empty_like(q)
     d_sparse = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block)

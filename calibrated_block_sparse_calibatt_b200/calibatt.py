@@ -72,6 +72,7 @@ SIGNATURES = {
     "calibatt_block_energy": (_i32, [_vp, _vp, _P(Shape), _i32, _f32, _vp, _vp, ctypes.c_size_t, _vp]),
     "calibatt_select_blocks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp, _vp]),
     "calibatt_aggregate_masks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp]),
+    "calibatt_debug_exp2_fma": (_i32, [_vp, _vp, _i64, _vp]),
     "calibatt_device_status": (_i32, [_vp, _P(_i32), _i32]),
     "calibatt_set_wait_timeout_ms": (_i32, [_i32]),
     "calibatt_device_sm_count": (_i32, [_P(_i32)]),
@@ -169,6 +170,10 @@ def lpt_schedule(cost, n_bins):
     mk = ctypes.c_int64(0)
     check(LIB.calibatt_lpt_schedule(c.size, _ptr(c), n_bins, _ptr(bin_ptr), _ptr(order), ctypes.byref(mk)))
     return bin_ptr, order[:c.size], mk.value
+
+
+def calibatt_debug_exp2_fma(x, y, stream=None):
+    check(LIB.calibatt_debug_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
 def set_wait_timeout_ms(ms: int) -> None:

@@ -14,8 +14,9 @@
 //   warp  4    producer: TMA loads of Q and of K/V tiles gathered by block
 //              index (or a plain-load gather of anchor Q rows)
 //   warp  5    TMEM allocator and MMA issuer (one lane issues tcgen05.mma)
-// Tensor memory (512 columns): S = Q K^T at 0..127 (f32), P (bf16 pairs) at
-// 128..191, O accumulator at 256..256+D.
+// Tensor memory (512 columns): S = Q K^T at 0..127 (f32), two P buffers
+// (bf16 pairs) at 128..191 and 192..255, O accumulator at 256..256+D.  With P
+// double-buffered the softmax writes P_{j+1} while O += P_j V_j still runs.
 // Pipelines (mbarriers): Q 1 stage, K 3 stages, V 3 stages; S/P/O handshakes
 // between the MMA warp and the softmax warps.  Per key block j the MMA warp
 // issues S_j = Q K_j^T as soon as the softmax warps have read S_{j-1} out of
@@ -38,9 +39,12 @@ constexpr int kKStages = 3;
 constexpr int kVStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
-constexpr uint32_t kColP = 128;
+constexpr uint32_t kColP = 128;  // P buffer b at kColP + 64 * b
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleLog2 = 8.0f;
+// One pair in kPolyEvery of exponentials runs on the FMA pipe (exp2_fma)
+// instead of the MUFU unit, which would otherwise bound the softmax at D=128.
+constexpr int kPolyEvery = 4;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -55,8 +59,10 @@ struct Layout {
   static constexpr int bQFull = 0, bQEmpty = 1;
   static constexpr int bKFull = 2, bKEmpty = bKFull + kKStages;
   static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
-  static constexpr int bSFull = bVEmpty + kVStages, bSFree = bSFull + 1, bPFull = bSFree + 1;
-  static constexpr int bPVDone = bPFull + 1, bOFree = bPVDone + 1, bDrain = bOFree + 1;
+  static constexpr int bSFull = bVEmpty + kVStages, bSFree = bSFull + 1;
+  static constexpr int bPFull = bSFree + 1;      // [2], one per P buffer
+  static constexpr int bPVDone = bPFull + 2;     // [2], P.V reading P buffer b finished
+  static constexpr int bOFree = bPVDone + 2, bDrain = bOFree + 1;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
   static constexpr int kUsed = kMisc + 16;
@@ -236,10 +242,11 @@ __device__ void mma_role(const TcParams& p, uint32_t base, uint32_t tmem, const 
   bool ok = true;
 
   // O += P_t V_t for key-block iteration t (global counter); `first` zeroes O.
+  // P_t lives in tensor-memory buffer t & 1.
   auto issue_pv = [&](uint32_t t, bool first) -> bool {
-    const uint32_t vs = t % kVStages;
+    const uint32_t vs = t % kVStages, pb = t & 1;
     if (!W.wait(bar(L::bVFull + vs), (t / kVStages) & 1, 7)) return false;
-    if (!W.wait(bar(L::bPFull), t & 1, 8)) return false;
+    if (!W.wait(bar(L::bPFull + pb), (t >> 1) & 1, 8)) return false;
     if (first && item > 0 && !W.wait(bar(L::bOFree), (item - 1) & 1, 9)) return false;
     tc_fence_after();
     if (lane == 0) {
@@ -247,11 +254,11 @@ __device__ void mma_role(const TcParams& p, uint32_t base, uint32_t tmem, const 
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         // B = V (MN-major): 16 keys per step = 2048 bytes; next 64 columns of D at +16 KB.
-        mma_ts(tmem + kColO, tmem + kColP + s * 8, sw128_desc(v_base + s * 2048, kChunkBytes, 1024),
+        mma_ts(tmem + kColO, tmem + kColP + pb * 64 + s * 8, sw128_desc(v_base + s * 2048, kChunkBytes, 1024),
                kIdescO, (first && s == 0) ? 0u : 1u);
       }
       mma_commit(bar(L::bVEmpty + vs));
-      mma_commit(bar(L::bPVDone));
+      mma_commit(bar(L::bPVDone + pb));
     }
     __syncwarp();
     return true;
@@ -307,6 +314,12 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_off + kColS;
   const uint32_t tP = tmem + lane_off + kColP;
+  // Waits until O += P_t V_t (key-block iteration t) has completed.
+  auto wait_pv = [&](uint32_t t, int where) -> bool {
+    if (!W.wait(bar(L::bPVDone + (t & 1)), (t >> 1) & 1, where)) return false;
+    tc_fence_after();
+    return true;
+  };
   const uint32_t tO = tmem + lane_off + kColO;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
@@ -340,15 +353,16 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mx_s = mx * sl2;
-      if (j > 0) {
-        // P and O of the previous block are in use until its P.V completes.
-        if (!W.wait(bar(L::bPVDone), (kv - 1) & 1, 11)) { ok = false; break; }
-        tc_fence_after();
-      }
-      if (mx_s > m_ref + kRescaleLog2) {
-        const float alpha = fast_exp2(m_ref - mx_s);
+      // The decision is taken per warp: tcgen05.ld/st are .sync.aligned and
+      // must be executed by all 32 lanes together.  Rows of a rescaling warp
+      // whose own maximum did not grow get alpha = 1.
+      if (__any_sync(0xFFFFFFFFu, mx_s > m_ref + kRescaleLog2)) {
+        const float m_new = fmaxf(m_ref, mx_s);
+        const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_ref - m_new);
         l *= alpha;
         if (j > 0) {
+          // O is stable once the previous block's P.V has completed.
+          if (!wait_pv(kv - 1, 11)) { ok = false; break; }
 #pragma unroll 1
           for (int ch = 0; ch < HD / 32; ++ch) {
             uint32_t o[32];
@@ -359,32 +373,35 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
           }
           tmem_wait_st();
         }
-        m_ref = mx_s;
+        m_ref = m_new;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       uint32_t pk[64];
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = fast_exp2(fmaf(s[2 * c], sl2, -m_use));
-        const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -m_use));
+        const float x0 = fmaf(s[2 * c], sl2, -m_use);
+        const float x1 = fmaf(s[2 * c + 1], sl2, -m_use);
+        const bool poly = (c % kPolyEvery) == kPolyEvery - 1;
+        const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
+        const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
         ls[c & 7] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      tmem_st_x64(tP, pk);
+      // P buffer kv & 1 was last read by the P.V of iteration kv - 2.
+      const uint32_t pb = kv & 1;
+      if (kv >= 2 && !wait_pv(kv - 2, 13)) { ok = false; break; }
+      tmem_st_x64(tP + pb * 64, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(L::bPFull));
+      mbar_arrive(bar(L::bPFull + pb));
       ++kv;
     }
     if (!ok) break;
 
     // ------------------------------------------------------------ epilogue
-    if (it.n > 0) {
-      if (!W.wait(bar(L::bPVDone), (kv - 1) & 1, 12)) break;
-      tc_fence_after();
-    }
+    if (it.n > 0 && !wait_pv(kv - 1, 12)) break;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const int64_t bh_off = static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
     // Destination rows of this thread's output.
@@ -469,8 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     }
     mbar_init(bar(L::bSFull), 1);
     mbar_init(bar(L::bSFree), 128);
-    mbar_init(bar(L::bPFull), 128);
-    mbar_init(bar(L::bPVDone), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(L::bPFull + b), 128);
+      mbar_init(bar(L::bPVDone + b), 1);
+    }
     mbar_init(bar(L::bOFree), 128);
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = 0;
@@ -517,7 +536,20 @@ cudaError_t launch_one(const TcParams& p, int grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    y[i] = exp2_fma(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  exp2_fma_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 size_t tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? Layout<64>::kBytes : Layout<128>::kBytes;

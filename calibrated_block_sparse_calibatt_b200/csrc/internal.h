@@ -91,6 +91,8 @@ cudaError_t launch_select_blocks(const float* energy, int64_t n_rows, int32_t nk
 cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,
                              uint8_t* mask, cudaStream_t s);
 
+cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s);
+
 // Dynamic shared memory the tensor-core kernel needs for a head dimension.
 size_t tc_smem_bytes(int head_dim);
 

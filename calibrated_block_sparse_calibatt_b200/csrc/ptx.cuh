@@ -198,6 +198,22 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA and integer pipes, for x <= 126 (Cody-Waite reduction and a
+// cubic fitted by Remez exchange to the relative error of 2^f on [-1/2, 1/2],
+// max relative error 7.5e-5; coefficients from csrc/fit_exp2_poly.py).
+// n = rint(x) comes from adding 1.5 * 2^23 (the integer lands in the low
+// mantissa bits), 2^n is added to the exponent field of the polynomial.
+// Inputs below -125 (including -inf) return about 2^-125 instead of 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(5.517166906e-02f, f, 2.426111222e-01f);
+  p = fmaf(p, f, 6.932609855e-01f);
+  p = fmaf(p, f, 9.999280735e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"

@@ -253,6 +253,13 @@ calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32
  * Returns CALIBATT_ERR_TIMEOUT when the word is non-zero. */
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);
 
+/* Evaluates, on the device, the FMA-pipe base-2 exponential that the
+ * tensor-core softmax uses for part of its probabilities (no counterpart in
+ * the paper; exposed so its error bound can be tested): y[i] = 2^x[i] with
+ * relative error below 1e-4 for -125 <= x <= 126, about 2^-125 for smaller x.
+ * x, y: device float32[n]. */
+calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, void* stream);
+
 /* Time limit of every in-kernel barrier wait, in milliseconds (default 4000;
  * applies to launches made after the call). */
 calibatt_status calibatt_set_wait_timeout_ms(int32_t ms);

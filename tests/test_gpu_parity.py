@@ -358,3 +358,21 @@ def test_energy_select_union_tiny(C, std, tau):
     ref_union = O.aggregate_masks(np.stack(ref_masks), 4, 0.25)
     assert (union.cpu().numpy().astype(bool)[all_ok] == ref_union[all_ok]).all()
     assert all_ok.mean() > 0.5
+
+
+def test_fma_exp2_error_bound(C):
+    rng = np.random.default_rng(22)
+    x = np.concatenate([rng.uniform(-125, 126, 200000), np.arange(-125, 127, 0.25),
+                        [0.0, -0.5, 0.5, 8.0, -1e-7, 1e-7]]).astype(np.float32)
+    xt = torch.from_numpy(x).cuda()
+    y = torch.empty_like(xt)
+    C.calibatt_debug_exp2_fma(xt, y)
+    _check_status(C)
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(y.cpu().numpy().astype(np.float64) / ref - 1.0)
+    assert rel.max() < 1e-4, rel.max()
+    low = torch.tensor([-126.0, -200.0, float("-inf")], device="cuda")
+    yl = torch.empty_like(low)
+    C.calibatt_debug_exp2_fma(low, yl)
+    _check_status(C)
+    assert (yl >= 0).all() and (yl < 1e-37).all()
