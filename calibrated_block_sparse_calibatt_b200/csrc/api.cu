@@ -104,6 +104,42 @@ void lpt(int32_t n, const int64_t* cost, int32_t bins, int32_t* bin_ptr, int32_t
   if (makespan) *makespan = mk;
 }
 
+// LPT over consecutive groups of items: inside a group, items in descending
+// cost go to the least-loaded bin; bin loads carry over from group to group,
+// and every bin lists its items group by group.  With one group per few heads
+// the persistent CTAs move through the heads roughly together, so the keys and
+// values of the heads in flight stay resident in L2.
+void lpt_grouped(int32_t n, const int64_t* cost, const int32_t* group, int32_t bins, int32_t* bin_ptr,
+                 int32_t* order) {
+  std::vector<int32_t> idx(n);
+  std::iota(idx.begin(), idx.end(), 0);
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) {
+    return group[a] != group[b] ? group[a] < group[b] : cost[a] > cost[b];
+  });
+  using Slot = std::pair<int64_t, int32_t>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int32_t b = 0; b < bins; ++b) heap.push({0, b});
+  std::vector<std::vector<int32_t>> per_bin(bins);
+  for (int32_t i : idx) {
+    Slot s = heap.top();
+    heap.pop();
+    per_bin[s.second].push_back(i);
+    heap.push({s.first + cost[i], s.second});
+  }
+  int32_t pos = 0;
+  for (int32_t b = 0; b < bins; ++b) {
+    bin_ptr[b] = pos;
+    for (int32_t i : per_bin[b]) order[pos++] = i;
+  }
+  bin_ptr[bins] = pos;
+}
+
+// Heads whose keys and values (at head_dim 128) fit together in about 80 MB of L2.
+int32_t heads_per_group(int32_t nq) {
+  const int64_t per_head = static_cast<int64_t>(nq) * 128 * 128 * 2 * 2;
+  return static_cast<int32_t>(std::max<int64_t>(1, (80ll << 20) / per_head));
+}
+
 // ------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -594,23 +630,27 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
   // Work items of the sparse heads and their LPT schedule over the grid.
   std::vector<uint32_t> items;
   std::vector<int64_t> cost;
+  std::vector<int32_t> group;
   int32_t n_sparse = 0, n_rep = 0;
   int64_t retained = 0;
+  const int32_t hpg = heads_per_group(nq);
   for (int h = 0; h < H; ++h) {
     if (repetitive && repetitive[h]) {
       ++n_rep;
       continue;
     }
+    const int32_t g = n_sparse / hpg;
     ++n_sparse;
     const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
     for (int r = 0; r < nq; ++r) {
       items.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
       cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);  // +2: Q load and epilogue
+      group.push_back(g);
       retained += rp[r + 1] - rp[r];
     }
   }
   std::vector<int32_t> cta_ptr(d->G + 1), order(items.size());
-  lpt(static_cast<int32_t>(items.size()), cost.data(), d->G, cta_ptr.data(), order.data(), nullptr);
+  lpt_grouped(static_cast<int32_t>(items.size()), cost.data(), group.data(), d->G, cta_ptr.data(), order.data());
   std::vector<uint32_t> sched(items.size());
   for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
   int prev = 0;

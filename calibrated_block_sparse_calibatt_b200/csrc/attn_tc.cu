@@ -9,15 +9,16 @@
 // path -- normalised and written to the output, once per query on the sparse
 // path and to every row an anchor serves on the anchor path.
 //
-// CTA layout (192 threads, one CTA per SM, persistent):
-//   warps 0-3  softmax + epilogue; thread t owns query row t = TMEM lane t
-//   warp  4    producer: TMA loads of Q and of K/V tiles gathered by block
+// CTA layout (320 threads, one CTA per SM, persistent):
+//   warps 0-7  softmax + epilogue; warp w owns query rows 32*(w%4)..+31 (its
+//              TMEM lane quarter) and score columns 64*(w/4)..+63
+//   warp  8    producer: TMA loads of Q and of K/V tiles gathered by block
 //              index (or a plain-load gather of anchor Q rows)
-//   warp  5    TMEM allocator and MMA issuer (one lane issues tcgen05.mma)
+//   warp  9    TMEM allocator and MMA issuer (one lane issues tcgen05.mma)
 // Tensor memory (512 columns): S = Q K^T at 0..127 (f32), two P buffers
 // (bf16 pairs) at 128..191 and 192..255, O accumulator at 256..256+D.  With P
 // double-buffered the softmax writes P_{j+1} while O += P_j V_j still runs.
-// Pipelines (mbarriers): Q 1 stage, K 3 stages, V 3 stages; S/P/O handshakes
+// Pipelines (mbarriers): Q 1 stage, K 3 stages, V 2 stages; S/P/O handshakes
 // between the MMA warp and the softmax warps.  Per key block j the MMA warp
 // issues S_j = Q K_j^T as soon as the softmax warps have read S_{j-1} out of
 // tensor memory, then O += P_{j-1} V_{j-1}, so the tensor core works on the
@@ -34,9 +35,12 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 8 softmax warps, producer, MMA
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxThreads = 256;
 constexpr int kKStages = 3;
-constexpr int kVStages = 3;
+constexpr int kVStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColP = 128;  // P buffer b at kColP + 64 * b
@@ -65,7 +69,8 @@ struct Layout {
   static constexpr int bOFree = bPVDone + 2, bDrain = bOFree + 1;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
-  static constexpr int kUsed = kMisc + 16;
+  static constexpr int kXchg = kMisc + 16;  // float [2][2][128] row maxima + [2][128] row sums
+  static constexpr int kUsed = kXchg + (512 + 256) * 4;
   // +1024 for aligning the base; at least 120 KB so only one CTA fits per SM
   // (each CTA holds all 512 tensor-memory columns).
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
@@ -305,81 +310,97 @@ __device__ void mma_role(const TcParams& p, uint32_t base, uint32_t tmem, const 
 }
 
 // --------------------------------------------------------- softmax/epilogue
+// Eight warps: warp w handles query rows 32*(w%4) .. +31 (its TMEM lane
+// quarter) and score columns 64*(w/4) .. +63.  The two warps sharing rows (w
+// and w+4) exchange their partial row maxima once per key block, and their
+// partial row sums at the end, through shared memory at a pair barrier
+// (bar.red.or, 64 threads).  The barrier also carries "a wait failed" so that
+// both warps of a pair always leave the loop together.
 template <int HD, bool ANCHOR>
-__device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W,
-                             int warp, int lane) {
+__device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
+                             const Waiter& W, int warp, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
-  const int row = warp * 32 + lane;  // query row within the tile == TMEM lane
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem + lane_off + kColS;
-  const uint32_t tP = tmem + lane_off + kColP;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
+  const int pair_bar = 1 + quarter;     // named barrier shared with the partner warp
+  float* xchg = reinterpret_cast<float*>(gbase + L::kXchg);  // [2 buffers][2 halves][128 rows]
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tS = tmem + lane_off + kColS + half * 64;
+  const uint32_t tP = tmem + lane_off + kColP + half * 32;
+  const uint32_t tO = tmem + lane_off + kColO + half * (HD / 2);
+  const int ragged_cols = p.seq_len % 128;
+  const int col0 = half * 64;
+  const float sl2 = p.scale_log2;
   // Waits until O += P_t V_t (key-block iteration t) has completed.
   auto wait_pv = [&](uint32_t t, int where) -> bool {
     if (!W.wait(bar(L::bPVDone + (t & 1)), (t >> 1) & 1, where)) return false;
     tc_fence_after();
     return true;
   };
-  const uint32_t tO = tmem + lane_off + kColO;
-  const int ragged_cols = p.seq_len % 128;
-  const float sl2 = p.scale_log2;
   Cursor<ANCHOR> cur;
   cur.init(p);
   Item it;
   uint32_t kv = 0;
   bool ok = true;
-  while (ok && cur.next(p, it)) {
+  while (cur.next(p, it)) {
     float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < it.n; ++j) {
-      if (!W.wait(bar(L::bSFull), kv & 1, 10)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld_x128(tS, sr);
+      ok = ok && W.wait(bar(L::bSFull), kv & 1, 10);
+      if (ok) tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld_x64(tS, sr);
       tc_fence_before();
-      mbar_arrive(bar(L::bSFree));
-      float s[128];
+      if (ok) mbar_arrive(bar(L::bSFree));
+      float s[64];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
       if (j == it.n - 1 && it.ragged_last) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= ragged_cols) s[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c)
+          if (col0 + c >= ragged_cols) s[c] = -INFINITY;
       }
       float mx8[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx8[a] = s[a];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mx_s = mx * sl2;
-      // The decision is taken per warp: tcgen05.ld/st are .sync.aligned and
-      // must be executed by all 32 lanes together.  Rows of a rescaling warp
-      // whose own maximum did not grow get alpha = 1.
+      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      float* xb = xchg + (kv & 1) * 256;
+      xb[half * 128 + row] = mx_half;
+      if (bar_red_or(pair_bar, 64, !ok)) { ok = false; break; }
+      const float mx_s = fmaxf(mx_half, xb[(1 - half) * 128 + row]) * sl2;
+      // The decision is taken per warp (tcgen05.ld/st are .sync.aligned and
+      // need all 32 lanes); both warps of a pair see the same row maxima and
+      // so decide alike.  Rows of a rescaling warp whose maximum did not grow
+      // get alpha = 1.
       if (__any_sync(0xFFFFFFFFu, mx_s > m_ref + kRescaleLog2)) {
         const float m_new = fmaxf(m_ref, mx_s);
         const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_ref - m_new);
         l *= alpha;
         if (j > 0) {
           // O is stable once the previous block's P.V has completed.
-          if (!wait_pv(kv - 1, 11)) { ok = false; break; }
+          ok = ok && wait_pv(kv - 1, 11);
+          if (ok) {
 #pragma unroll 1
-          for (int ch = 0; ch < HD / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_x32(tO + ch * 32, o);
+            for (int ch = 0; ch < HD / 64; ++ch) {
+              uint32_t o[32];
+              tmem_ld_x32(tO + ch * 32, o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st_x32(tO + ch * 32, o);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st_x32(tO + ch * 32, o);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
         }
         m_ref = m_new;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint32_t pk[64];
+      uint32_t pk[32];
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
+      for (int c = 0; c < 32; ++c) {
         const float x0 = fmaf(s[2 * c], sl2, -m_use);
         const float x1 = fmaf(s[2 * c + 1], sl2, -m_use);
         const bool poly = (c % kPolyEvery) == kPolyEvery - 1;
@@ -391,18 +412,25 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       // P buffer kv & 1 was last read by the P.V of iteration kv - 2.
       const uint32_t pb = kv & 1;
-      if (kv >= 2 && !wait_pv(kv - 2, 13)) { ok = false; break; }
-      tmem_st_x64(tP + pb * 64, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(L::bPFull + pb));
+      if (kv >= 2) ok = ok && wait_pv(kv - 2, 13);
+      if (ok) {
+        tmem_st_x32(tP + pb * 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::bPFull + pb));
+      }
       ++kv;
     }
-    if (!ok) break;
 
     // ------------------------------------------------------------ epilogue
-    if (it.n > 0 && !wait_pv(kv - 1, 12)) break;
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    // (A failed wait is acted on at the pair barrier below, which both warps
+    // of the pair reach; leaving earlier could strand the partner there.)
+    if (it.n > 0) ok = ok && wait_pv(kv - 1, 12);
+    float* xl = xchg + 512;  // partial row sums
+    xl[half * 128 + row] = l;
+    if (bar_red_or(pair_bar, 64, !ok)) { ok = false; break; }
+    const float l_row = l + xl[(1 - half) * 128 + row];
+    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
     const int64_t bh_off = static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
     // Destination rows of this thread's output.
     int64_t dst_token = -1;
@@ -426,7 +454,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
       }
     }
 #pragma unroll 1
-    for (int ch = 0; ch < HD / 32; ++ch) {
+    for (int ch = 0; ch < HD / 64; ++ch) {
       uint32_t o[32];
       if (it.n > 0) {
         tmem_ld_x32(tO + ch * 32, o);
@@ -442,19 +470,20 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint32_t tmem, co
         pkd[g].z = pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv_l, __uint_as_float(o[8 * g + 5]) * inv_l);
         pkd[g].w = pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv_l, __uint_as_float(o[8 * g + 7]) * inv_l);
       }
+      const int dcol = half * (HD / 2) + ch * 32;
 #pragma unroll 1
       for (int d = 0; d < n_dst; ++d) {
         const int64_t token = ANCHOR
             ? (static_cast<int64_t>(anchor_f) * p.anc.rows + lo + d) * p.anc.cols + anchor_w
             : dst_token;
-        uint4* dst = reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + ch * 32);
+        uint4* dst = reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + dcol);
 #pragma unroll
         for (int g = 0; g < 4; ++g) dst[g] = pkd[g];
       }
     }
-    if (!ANCHOR && p.lse != nullptr && dst_token >= 0) {
+    if (!ANCHOR && half == 0 && p.lse != nullptr && dst_token >= 0) {
       p.lse[(static_cast<int64_t>(it.b) * p.heads + it.h) * p.seq_len + dst_token] =
-          it.n > 0 ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          it.n > 0 ? (m_ref + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     mbar_arrive(bar(L::bOFree));
@@ -485,22 +514,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       mbar_init(bar(L::bVEmpty + s), 1);
     }
     mbar_init(bar(L::bSFull), 1);
-    mbar_init(bar(L::bSFree), 128);
+    mbar_init(bar(L::bSFree), kSoftmaxThreads);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(L::bPFull + b), 128);
+      mbar_init(bar(L::bPFull + b), kSoftmaxThreads);
       mbar_init(bar(L::bPVDone + b), 1);
     }
-    mbar_init(bar(L::bOFree), 128);
+    mbar_init(bar(L::bOFree), kSoftmaxThreads);
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0 && !ANCHOR) {
+  if (warp == kProducerWarp && lane == 0 && !ANCHOR) {
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -510,17 +539,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     producer_role<HD, ANCHOR>(p, base, W, lane);
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     mma_role<HD, ANCHOR>(p, base, tmem, W, lane);
   } else {
-    softmax_role<HD, ANCHOR>(p, base, tmem, W, warp, lane);
+    softmax_role<HD, ANCHOR>(p, base, gbase, tmem, W, warp, lane);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -143,7 +143,10 @@ calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq
  * Every CSR is validated as calibatt_csr_validate (no diagonal requirement),
  * converted to 16-bit indices, copied to the device (synchronously), and a
  * longest-processing-time schedule of the layer's (head, query block) work
- * is built for the dictionary's num_ctas. */
+ * is built for the dictionary's num_ctas: heads are taken in groups whose
+ * keys and values fit in about 80 MB of L2, and the schedule keeps one
+ * running LPT balance across the groups while listing each CTA's items group
+ * by group, so the persistent CTAs work on the same few heads at a time. */
 calibatt_status calibatt_dict_set_layer(calibatt_dict* dict, int32_t t, int32_t l,
                                         const int32_t* row_ptr, const int32_t* col_idx,
                                         const uint8_t* repetitive);
