@@ -82,6 +82,13 @@ constexpr float kRescaleLog2 = 8.0f;
 #define CALIBATT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
+// Exponential phases of consecutive key blocks (which alternate between the
+// two streams) take turns on the MUFU unit instead of overlapping (1 = on;
+// measured slower than free overlap on B200, so off by default).
+#ifndef CALIBATT_EXP_TURNS
+#define CALIBATT_EXP_TURNS 0
+#endif
+constexpr bool kExpTurns = CALIBATT_EXP_TURNS != 0;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -100,7 +107,8 @@ struct Layout {
   static constexpr int bPFull = bSFull + 2;          // [2] probabilities of stream s ready
   static constexpr int bPVDone = bPFull + 2;         // [2] O_s += P_s V finished
   static constexpr int bOFree = bPVDone + 2;         // epilogue has read O_0 and O_1
-  static constexpr int bDrain = bOFree + 1;
+  static constexpr int bTurn = bOFree + 1;           // [2] stream s may start its exponentials
+  static constexpr int bDrain = bTurn + 2;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
   static constexpr int kXchg = kMisc + 16;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
@@ -391,6 +399,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   Item it;
   uint32_t kv = 0, item = 0;
   uint32_t t_me = 0, t_other = 0;  // key blocks of this / the other stream so far (global)
+  uint32_t turns = 0;                // turns this stream has waited for
   bool ok = true;
   while (cur.next(p, it)) {
     const int n_s = (it.n + 1 - s) / 2;  // blocks of this stream in the item
@@ -420,7 +429,8 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sc[c + a], sc[c + a + 8]);
       }
-      const float mx_s = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
+      const float mx_s =
+          fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
       // The decision is taken per warp (tcgen05.ld/st are .sync.aligned and
       // need all 32 lanes); rows of a rescaling warp whose maximum did not grow
       // get alpha = 1.  O_s itself is rescaled after the probabilities are
@@ -434,28 +444,39 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         l *= alpha;
         m_ref = m_new;
       }
-      CALIBATT_TRACE_EVENT(lane == 0, 48 + warp, kv + j);
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // Wait for this block's turn on the MUFU unit: the previous key block
+      // (of the other stream, or the last block of the previous item) has
+      // finished its exponentials.
+      const uint32_t g = kv + j;
+      if (kExpTurns && g > 0) {
+        ok = ok && W.wait(bar(L::bTurn + s), turns & 1, 14);
+        ++turns;
+      }
       // Probabilities in four chunks of 32 keys; each chunk's 16 packed
       // columns go to tensor memory (over the already-read scores) at once.
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh) {
         uint32_t pk[16];
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
           const int c = hh * 16 + cc;
-          const float x0 = fmaf(sc[2 * c], sl2, -m_use);
-          const float x1 = fmaf(sc[2 * c + 1], sl2, -m_use);
+          float x0, x1;
+          fma2(x0, x1, sc[2 * c], sc[2 * c + 1], sl2, sl2, -m_use, -m_use);
           const bool poly = kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1;
           const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
           const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
-          ls[c & 7] += p0 + p1;
+          if (cc & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
           pk[cc] = pack_bf16x2(p0, p1);
         }
         if (ok) tmem_st_x16(tS + hh * 16, pk);
       }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      l += (la + lb) + (lc + ld);
+      // Hand the MUFU unit to the next key block in issue order: the other
+      // stream within the item, or stream 0 of the next item.
+      if (kExpTurns && ok) mbar_arrive(bar(L::bTurn + ((j + 1 < it.n) ? 1 - s : 0)));
+      CALIBATT_TRACE_EVENT(lane == 0, 48 + warp, kv + j);
       if (rescale && k > 0) {
         // O_s is stable once this stream's previous P.V has completed.
         ok = ok && wait_pv(s, t_me - 1, 11);
@@ -607,6 +628,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       mbar_init(bar(L::bPVDone + s), 1);
     }
     mbar_init(bar(L::bOFree), kSoftmaxThreads);
+    mbar_init(bar(L::bTurn + 0), kGroupThreads);
+    mbar_init(bar(L::bTurn + 1), kGroupThreads);
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
