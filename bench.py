@@ -97,6 +97,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def measured_traffic(tiles):
+    """DRAM bytes per launch of the sparse kernel from the committed ncu capture
+    (profiles/tc_attn_sparse_720p_traffic.json), scaled by retained tiles; None
+    when the kernel source changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "tc_attn_sparse_720p_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    src = os.path.join(ROOT, t["kernel_source"])
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != t["kernel_source_sha256"]:
+        return None
+    return t["dram_bytes_per_retained_tile"] * tiles
+
+
 def build_dict(C, masks, heads, nb, block, rep=None):
     rp, ci, rep_arr = C.masks_to_layer_csr(masks, heads, nb)
     d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, ci.size))
@@ -347,7 +363,9 @@ def main():
                        "l2": "inputs 2.32 GB > 126 MB L2, no flush", "parallelism": f"replicas x{world}"},
             "pct_of_peak": achieved / pk["bf16_tflops"],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                         "frac": achieved / pk["bf16_tflops"], "traffic": measured_traffic(tiles),
+                         "traffic_unit": "bytes per launch (DRAM read + write)",
+                         "algorithmic_bytes": 4 * q.numel() * q.element_size(),
                          "peak_source": f"{pk['source']} burst bf16"},
             "clocks": clk.summary(),
             "e2e": e2e,
