@@ -22,7 +22,7 @@ LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libcalibatt.so")
 BUILD = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu"]
+SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu", "energy_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -70,6 +70,7 @@ SIGNATURES = {
                                        _vp, _i32, _f32, _vp, _vp]),
     "calibatt_block_energy_workspace_size": (_i32, [_P(Shape), _P(ctypes.c_size_t)]),
     "calibatt_block_energy": (_i32, [_vp, _vp, _P(Shape), _i32, _f32, _vp, _vp, ctypes.c_size_t, _vp]),
+    "calibatt_block_energy_noalloc": (_i32, [_vp, _vp, _P(Shape), _i32, _f32, _vp, _vp]),
     "calibatt_select_blocks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp, _vp]),
     "calibatt_aggregate_masks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp]),
     "calibatt_debug_exp2_fma": (_i32, [_vp, _vp, _i64, _vp]),
@@ -291,6 +292,13 @@ def calibatt_block_energy(q, k, energy, workspace, block, softmax_scale=0.0, str
     nbytes = workspace.numel() * workspace.element_size()
     check(LIB.calibatt_block_energy(_ptr(q), _ptr(k), ctypes.byref(shape), block, float(softmax_scale),
                                     _ptr(energy), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def calibatt_block_energy_noalloc(q, k, energy, block, softmax_scale=0.0, stream=None):
+    """Block energies without any device allocation (scratch built into the library)."""
+    shape = shape_of(q)
+    check(LIB.calibatt_block_energy_noalloc(_ptr(q), _ptr(k), ctypes.byref(shape), block, float(softmax_scale),
+                                            _ptr(energy), _stream(stream)))
 
 
 def calibatt_select_blocks(energy, tau, mask, count_accum=None, stream=None):

@@ -279,6 +279,17 @@ float scale_log2_of(float softmax_scale, int head_dim) {
 
 }  // namespace
 
+namespace calibatt {
+void set_last_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+}  // namespace calibatt
+
 // ================================================================ dictionary
 
 struct calibatt_dict {

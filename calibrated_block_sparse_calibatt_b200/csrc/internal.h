@@ -93,6 +93,9 @@ cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts
 
 cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s);
 
+// Records a failure message for calibatt_last_error() on the calling thread.
+void set_last_error(const char* fmt, ...);
+
 // Dynamic shared memory the tensor-core kernel needs for a head dimension.
 size_t tc_smem_bytes(int head_dim);
 

@@ -231,6 +231,27 @@ calibatt_status calibatt_block_energy(const void* q, const void* k,
                                       float softmax_scale, float* energy, void* workspace,
                                       size_t workspace_bytes, void* stream);
 
+/* The same block energies as calibatt_block_energy, for callers that may not
+ * allocate device memory (the paper has no counterpart; this is a deployment
+ * variant).  Some processes cannot call cudaMalloc when they calibrate: a
+ * server that reserved all device memory at start-up for weights and caches,
+ * a host runtime that owns the allocator and forbids plug-ins to go around
+ * it, or an integration whose host code may not call the CUDA memory API.
+ * This entry point allocates nothing: its row log-sum-exp scratch is a fixed
+ * array inside the library, 2^20 float32 rows (4 MiB, held on every GPU that
+ * loads the library until the process exits), so batch * heads * seq_len
+ * must not exceed 2^20 (CALIBATT_ERR_INVALID_ARG otherwise, with a message;
+ * use calibatt_block_energy and a caller workspace for larger problems).
+ * All calls share that array and it keeps the previous call's contents
+ * (nothing in it needs clearing: every row is written before it is read);
+ * calls whose work overlaps on the GPU race on it, so order them on one
+ * stream.  The first call on each device looks up the array's device address
+ * with that device current; make that first call before capturing any
+ * stream.  Other arguments and errors as calibatt_block_energy. */
+calibatt_status calibatt_block_energy_noalloc(const void* q, const void* k,
+                                              const calibatt_shape* shape, int32_t block,
+                                              float softmax_scale, float* energy, void* stream);
+
 /* Top-mass selection (Key Designs 1, after Eq. (5)) for n_rows rows of nk
  * energies (device float32 [n_rows, nk], nk <= 4096): order each row by
  * energy descending, ties to the lower key block; keep the shortest prefix
