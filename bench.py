@@ -113,6 +113,27 @@ def measured_traffic(tiles):
     return t["dram_bytes_per_retained_tile"] * tiles
 
 
+def rank_seed(base, rank):
+    """Input seed of a rank: every rank times an independent layer (weak scaling)."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Largest value of x over the ranks of the default process group (x itself
+    when there is none); every rank must call it in the same order."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flop_per_rank, world, ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flop_per_rank / (ms * 1e-3) / 1e12
+
+
 def build_dict(C, masks, heads, nb, block, rep=None):
     rp, ci, rep_arr = C.masks_to_layer_csr(masks, heads, nb)
     d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, ci.size))
@@ -252,7 +273,8 @@ def main():
     import dataclasses
     wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
     masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])
-    q, k, v = W.make_qkv(wl.seed + 7919 * rank, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    q, k, v = W.make_qkv(rank_seed(wl.seed, rank), 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std,
+                         "cuda")
     o = torch.empty_like(q)
     d_sparse = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block)
     tiles = d_sparse.layer_info(0, 0)["retained_tiles"]
@@ -278,13 +300,9 @@ def main():
             dist.barrier()
     if C.device_status() != 0:
         raise RuntimeError("device wait timed out during the benchmark")
-    total_ms = sum(per_call)
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(per_call), dist, "cuda")
     ms = total_ms / args.steps
-    value = world * flop / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(flop, world, ms)
     avg_launch_ms = statistics.mean(per_call)
     achieved = flop / (avg_launch_ms * 1e-3) / 1e12
 
@@ -294,9 +312,9 @@ def main():
         ones = [np.ones((wl.num_blocks, wl.num_blocks), bool)] * wl.heads
         d_dense = build_dict(C, ones, wl.heads, wl.num_blocks, wl.block)
         dense_tiles = d_dense.layer_info(0, 0)["retained_tiles"]
-        dense_ms = statistics.mean(time_calls(
+        dense_ms = max_over_ranks(statistics.mean(time_calls(
             torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d_dense, 0, 0, wl.block, stream=stream),
-            max(3, args.steps // 4), 2, stream))
+            max(3, args.steps // 4), 2, stream)), dist, "cuda")
         d_dense.close()
         extras["dense"] = {"ms_per_call": dense_ms,
                            "tflops": dense_tiles * FLOP_PER_TILE / (dense_ms * 1e-3) / 1e12,
@@ -307,14 +325,14 @@ def main():
         d_dual = build_dict(C, [dmasks[h] for h in range(wd.heads)], wd.heads, wd.num_blocks, wd.block)
         dual_tiles = d_dual.layer_info(0, 0)["retained_tiles"]
         anchor_tiles = len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128) * wd.num_blocks
-        dual_ms = statistics.mean(time_calls(
+        dual_ms = max_over_ranks(statistics.mean(time_calls(
             torch, lambda: C.calibatt_dual_path_attn(q, k, v, o, d_dual, 0, 0, wd.frames, wd.rows, wd.cols,
                                                      wd.anchors, wd.block, stream=stream),
-            max(3, args.steps // 4), 2, stream))
-        anchor_ms = statistics.mean(time_calls(
+            max(3, args.steps // 4), 2, stream)), dist, "cuda")
+        anchor_ms = max_over_ranks(statistics.mean(time_calls(
             torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
                                                   list(rep_heads), stream=stream),
-            max(3, args.steps // 4), 2, stream))
+            max(3, args.steps // 4), 2, stream)), dist, "cuda")
         d_dual.close()
         bcast_bytes = len(rep_heads) * wd.seq_len * wd.head_dim * 2
         extras["dual_path_720p"] = {
@@ -341,9 +359,9 @@ def main():
             ho.copy_(o, non_blocking=True)
 
         e2e_steps = max(3, args.steps // 4)
-        e2e_ms = statistics.mean(time_calls(torch, e2e_step, e2e_steps, 2, stream))
+        e2e_ms = max_over_ranks(statistics.mean(time_calls(torch, e2e_step, e2e_steps, 2, stream)), dist, "cuda")
         nbytes = 3 * q.numel() * q.element_size()
-        e2e = {"value": world * flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": aggregate_tflops(flop, world, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": o.numel() * o.element_size()}
         del hq, hk, hv, ho, dq, dk, dv
 
