@@ -10,30 +10,37 @@
 // an anchor serves on the anchor path.
 //
 // Two softmax streams per query tile.  Key blocks at even list positions go
-// to stream 0 and odd positions to stream 1; each stream keeps its own running
-// maximum m, row sum l and output accumulator O in tensor memory, and the
-// epilogue merges them exactly:
-//   m = max(m0, m1),  a_s = 2^(m_s - m),  O = (a0 O0 + a1 O1) / (a0 l0 + a1 l1).
-// The MMA warp issues S(j) = Q K_j^T, then O_s += P(j-1) V_{j-1} for the other
-// stream, then S(j+1), ... so the tensor core computes one stream's products
-// while the other stream's softmax warps exponentiate.  K and V tiles are still
-// loaded once each, in list order.
+// to stream 0 and odd positions to stream 1, and both streams accumulate into
+// ONE output accumulator O in tensor memory.  That works because the
+// reference maximum is a single in-order sequence m(0) <= m(1) <= ...: the
+// softmax of block j takes m(j-1) from the other stream (published as soon as
+// that block's row maximum is known, long before its exponentials end), keeps
+// it unless a row maximum exceeds it by more than 2^8 (exp2 domain), and
+// publishes m(j).  P(j) = 2^(s*log2e*scale - m(j)) <= 256.  When m grows at
+// block j, O is rescaled by 2^(m(j-1) - m(j)) after P(j-1).V has landed and
+// before P(j).V is issued (it waits for P(j)), so O always carries the
+// reference of the last block accumulated.  Each stream keeps its own row sum
+// relative to the reference of its latest block; the epilogue combines the
+// two sums against the final reference.
 //
-// CTA layout (352 threads, one CTA per SM, persistent):
+// Freeing the second accumulator leaves room for three score buffers: S(j)
+// lives in buffer j mod 3 and S(j+3) can run as soon as P(j).V is done, so a
+// stream finds the scores of its next block ready when its current block
+// ends, and the tensor core's P.V + S work is off the softmax chain.
+//
+// CTA layout (384 threads, one CTA per SM, persistent):
 //   warps 0-3  softmax of stream 0, warps 4-7 softmax of stream 1: thread t of
 //              a group owns query row t (TMEM lane t) and a whole 128-key score
 //              row; in the epilogue the two groups split the output columns
 //   warp  8    producer of Q (TMA, or a plain-load gather of anchor rows)
 //              and of the K tiles gathered by block index
-//   warp  9    TMEM allocator and MMA issuer (one lane issues tcgen05.mma)
+//   warp  9    TMEM allocator; one lane issues the S = Q K^T MMAs
 //   warp 10    producer of the V tiles
-// Tensor memory (512 columns): stream s has S_s at 128*s (f32 scores; its bf16
-// probabilities P_s overwrite the first 64 columns once the scores are in
-// registers) and O_s at 256 + 128*s.  S_s(j+2) is issued after O_s += P_s(j) V_j
-// on the same thread, and tcgen05 MMAs from one thread run in issue order, so
-// the P values are read before the next scores overwrite them.
-// The softmax keeps a reference maximum per stream and only rescales O_s and
-// l_s when a row maximum exceeds it by more than 2^8 (exp2 domain), so P <= 256.
+//   warp 11    one lane issues the O += P V MMAs
+// Tensor memory (512 columns): score buffer b at 128*b, b = 0..2 (f32 scores;
+// the bf16 probabilities overwrite its first 64 columns once the scores are in
+// registers), O at 384.  S(j+3) reuses the buffer of P(j); its issuer waits
+// until P(j).V has completed before overwriting it.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -54,41 +61,77 @@ __device__ unsigned long long g_trace[kTraceEvents * kTraceIters];
 __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
   if (blockIdx.x == 0 && idx < kTraceIters) g_trace[ev * kTraceIters + idx] = clock64();
 }
+// Per-CTA totals of the MMA thread's time by phase (clock reads only inside
+// the loop; one store per phase at the end).
+__device__ unsigned long long g_mma_prof[1024 * 8];
+#define CALIBATT_PROF_T(var) const long long var = clock64()
+#define CALIBATT_PROF_ADD(slot, t0) prof[slot] += clock64() - (t0)
 #define CALIBATT_TRACE_EVENT(cond, ev, idx) \
   do {                                     \
     if (cond) trace_event(ev, idx);        \
   } while (0)
+// Stores from the MMA-issuing thread delay its next tcgen05.mma, so its
+// events are recorded only on request.
+#ifdef CALIBATT_TRACE_MMA
+constexpr bool kTraceMma = true;
+#else
+constexpr bool kTraceMma = false;
+#endif
 #else
 #define CALIBATT_TRACE_EVENT(cond, ev, idx) \
   do {                                     \
   } while (0)
+#define CALIBATT_PROF_T(var) \
+  do {                       \
+  } while (0)
+#define CALIBATT_PROF_ADD(slot, t0) \
+  do {                              \
+  } while (0)
 #endif
 
-constexpr int kThreads = 352;       // 8 softmax warps, Q/K producer, MMA, V producer
+// Three full warpgroups so registers can be moved between them (setmaxnreg
+// acts per warpgroup): two softmax groups and one for the producers, the MMA
+// issuer and a spare warp.  At launch every thread has kLaunchRegs; the
+// softmax groups then raise theirs to kSoftmaxRegs and the third group drops
+// to kOtherRegs, keeping 128 * (2 * kSoftmaxRegs + kOtherRegs) within the
+// 384 * kLaunchRegs the CTA was launched with.
+constexpr int kThreads = 384;       // 8 softmax warps, Q/K producer, MMA, V producer, spare
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split");
+constexpr int kEndBarrier = 5;      // named barrier id (1-4: softmax warp pairs)
 constexpr int kProducerWarp = 8;    // Q and K tiles
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;         // TMEM allocator, issues S = Q K^T
+constexpr int kPvWarp = 11;         // issues O += P V
 constexpr int kVProducerWarp = 10;  // V tiles
 constexpr int kGroupThreads = 128;  // softmax threads per stream
 constexpr int kSoftmaxThreads = 256;
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
+#ifndef CALIBATT_K_STAGES
+#define CALIBATT_K_STAGES 3
+#endif
+#ifndef CALIBATT_V_STAGES
+#define CALIBATT_V_STAGES 2
+#endif
+// Key blocks ahead of the current one whose K/V tiles the producers ask L2 to
+// fetch (0 = no prefetch).
+#ifndef CALIBATT_L2_PREFETCH
+#define CALIBATT_L2_PREFETCH 0
+#endif
+constexpr int kKStages = CALIBATT_K_STAGES;
+constexpr int kVStages = CALIBATT_V_STAGES;
+constexpr int kL2Prefetch = CALIBATT_L2_PREFETCH;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // S_s (and P_s) at kColS + 128 * s
-constexpr uint32_t kColO = 256;  // O_s at kColO + 128 * s
+constexpr int kSBufs = 3;         // score buffers, S(j) in buffer j mod 3
+constexpr uint32_t kColS = 0;    // score buffer b at kColS + 128 * b
+constexpr uint32_t kColO = 384;  // the output accumulator O
 constexpr float kRescaleLog2 = 8.0f;
-// One pair in kPolyEvery of exponentials runs on the FMA pipe (exp2_fma)
-// instead of the MUFU unit (0 = all on MUFU).
+// One pair in kPolyEvery of exponentials runs on the FMA pipe (exp2_fma2)
+// instead of the MUFU unit (0 = all on MUFU; measured fastest on B200).
 #ifndef CALIBATT_POLY_EVERY
 #define CALIBATT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
-// Exponential phases of consecutive key blocks (which alternate between the
-// two streams) take turns on the MUFU unit instead of overlapping (1 = on;
-// measured slower than free overlap on B200, so off by default).
-#ifndef CALIBATT_EXP_TURNS
-#define CALIBATT_EXP_TURNS 0
-#endif
-constexpr bool kExpTurns = CALIBATT_EXP_TURNS != 0;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -103,16 +146,18 @@ struct Layout {
   static constexpr int bQFull = 0, bQEmpty = 1;
   static constexpr int bKFull = 2, bKEmpty = bKFull + kKStages;
   static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
-  static constexpr int bSFull = bVEmpty + kVStages;  // [2] scores of stream s ready
-  static constexpr int bPFull = bSFull + 2;          // [2] probabilities of stream s ready
-  static constexpr int bPVDone = bPFull + 2;         // [2] O_s += P_s V finished
-  static constexpr int bOFree = bPVDone + 2;         // epilogue has read O_0 and O_1
-  static constexpr int bTurn = bOFree + 1;           // [2] stream s may start its exponentials
-  static constexpr int bDrain = bTurn + 2;
+  static constexpr int bSFull = bVEmpty + kVStages;  // [3] scores in buffer b ready
+  static constexpr int bPFull = bSFull + kSBufs;     // [3] probabilities in buffer b ready
+  static constexpr int bPFree = bPFull + kSBufs;     // [3] P.V of the block in buffer b finished
+  static constexpr int bMReady = bPFree + kSBufs;    // [2 streams][4 warps] m of a block published
+  static constexpr int bOFull = bMReady + 8;         // every P.V of the item finished
+  static constexpr int bOFree = bOFull + 1;          // epilogue has read O
+  static constexpr int bDrain = bOFree + 1;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
   static constexpr int kXchg = kMisc + 16;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
-  static constexpr int kUsed = kXchg + 2 * 2 * 2 * 128 * 4;
+  static constexpr int kMSlot = kXchg + 2 * 2 * 2 * 128 * 4;  // float [2 streams][128 rows]
+  static constexpr int kUsed = kMSlot + 2 * 128 * 4;
   // +1024 for aligning the base; at least 120 KB so only one CTA fits per SM
   // (each CTA holds all 512 tensor-memory columns).
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
@@ -263,7 +308,17 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
         mbar_arrive_expect_tx(bar(kFull + slot), L::kTile);
         tma_tile<HD>(base + kRing + slot * L::kTile, map, bar(kFull + slot), p, c * 128, it.h, it.b);
       }
-      CALIBATT_TRACE_EVENT(lane == 0, V ? 2 : 1, kv);
+      if (kL2Prefetch > 0 && j + kL2Prefetch < it.n) {
+        const int jj = j + kL2Prefetch;
+        const int cp = ANCHOR ? jj : static_cast<int>(it.cols[jj]);
+        if (lane == 0) {
+          int c1, c2, c3;
+          map_coords(p, cp * 128, it.h, it.b, c1, c2, c3);
+#pragma unroll
+          for (int ch = 0; ch < HD / 64; ++ch) tma_prefetch_4d(map, ch * 64, c1, c2, c3);
+        }
+      }
+      CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, V ? 2 : 1, kv);
       ++issued;
       ++kv;
     }
@@ -277,92 +332,97 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
 
 
 // -------------------------------------------------------------------- MMA
+// Two issuing threads share the tensor core: warp 9 issues every S(j) and
+// warp 11 every O += P(j) V_j.  A wait on an mbarrier by the issuing thread
+// leaves the tensor core idle once its queue drains, so with one issuer every
+// wait is a bubble; with two, one thread's MMAs run while the other waits.
+// Ordering between them goes through barriers: S(j) waits for p_free of its
+// buffer (P(j - 3) V_{j-3} complete) before overwriting it.
 template <int HD, bool ANCHOR>
-__device__ void mma_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
+__device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0);
-  constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, 1);
   Cursor<ANCHOR> cur;
   cur.init(p);
   Item it;
-  uint32_t kv = 0, item = 0;  // global key-block iteration, item counter
-  uint32_t ta = 0, tb = 0;    // key blocks issued to stream 0 / stream 1 (global)
+  uint32_t g = 0, item = 0;  // global key-block iteration, item counter
   bool ok = true;
-
-  // O_s += P_s(g) V_g for the item-local block index jl (stream jl & 1) whose
-  // global iteration is g and whose per-stream ordinal is ts.
-  auto issue_pv = [&](int jl, uint32_t g, uint32_t ts) -> bool {
-    const int s = jl & 1;
-    const uint32_t vs = g % kVStages;
-    if (!W.wait(bar(L::bVFull + vs), (g / kVStages) & 1, 7)) return false;
-    if (!W.wait(bar(L::bPFull + s), ts & 1, 8)) return false;
-    if (jl == 0 && item > 0 && !W.wait(bar(L::bOFree), (item - 1) & 1, 9)) return false;
-    tc_fence_after();
-    CALIBATT_TRACE_EVENT(lane == 0, 4, g);
-    if (lane == 0) {
-      const uint32_t v_base = base + L::kV + vs * L::kTile;
-      const bool first = jl < 2;  // first block of this stream in the item
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        // A = P_s in tensor memory (16 keys = 8 columns per step); B = V
-        // (MN-major): 16 keys per step = 2048 bytes; next 64 columns of D at +16 KB.
-        mma_ts(tmem + kColO + s * 128, tmem + kColS + s * 128 + k * 8,
-               sw128_desc(v_base + k * 2048, kChunkBytes, 1024), kIdescO, (first && k == 0) ? 0u : 1u);
-      }
-      mma_commit(bar(L::bVEmpty + vs));
-      mma_commit(bar(L::bPVDone + s));
-    }
-    __syncwarp();
-    return true;
-  };
-
   while (ok && cur.next(p, it)) {
     if (!W.wait(bar(L::bQFull), item & 1, 4)) break;
     tc_fence_after();
-    const uint32_t kv0 = kv, ta0 = ta, tb0 = tb;
-    // Per-stream ordinal of item-local block jl.
-    auto ordinal = [&](int jl) -> uint32_t { return ((jl & 1) ? tb0 : ta0) + (jl >> 1); };
-    for (int j = 0; j < it.n; ++j) {
-      const int s = j & 1;
-      const uint32_t ks = kv % kKStages;
-      if (!W.wait(bar(L::bKFull + ks), (kv / kKStages) & 1, 5)) { ok = false; break; }
+    for (int j = 0; j < it.n; ++j, ++g) {
+      const uint32_t ks = g % kKStages, sb = g % kSBufs;
+      // The buffer's previous probabilities (block g - 3) must have been consumed.
+      if (g >= kSBufs && !W.wait(bar(L::bPFree + sb), ((g - kSBufs) / kSBufs) & 1, 6)) { ok = false; break; }
+      if (!W.wait(bar(L::bKFull + ks), (g / kKStages) & 1, 5)) { ok = false; break; }
       tc_fence_after();
-      CALIBATT_TRACE_EVENT(lane == 0, 3, kv);
       if (lane == 0) {
         const uint32_t k_base = base + L::kK + ks * L::kTile;
+        const uint32_t d = tmem + kColS + sb * 128;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           // K-major operands: 16 columns = 32 bytes per step inside a 64-column chunk.
           const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + kColS + s * 128, sw128_desc(base + L::kQ + off, 16, 1024),
-                 sw128_desc(k_base + off, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+          mma_ss(d, sw128_desc(base + L::kQ + off, 16, 1024), sw128_desc(k_base + off, 16, 1024), kIdescS,
+                 k > 0 ? 1u : 0u);
         }
         mma_commit(bar(L::bKEmpty + ks));
-        mma_commit(bar(L::bSFull + s));
+        mma_commit(bar(L::bSFull + sb));
         if (j == it.n - 1) mma_commit(bar(L::bQEmpty));
       }
       __syncwarp();
-      if (s) ++tb; else ++ta;
-      // The previous block belongs to the other stream; its P.V goes next, so
-      // each stream's P(j) is consumed before that stream's S(j + 2) is issued.
-      if (j >= 1) {
-        const int jp = j - 1;
-        if (!issue_pv(jp, kv0 + jp, ordinal(jp))) { ok = false; break; }
-      }
-      ++kv;
     }
     if (!ok) break;
-    if (it.n >= 1) {
-      const int jp = it.n - 1;
-      if (!issue_pv(jp, kv0 + jp, ordinal(jp))) break;
-    } else if (lane == 0) {
-      mbar_arrive(bar(L::bQEmpty));
-    }
+    if (it.n == 0 && lane == 0) mbar_arrive(bar(L::bQEmpty));
     __syncwarp();
     ++item;
   }
-  // Every MMA this warp issued must finish before tensor memory is freed.
+  // Every MMA this thread issued must finish before tensor memory is freed.
+  if (lane == 0) mma_commit(bar(L::bDrain));
+  __syncwarp();
+  drain_wait(bar(L::bDrain), 0);
+}
+
+template <int HD, bool ANCHOR>
+__device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
+  using L = Layout<HD>;
+  auto bar = [&](int i) { return base + L::kBar + 8u * i; };
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, 1);
+  Cursor<ANCHOR> cur;
+  cur.init(p);
+  Item it;
+  uint32_t g = 0, item = 0;
+  bool ok = true;
+  while (ok && cur.next(p, it)) {
+    // The epilogue of the previous item has read O (waited for every item,
+    // empty ones included, so each phase of o_free is consumed in order).
+    if (item > 0 && !W.wait(bar(L::bOFree), (item - 1) & 1, 9)) break;
+    for (int j = 0; j < it.n; ++j, ++g) {
+      const uint32_t vs = g % kVStages, sb = g % kSBufs;
+      if (!W.wait(bar(L::bVFull + vs), (g / kVStages) & 1, 7)) { ok = false; break; }
+      if (!W.wait(bar(L::bPFull + sb), (g / kSBufs) & 1, 8)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t v_base = base + L::kV + vs * L::kTile;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          // A = P in tensor memory (16 keys = 8 columns per step); B = V
+          // (MN-major): 16 keys per step = 2048 bytes; next 64 columns of D at +16 KB.
+          mma_ts(tmem + kColO, tmem + kColS + sb * 128 + k * 8,
+                 sw128_desc(v_base + k * 2048, kChunkBytes, 1024), kIdescO, (j == 0 && k == 0) ? 0u : 1u);
+        }
+        mma_commit(bar(L::bVEmpty + vs));
+        mma_commit(bar(L::bPFree + sb));
+        if (j == it.n - 1) mma_commit(bar(L::bOFull));
+      }
+      __syncwarp();
+    }
+    if (!ok) break;
+    if (it.n == 0 && lane == 0) mbar_arrive(bar(L::bOFull));
+    __syncwarp();
+    ++item;
+  }
   if (lane == 0) mma_commit(bar(L::bDrain));
   __syncwarp();
   drain_wait(bar(L::bDrain), 0);
@@ -373,7 +433,7 @@ __device__ void mma_role(const TcParams& p, uint32_t base, uint32_t tmem, const 
 // group owns query row t.  In the epilogue the two groups exchange (m_s, l_s)
 // through shared memory at a pair barrier (warps w and w+4, bar.red.or, which
 // also carries "a wait failed" so both warps leave together), then group s
-// writes output columns [s*D/2, (s+1)*D/2) of the merged result.
+// writes output columns [s*D/2, (s+1)*D/2) of O / l.
 template <int HD, bool ANCHOR>
 __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
                              const Waiter& W, int warp, int lane) {
@@ -383,35 +443,32 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
   const int pair_bar = 1 + quarter;     // named barrier shared with the partner warp
   float* xchg = reinterpret_cast<float*>(gbase + L::kXchg);
+  float* mslot = reinterpret_cast<float*>(gbase + L::kMSlot);
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tS = tmem + lane_off + kColS + s * 128;   // this stream's scores / probabilities
-  const uint32_t tO0 = tmem + lane_off + kColO;            // O_0 (O_1 at +128)
+  const uint32_t tS0 = tmem + lane_off + kColS;  // score buffer 0 (buffer b at +128 b)
+  const uint32_t tO = tmem + lane_off + kColO;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
-  // Waits until the P.V numbered ts of stream st has completed.
-  auto wait_pv = [&](int st, uint32_t ts, int where) -> bool {
-    if (!W.wait(bar(L::bPVDone + st), ts & 1, where)) return false;
-    tc_fence_after();
-    return true;
-  };
   Cursor<ANCHOR> cur;
   cur.init(p);
   Item it;
   uint32_t kv = 0, item = 0;
   uint32_t t_me = 0, t_other = 0;  // key blocks of this / the other stream so far (global)
-  uint32_t turns = 0;                // turns this stream has waited for
   bool ok = true;
   while (cur.next(p, it)) {
     const int n_s = (it.n + 1 - s) / 2;  // blocks of this stream in the item
-    float m_ref = -INFINITY, l = 0.f;
+    const uint32_t t_other0 = t_other;
+    float m_own = -INFINITY, l = 0.f;    // this stream's row sum, relative to m_own
     for (int k = 0; k < n_s; ++k) {
       const int j = 2 * k + s;  // item-local block index
-      ok = ok && W.wait(bar(L::bSFull + s), t_me & 1, 10);
+      const uint32_t g = kv + j;
+      const uint32_t tS = tS0 + (g % kSBufs) * 128;
+      ok = ok && W.wait(bar(L::bSFull + g % kSBufs), (g / kSBufs) & 1, 10);
       if (ok) tc_fence_after();
-      CALIBATT_TRACE_EVENT(lane == 0, 32 + warp, kv + j);
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 32 + warp, g);
       uint32_t sr[128];
       tmem_ld_x128(tS, sr);
-      CALIBATT_TRACE_EVENT(lane == 0, 40 + warp, kv + j);
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 40 + warp, g);
       float sc[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sc[c] = __uint_as_float(sr[c]);
@@ -431,28 +488,31 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       }
       const float mx_s =
           fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
+      // m(j - 1), published by the partner warp of the other stream (same
+      // rows; block j - 1 is that stream's block number t_other0 + (j - 1) / 2
+      // in global order).  The partner cannot publish again before it has
+      // read m(j), so the barrier is never two phases ahead of this wait.
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        const uint32_t prev_ord = t_other0 + static_cast<uint32_t>(j - 1) / 2;
+        ok = ok && W.wait(bar(L::bMReady + (1 - s) * 4 + quarter), prev_ord & 1, 13);
+        m_prev = mslot[(1 - s) * 128 + row];
+      }
       // The decision is taken per warp (tcgen05.ld/st are .sync.aligned and
       // need all 32 lanes); rows of a rescaling warp whose maximum did not grow
-      // get alpha = 1.  O_s itself is rescaled after the probabilities are
-      // written (the scores are no longer live then); it only has to happen
-      // before this block's P.V, which waits for p_full.
-      const bool rescale = __any_sync(0xFFFFFFFFu, mx_s > m_ref + kRescaleLog2);
-      float alpha = 1.f;
-      if (rescale) {
-        const float m_new = fmaxf(m_ref, mx_s);
-        alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_ref - m_new);
-        l *= alpha;
-        m_ref = m_new;
+      // keep their reference (alpha = 1).
+      const bool rescale = __any_sync(0xFFFFFFFFu, mx_s > m_prev + kRescaleLog2);
+      const float m_j = rescale ? fmaxf(m_prev, mx_s) : m_prev;
+      // O's factor; O is still zero while m_prev = -inf (every earlier P was 0).
+      const float alpha = (m_prev == -INFINITY) ? 0.f : fast_exp2(m_prev - m_j);
+      mslot[s * 128 + row] = m_j;
+      if (ok) mbar_arrive(bar(L::bMReady + s * 4 + quarter));
+      if (m_j != m_own) {
+        l = (m_own == -INFINITY) ? 0.f : l * fast_exp2(m_own - m_j);
+        m_own = m_j;
       }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // Wait for this block's turn on the MUFU unit: the previous key block
-      // (of the other stream, or the last block of the previous item) has
-      // finished its exponentials.
-      const uint32_t g = kv + j;
-      if (kExpTurns && g > 0) {
-        ok = ok && W.wait(bar(L::bTurn + s), turns & 1, 14);
-        ++turns;
-      }
+      const float m_use = (m_j == -INFINITY) ? 0.f : m_j;
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 56 + warp, g);
       // Probabilities in four chunks of 32 keys; each chunk's 16 packed
       // columns go to tensor memory (over the already-read scores) at once.
       float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
@@ -464,70 +524,70 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
           const int c = hh * 16 + cc;
           float x0, x1;
           fma2(x0, x1, sc[2 * c], sc[2 * c + 1], sl2, sl2, -m_use, -m_use);
-          const bool poly = kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1;
-          const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
-          const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
+          float p0, p1;
+          if (kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1) {
+            exp2_fma2(p0, p1, x0, x1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
           if (cc & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
           pk[cc] = pack_bf16x2(p0, p1);
         }
         if (ok) tmem_st_x16(tS + hh * 16, pk);
       }
       l += (la + lb) + (lc + ld);
-      // Hand the MUFU unit to the next key block in issue order: the other
-      // stream within the item, or stream 0 of the next item.
-      if (kExpTurns && ok) mbar_arrive(bar(L::bTurn + ((j + 1 < it.n) ? 1 - s : 0)));
-      CALIBATT_TRACE_EVENT(lane == 0, 48 + warp, kv + j);
-      if (rescale && k > 0) {
-        // O_s is stable once this stream's previous P.V has completed.
-        ok = ok && wait_pv(s, t_me - 1, 11);
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 48 + warp, g);
+      if (rescale && j > 0) {
+        // O carries m(j - 1) once P(j - 1).V has completed; P(j).V waits for
+        // p_full below, so nothing else touches these rows of O meanwhile.
+        // (The previous phase of that buffer's p_free, block j - 4, completed
+        // before S(j - 1) was issued; the next, block j + 2, needs P(j + 2):
+        // so the parity names P(j - 1).V.)
+        ok = ok && W.wait(bar(L::bPFree + (g - 1) % kSBufs), ((g - 1) / kSBufs) & 1, 11);
         if (ok) {
-          const uint32_t tOs = tO0 + s * 128;
+          tc_fence_after();
 #pragma unroll 1
           for (int ch = 0; ch < HD / 32; ++ch) {
             uint32_t o[32];
-            tmem_ld_x32(tOs + ch * 32, o);
+            tmem_ld_x32(tO + ch * 32, o);
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st_x32(tOs + ch * 32, o);
+            tmem_st_x32(tO + ch * 32, o);
           }
         }
       }
       if (ok) {
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::bPFull + s));
+        mbar_arrive(bar(L::bPFull + g % kSBufs));
       }
-      CALIBATT_TRACE_EVENT(lane == 0, 20 + warp, kv + j);
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 20 + warp, g);
       ++t_me;
     }
-    // The other stream's block count, to track its P.V completions too.
+    // The other stream's block count, to name its P.V completions.
     t_other += (it.n + s) / 2;
-    const uint32_t ta = s == 0 ? t_me : t_other, tb = s == 0 ? t_other : t_me;
-    kv += it.n;
 
     // ------------------------------------------------------------ epilogue
     // (A failed wait is acted on at the pair barrier below, which both warps
     // of the pair reach; leaving earlier could strand the partner there.)
-    const int n0 = (it.n + 1) / 2, n1 = it.n / 2;
-    if (n0 > 0) ok = ok && wait_pv(0, ta - 1, 12);
-    if (n1 > 0) ok = ok && wait_pv(1, tb - 1, 12);
+    ok = ok && W.wait(bar(L::bOFull), item & 1, 12);
+    if (ok) tc_fence_after();
+    kv += it.n;
     CALIBATT_TRACE_EVENT(lane == 0 && warp == 0, 10, kv);
     // Exchange buffer alternates by item so the partner's read of the
     // previous item's values can never meet this item's writes.
     float* xb = xchg + (item & 1) * 512;
-    xb[(s * 2 + 0) * 128 + row] = m_ref;
+    xb[(s * 2 + 0) * 128 + row] = m_own;
     xb[(s * 2 + 1) * 128 + row] = l;
     if (bar_red_or(pair_bar, 64, !ok)) { ok = false; break; }
     const float m_o = xb[((1 - s) * 2 + 0) * 128 + row];
     const float l_o = xb[((1 - s) * 2 + 1) * 128 + row];
-    const float m0 = s == 0 ? m_ref : m_o, m1 = s == 0 ? m_o : m_ref;
-    const float l0 = s == 0 ? l : l_o, l1 = s == 0 ? l_o : l;
-    const float m = fmaxf(m0, m1);
-    const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - m);
-    const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - m);
-    const float l_row = l0 * a0 + l1 * a1;
+    // References only grow along the list, so the larger one is m of the last block.
+    const float m = fmaxf(m_own, m_o);
+    const float l_row = (m_own == -INFINITY ? 0.f : l * fast_exp2(m_own - m)) +
+                        (m_o == -INFINITY ? 0.f : l_o * fast_exp2(m_o - m));
     const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-    const float w0 = a0 * inv_l, w1 = a1 * inv_l;
     const int64_t bh_off = static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
     // Destination rows of this thread's output.
     int64_t dst_token = -1;
@@ -553,26 +613,19 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
 #pragma unroll 1
     for (int ch = 0; ch < HD / 64; ++ch) {
       const int col = s * (HD / 2) + ch * 32;  // this group's output columns
-      uint32_t o0[32], o1[32];
-      if (n0 > 0) {
-        tmem_ld_x32(tO0 + col, o0);
+      uint32_t o[32];
+      if (it.n > 0) {
+        tmem_ld_x32(tO + col, o);
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) o0[c] = 0u;
-      }
-      if (n1 > 0) {
-        tmem_ld_x32(tO0 + 128 + col, o1);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o1[c] = 0u;
+        for (int c = 0; c < 32; ++c) o[c] = 0u;
       }
       uint4 pkd[4];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          v[e] = __uint_as_float(o0[8 * g + e]) * w0 + __uint_as_float(o1[8 * g + e]) * w1;
+        for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * g + e]) * inv_l;
         pkd[g].x = pack_bf16x2(v[0], v[1]);
         pkd[g].y = pack_bf16x2(v[2], v[3]);
         pkd[g].z = pack_bf16x2(v[4], v[5]);
@@ -622,15 +675,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       mbar_init(bar(L::bVFull + s), 1);
       mbar_init(bar(L::bVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::bSFull + s), 1);
-      mbar_init(bar(L::bPFull + s), kGroupThreads);
-      mbar_init(bar(L::bPVDone + s), 1);
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(bar(L::bSFull + b), 1);
+      mbar_init(bar(L::bPFull + b), kGroupThreads);
     }
+    for (int b = 0; b < kSBufs; ++b) mbar_init(bar(L::bPFree + b), 1);
+    for (int w = 0; w < 8; ++w) mbar_init(bar(L::bMReady + w), 32);
+    mbar_init(bar(L::bOFull), 1);
     mbar_init(bar(L::bOFree), kSoftmaxThreads);
-    mbar_init(bar(L::bTurn + 0), kGroupThreads);
-    mbar_init(bar(L::bTurn + 1), kGroupThreads);
-    mbar_init(bar(L::bDrain), 1);
+    mbar_init(bar(L::bDrain), 2);  // one commit from each MMA-issuing thread
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -649,21 +702,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == kProducerWarp) {
-    producer_role<HD, ANCHOR, false>(p, base, W, lane);
-  } else if (warp == kVProducerWarp) {
-    producer_role<HD, ANCHOR, true>(p, base, W, lane);
-  } else if (warp == kMmaWarp) {
-    mma_role<HD, ANCHOR>(p, base, tmem, W, lane);
+  // After the register split the two kinds of warpgroup never share code
+  // again: each ends with its own copy of the final CTA barrier.
+  if (warp >= 8) {
+    reg_dealloc<kOtherRegs>();
+    if (warp == kProducerWarp) {
+      producer_role<HD, ANCHOR, false>(p, base, W, lane);
+    } else if (warp == kVProducerWarp) {
+      producer_role<HD, ANCHOR, true>(p, base, W, lane);
+    } else if (warp == kMmaWarp) {
+      mma_s_role<HD, ANCHOR>(p, base, tmem, W, lane);
+    } else if (warp == kPvWarp) {
+      mma_pv_role<HD, ANCHOR>(p, base, tmem, W, lane);
+    }
+    tc_fence_before();
+    cta_bar_sync(kEndBarrier, kThreads);
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
   } else {
+    reg_alloc<kSoftmaxRegs>();
     softmax_role<HD, ANCHOR>(p, base, gbase, tmem, W, warp, lane);
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tc_fence_before();
+    cta_bar_sync(kEndBarrier, kThreads);
   }
 }
 
@@ -671,16 +733,32 @@ template <int HD, bool ANCHOR>
 cudaError_t launch_one(const TcParams& p, int grid, cudaStream_t s) {
   auto kern = tc_attn_kernel<HD, ANCHOR>;
   const int bytes = Layout<HD>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // The register split above assumes the CTA is launched with kLaunchRegs per
+  // thread; with fewer, setmaxnreg.inc could never be satisfied.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, bytes, s>>>(p);
   return cudaGetLastError();
 }
 
+// Even elements go through the packed pair routine the softmax uses (with their
+// odd neighbour), a trailing odd element through the scalar one.
 __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    y[i] = exp2_fma(x[i]);
+  for (int64_t i = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); i < n;
+       i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (i + 1 < n) {
+      float y0, y1;
+      exp2_fma2(y0, y1, x[i], x[i + 1]);
+      y[i] = y0;
+      y[i + 1] = y1;
+    } else {
+      y[i] = exp2_fma(x[i]);
+    }
+  }
 }
 
 }  // namespace
@@ -689,6 +767,11 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__
 extern "C" int calibatt_trace_read(unsigned long long* host, int max_records) {
   const int n = static_cast<int>(kTraceEvents * kTraceIters);
   cudaMemcpyFromSymbol(host, g_trace, sizeof(unsigned long long) * (n < max_records ? n : max_records));
+  return n;
+}
+extern "C" int calibatt_mma_prof_read(unsigned long long* host, int max_records) {
+  const int n = 1024 * 8;
+  cudaMemcpyFromSymbol(host, g_mma_prof, sizeof(unsigned long long) * (n < max_records ? n : max_records));
   return n;
 }
 extern "C" void calibatt_trace_reset() {

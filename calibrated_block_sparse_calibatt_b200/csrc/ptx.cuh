@@ -114,6 +114,20 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// Per-warpgroup register reallocation (all four warps of the group execute it).
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ void cta_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ----------------------------------------------------------------------- TMA
 
 // 4-D tiled bulk tensor load global -> shared, completing on an mbarrier.
@@ -124,6 +138,14 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+
+// Asks L2 to fetch a tile of a tensor (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -250,6 +272,22 @@ __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, f
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// exp2_fma for two values with packed f32x2 arithmetic (same reduction, same
+// cubic, same bounds): about six issue slots for two results.
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0, t1, u0, u1, f0, f1, p0, p1;
+  add2(t0, t1, x0, x1, 12582912.0f, 12582912.0f);
+  add2(u0, u1, t0, t1, -12582912.0f, -12582912.0f);
+  fma2(f0, f1, u0, u1, -1.0f, -1.0f, x0, x1);
+  fma2(p0, p1, f0, f1, 5.517166906e-02f, 5.517166906e-02f, 2.426111222e-01f, 2.426111222e-01f);
+  fma2(p0, p1, p0, p1, f0, f1, 6.932609855e-01f, 6.932609855e-01f);
+  fma2(p0, p1, p0, p1, f0, f1, 9.999280735e-01f, 9.999280735e-01f);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
