@@ -23,10 +23,11 @@
 // relative to the reference of its latest block; the epilogue combines the
 // two sums against the final reference.
 //
-// Freeing the second accumulator leaves room for three score buffers: S(j)
-// lives in buffer j mod 3 and S(j+3) can run as soon as P(j).V is done, so a
-// stream finds the scores of its next block ready when its current block
-// ends, and the tensor core's P.V + S work is off the softmax chain.
+// Freeing the second accumulator leaves room for separate score and
+// probability buffers per stream: a stream's next S is issued as soon as its
+// softmax warps have loaded the current scores into registers, so it finds
+// the scores of its next block ready when its current block ends, and the
+// tensor core's P.V + S work is off the softmax chain.
 //
 // CTA layout (384 threads, one CTA per SM, persistent):
 //   warps 0-3  softmax of stream 0, warps 4-7 softmax of stream 1: thread t of
@@ -37,10 +38,8 @@
 //   warp  9    TMEM allocator; one lane issues the S = Q K^T MMAs
 //   warp 10    producer of the V tiles
 //   warp 11    one lane issues the O += P V MMAs
-// Tensor memory (512 columns): score buffer b at 128*b, b = 0..2 (f32 scores;
-// the bf16 probabilities overwrite its first 64 columns once the scores are in
-// registers), O at 384.  S(j+3) reuses the buffer of P(j); its issuer waits
-// until P(j).V has completed before overwriting it.
+// Tensor memory (512 columns): stream s has its f32 scores S_s at 128*s and
+// its bf16 probabilities P_s at 256 + 64*s; O is at 384.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -97,8 +96,8 @@ constexpr bool kTraceMma = false;
 // 384 * kLaunchRegs the CTA was launched with.
 constexpr int kThreads = 384;       // 8 softmax warps, Q/K producer, MMA, V producer, spare
 constexpr int kLaunchRegs = 168;
-constexpr int kSoftmaxRegs = 224;
-constexpr int kOtherRegs = 56;
+constexpr int kSoftmaxRegs = 232;
+constexpr int kOtherRegs = 40;
 static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kThreads * kLaunchRegs, "register split");
 constexpr int kEndBarrier = 5;      // named barrier id (1-4: softmax warp pairs)
 constexpr int kProducerWarp = 8;    // Q and K tiles
@@ -122,8 +121,8 @@ constexpr int kKStages = CALIBATT_K_STAGES;
 constexpr int kVStages = CALIBATT_V_STAGES;
 constexpr int kL2Prefetch = CALIBATT_L2_PREFETCH;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 3;         // score buffers, S(j) in buffer j mod 3
-constexpr uint32_t kColS = 0;    // score buffer b at kColS + 128 * b
+constexpr uint32_t kColS = 0;    // stream s's f32 scores at kColS + 128 * s
+constexpr uint32_t kColP = 256;  // stream s's bf16 probabilities at kColP + 64 * s
 constexpr uint32_t kColO = 384;  // the output accumulator O
 constexpr float kRescaleLog2 = 8.0f;
 // One pair in kPolyEvery of exponentials runs on the FMA pipe (exp2_fma2)
@@ -132,6 +131,18 @@ constexpr float kRescaleLog2 = 8.0f;
 #define CALIBATT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
+// Probabilities packed to bf16 with integer ops (round half up) instead of
+// the conversion instruction.
+#ifndef CALIBATT_PACK_INT
+#define CALIBATT_PACK_INT 0
+#endif
+constexpr bool kPackInt = CALIBATT_PACK_INT != 0;
+// Where the softmax waits for its previous P to be consumed: before the
+// exponentials (1) or after the first chunk of them (0).
+#ifndef CALIBATT_PFREE_EARLY
+#define CALIBATT_PFREE_EARLY 1
+#endif
+constexpr bool kPFreeEarly = CALIBATT_PFREE_EARLY != 0;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -146,18 +157,19 @@ struct Layout {
   static constexpr int bQFull = 0, bQEmpty = 1;
   static constexpr int bKFull = 2, bKEmpty = bKFull + kKStages;
   static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
-  static constexpr int bSFull = bVEmpty + kVStages;  // [3] scores in buffer b ready
-  static constexpr int bPFull = bSFull + kSBufs;     // [3] probabilities in buffer b ready
-  static constexpr int bPFree = bPFull + kSBufs;     // [3] P.V of the block in buffer b finished
-  static constexpr int bMReady = bPFree + kSBufs;    // [2 streams][4 warps] m of a block published
-  static constexpr int bOFull = bMReady + 8;         // every P.V of the item finished
+  static constexpr int bSFull = bVEmpty + kVStages;  // [2] scores of stream s ready
+  static constexpr int bSFree = bSFull + 2;          // [2] stream s has read its scores
+  static constexpr int bPFull = bSFree + 2;          // [2] probabilities of stream s ready
+  static constexpr int bPFree = bPFull + 2;          // [2] P.V of stream s's block finished
+  static constexpr int bOFull = bPFree + 2;          // every P.V of the item finished
   static constexpr int bOFree = bOFull + 1;          // epilogue has read O
   static constexpr int bDrain = bOFree + 1;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
   static constexpr int kXchg = kMisc + 16;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
-  static constexpr int kMSlot = kXchg + 2 * 2 * 2 * 128 * 4;  // float [2 streams][128 rows]
-  static constexpr int kUsed = kMSlot + 2 * 128 * 4;
+  // {m bits, stream ordinal + 1} [2 streams][128 rows], 8-byte slots
+  static constexpr int kMSlot = kXchg + 2 * 2 * 2 * 128 * 4;
+  static constexpr int kUsed = kMSlot + 2 * 128 * 8;
   // +1024 for aligning the base; at least 120 KB so only one CTA fits per SM
   // (each CTA holds all 512 tensor-memory columns).
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
@@ -336,8 +348,9 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
 // warp 11 every O += P(j) V_j.  A wait on an mbarrier by the issuing thread
 // leaves the tensor core idle once its queue drains, so with one issuer every
 // wait is a bubble; with two, one thread's MMAs run while the other waits.
-// Ordering between them goes through barriers: S(j) waits for p_free of its
-// buffer (P(j - 3) V_{j-3} complete) before overwriting it.
+// Block j belongs to stream j mod 2 of its item; t is its ordinal within
+// that stream over the whole launch, and the barriers of stream s count
+// those ordinals.
 template <int HD, bool ANCHOR>
 __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
   using L = Layout<HD>;
@@ -346,20 +359,26 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
   Cursor<ANCHOR> cur;
   cur.init(p);
   Item it;
-  uint32_t g = 0, item = 0;  // global key-block iteration, item counter
+  uint32_t g = 0, item = 0;      // global key-block iteration, item counter
+  uint32_t t0 = 0, t1 = 0;       // blocks issued per stream
   bool ok = true;
   while (ok && cur.next(p, it)) {
     if (!W.wait(bar(L::bQFull), item & 1, 4)) break;
     tc_fence_after();
     for (int j = 0; j < it.n; ++j, ++g) {
-      const uint32_t ks = g % kKStages, sb = g % kSBufs;
-      // The buffer's previous probabilities (block g - 3) must have been consumed.
-      if (g >= kSBufs && !W.wait(bar(L::bPFree + sb), ((g - kSBufs) / kSBufs) & 1, 6)) { ok = false; break; }
+      const int s = j & 1;
+      const uint32_t t = s ? t1++ : t0++;
+      const uint32_t ks = g % kKStages;
+      // The stream's previous scores must be in its softmax warps' registers.
+      CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 6, g);
+      if (t > 0 && !W.wait(bar(L::bSFree + s), (t - 1) & 1, 6)) { ok = false; break; }
+      CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 7, g);
       if (!W.wait(bar(L::bKFull + ks), (g / kKStages) & 1, 5)) { ok = false; break; }
       tc_fence_after();
+      CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 3, g);
       if (lane == 0) {
         const uint32_t k_base = base + L::kK + ks * L::kTile;
-        const uint32_t d = tmem + kColS + sb * 128;
+        const uint32_t d = tmem + kColS + s * 128;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           // K-major operands: 16 columns = 32 bytes per step inside a 64-column chunk.
@@ -368,7 +387,7 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
                  k > 0 ? 1u : 0u);
         }
         mma_commit(bar(L::bKEmpty + ks));
-        mma_commit(bar(L::bSFull + sb));
+        mma_commit(bar(L::bSFull + s));
         if (j == it.n - 1) mma_commit(bar(L::bQEmpty));
       }
       __syncwarp();
@@ -393,15 +412,18 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
   cur.init(p);
   Item it;
   uint32_t g = 0, item = 0;
+  uint32_t t0 = 0, t1 = 0;
   bool ok = true;
   while (ok && cur.next(p, it)) {
     // The epilogue of the previous item has read O (waited for every item,
     // empty ones included, so each phase of o_free is consumed in order).
     if (item > 0 && !W.wait(bar(L::bOFree), (item - 1) & 1, 9)) break;
     for (int j = 0; j < it.n; ++j, ++g) {
-      const uint32_t vs = g % kVStages, sb = g % kSBufs;
+      const int s = j & 1;
+      const uint32_t t = s ? t1++ : t0++;
+      const uint32_t vs = g % kVStages;
       if (!W.wait(bar(L::bVFull + vs), (g / kVStages) & 1, 7)) { ok = false; break; }
-      if (!W.wait(bar(L::bPFull + sb), (g / kSBufs) & 1, 8)) { ok = false; break; }
+      if (!W.wait(bar(L::bPFull + s), t & 1, 8)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t v_base = base + L::kV + vs * L::kTile;
@@ -409,11 +431,11 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
         for (int k = 0; k < 8; ++k) {
           // A = P in tensor memory (16 keys = 8 columns per step); B = V
           // (MN-major): 16 keys per step = 2048 bytes; next 64 columns of D at +16 KB.
-          mma_ts(tmem + kColO, tmem + kColS + sb * 128 + k * 8,
+          mma_ts(tmem + kColO, tmem + kColP + s * 64 + k * 8,
                  sw128_desc(v_base + k * 2048, kChunkBytes, 1024), kIdescO, (j == 0 && k == 0) ? 0u : 1u);
         }
         mma_commit(bar(L::bVEmpty + vs));
-        mma_commit(bar(L::bPFree + sb));
+        mma_commit(bar(L::bPFree + s));
         if (j == it.n - 1) mma_commit(bar(L::bOFull));
       }
       __syncwarp();
@@ -443,9 +465,14 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
   const int pair_bar = 1 + quarter;     // named barrier shared with the partner warp
   float* xchg = reinterpret_cast<float*>(gbase + L::kXchg);
-  float* mslot = reinterpret_cast<float*>(gbase + L::kMSlot);
+  // Row `row`'s reference maximum is handed between the two threads that own
+  // the row (one per stream) through an 8-byte slot {m, ordinal + 1} written
+  // in one store; the reader spins (bounded) until the ordinal it needs shows.
+  const uint32_t my_slot = smem_addr(gbase + L::kMSlot) + (s * 128 + row) * 8;
+  const uint32_t other_slot = smem_addr(gbase + L::kMSlot) + ((1 - s) * 128 + row) * 8;
   const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tS0 = tmem + lane_off + kColS;  // score buffer 0 (buffer b at +128 b)
+  const uint32_t tS = tmem + lane_off + kColS + s * 128;  // this stream's scores
+  const uint32_t tP = tmem + lane_off + kColP + s * 64;   // and probabilities
   const uint32_t tO = tmem + lane_off + kColO;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
@@ -461,13 +488,15 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
     float m_own = -INFINITY, l = 0.f;    // this stream's row sum, relative to m_own
     for (int k = 0; k < n_s; ++k) {
       const int j = 2 * k + s;  // item-local block index
-      const uint32_t g = kv + j;
-      const uint32_t tS = tS0 + (g % kSBufs) * 128;
-      ok = ok && W.wait(bar(L::bSFull + g % kSBufs), (g / kSBufs) & 1, 10);
+      [[maybe_unused]] const uint32_t g = kv + j;
+      ok = ok && W.wait(bar(L::bSFull + s), t_me & 1, 10);
       if (ok) tc_fence_after();
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 32 + warp, g);
       uint32_t sr[128];
       tmem_ld_x128(tS, sr);
+      // The scores are in registers: the next S of this stream may overwrite them.
+      tc_fence_before();
+      if (ok) mbar_arrive(bar(L::bSFree + s));
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 40 + warp, g);
       float sc[128];
 #pragma unroll
@@ -492,26 +521,27 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       // rows; block j - 1 is that stream's block number t_other0 + (j - 1) / 2
       // in global order).  The partner cannot publish again before it has
       // read m(j), so the barrier is never two phases ahead of this wait.
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 12 + s, g);
       float m_prev = -INFINITY;
       if (j > 0) {
         const uint32_t prev_ord = t_other0 + static_cast<uint32_t>(j - 1) / 2;
-        ok = ok && W.wait(bar(L::bMReady + (1 - s) * 4 + quarter), prev_ord & 1, 13);
-        m_prev = mslot[(1 - s) * 128 + row];
+        ok = ok && W.spin_slot(other_slot, prev_ord + 1u, 13, m_prev);
       }
-      // The decision is taken per warp (tcgen05.ld/st are .sync.aligned and
-      // need all 32 lanes); rows of a rescaling warp whose maximum did not grow
-      // keep their reference (alpha = 1).
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 14 + s, g);
       const bool rescale = __any_sync(0xFFFFFFFFu, mx_s > m_prev + kRescaleLog2);
       const float m_j = rescale ? fmaxf(m_prev, mx_s) : m_prev;
-      // O's factor; O is still zero while m_prev = -inf (every earlier P was 0).
-      const float alpha = (m_prev == -INFINITY) ? 0.f : fast_exp2(m_prev - m_j);
-      mslot[s * 128 + row] = m_j;
-      if (ok) mbar_arrive(bar(L::bMReady + s * 4 + quarter));
+      st_shared_v2(my_slot, __float_as_uint(m_j), t_me + 1u);
       if (m_j != m_own) {
         l = (m_own == -INFINITY) ? 0.f : l * fast_exp2(m_own - m_j);
         m_own = m_j;
       }
       const float m_use = (m_j == -INFINITY) ? 0.f : m_j;
+      CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 16 + s, g);
+      if (kPFreeEarly && t_me > 0) {
+        // P of this stream's previous block must have been consumed by its P.V.
+        ok = ok && W.wait(bar(L::bPFree + s), (t_me - 1) & 1, 14);
+        if (ok) tc_fence_after();
+      }
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 56 + warp, g);
       // Probabilities in four chunks of 32 keys; each chunk's 16 packed
       // columns go to tensor memory (over the already-read scores) at once.
@@ -532,21 +562,30 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
             p1 = fast_exp2(x1);
           }
           if (cc & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
-          pk[cc] = pack_bf16x2(p0, p1);
+          pk[cc] = kPackInt ? pack_bf16x2_nonneg(p0, p1) : pack_bf16x2(p0, p1);
         }
-        if (ok) tmem_st_x16(tS + hh * 16, pk);
+        if (!kPFreeEarly && hh == 0 && t_me > 0) {
+          // P of this stream's previous block must have been consumed by its
+          // P.V (waited here, after the first exponentials, to hide the wait).
+          ok = ok && W.wait(bar(L::bPFree + s), (t_me - 1) & 1, 14);
+          if (ok) tc_fence_after();
+        }
+        if (ok) tmem_st_x16(tP + hh * 16, pk);
       }
       l += (la + lb) + (lc + ld);
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 48 + warp, g);
       if (rescale && j > 0) {
         // O carries m(j - 1) once P(j - 1).V has completed; P(j).V waits for
         // p_full below, so nothing else touches these rows of O meanwhile.
-        // (The previous phase of that buffer's p_free, block j - 4, completed
-        // before S(j - 1) was issued; the next, block j + 2, needs P(j + 2):
-        // so the parity names P(j - 1).V.)
-        ok = ok && W.wait(bar(L::bPFree + (g - 1) % kSBufs), ((g - 1) / kSBufs) & 1, 11);
+        // (The other stream's previous P.V, block j - 3, completed before
+        // this stream's P.V of block j - 2, seen above; its next, block
+        // j + 1, needs P(j): so the parity names P(j - 1).V.)
+        const uint32_t prev_ord = t_other0 + static_cast<uint32_t>(j - 1) / 2;
+        ok = ok && W.wait(bar(L::bPFree + (1 - s)), prev_ord & 1, 11);
         if (ok) {
           tc_fence_after();
+          // O's factor; O is still zero while m_prev = -inf (every earlier P was 0).
+          const float alpha = (m_prev == -INFINITY) ? 0.f : fast_exp2(m_prev - m_j);
 #pragma unroll 1
           for (int ch = 0; ch < HD / 32; ++ch) {
             uint32_t o[32];
@@ -560,7 +599,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       if (ok) {
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::bPFull + g % kSBufs));
+        mbar_arrive(bar(L::bPFull + s));
       }
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 20 + warp, g);
       ++t_me;
@@ -675,15 +714,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       mbar_init(bar(L::bVFull + s), 1);
       mbar_init(bar(L::bVEmpty + s), 1);
     }
-    for (int b = 0; b < kSBufs; ++b) {
-      mbar_init(bar(L::bSFull + b), 1);
-      mbar_init(bar(L::bPFull + b), kGroupThreads);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(bar(L::bSFull + st), 1);
+      mbar_init(bar(L::bSFree + st), kGroupThreads);
+      mbar_init(bar(L::bPFull + st), kGroupThreads);
+      mbar_init(bar(L::bPFree + st), 1);
     }
-    for (int b = 0; b < kSBufs; ++b) mbar_init(bar(L::bPFree + b), 1);
-    for (int w = 0; w < 8; ++w) mbar_init(bar(L::bMReady + w), 32);
     mbar_init(bar(L::bOFull), 1);
     mbar_init(bar(L::bOFree), kSoftmaxThreads);
     mbar_init(bar(L::bDrain), 2);  // one commit from each MMA-issuing thread
+    for (int i = 0; i < 256; ++i) st_shared_v2(base + L::kMSlot + i * 8, 0u, 0u);  // tag 0: no m yet
     *abort_flag = 0;
     fence_mbar_init();
   }

@@ -96,7 +96,38 @@ struct Waiter {
     }
     return __all_sync(0xFFFFFFFFu, ok);
   }
+
+  // Per-thread bounded spin on an 8-byte shared-memory slot {value, tag}
+  // until tag == want; returns the value through `out`.  Lanes may leave at
+  // different times; the result is made warp-uniform at the end.
+  __device__ __forceinline__ bool spin_slot(uint32_t slot, uint32_t want, int where, float& out) const {
+    uint32_t v, tag;
+    asm volatile("ld.volatile.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v), "=r"(tag) : "r"(slot) : "memory");
+    bool ok = tag == want;
+    if (!ok) {
+      const unsigned long long t0 = globaltimer();
+#pragma unroll 1
+      for (uint32_t i = 1;; ++i) {
+        asm volatile("ld.volatile.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v), "=r"(tag) : "r"(slot) : "memory");
+        if (tag == want) { ok = true; break; }
+        if ((i & 255u) == 0u) {
+          if (*abort_flag) break;
+          if (globaltimer() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            if (status) atomicCAS(status, 0, 4 | (where << 8));
+            break;
+          }
+        }
+      }
+    }
+    out = __uint_as_float(v);
+    return __all_sync(0xFFFFFFFFu, ok);
+  }
 };
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
 
 // Named-barrier reduction: the `nthreads` threads arriving at barrier `id`
 // all receive the OR of their predicates.  Used both to meet a partner warp
