@@ -60,11 +60,6 @@ __device__ unsigned long long g_trace[kTraceEvents * kTraceIters];
 __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
   if (blockIdx.x == 0 && idx < kTraceIters) g_trace[ev * kTraceIters + idx] = clock64();
 }
-// Per-CTA totals of the MMA thread's time by phase (clock reads only inside
-// the loop; one store per phase at the end).
-__device__ unsigned long long g_mma_prof[1024 * 8];
-#define CALIBATT_PROF_T(var) const long long var = clock64()
-#define CALIBATT_PROF_ADD(slot, t0) prof[slot] += clock64() - (t0)
 #define CALIBATT_TRACE_EVENT(cond, ev, idx) \
   do {                                     \
     if (cond) trace_event(ev, idx);        \
@@ -79,12 +74,6 @@ constexpr bool kTraceMma = false;
 #else
 #define CALIBATT_TRACE_EVENT(cond, ev, idx) \
   do {                                     \
-  } while (0)
-#define CALIBATT_PROF_T(var) \
-  do {                       \
-  } while (0)
-#define CALIBATT_PROF_ADD(slot, t0) \
-  do {                              \
   } while (0)
 #endif
 
@@ -112,14 +101,8 @@ constexpr int kSoftmaxThreads = 256;
 #ifndef CALIBATT_V_STAGES
 #define CALIBATT_V_STAGES 2
 #endif
-// Key blocks ahead of the current one whose K/V tiles the producers ask L2 to
-// fetch (0 = no prefetch).
-#ifndef CALIBATT_L2_PREFETCH
-#define CALIBATT_L2_PREFETCH 0
-#endif
 constexpr int kKStages = CALIBATT_K_STAGES;
 constexpr int kVStages = CALIBATT_V_STAGES;
-constexpr int kL2Prefetch = CALIBATT_L2_PREFETCH;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;    // stream s's f32 scores at kColS + 128 * s
 constexpr uint32_t kColP = 256;  // stream s's bf16 probabilities at kColP + 64 * s
@@ -131,18 +114,7 @@ constexpr float kRescaleLog2 = 8.0f;
 #define CALIBATT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
-// Probabilities packed to bf16 with integer ops (round half up) instead of
-// the conversion instruction.
-#ifndef CALIBATT_PACK_INT
-#define CALIBATT_PACK_INT 0
-#endif
-constexpr bool kPackInt = CALIBATT_PACK_INT != 0;
-// Where the softmax waits for its previous P to be consumed: before the
-// exponentials (1) or after the first chunk of them (0).
-#ifndef CALIBATT_PFREE_EARLY
-#define CALIBATT_PFREE_EARLY 1
-#endif
-constexpr bool kPFreeEarly = CALIBATT_PFREE_EARLY != 0;
+
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
@@ -319,16 +291,6 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(kFull + slot), L::kTile);
         tma_tile<HD>(base + kRing + slot * L::kTile, map, bar(kFull + slot), p, c * 128, it.h, it.b);
-      }
-      if (kL2Prefetch > 0 && j + kL2Prefetch < it.n) {
-        const int jj = j + kL2Prefetch;
-        const int cp = ANCHOR ? jj : static_cast<int>(it.cols[jj]);
-        if (lane == 0) {
-          int c1, c2, c3;
-          map_coords(p, cp * 128, it.h, it.b, c1, c2, c3);
-#pragma unroll
-          for (int ch = 0; ch < HD / 64; ++ch) tma_prefetch_4d(map, ch * 64, c1, c2, c3);
-        }
       }
       CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, V ? 2 : 1, kv);
       ++issued;
@@ -537,7 +499,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       }
       const float m_use = (m_j == -INFINITY) ? 0.f : m_j;
       CALIBATT_TRACE_EVENT(lane == 0 && quarter == 0, 16 + s, g);
-      if (kPFreeEarly && t_me > 0) {
+      if (t_me > 0) {
         // P of this stream's previous block must have been consumed by its P.V.
         ok = ok && W.wait(bar(L::bPFree + s), (t_me - 1) & 1, 14);
         if (ok) tc_fence_after();
@@ -562,13 +524,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
             p1 = fast_exp2(x1);
           }
           if (cc & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
-          pk[cc] = kPackInt ? pack_bf16x2_nonneg(p0, p1) : pack_bf16x2(p0, p1);
-        }
-        if (!kPFreeEarly && hh == 0 && t_me > 0) {
-          // P of this stream's previous block must have been consumed by its
-          // P.V (waited here, after the first exponentials, to hide the wait).
-          ok = ok && W.wait(bar(L::bPFree + s), (t_me - 1) & 1, 14);
-          if (ok) tc_fence_after();
+          pk[cc] = pack_bf16x2(p0, p1);
         }
         if (ok) tmem_st_x16(tP + hh * 16, pk);
       }
@@ -807,11 +763,6 @@ __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__
 extern "C" int calibatt_trace_read(unsigned long long* host, int max_records) {
   const int n = static_cast<int>(kTraceEvents * kTraceIters);
   cudaMemcpyFromSymbol(host, g_trace, sizeof(unsigned long long) * (n < max_records ? n : max_records));
-  return n;
-}
-extern "C" int calibatt_mma_prof_read(unsigned long long* host, int max_records) {
-  const int n = 1024 * 8;
-  cudaMemcpyFromSymbol(host, g_mma_prof, sizeof(unsigned long long) * (n < max_records ? n : max_records));
   return n;
 }
 extern "C" void calibatt_trace_reset() {
