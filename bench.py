@@ -234,6 +234,100 @@ def run_reference(args, rank, world):
     del torch
 
 
+def run_sweep(args, C, torch, stream, pk):
+    """Schedule sweep: a dictionary holding every (timestep, layer) record of
+    the schedule, then one dual-path call per (t, l) on fresh seeded inputs,
+    timed with CUDA events; the dense path is timed on a sample of the calls."""
+    import time
+    wl = W.WORKLOADS["720p_sweep"]
+    T, L, H, nb = args.sweep_steps, args.sweep_layers, wl.heads, wl.num_blocks
+    t_build = time.time()
+    nnz = sum(W.sweep_record_blocks(wl, t, l, h, T) for t in range(T) for l in range(L) for h in range(H))
+    dct = C.MaskDictionary(T, L, H, nb, nb, wl.block, nnz)
+    for t in range(T):
+        for l in range(L):
+            masks, rep = W.sweep_layer_masks(wl, t, l, "cuda", T)
+            rp, ci = W.layer_csr(masks)
+            rep_arr = np.zeros(H, np.uint8)
+            rep_arr[list(rep)] = 1
+            dct.set_layer(t, l, rp, ci, rep_arr)
+    build_s = time.time() - t_build
+    info = dct.info()
+    anchor_tiles_per_head = -(-wl.frames * len(wl.anchors) * wl.cols // 128) * nb
+    tiles = 0
+    for t in range(T):
+        for l in range(L):
+            li = dct.layer_info(t, l)
+            tiles += li["retained_tiles"] + li["repetitive_heads"] * anchor_tiles_per_head
+    o = None
+
+    def call(q, k, v, o, t, l):
+        C.calibatt_dual_path_attn(q, k, v, o, dct, t, l, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block,
+                                  stream=stream)
+
+    q, k, v = W.make_qkv(W.seed_for("sweep-qkv", 0, 0) % (1 << 62), 1, wl.seq_len, H, wl.head_dim, "bf16",
+                         wl.input_std, "cuda")
+    o = torch.empty_like(q)
+    for _ in range(args.warmup):
+        call(q, k, v, o, 0, 0)
+    torch.cuda.synchronize()
+    evs = []
+    with ClockSampler(0) as clk:
+        for t in range(T):
+            for l in range(L):
+                del q, k, v
+                q, k, v = W.make_qkv(W.seed_for("sweep-qkv", t, l) % (1 << 62), 1, wl.seq_len, H, wl.head_dim,
+                                     "bf16", wl.input_std, "cuda")
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                call(q, k, v, o, t, l)
+                b.record(stream)
+                evs.append((a, b))
+        torch.cuda.synchronize()
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out during the sweep")
+    per_call = [a.elapsed_time(b) for a, b in evs]
+    sparse_s = sum(per_call) / 1e3
+    # dense path: all-ones masks for every head, on the inputs of a sample of the calls
+    ones = [np.ones((nb, nb), bool)] * H
+    d_dense = build_dict(C, ones, H, nb, wl.block)
+    dense_tiles = d_dense.layer_info(0, 0)["retained_tiles"]
+    picks = [(i * T // max(1, args.dense_sample), (i * 7) % L) for i in range(min(args.dense_sample, T * L))]
+    dense_ms = []
+    for t, l in picks:
+        q2, k2, v2 = W.make_qkv(W.seed_for("sweep-qkv", t, l) % (1 << 62), 1, wl.seq_len, H, wl.head_dim, "bf16",
+                                wl.input_std, "cuda")
+        dense_ms.append(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_block_sparse_attn(q2, k2, v2, o, d_dense, 0, 0, wl.block, stream=stream),
+            1, 1, stream)))
+        del q2, k2, v2
+    d_dense.close()
+    dense_s = statistics.mean(dense_ms) * T * L / 1e3
+    value = tiles * FLOP_PER_TILE / sparse_s / 1e12
+    line = {
+        "metric": "effective TFLOP/s (retained blocks) and ms/call, % of B200 BF16 tensor peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": T * L, "warmup": args.warmup,
+        "ms_per_step": sparse_s * 1e3 / (T * L), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "wan2.1-14b-720p schedule sweep, dual path (block-sparse + anchor heads)",
+                   "timesteps": T, "layers": L, "heads": H, "repetitive_heads_per_call": W.SWEEP_REPETITIVE,
+                   "anchors": list(wl.anchors), "density": "0.60 -> 0.20 over the timesteps",
+                   "inputs": "fresh seeded Q/K/V per call (2.32 GB > L2)", "parallelism": "replicas x1"},
+        "pct_of_peak": value / pk["bf16_tflops"],
+        "clocks": clk.summary(),
+        "sweep": {"sparse_total_s": sparse_s, "dense_total_s": dense_s,
+                  "dense_total_basis": f"mean of {len(dense_ms)} sampled calls x {T * L} calls",
+                  "dense_ms_per_call": statistics.mean(dense_ms), "speedup_vs_dense": dense_s / sparse_s,
+                  "effective_tiles": tiles, "dense_tiles_per_call": dense_tiles,
+                  "dictionary_device_bytes": info["device_bytes"], "dictionary_blocks": info["nnz"],
+                  "dictionary_build_s": build_s,
+                  "min_ms_per_call": min(per_call), "max_ms_per_call": max(per_call)},
+        "gpu_launches": 2 * T * L,
+    }
+    print(json.dumps(line), flush=True)
+    dct.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -244,6 +338,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the dense / dual-path / e2e legs")
     ap.add_argument("--heads", type=int, default=40,
                     help="heads of the 720p layer (fewer heads = smaller case for profiling)")
+    ap.add_argument("--workload", default="720p", choices=["720p", "sweep"],
+                    help="sweep: the mask-dictionary schedule sweep (one dual-path 720p call per "
+                         "timestep and layer), reported as aggregate time against the dense path")
+    ap.add_argument("--sweep-steps", type=int, default=W.SWEEP_STEPS)
+    ap.add_argument("--sweep-layers", type=int, default=W.SWEEP_LAYERS)
+    ap.add_argument("--dense-sample", type=int, default=50,
+                    help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -270,6 +371,11 @@ def main():
 
     pk = peaks()
     stream = torch.cuda.current_stream()
+    if args.workload == "sweep":
+        if world > 1:
+            raise SystemExit("the sweep workload runs on one GPU")
+        run_sweep(args, C, torch, stream, pk)
+        return
     import dataclasses
     wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
     masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])

@@ -210,28 +210,42 @@ def _sampled_blocks(rng, nb, k):
     return sorted({0, nb - 1, *mid.tolist()})
 
 
+def _f32(t):
+    return t.detach().float().cpu().numpy()
+
+
+def _block_rows(blocks, seq_len):
+    return np.concatenate([np.arange(r * 128, min(seq_len, (r + 1) * 128)) for r in blocks])
+
+
 @pytest.mark.parametrize("name", ["480p", "720p"])
 def test_full_size_sparse_sampled(C, name):
+    """Every head at full size, 8 sampled q-blocks each including the first and
+    the ragged last one, against the oracle (evaluated in spawned workers)."""
+    import _oracle_jobs as J
+
     wl = W.WORKLOADS[name]
     q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
     masks, _ = W.workload_masks(wl)
     masks = [masks[h] for h in range(wl.heads)]
     out, _ = _run_sparse(C, q, k, v, masks, wl.block)
     rng = np.random.default_rng(1)
-    errs = []
-    heads_deep = set(rng.choice(wl.heads, 3, replace=False).tolist())
+    jobs, got = [], []
     for h in range(wl.heads):
-        blocks = _sampled_blocks(rng, wl.num_blocks, 8 if h in heads_deep else 3)
-        rows = np.concatenate([np.arange(r * 128, min(wl.seq_len, (r + 1) * 128)) for r in blocks])
-        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
-        ref, _ = O.block_sparse_attention(qh, kh, vh, masks[h], wl.block, rows=rows)
-        got = _np(out[0, torch.as_tensor(rows, device=q.device), h])
-        errs.append(np.abs(got - ref))
-    err = np.concatenate([e.ravel() for e in errs])
+        rows = _block_rows(_sampled_blocks(rng, wl.num_blocks, 8), wl.seq_len)
+        jobs.append((_f32(q[0, rows, h]), _f32(k[0, :wl.seq_len, h]), _f32(v[0, :wl.seq_len, h]), masks[h],
+                     wl.block, rows))
+        got.append(_np(out[0, torch.as_tensor(rows, device=q.device), h]))
+    refs = J.sparse_rows_many(jobs)
+    err = np.concatenate([np.abs(g - r).ravel() for g, r in zip(got, refs)])
     assert err.max() <= BF16_MAX and err.mean() <= BF16_MEAN, (err.max(), err.mean())
 
 
 def test_full_size_dual_path_sampled(C):
+    """The dual-path 720p layer: every anchor head on sampled rows of two frames,
+    every sparse head on 8 sampled q-blocks, broadcast rows bitwise equal."""
+    import _oracle_jobs as J
+
     wl = W.WORKLOADS["720p_dual"]
     q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
     masks, rep_heads = W.workload_masks(wl)
@@ -247,26 +261,25 @@ def test_full_size_dual_path_sampled(C):
     # anchor heads: rows of two frames, including the last frame's last row
     f_rows = np.concatenate([np.arange(f * wl.tokens_per_frame, (f + 1) * wl.tokens_per_frame)
                              for f in (int(rng.integers(0, wl.frames - 1)), wl.frames - 1)])
-    sample = f_rows[rng.choice(len(f_rows), 600, replace=False)]
-    for h in rep_heads[:4]:
-        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
-        ref, _ = O.anchor_attention(qh, kh, vh, wl.frames, wl.rows, wl.cols, wl.anchors, rows=sample)
-        got = _np(out[0, torch.as_tensor(sample, device=q.device), h])
-        _assert_close(got, ref, "bf16")
+    sample = np.union1d(f_rows[rng.choice(len(f_rows), 400, replace=False)], [wl.seq_len - 1])
+    a_jobs = [(_f32(q[0, :wl.seq_len, h]), _f32(k[0, :wl.seq_len, h]), _f32(v[0, :wl.seq_len, h]),
+               wl.frames, wl.rows, wl.cols, wl.anchors, sample) for h in rep_heads]
+    # sparse heads: 8 sampled q-blocks each
+    sparse_heads = [h for h in range(wl.heads) if h not in rep_heads]
+    s_rows = {h: _block_rows(_sampled_blocks(rng, wl.num_blocks, 8), wl.seq_len) for h in sparse_heads}
+    s_jobs = [(_f32(q[0, s_rows[h], h]), _f32(k[0, :wl.seq_len, h]), _f32(v[0, :wl.seq_len, h]), masks[h],
+               wl.block, s_rows[h]) for h in sparse_heads]
+    a_refs = J.anchor_rows_many(a_jobs)
+    for h, ref in zip(rep_heads, a_refs):
+        _assert_close(_np(out[0, torch.as_tensor(sample, device=q.device), h]), ref, "bf16")
+    s_refs = J.sparse_rows_many(s_jobs)
+    for h, ref in zip(sparse_heads, s_refs):
+        _assert_close(_np(out[0, torch.as_tensor(s_rows[h], device=q.device), h]), ref, "bf16")
     # broadcast rows are bitwise copies of their anchor rows, for every repetitive head
     near = O.nearest_anchor_rows(wl.rows, wl.anchors)
     o = out.view(1, wl.frames, wl.rows, wl.cols, wl.heads, wl.head_dim)[..., list(rep_heads), :]
     for rho in range(wl.rows):
         assert torch.equal(o[:, :, rho], o[:, :, near[rho]])
-    # sparse heads: three sampled q-blocks each for four heads
-    sparse_heads = [h for h in range(wl.heads) if h not in rep_heads][:4]
-    for h in sparse_heads:
-        blocks = _sampled_blocks(rng, wl.num_blocks, 3)
-        rows = np.concatenate([np.arange(r * 128, min(wl.seq_len, (r + 1) * 128)) for r in blocks])
-        qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
-        ref, _ = O.block_sparse_attention(qh, kh, vh, masks[h], wl.block, rows=rows)
-        got = _np(out[0, torch.as_tensor(rows, device=q.device), h])
-        _assert_close(got, ref, "bf16")
 
 
 # --------------------------------------------------------- offline calibration
@@ -376,3 +389,52 @@ def test_fma_exp2_error_bound(C):
     C.calibatt_debug_exp2_fma(low, yl)
     _check_status(C)
     assert (yl >= 0).all() and (yl < 1e-37).all()
+
+
+def test_sweep_records_sampled(C):
+    """Records of the schedule sweep in one dictionary spanning all 50 x 40
+    (timestep, layer) slots: the dual-path call of (t, l) must use that
+    record's masks and anchor heads (checked against the oracle on sampled
+    rows), and retained-tile counts must match the recipe."""
+    wl = W.WORKLOADS["720p_sweep"]
+    nb = wl.num_blocks
+    records = [(0, 0), (25, 17), (49, 39)]
+    nnz = sum(W.sweep_record_blocks(wl, t, l, h) for t, l in records for h in range(wl.heads))
+    rng = np.random.default_rng(5)
+    with C.MaskDictionary(W.SWEEP_STEPS, W.SWEEP_LAYERS, wl.heads, nb, nb, wl.block, nnz) as dct:
+        host = {}
+        for t, l in records:
+            masks, rep = W.sweep_layer_masks(wl, t, l, "cuda")
+            rp, ci = W.layer_csr(masks)
+            rep_arr = np.zeros(wl.heads, np.uint8)
+            rep_arr[list(rep)] = 1
+            dct.set_layer(t, l, rp, ci, rep_arr)
+            host[(t, l)] = (masks.cpu().numpy(), rep)
+            li = dct.layer_info(t, l)
+            assert li["repetitive_heads"] == W.SWEEP_REPETITIVE
+            assert li["retained_tiles"] == sum(W.sweep_record_blocks(wl, t, l, h) for h in range(wl.heads))
+        for t, l in records:
+            masks, rep = host[(t, l)]
+            q, k, v = W.make_qkv(W.seed_for("sweep-qkv", t, l) % (1 << 62), 1, wl.seq_len, wl.heads,
+                                 wl.head_dim, "bf16", wl.input_std, "cuda")
+            out = torch.full_like(q, float("nan"))
+            C.calibatt_dual_path_attn(q, k, v, out, dct, t, l, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
+            _check_status(C)
+            assert not torch.isnan(out).any()
+            sparse_heads = [h for h in range(wl.heads) if h not in rep]
+            for h in rng.choice(sparse_heads, 2, replace=False):
+                blocks = _sampled_blocks(rng, nb, 3)
+                rows = np.concatenate([np.arange(r * 128, min(wl.seq_len, (r + 1) * 128)) for r in blocks])
+                qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
+                ref, _ = O.block_sparse_attention(qh, kh, vh, masks[h], wl.block, rows=rows)
+                _assert_close(_np(out[0, torch.as_tensor(rows, device=q.device), h]), ref, "bf16")
+            h = int(rng.choice(rep))
+            sample = np.sort(rng.choice(wl.seq_len, 300, replace=False))
+            qh, kh, vh = _np(q[0, :, h]), _np(k[0, :, h]), _np(v[0, :, h])
+            ref, _ = O.anchor_attention(qh, kh, vh, wl.frames, wl.rows, wl.cols, wl.anchors, rows=sample)
+            _assert_close(_np(out[0, torch.as_tensor(sample, device=q.device), h]), ref, "bf16")
+            near = O.nearest_anchor_rows(wl.rows, wl.anchors)
+            o = out.view(1, wl.frames, wl.rows, wl.cols, wl.heads, wl.head_dim)[..., list(rep), :]
+            for rho in range(wl.rows):
+                assert torch.equal(o[:, :, rho], o[:, :, near[rho]])
+            del q, k, v, out

@@ -54,3 +54,40 @@ def test_mask_to_csr_roundtrip():
 def test_sweep_density_ramp():
     assert abs(W.sweep_density(0, 50, 1) - 0.60) <= 0.03 + 1e-12
     assert abs(W.sweep_density(49, 50, 1) - 0.20) <= 0.03 + 1e-12
+
+
+def test_sweep_recipe_small():
+    """The schedule-sweep mask recipe on a small geometry: exact retained-block
+    counts from the recipe alone, diagonal and first-frame key blocks kept, an
+    empty mask for anchor-path heads, the density ramp, determinism, and the
+    per-head CSR layout."""
+    import dataclasses
+
+    wl = dataclasses.replace(W.WORKLOADS["720p_sweep"], frames=4, rows=8, cols=16, block=64, heads=12)
+    nb = wl.num_blocks
+    for t, l in [(0, 0), (30, 3), (49, 7)]:
+        masks, rep = W.sweep_layer_masks(wl, t, l)
+        assert rep == W.sweep_repetitive_heads(t, l, wl.heads) and len(rep) == W.SWEEP_REPETITIVE
+        m = masks.numpy()
+        first = np.arange(nb) * wl.block < wl.tokens_per_frame
+        for h in range(wl.heads):
+            assert m[h].sum() == W.sweep_record_blocks(wl, t, l, h)
+            if h in rep:
+                assert not m[h].any()
+            else:
+                assert m[h][np.arange(nb), np.arange(nb)].all()
+                assert m[h][:, first].all()
+        again, _ = W.sweep_layer_masks(wl, t, l)
+        assert np.array_equal(again.numpy(), m)
+        rp, ci = W.layer_csr(masks)
+        assert rp.shape == (wl.heads, nb + 1) and rp.dtype == np.int32 and (rp[:, 0] == 0).all()
+        off = 0
+        for h in range(wl.heads):
+            r, c = W.mask_to_csr(m[h])
+            assert np.array_equal(rp[h], r)
+            assert np.array_equal(ci[off:off + c.size], c)
+            off += c.size
+        assert off == ci.size
+    d0 = [W.sweep_record_density(0, 0, h) for h in range(20)]
+    d49 = [W.sweep_record_density(49, 0, h) for h in range(20)]
+    assert all(0.57 <= d <= 0.63 for d in d0) and all(0.17 <= d <= 0.23 for d in d49)

@@ -31,6 +31,12 @@ __all__ = [
     "sweep_density",
     "seed_for",
     "mask_to_csr",
+    "SWEEP_STEPS",
+    "SWEEP_LAYERS",
+    "sweep_record_density",
+    "sweep_repetitive_heads",
+    "sweep_layer_masks",
+    "layer_csr",
 ]
 
 
@@ -229,3 +235,106 @@ def ceil_div(a, b):
 def count_bytes(*arrays):
     return int(sum(a.numel() * a.element_size() for a in arrays))
 
+
+
+# ------------------------------------------------------------- schedule sweep
+# One 720p-shaped call per (timestep t, layer l) of a 50-step, 40-layer
+# schedule; per-(t, l, h) seeded masks whose density ramps from 60 % at the
+# first timestep to 20 % at the last, and 10 of the 40 heads of every call on
+# the anchor path.
+
+SWEEP_STEPS = 50
+SWEEP_LAYERS = 40
+SWEEP_REPETITIVE = 10
+
+
+def sweep_record_density(t, l, h, steps=SWEEP_STEPS):
+    """Target block density of record (t, l, h) of the sweep."""
+    return sweep_density(t, steps, seed_for("sweep-density", t, l, h) % (1 << 32))
+
+
+def sweep_repetitive_heads(t, l, heads=40, n=SWEEP_REPETITIVE):
+    """Heads of call (t, l) on the anchor path."""
+    return repetitive_heads(seed_for("sweep-repetitive", t, l) % (1 << 32), heads, n)
+
+
+def _band_counts(num_blocks, block, tokens_per_frame):
+    """Blocks kept by band_mask for every half-width w = 0 .. last frame."""
+    frames = ((num_blocks - 1) * block) // tokens_per_frame + 1
+    return [int(band_mask(num_blocks, block, tokens_per_frame, w).sum()) for w in range(frames + 1)]
+
+
+_BAND_COUNTS = {}
+
+
+def sweep_record_blocks(wl, t, l, h, steps=SWEEP_STEPS):
+    """Retained blocks of record (t, l, h) (0 for heads on the anchor path), from
+    the recipe alone: the band of the largest half-width within the target,
+    topped up with random blocks to round(density * nb^2)."""
+    if h in sweep_repetitive_heads(t, l, wl.heads):
+        return 0
+    key = (wl.num_blocks, wl.block, wl.tokens_per_frame)
+    if key not in _BAND_COUNTS:
+        _BAND_COUNTS[key] = _band_counts(*key)
+    counts = _BAND_COUNTS[key]
+    want = int(round(sweep_record_density(t, l, h, steps) * wl.num_blocks ** 2))
+    w = max([0] + [i for i, c in enumerate(counts) if c <= want])
+    return max(want, counts[w])
+
+
+def sweep_layer_masks(wl, t, l, device="cpu", steps=SWEEP_STEPS):
+    """Block masks of call (t, l) of the sweep: a bool tensor [H, nb, nb] on
+    `device` (all False for the heads on the anchor path) and the tuple of
+    anchor-path heads.
+
+    The structure follows synthetic_block_mask (band of the largest half-width
+    within the target, every first-frame key block, the diagonal), and the
+    random top-up is the round(density * nb^2) - |band| free blocks with the
+    smallest uniform keys drawn by torch's generator on `device` with seed
+    seed_for("sweep-fill", t, l, h): a uniform random subset, drawn fast enough
+    on the GPU for the 2,000 calls of the sweep.  The masks depend on the
+    device whose generator drew them."""
+    import torch
+
+    nb = wl.num_blocks
+    rep = sweep_repetitive_heads(t, l, wl.heads)
+    key = (nb, wl.block, wl.tokens_per_frame)
+    if key not in _BAND_COUNTS:
+        _BAND_COUNTS[key] = _band_counts(*key)
+    counts = _BAND_COUNTS[key]
+    idx = torch.arange(nb, device=device)
+    frame = (idx * wl.block) // wl.tokens_per_frame
+    first = (idx * wl.block < wl.tokens_per_frame)[None, :]
+    eye = torch.eye(nb, dtype=torch.bool, device=device)
+    masks = torch.zeros((wl.heads, nb, nb), dtype=torch.bool, device=device)
+    for h in range(wl.heads):
+        if h in rep:
+            continue
+        want = int(round(sweep_record_density(t, l, h, steps) * nb * nb))
+        w = max([0] + [i for i, c in enumerate(counts) if c <= want])
+        band = ((frame[:, None] - frame[None, :]).abs() <= w) | first | eye
+        extra = want - counts[w]
+        if extra > 0:
+            g = torch.Generator(device=device)
+            g.manual_seed(seed_for("sweep-fill", t, l, h))
+            keys = torch.rand(nb * nb, generator=g, device=device)
+            keys[band.view(-1)] = 2.0
+            pick = torch.argsort(keys)[:extra]
+            flat = band.view(-1).clone()
+            flat[pick] = True
+            band = flat.view(nb, nb)
+        masks[h] = band
+    return masks, rep
+
+
+def layer_csr(masks):
+    """Per-head CSR of a [H, nb, nb] bool tensor, on the host: row_ptr int32
+    [H, nb + 1] (each head's starting at 0) and the heads' column lists
+    concatenated in head order (int32)."""
+    import torch
+
+    counts = masks.sum(dim=2, dtype=torch.int32)
+    row_ptr = torch.zeros((masks.shape[0], masks.shape[1] + 1), dtype=torch.int32, device=masks.device)
+    row_ptr[:, 1:] = torch.cumsum(counts, dim=1, dtype=torch.int32)
+    col_idx = torch.nonzero(masks)[:, 2].to(torch.int32)
+    return row_ptr.cpu().numpy(), col_idx.cpu().numpy()
