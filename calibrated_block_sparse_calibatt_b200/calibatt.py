@@ -60,6 +60,7 @@ SIGNATURES = {
     "calibatt_lpt_schedule": (_i32, [_i32, _vp, _i32, _vp, _vp, _P(_i64)]),
     "calibatt_dict_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P(_vp)]),
     "calibatt_dict_set_layer": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
+    "calibatt_dict_set_anchor_geometry": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32]),
     "calibatt_dict_info": (_i32, [_vp, _P(_i64), _P(_i64), _P(_i32)]),
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
@@ -212,6 +213,12 @@ class MaskDictionary:
         rep = None if repetitive is None else np.ascontiguousarray(np.asarray(repetitive, dtype=np.uint8))
         check(LIB.calibatt_dict_set_layer(self.handle, t, l, _ptr(rp), _ptr(ci) if ci.size else None,
                                           _ptr(rep) if rep is not None else None))
+
+    def set_anchor_geometry(self, frames, rows, cols, anchor_rows):
+        """Anchor geometry of the dual path; set before the first layer so
+        that calibatt_dual_path_attn runs each layer in one launch."""
+        a = _i32_array(anchor_rows).reshape(-1)
+        check(LIB.calibatt_dict_set_anchor_geometry(self.handle, frames, rows, cols, _ptr(a), a.size))
 
     def info(self):
         b, n, g = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int32(0)

@@ -307,8 +307,24 @@ struct calibatt_dict {
   std::vector<int32_t> n_sparse;    // [T*L]
   std::vector<int32_t> n_rep;       // [T*L]
   std::vector<int64_t> retained;    // [T*L]
+  // Anchor geometry of the dual path (calibatt_dict_set_anchor_geometry) and
+  // the joint sparse + anchor schedules built with it, one per layer.
+  bool has_geom = false;
+  int32_t g_frames = 0, g_rows = 0, g_cols = 0, g_tiles = 0;
+  std::vector<int32_t> g_anchors;
+  int64_t f_stride = 0;              // item slots per layer
+  uint32_t* d_fitems = nullptr;
+  int32_t* d_fcta_ptr = nullptr;
 
   int64_t layer(int t, int l) const { return static_cast<int64_t>(t) * L + l; }
+
+  LayerSchedule fused_schedule(int t, int l) const {
+    LayerSchedule s = schedule(t, l);
+    const int64_t ly = layer(t, l);
+    s.items = d_fitems + ly * f_stride;
+    s.cta_ptr = d_fcta_ptr + ly * (G + 1);
+    return s;
+  }
 
   LayerSchedule schedule(int t, int l) const {
     const int64_t ly = layer(t, l);
@@ -328,6 +344,10 @@ struct calibatt_dict {
     cudaFree(d_col);
     cudaFree(d_items);
     cudaFree(d_cta_ptr);
+    cudaFree(d_fitems);
+    cudaFree(d_fcta_ptr);
+    d_fitems = nullptr;
+    d_fcta_ptr = nullptr;
     d_row_ptr = nullptr;
     d_col_base = nullptr;
     d_col = nullptr;
@@ -374,7 +394,7 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
     p.sched = sch;
     p.status = status_word_ptr();
     p.timeout_ns = g_timeout_ns.load();
-    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, false, d->G, stream);
+    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeSparse, d->G, stream);
     if (e != cudaSuccess) return cuda_fail(e, "block-sparse tensor-core launch");
     return CALIBATT_OK;
   }
@@ -471,7 +491,7 @@ calibatt_status launch_anchor(const void* q, const void* k, const void* v, void*
     if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
     const int64_t items = static_cast<int64_t>(n_heads) * g.tiles_per_head;
     const int grid = static_cast<int>(std::min<int64_t>(sms, items));
-    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, true, grid, stream);
+    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeAnchor, grid, stream);
     if (e != cudaSuccess) return cuda_fail(e, "anchor tensor-core launch");
     return CALIBATT_OK;
   }
@@ -494,6 +514,46 @@ calibatt_status launch_anchor(const void* q, const void* k, const void* v, void*
   const int64_t n_items = static_cast<int64_t>(s.batch) * n_heads * g.tiles_per_head;
   cudaError_t e = calibatt::launch_simt_attn(p, s.head_dim, block, s.dtype, true, static_cast<int>(n_items), stream);
   if (e != cudaSuccess) return cuda_fail(e, "anchor CUDA-core launch");
+  return CALIBATT_OK;
+}
+
+// One persistent launch over the joint sparse + anchor schedule of a layer
+// (the dictionary's anchor geometry matches the call's).
+calibatt_status launch_fused(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
+                             const calibatt_dict* d, int32_t t, int32_t l, float softmax_scale, float* lse,
+                             cudaStream_t stream) {
+  AnchorGeom g;
+  std::memset(&g, 0, sizeof(g));
+  g.frames = d->g_frames;
+  g.rows = d->g_rows;
+  g.cols = d->g_cols;
+  g.n_anchors = static_cast<int32_t>(d->g_anchors.size());
+  g.anchor_tokens = g.frames * g.n_anchors * g.cols;
+  g.tiles_per_head = d->g_tiles;
+  anchor_groups(g.rows, d->g_anchors.data(), g.n_anchors, g);
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  calibatt_status st;
+  if ((st = encode_qkv_map(&p.tm_q, q, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+  if ((st = encode_qkv_map(&p.tm_k, k, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+  if ((st = encode_qkv_map(&p.tm_v, v, s, &p.pos_n, &p.pos_h, &p.pos_b)) != CALIBATT_OK) return st;
+  p.q = static_cast<const uint16_t*>(q);
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.sb = s.stride_b;
+  p.sn = s.stride_n;
+  p.sh = s.stride_h;
+  p.batch = s.batch;
+  p.seq_len = s.seq_len;
+  p.heads = s.heads;
+  p.nb = ceil_div(s.seq_len, 128);
+  p.scale_log2 = scale_log2_of(softmax_scale, s.head_dim);
+  p.sched = d->fused_schedule(t, l);
+  p.anc = g;
+  p.status = status_word_ptr();
+  p.timeout_ns = g_timeout_ns.load();
+  cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeFused, d->G, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dual-path tensor-core launch");
   return CALIBATT_OK;
 }
 
@@ -664,6 +724,48 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
   lpt_grouped(static_cast<int32_t>(items.size()), cost.data(), group.data(), d->G, cta_ptr.data(), order.data());
   std::vector<uint32_t> sched(items.size());
   for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
+  // Joint schedule of the dual path.  All anchor tiles of the repetitive
+  // heads come first, as one group in head order (a tile visits all nq key
+  // blocks; its epilogue writes about rows / n_anchors output rows per query,
+  // counted as that many extra blocks): the equal-cost tiles go round-robin
+  // over the CTAs, so the grid works on two or three heads at a time.  The
+  // sparse items follow in the L2 groups of the sparse-only schedule, with the
+  // running balance starting from the anchor loads.  (Interleaving both kinds
+  // in head-order groups let CTAs drift several groups apart behind the large
+  // anchor tiles, and the keys and values of the heads in flight no longer
+  // fitted in L2.)
+  std::vector<uint32_t> fsched;
+  std::vector<int32_t> fcta_ptr;
+  if (d->has_geom) {
+    std::vector<uint32_t> fitems;
+    std::vector<int64_t> fcost;
+    std::vector<int32_t> fgroup;
+    const int64_t bcast = std::max<int64_t>(1, d->g_rows / static_cast<int64_t>(d->g_anchors.size()));
+    int32_t sparse_rank = 0;
+    for (int h = 0; h < H; ++h) {
+      if (repetitive && repetitive[h]) {
+        for (int tile = 0; tile < d->g_tiles; ++tile) {
+          fitems.push_back(calibatt::kItemAnchorBit | (static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(tile));
+          fcost.push_back(static_cast<int64_t>(nq) + 2 + bcast);
+          fgroup.push_back(0);
+        }
+      } else {
+        const int32_t g = 1 + sparse_rank++ / hpg;
+        const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+        for (int r = 0; r < nq; ++r) {
+          fitems.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
+          fcost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
+          fgroup.push_back(g);
+        }
+      }
+    }
+    fcta_ptr.assign(d->G + 1, 0);
+    std::vector<int32_t> forder(fitems.size());
+    lpt_grouped(static_cast<int32_t>(fitems.size()), fcost.data(), fgroup.data(), d->G, fcta_ptr.data(),
+                forder.data());
+    fsched.resize(fitems.size());
+    for (size_t i = 0; i < fitems.size(); ++i) fsched[i] = fitems[forder[i]];
+  }
   int prev = 0;
   cudaGetDevice(&prev);
   if (prev != d->device) cudaSetDevice(d->device);
@@ -677,6 +779,12 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(d->d_cta_ptr + ly * (d->G + 1), cta_ptr.data(), sizeof(int32_t) * (d->G + 1), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && d->has_geom && !fsched.empty())
+    e = cudaMemcpy(d->d_fitems + ly * d->f_stride, fsched.data(), sizeof(uint32_t) * fsched.size(),
+                   cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && d->has_geom)
+    e = cudaMemcpy(d->d_fcta_ptr + ly * (d->G + 1), fcta_ptr.data(), sizeof(int32_t) * (d->G + 1),
+                   cudaMemcpyHostToDevice);
   if (prev != d->device) cudaSetDevice(prev);
   if (e != cudaSuccess) return cuda_fail(e, "dictionary upload");
   d->nnz_used += nnz;
@@ -685,6 +793,54 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
   d->n_rep[ly] = n_rep;
   d->retained[ly] = retained;
   d->layer_set[ly] = 1;
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* d, int32_t frames, int32_t rows, int32_t cols,
+                                                  const int32_t* anchor_rows, int32_t n_anchors) {
+  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+  if (d->has_geom) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry is already set");
+  for (uint8_t set : d->layer_set)
+    if (set) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry must be set before the first layer");
+  if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
+  const int64_t tokens = static_cast<int64_t>(frames) * rows * cols;
+  if (ceil_div(tokens, d->block) != d->nq)
+    return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld tokens do not make the dictionary's %d blocks",
+                (long long)tokens, d->nq);
+  if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
+  for (int a = 0; a < n_anchors; ++a) {
+    if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
+    if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
+  }
+  if (d->H > 32767) return fail(CALIBATT_ERR_UNSUPPORTED, "joint schedules need H <= 32767");
+  const int64_t tiles = ceil_div(static_cast<int64_t>(frames) * n_anchors * cols, 128);
+  if (tiles > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 anchor tiles per head");
+  const int64_t layers = static_cast<int64_t>(d->T) * d->L;
+  const int64_t stride = static_cast<int64_t>(d->H) * std::max<int64_t>(d->nq, tiles);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != d->device) cudaSetDevice(d->device);
+  cudaError_t e = cudaMalloc(&d->d_fitems, sizeof(uint32_t) * layers * stride);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_fcta_ptr, sizeof(int32_t) * layers * (d->G + 1));
+  if (prev != d->device) cudaSetDevice(prev);
+  if (e != cudaSuccess) {
+    cudaFree(d->d_fitems);
+    cudaFree(d->d_fcta_ptr);
+    d->d_fitems = nullptr;
+    d->d_fcta_ptr = nullptr;
+    return cuda_fail(e, "joint schedule allocation");
+  }
+  d->device_bytes += static_cast<int64_t>(sizeof(uint32_t) * layers * stride + sizeof(int32_t) * layers * (d->G + 1));
+  d->f_stride = stride;
+  d->g_frames = frames;
+  d->g_rows = rows;
+  d->g_cols = cols;
+  d->g_tiles = static_cast<int32_t>(tiles);
+  d->g_anchors.assign(anchor_rows, anchor_rows + n_anchors);
+  d->has_geom = true;
   return CALIBATT_OK;
 }
 
@@ -755,6 +911,30 @@ calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void
                                         int32_t t, int32_t l, int32_t frames, int32_t rows, int32_t cols,
                                         const int32_t* anchor_rows, int32_t n_anchors, float softmax_scale,
                                         float* lse, void* stream) {
+  // One launch when the dictionary carries this call's anchor geometry and
+  // the tensor-core path applies; otherwise the sparse and anchor launches.
+  if (dict && shape && dict->has_geom && shape->dtype == CALIBATT_DTYPE_BF16 && block == 128 &&
+      frames == dict->g_frames && rows == dict->g_rows && cols == dict->g_cols && anchor_rows &&
+      n_anchors == static_cast<int32_t>(dict->g_anchors.size()) &&
+      std::equal(dict->g_anchors.begin(), dict->g_anchors.end(), anchor_rows)) {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+    if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
+    if (dict->H != shape->heads)
+      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
+    if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
+    if (dict->nq != ceil_div(shape->seq_len, block))
+      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq,
+                  shape->seq_len, ceil_div(shape->seq_len, block));
+    if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
+      return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
+                  shape->seq_len);
+    if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    const int64_t ly = dict->layer(t, l);
+    if (dict->n_sparse[ly] + dict->n_rep[ly] == 0) return CALIBATT_OK;
+    return launch_fused(q, k, v, o, *shape, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
+  }
   calibatt_status st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
   if (st != CALIBATT_OK) return st;
   const int64_t ly = dict->layer(t, l);

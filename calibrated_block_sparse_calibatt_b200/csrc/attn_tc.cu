@@ -57,8 +57,17 @@ using namespace ptx;
 constexpr unsigned kTraceIters = 4096;
 constexpr unsigned kTraceEvents = 64;
 __device__ unsigned long long g_trace[kTraceEvents * kTraceIters];
+// Start and end (globaltimer, ns) of every CTA.
+__device__ unsigned long long g_cta_span[2 * 1024];
+#ifndef CALIBATT_TRACE_OFFSET
+#define CALIBATT_TRACE_OFFSET 0
+#endif
+#ifndef CALIBATT_TRACE_CTA
+#define CALIBATT_TRACE_CTA 0
+#endif
 __device__ __forceinline__ void trace_event(int ev, uint32_t idx) {
-  if (blockIdx.x == 0 && idx < kTraceIters) g_trace[ev * kTraceIters + idx] = clock64();
+  idx -= CALIBATT_TRACE_OFFSET;
+  if (blockIdx.x == CALIBATT_TRACE_CTA && idx < kTraceIters) g_trace[ev * kTraceIters + idx] = clock64();
 }
 #define CALIBATT_TRACE_EVENT(cond, ev, idx) \
   do {                                     \
@@ -152,15 +161,17 @@ struct Item {
   int n;                     // key blocks to visit
   const uint16_t* cols;      // retained key blocks (sparse), nullptr = 0..n-1
   bool ragged_last;          // last visited key block is the partial one
+  bool anchor;               // anchor-row tile (gathered queries, broadcast epilogue)
 };
 
+
 // Walks this CTA's work items in the same order in every role.
-template <bool ANCHOR>
+template <int MODE>
 struct Cursor {
   int b, idx, begin, end, step;
   __device__ void init(const TcParams& p) {
     b = 0;
-    if (ANCHOR) {
+    if (MODE == kModeAnchor) {
       begin = blockIdx.x;
       end = p.anc.n_heads * p.anc.tiles_per_head;
       step = gridDim.x;
@@ -175,15 +186,23 @@ struct Cursor {
     while (b < p.batch) {
       if (idx < end) {
         it.b = b;
-        if (ANCHOR) {
-          it.h = p.anc.head_ids[idx / p.anc.tiles_per_head];
-          it.tile = idx % p.anc.tiles_per_head;
+        uint32_t w = 0;
+        if (MODE != kModeAnchor) w = p.sched.items[idx];
+        if (MODE == kModeAnchor || (MODE == kModeFused && (w & kItemAnchorBit))) {
+          it.anchor = true;
+          if (MODE == kModeAnchor) {
+            it.h = p.anc.head_ids[idx / p.anc.tiles_per_head];
+            it.tile = idx % p.anc.tiles_per_head;
+          } else {
+            it.h = static_cast<int>((w >> 16) & 0x7FFFu);
+            it.tile = static_cast<int>(w & 0xFFFFu);
+          }
           it.n = p.nb;
           it.cols = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
         } else {
-          const uint32_t w = p.sched.items[idx];
-          it.h = static_cast<int>(w >> 16);
+          it.anchor = false;
+          it.h = static_cast<int>(MODE == kModeFused ? (w >> 16) & 0x7FFFu : w >> 16);
           it.tile = static_cast<int>(w & 0xFFFFu);
           const int32_t* rp = p.sched.row_ptr + static_cast<int64_t>(it.h) * (p.sched.nq + 1);
           const int s0 = rp[it.tile];
@@ -229,7 +248,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // --------------------------------------------------------------- producers
 // Q/K producer (V == false) and V producer (V == true) walk the same items and
 // key blocks; each lets its own in-flight bulk copies land before exiting.
-template <int HD, bool ANCHOR, bool V>
+template <int HD, int MODE, bool V>
 __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
@@ -238,35 +257,50 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
   constexpr int kEmpty = V ? L::bVEmpty : L::bKEmpty;
   constexpr int kRing = V ? L::kV : L::kK;
   const CUtensorMap* map = V ? &p.tm_v : &p.tm_k;
-  Cursor<ANCHOR> cur;
+  Cursor<MODE> cur;
   cur.init(p);
   Item it;
-  uint32_t kv = 0, item = 0, issued = 0, q_issued = 0;
+  uint32_t kv = 0, item = 0, issued = 0, q_items = 0;
   bool ok = true;
   while (ok && cur.next(p, it)) {
     if (!V) {
       if (item > 0 && !W.wait(bar(L::bQEmpty), (item - 1) & 1, 1)) break;
-      if (ANCHOR) {
+      CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 9, item + CALIBATT_TRACE_OFFSET);
+      if (it.anchor) {
         // Gather this tile's 128 anchor-row queries into the 128-byte swizzled
         // K-major layout the MMA expects (16-byte unit u of row r lands at
         // chunk u/8, row r, position (u%8) ^ (r%8)).
         constexpr int kUnits = HD / 8;
         const int per_frame = p.anc.n_anchors * p.anc.cols;
         const uint16_t* qb = p.q + static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
-        for (int idx = lane; idx < 128 * kUnits; idx += 32) {
-          const int r = idx / kUnits, u = idx % kUnits;
-          const int pq = it.tile * 128 + r;
-          uint4 val = make_uint4(0u, 0u, 0u, 0u);
-          if (pq < p.anc.anchor_tokens) {
-            const int f = pq / per_frame, rem = pq % per_frame;
-            const int a = rem / p.anc.cols, w = rem % p.anc.cols;
-            const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + p.anc.anchor_row[a]) * p.anc.cols + w;
-            val = __ldg(reinterpret_cast<const uint4*>(qb + token * p.sn + u * 8));
+        // Two 16-byte loads in flight per lane before their stores (the
+        // producer warpgroup has 40 registers per thread).
+        constexpr int kBatch = 2;
+        static_assert((128 * kUnits) % (32 * kBatch) == 0, "gather batches");
+        for (int i0 = lane; i0 < 128 * kUnits; i0 += 32 * kBatch) {
+          uint4 val[kBatch];
+#pragma unroll
+          for (int e = 0; e < kBatch; ++e) {
+            const int idx = i0 + 32 * e;
+            const int r = idx / kUnits, u = idx % kUnits;
+            const int pq = it.tile * 128 + r;
+            val[e] = make_uint4(0u, 0u, 0u, 0u);
+            if (pq < p.anc.anchor_tokens) {
+              const int f = pq / per_frame, rem = pq % per_frame;
+              const int a = rem / p.anc.cols, w = rem % p.anc.cols;
+              const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + p.anc.anchor_row[a]) * p.anc.cols + w;
+              val[e] = __ldg(reinterpret_cast<const uint4*>(qb + token * p.sn + u * 8));
+            }
           }
-          const uint32_t dst = base + L::kQ + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val.x), "r"(val.y),
-                       "r"(val.z), "r"(val.w)
-                       : "memory");
+#pragma unroll
+          for (int e = 0; e < kBatch; ++e) {
+            const int idx = i0 + 32 * e;
+            const int r = idx / kUnits, u = idx % kUnits;
+            const uint32_t dst = base + L::kQ + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val[e].x), "r"(val[e].y),
+                         "r"(val[e].z), "r"(val[e].w)
+                         : "memory");
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -276,14 +310,14 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
           mbar_arrive_expect_tx(bar(L::bQFull), L::kTile);
           tma_tile<HD>(base + L::kQ, &p.tm_q, bar(L::bQFull), p, it.tile * 128, it.h, it.b);
         }
-        ++q_issued;
       }
+      ++q_items;  // every item completes one phase of q_full, whichever way its Q came
     }
     uint32_t my_col = 0;
     for (int j = 0; j < it.n; ++j) {
       if ((j & 31) == 0) {
         const int jj = j + lane;
-        my_col = ANCHOR ? static_cast<uint32_t>(jj) : (jj < it.n ? it.cols[jj] : 0u);
+        my_col = it.anchor ? static_cast<uint32_t>(jj) : (jj < it.n ? it.cols[jj] : 0u);
       }
       const int c = static_cast<int>(__shfl_sync(0xFFFFFFFFu, my_col, j & 31));
       const uint32_t slot = kv % kStages, use = kv / kStages;
@@ -301,7 +335,9 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
   // Let every bulk copy this warp issued land before the CTA can exit.
   for (uint32_t s = 0; s < static_cast<uint32_t>(kStages); ++s)
     if (issued > s) drain_wait(bar(kFull + s), ((issued - 1 - s) / kStages) & 1);
-  if (q_issued > 0) drain_wait(bar(L::bQFull), (q_issued - 1) & 1);
+  // Only the last item's Q copy can still be in flight (each earlier one was
+  // consumed before the next Q load): wait for that phase of q_full.
+  if (q_items > 0) drain_wait(bar(L::bQFull), (q_items - 1) & 1);
 }
 
 
@@ -313,12 +349,12 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
 // Block j belongs to stream j mod 2 of its item; t is its ordinal within
 // that stream over the whole launch, and the barriers of stream s count
 // those ordinals.
-template <int HD, bool ANCHOR>
+template <int HD, int MODE>
 __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0);
-  Cursor<ANCHOR> cur;
+  Cursor<MODE> cur;
   cur.init(p);
   Item it;
   uint32_t g = 0, item = 0;      // global key-block iteration, item counter
@@ -327,6 +363,7 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
   while (ok && cur.next(p, it)) {
     if (!W.wait(bar(L::bQFull), item & 1, 4)) break;
     tc_fence_after();
+    CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 8, item + CALIBATT_TRACE_OFFSET);
     for (int j = 0; j < it.n; ++j, ++g) {
       const int s = j & 1;
       const uint32_t t = s ? t1++ : t0++;
@@ -365,12 +402,12 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
   drain_wait(bar(L::bDrain), 0);
 }
 
-template <int HD, bool ANCHOR>
+template <int HD, int MODE>
 __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, const Waiter& W, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, 1);
-  Cursor<ANCHOR> cur;
+  Cursor<MODE> cur;
   cur.init(p);
   Item it;
   uint32_t g = 0, item = 0;
@@ -418,7 +455,7 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
 // through shared memory at a pair barrier (warps w and w+4, bar.red.or, which
 // also carries "a wait failed" so both warps leave together), then group s
 // writes output columns [s*D/2, (s+1)*D/2) of O / l.
-template <int HD, bool ANCHOR>
+template <int HD, int MODE>
 __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
                              const Waiter& W, int warp, int lane) {
   using L = Layout<HD>;
@@ -438,7 +475,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   const uint32_t tO = tmem + lane_off + kColO;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
-  Cursor<ANCHOR> cur;
+  Cursor<MODE> cur;
   cur.init(p);
   Item it;
   uint32_t kv = 0, item = 0;
@@ -569,7 +606,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
     ok = ok && W.wait(bar(L::bOFull), item & 1, 12);
     if (ok) tc_fence_after();
     kv += it.n;
-    CALIBATT_TRACE_EVENT(lane == 0 && warp == 0, 10, kv);
+    CALIBATT_TRACE_EVENT(lane == 0 && warp == 0, 10, item + CALIBATT_TRACE_OFFSET);
     // Exchange buffer alternates by item so the partner's read of the
     // previous item's values can never meet this item's writes.
     float* xb = xchg + (item & 1) * 512;
@@ -587,7 +624,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
     // Destination rows of this thread's output.
     int64_t dst_token = -1;
     int n_dst = 0, anchor_f = 0, anchor_w = 0, lo = 0;
-    if (ANCHOR) {
+    if (it.anchor) {
       const int pq = it.tile * 128 + row;
       if (pq < p.anc.anchor_tokens) {
         const int per_frame = p.anc.n_anchors * p.anc.cols;
@@ -628,7 +665,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       }
 #pragma unroll 1
       for (int d = 0; d < n_dst; ++d) {
-        const int64_t token = ANCHOR
+        const int64_t token = it.anchor
             ? (static_cast<int64_t>(anchor_f) * p.anc.rows + lo + d) * p.anc.cols + anchor_w
             : dst_token;
         uint4* dst = reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + col);
@@ -636,18 +673,18 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         for (int g = 0; g < 4; ++g) dst[g] = pkd[g];
       }
     }
-    if (!ANCHOR && s == 0 && p.lse != nullptr && dst_token >= 0) {
+    if (!it.anchor && s == 0 && p.lse != nullptr && dst_token >= 0) {
       p.lse[(static_cast<int64_t>(it.b) * p.heads + it.h) * p.seq_len + dst_token] =
           it.n > 0 ? (m + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     mbar_arrive(bar(L::bOFree));
-    CALIBATT_TRACE_EVENT(lane == 0 && warp == 0, 11, kv);
+    CALIBATT_TRACE_EVENT(lane == 0 && warp == 0, 11, item + CALIBATT_TRACE_OFFSET);
     ++item;
   }
 }
 
-template <int HD, bool ANCHOR>
+template <int HD, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<HD>;
   extern __shared__ uint8_t smem_raw[];
@@ -658,6 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+#ifdef CALIBATT_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x] = globaltimer();
+#endif
   if (threadIdx.x == 0) {
     auto bar = [&](int i) { return base + L::kBar + 8u * i; };
     mbar_init(bar(L::bQFull), 1);
@@ -683,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0 && !ANCHOR) {
+  if (warp == kProducerWarp && lane == 0 && MODE != kModeAnchor) {
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
   }
@@ -703,13 +743,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   if (warp >= 8) {
     reg_dealloc<kOtherRegs>();
     if (warp == kProducerWarp) {
-      producer_role<HD, ANCHOR, false>(p, base, W, lane);
+      producer_role<HD, MODE, false>(p, base, W, lane);
     } else if (warp == kVProducerWarp) {
-      producer_role<HD, ANCHOR, true>(p, base, W, lane);
+      producer_role<HD, MODE, true>(p, base, W, lane);
     } else if (warp == kMmaWarp) {
-      mma_s_role<HD, ANCHOR>(p, base, tmem, W, lane);
+      mma_s_role<HD, MODE>(p, base, tmem, W, lane);
     } else if (warp == kPvWarp) {
-      mma_pv_role<HD, ANCHOR>(p, base, tmem, W, lane);
+      mma_pv_role<HD, MODE>(p, base, tmem, W, lane);
     }
     tc_fence_before();
     cta_bar_sync(kEndBarrier, kThreads);
@@ -717,17 +757,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
       tc_fence_after();
       tmem_dealloc(tmem, kTmemCols);
     }
+#ifdef CALIBATT_TRACE
+    if (warp == kMmaWarp && lane == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x + 1] = globaltimer();
+#endif
   } else {
     reg_alloc<kSoftmaxRegs>();
-    softmax_role<HD, ANCHOR>(p, base, gbase, tmem, W, warp, lane);
+    softmax_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
     tc_fence_before();
     cta_bar_sync(kEndBarrier, kThreads);
   }
 }
 
-template <int HD, bool ANCHOR>
+template <int HD, int MODE>
 cudaError_t launch_one(const TcParams& p, int grid, cudaStream_t s) {
-  auto kern = tc_attn_kernel<HD, ANCHOR>;
+  auto kern = tc_attn_kernel<HD, MODE>;
   const int bytes = Layout<HD>::kBytes;
   // The register split above assumes the CTA is launched with kLaunchRegs per
   // thread; with fewer, setmaxnreg.inc could never be satisfied.
@@ -765,6 +808,11 @@ extern "C" int calibatt_trace_read(unsigned long long* host, int max_records) {
   cudaMemcpyFromSymbol(host, g_trace, sizeof(unsigned long long) * (n < max_records ? n : max_records));
   return n;
 }
+extern "C" int calibatt_cta_span_read(unsigned long long* host, int max_records) {
+  const int n = 2 * 1024;
+  cudaMemcpyFromSymbol(host, g_cta_span, sizeof(unsigned long long) * (n < max_records ? n : max_records));
+  return n;
+}
 extern "C" void calibatt_trace_reset() {
   cudaMemset(nullptr, 0, 0);
   static unsigned long long zeros[kTraceEvents * kTraceIters];
@@ -783,9 +831,17 @@ size_t tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? Layout<64>::kBytes : Layout<128>::kBytes;
 }
 
-cudaError_t launch_tc_attn(const TcParams& p, int head_dim, bool anchor, int grid, cudaStream_t s) {
-  if (head_dim == 128) return anchor ? launch_one<128, true>(p, grid, s) : launch_one<128, false>(p, grid, s);
-  if (head_dim == 64) return anchor ? launch_one<64, true>(p, grid, s) : launch_one<64, false>(p, grid, s);
+cudaError_t launch_tc_attn(const TcParams& p, int head_dim, int mode, int grid, cudaStream_t s) {
+  if (head_dim == 128) {
+    if (mode == kModeSparse) return launch_one<128, kModeSparse>(p, grid, s);
+    if (mode == kModeAnchor) return launch_one<128, kModeAnchor>(p, grid, s);
+    if (mode == kModeFused) return launch_one<128, kModeFused>(p, grid, s);
+  }
+  if (head_dim == 64) {
+    if (mode == kModeSparse) return launch_one<64, kModeSparse>(p, grid, s);
+    if (mode == kModeAnchor) return launch_one<64, kModeAnchor>(p, grid, s);
+    if (mode == kModeFused) return launch_one<64, kModeFused>(p, grid, s);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -81,7 +81,17 @@ struct EnergyParams {
   float scale_log2;
 };
 
-cudaError_t launch_tc_attn(const TcParams& p, int head_dim, bool anchor, int grid, cudaStream_t s);
+// Tensor-core kernel modes: block-sparse items only, anchor tiles only, or
+// both kinds in one persistent launch under a joint schedule (dual path).
+constexpr int kModeSparse = 0;
+constexpr int kModeAnchor = 1;
+constexpr int kModeFused = 2;
+// Work-item word of the dictionary schedules: bit 31 marks an anchor tile
+// (fused schedules only), bits 16-30 the head, bits 0-15 the query block or
+// anchor tile.
+constexpr uint32_t kItemAnchorBit = 0x80000000u;
+
+cudaError_t launch_tc_attn(const TcParams& p, int head_dim, int mode, int grid, cudaStream_t s);
 cudaError_t launch_simt_attn(const SimtParams& p, int head_dim, int block, int dtype, bool anchor,
                              int n_items, cudaStream_t s);
 cudaError_t launch_block_energy(const EnergyParams& p, int head_dim, int block, int dtype,

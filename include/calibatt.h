@@ -151,6 +151,23 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* dict, int32_t t, int32_t 
                                         const int32_t* row_ptr, const int32_t* col_idx,
                                         const uint8_t* repetitive);
 
+/* Records the anchor geometry of the dual path (Key Designs 3: anchor rows
+ * of each frame, every other row served by its nearest anchor row, ties to
+ * the lower one) so that every layer set afterwards also gets a joint
+ * schedule of its block-sparse work items and the anchor-row tiles of its
+ * repetitive heads.  calibatt_dual_path_attn then runs a layer in ONE
+ * persistent launch when its call passes the same frames, rows, cols and
+ * anchor rows, a bf16 shape and block 128 (otherwise two launches, as
+ * without a geometry).  Host inputs: anchor_rows int32[n_anchors], strictly
+ * ascending in [0, rows), 1 <= n_anchors <= 16; frames*rows*cols tokens must
+ * make the dictionary's nq blocks.  Must be called at most once, before the
+ * first calibatt_dict_set_layer; allocates the joint schedules on the device
+ * (CALIBATT_ERR_CUDA if that fails).  CALIBATT_ERR_UNSUPPORTED for H > 32767
+ * or more than 65535 anchor tiles per head. */
+calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* dict, int32_t frames, int32_t rows,
+                                                  int32_t cols, const int32_t* anchor_rows,
+                                                  int32_t n_anchors);
+
 /* Totals: device bytes held, retained blocks stored, persistent grid size. */
 calibatt_status calibatt_dict_info(const calibatt_dict* dict, int64_t* device_bytes,
                                    int64_t* nnz_total, int32_t* num_ctas);
@@ -204,7 +221,10 @@ calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v
  * anchor path and the rest through the block-sparse path, enqueued on one
  * stream (Key Designs 4: the repetition flag selects one path per head; the
  * paths are alternatives, never stacked).  Arguments as above; lse
- * (nullable) is written for the sparse heads only. */
+ * (nullable) is written for the sparse heads only.  With a matching
+ * calibatt_dict_set_anchor_geometry (bf16, block 128) both kinds of work run
+ * in one persistent launch under the layer's joint schedule; otherwise as
+ * calibatt_block_sparse_attn followed by calibatt_anchor_attn. */
 calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void* v, void* o,
                                         const calibatt_shape* shape, int32_t block,
                                         const calibatt_dict* dict, int32_t t, int32_t l,

@@ -438,3 +438,78 @@ def test_sweep_records_sampled(C):
             for rho in range(wl.rows):
                 assert torch.equal(o[:, :, rho], o[:, :, near[rho]])
             del q, k, v, out
+
+
+# ------------------------------------------------------- fused dual path (one launch)
+
+@pytest.mark.parametrize("d,frames,rows,cols,anchors", [
+    (128, 2, 8, 64, (0, 4)),          # N = 1024: 8 full blocks, 2 anchor tiles per head
+    (128, 3, 9, 40, (1, 4, 7)),       # N = 1080: ragged last block (56 tokens), ragged anchor tile
+    (64, 3, 9, 40, (2, 6)),           # head_dim 64, ties broken to the lower anchor
+])
+def test_fused_dual_path(C, d, frames, rows, cols, anchors):
+    """A dictionary carrying the anchor geometry runs the dual path in one
+    launch over a joint schedule: every row matches the oracle (block-sparse
+    heads with their LSE, anchor heads with the broadcast), and the result is
+    bitwise the one of the two-launch path (each work item is computed the
+    same way whatever CTA runs it)."""
+    n, h, block = frames * rows * cols, 5, 128
+    nb = O.num_blocks(n, block)
+    q, k, v = W.make_qkv(21, 1, n, h, d, "bf16", 1.0, "cuda")
+    rep_heads = (1, 3)
+    masks = _random_masks(9, h, nb, 0.45)
+    masks = [None if i in rep_heads else masks[i] for i in range(h)]
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    fused = torch.full_like(q, float("nan"))
+    two = torch.full_like(q, float("nan"))
+    lse_f = torch.full((1, h, n), float("nan"), device="cuda")
+    lse_t = torch.full((1, h, n), float("nan"), device="cuda")
+    with C.MaskDictionary(2, 1, h, nb, nb, block, 2 * max(1, ci.size)) as dg, \
+            C.MaskDictionary(1, 1, h, nb, nb, block, max(1, ci.size)) as dp:
+        dg.set_anchor_geometry(frames, rows, cols, anchors)
+        dg.set_layer(1, 0, rp, ci, rep)
+        dp.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_dual_path_attn(q, k, v, fused, dg, 1, 0, frames, rows, cols, anchors, block, lse=lse_f)
+        C.calibatt_dual_path_attn(q, k, v, two, dp, 0, 0, frames, rows, cols, anchors, block, lse=lse_t)
+        _check_status(C)
+    assert torch.equal(fused, two)
+    sparse = [i for i in range(h) if i not in rep_heads]
+    assert torch.equal(lse_f[:, sparse], lse_t[:, sparse])
+    qn, kn, vn = _np(q)[0], _np(k)[0], _np(v)[0]
+    got = _np(fused)[0]
+    for i in range(h):
+        if i in rep_heads:
+            ref, _ = O.anchor_attention(qn[:, i], kn[:, i], vn[:, i], frames, rows, cols, anchors)
+        else:
+            ref, ref_lse = O.block_sparse_attention(qn[:, i], kn[:, i], vn[:, i], masks[i], block)
+            np.testing.assert_allclose(lse_f[0, i].cpu().numpy(), ref_lse, atol=2e-2)
+        _assert_close(got[:, i], ref, "bf16")
+
+
+def test_fused_geometry_rules(C):
+    """The geometry is checked and must come before the first layer; a call
+    whose geometry differs from the dictionary's takes the two-launch path."""
+    n, h, nb = 1024, 2, 8
+    rp, ci, rep = C.masks_to_layer_csr([np.eye(nb, dtype=bool), None], h, nb)
+    with C.MaskDictionary(1, 1, h, nb, nb, 128, ci.size) as dg:
+        with pytest.raises(C.CalibattError):
+            dg.set_anchor_geometry(2, 8, 32, (0, 4))       # 512 tokens: not the dictionary's 8 blocks
+        with pytest.raises(C.CalibattError):
+            dg.set_anchor_geometry(2, 8, 64, (4, 0))       # not ascending
+        dg.set_anchor_geometry(2, 8, 64, (0, 4))
+        with pytest.raises(C.CalibattError):
+            dg.set_anchor_geometry(2, 8, 64, (0, 4))       # only once
+        dg.set_layer(0, 0, rp, ci, rep)
+        q, k, v = W.make_qkv(3, 1, n, h, 128, "bf16", 1.0, "cuda")
+        a, b = torch.empty_like(q), torch.empty_like(q)
+        C.calibatt_dual_path_attn(q, k, v, a, dg, 0, 0, 2, 8, 64, (0, 4))      # one launch
+        C.calibatt_dual_path_attn(q, k, v, b, dg, 0, 0, 2, 8, 64, (1, 4))      # other anchors: two launches
+        _check_status(C)
+        assert torch.equal(a[:, :, 0], b[:, :, 0])                           # the sparse head agrees
+        qn, kn, vn = _np(q)[0], _np(k)[0], _np(v)[0]
+        ref, _ = O.anchor_attention(qn[:, 1], kn[:, 1], vn[:, 1], 2, 8, 64, (1, 4))
+        _assert_close(_np(b)[0][:, 1], ref, "bf16")
+    with C.MaskDictionary(1, 1, h, nb, nb, 128, ci.size) as dl:
+        dl.set_layer(0, 0, rp, ci, rep)
+        with pytest.raises(C.CalibattError):
+            dl.set_anchor_geometry(2, 8, 64, (0, 4))       # after a layer
