@@ -238,6 +238,57 @@ def run_reference(args, rank, world):
     del torch
 
 
+def run_epilogue_probe(torch, B, C):
+    """Store rate of the anchor broadcast epilogue (the 12 repetitive heads of
+    the dual-path 720p layer).  The measurement build records, per CTA, the
+    nanoseconds its epilogues spend issuing the output stores of anchor tiles;
+    every output row of those heads is written once (N x D x 2 bytes per
+    head), so the aggregate rate while in the epilogue is bytes / (mean
+    per-CTA epilogue time)."""
+    import ctypes
+    lib = ctypes.CDLL(B.build(trace=True))
+    for name, (res, argt) in C.SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, argt
+    lib.calibatt_epilogue_probe_read.restype = ctypes.c_int
+    lib.calibatt_epilogue_probe_read.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    C.LIB = lib
+    wd = W.WORKLOADS["720p_dual"]
+    _, rep_heads = W.workload_masks(wd)
+    q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
+    o = torch.empty_like(q)
+
+    def call():
+        C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors, list(rep_heads))
+
+    call()
+    torch.cuda.synchronize()
+    lib.calibatt_trace_reset()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    call()
+    b.record()
+    torch.cuda.synchronize()
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out during the epilogue probe")
+    ns = (ctypes.c_ulonglong * 1024)()
+    items = (ctypes.c_ulonglong * 1024)()
+    lib.calibatt_epilogue_probe_read(ns, items, 1024)
+    used = [(ns[i], items[i]) for i in range(1024) if items[i] > 0]
+    total_bytes = len(rep_heads) * wd.seq_len * wd.head_dim * 2
+    mean_ns = sum(t for t, _ in used) / len(used)
+    n_items = sum(n for _, n in used)
+    print(json.dumps({"epilogue_probe": {
+        "workload": "dual-path 720p layer, anchor path of its 12 repetitive heads",
+        "anchor_tiles": n_items, "ctas": len(used), "output_bytes": total_bytes,
+        "epilogue_ns_per_tile": sum(t for t, _ in used) / n_items,
+        "bytes_per_tile": total_bytes / n_items,
+        "aggregate_gbs_in_epilogue": total_bytes / mean_ns,
+        "call_ms_measurement_build": a.elapsed_time(b),
+        "epilogue_share_of_call": mean_ns / (a.elapsed_time(b) * 1e6),
+        "peak_hbm_gbs": peaks()["hbm_gbs"]}}), flush=True)
+
+
 def run_sweep(args, C, torch, stream, pk):
     """Schedule sweep: a dictionary holding every (timestep, layer) record of
     the schedule, then one dual-path call per (t, l) on fresh seeded inputs,
@@ -348,6 +399,9 @@ def main():
                          "timestep and layer), reported as aggregate time against the dense path")
     ap.add_argument("--sweep-steps", type=int, default=W.SWEEP_STEPS)
     ap.add_argument("--sweep-layers", type=int, default=W.SWEEP_LAYERS)
+    ap.add_argument("--epilogue-probe", action="store_true",
+                    help="time the anchor broadcast epilogue with the library's measurement build "
+                         "(-DCALIBATT_TRACE) and print its store rate")
     ap.add_argument("--dense-sample", type=int, default=50,
                     help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
@@ -376,6 +430,9 @@ def main():
 
     pk = peaks()
     stream = torch.cuda.current_stream()
+    if args.epilogue_probe:
+        run_epilogue_probe(torch, B, C)
+        return
     if args.workload == "sweep":
         if world > 1:
             raise SystemExit("the sweep workload runs on one GPU")

@@ -21,6 +21,9 @@ INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libcalibatt.so")
 BUILD = os.path.join(ROOT, "_build")
+# Measurement variant: the same sources with -DCALIBATT_TRACE (pipeline and
+# epilogue timers compiled in); never loaded by the product path.
+LIB_TRACE = os.path.join(LIBDIR, "libcalibatt_trace.so")
 
 SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu", "energy_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,9 +38,10 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
-    obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+def _compile(src: str, verbose_ptxas: bool, trace: bool = False) -> str:
+    obj = os.path.join(BUILD, "trace" if trace else "", src.replace(".cu", ".o"))
+    cmd = [nvcc(), *ARCH, *FLAGS, *(["-DCALIBATT_TRACE"] if trace else []), "-c", os.path.join(CSRC, src),
+           "-o", obj]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -48,28 +52,30 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "calibatt.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compiles the library if any source is newer than it; returns its path."""
-    if not force and not verbose_ptxas and not _stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, trace: bool = False) -> str:
+    """Compiles the library (or, with trace=True, its measurement variant) if
+    any source is newer than it; returns its path."""
+    lib = LIB_TRACE if trace else LIB
+    if not force and not verbose_ptxas and not _stale(lib):
+        return lib
+    os.makedirs(os.path.join(BUILD, "trace") if trace else BUILD, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), SOURCES))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, trace), SOURCES))
+    tmp = lib + ".tmp"
     r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -59,6 +59,10 @@ constexpr unsigned kTraceEvents = 64;
 __device__ unsigned long long g_trace[kTraceEvents * kTraceIters];
 // Start and end (globaltimer, ns) of every CTA.
 __device__ unsigned long long g_cta_span[2 * 1024];
+// Per CTA: nanoseconds spent in the epilogue stores of anchor tiles, and the
+// number of such tiles (warp 0, lane 0 times its warp's stores).
+__device__ unsigned long long g_epi_ns[1024];
+__device__ unsigned long long g_epi_items[1024];
 #ifndef CALIBATT_TRACE_OFFSET
 #define CALIBATT_TRACE_OFFSET 0
 #endif
@@ -642,6 +646,9 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         n_dst = 1;
       }
     }
+#ifdef CALIBATT_TRACE
+    const unsigned long long t_epi = globaltimer();
+#endif
 #pragma unroll 1
     for (int ch = 0; ch < HD / 64; ++ch) {
       const int col = s * (HD / 2) + ch * 32;  // this group's output columns
@@ -673,6 +680,12 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         for (int g = 0; g < 4; ++g) dst[g] = pkd[g];
       }
     }
+#ifdef CALIBATT_TRACE
+    if (it.anchor && warp == 0 && lane == 0 && blockIdx.x < 1024) {
+      g_epi_ns[blockIdx.x] += globaltimer() - t_epi;
+      g_epi_items[blockIdx.x] += 1;
+    }
+#endif
     if (!it.anchor && s == 0 && p.lse != nullptr && dst_token >= 0) {
       p.lse[(static_cast<int64_t>(it.b) * p.heads + it.h) * p.seq_len + dst_token] =
           it.n > 0 ? (m + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
@@ -813,7 +826,16 @@ extern "C" int calibatt_cta_span_read(unsigned long long* host, int max_records)
   cudaMemcpyFromSymbol(host, g_cta_span, sizeof(unsigned long long) * (n < max_records ? n : max_records));
   return n;
 }
+extern "C" int calibatt_epilogue_probe_read(unsigned long long* ns, unsigned long long* items, int max_ctas) {
+  const int n = max_ctas < 1024 ? max_ctas : 1024;
+  cudaMemcpyFromSymbol(ns, g_epi_ns, sizeof(unsigned long long) * n);
+  cudaMemcpyFromSymbol(items, g_epi_items, sizeof(unsigned long long) * n);
+  return n;
+}
 extern "C" void calibatt_trace_reset() {
+  static unsigned long long zeros_cta[1024];
+  cudaMemcpyToSymbol(g_epi_ns, zeros_cta, sizeof(zeros_cta));
+  cudaMemcpyToSymbol(g_epi_items, zeros_cta, sizeof(zeros_cta));
   cudaMemset(nullptr, 0, 0);
   static unsigned long long zeros[kTraceEvents * kTraceIters];
   cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros));
