@@ -51,6 +51,21 @@ Pins (tests/test_oracle_pins.py, run with ``-m "not gpu"``):
   aggregate_masks: the worked example of the page, 64 prompts at rho = 0.5
       keep a block selected 32 times and drop one selected 31 times
       (tests/golden/aggregation_worked_example.json).
+  spatial_similarity / repetition_flags: anchor rows score exactly one;
+      frames whose rows repeat the anchor queries score one; rows attending
+      to disjoint keys score zero; a two-key closed form; a double-loop brute
+      force over (column, key) on a tiny case; Cauchy-Schwarz bounds; the
+      flag is the strict "exceeds" of the mean over prompts, frames and rows.
+
+Readings for the spatial-repetition branch (Key Designs 3):
+  * the attention "associated with a spatial row" is the post-softmax rows of
+    that row's W queries over all N keys, concatenated in column order into
+    one W*N vector; the nearest anchor row's vector is built the same way
+    from its W queries (the same columns);
+  * the mean runs over every spatial row of every frame, anchor rows
+    included (they score one), and over the calibration prompts;
+  * a head is repetitive when the mean is strictly greater than the
+    threshold (0.87 by default).
 """
 
 from __future__ import annotations
@@ -325,3 +340,52 @@ def aggregate_masks(masks_or_counts, n_prompts, rho):
         counts = a.astype(np.int64)
     mbar = counts.astype(np.float64) / float(n_prompts)
     return mbar >= float(rho)
+
+
+# ------------------------------------------------------ spatial repetition
+
+def attention_probability_rows(q_rows, k, seq_len, scale):
+    """Post-softmax attention rows P[i, :] of the given queries over keys 0..N-1."""
+    qq = _f64(q_rows)
+    kk = _f64(k)[:seq_len]
+    s = scale * (qq @ kk.T)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def spatial_similarity(q, k, frames, rows_per_frame, cols, anchors, scale=None):
+    """Spatial-repetition score of one head (Key Designs 3): for every frame f
+    and spatial row rho, the cosine similarity between the flattened attention
+    of the row's W = cols queries and that of the nearest anchor row's W
+    queries (same frame, same columns):
+
+        v(f, rho) = [P[(f, rho, 0), :], ..., P[(f, rho, W-1), :]]   (length W*N)
+        sim(f, rho) = <v(f, rho), v(f, a*(rho))> / (|v(f, rho)| |v(f, a*(rho))|)
+
+    q, k: [>= N, D] with N = frames * rows * cols.  Returns float64 [frames, rows]."""
+    n = frames * rows_per_frame * cols
+    q = _f64(q)
+    scale = default_scale(q.shape[1]) if scale is None else float(scale)
+    near = nearest_anchor_rows(rows_per_frame, anchors)
+    out = np.zeros((frames, rows_per_frame))
+    for f in range(frames):
+        base = f * rows_per_frame * cols
+        p_anchor = {}
+        for a in sorted(set(int(x) for x in near)):
+            p_anchor[a] = attention_probability_rows(q[base + a * cols: base + (a + 1) * cols], k, n, scale)
+        for rho in range(rows_per_frame):
+            pr = attention_probability_rows(q[base + rho * cols: base + (rho + 1) * cols], k, n, scale)
+            pa = p_anchor[int(near[rho])]
+            out[f, rho] = float(np.sum(pr * pa) / math.sqrt(float(np.sum(pr * pr)) * float(np.sum(pa * pa))))
+    return out
+
+
+def repetition_flags(similarities, threshold=0.87):
+    """Per-head repetition decision (Key Designs 3): the mean of the spatial
+    similarities over calibration prompts, frames and rows, and whether it
+    exceeds the threshold.  similarities: [prompts, heads, frames, rows].
+    Returns (mean float64 [heads], flag bool [heads])."""
+    s = _f64(similarities)
+    mean = s.reshape(s.shape[0], s.shape[1], -1).mean(axis=(0, 2))
+    return mean, mean > float(threshold)

@@ -270,3 +270,98 @@ def test_aggregation_from_stacked_masks_and_union():
     np.testing.assert_array_equal(union, masks.any(axis=0))
     inter = O.aggregate_masks(masks, 4, 1.0)
     np.testing.assert_array_equal(inter, masks.all(axis=0))
+
+
+# ------------------------------------------------------- spatial repetition
+
+def test_spatial_similarity_anchor_rows_score_one():
+    rng = np.random.default_rng(31)
+    frames, rows, cols, d = 2, 6, 5, 8
+    n = frames * rows * cols
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    sim = O.spatial_similarity(q, k, frames, rows, cols, (1, 4))
+    assert np.abs(sim[:, [1, 4]] - 1.0).max() < 1e-12
+    assert (sim >= 0).all() and (sim <= 1 + 1e-12).all()          # probabilities: Cauchy-Schwarz, non-negative
+
+
+def test_spatial_similarity_repeated_rows_score_one():
+    """A frame whose every spatial row repeats the anchor row's queries column
+    by column attends identically row by row: similarity one everywhere."""
+    rng = np.random.default_rng(32)
+    frames, rows, cols, d = 2, 5, 4, 6
+    n = frames * rows * cols
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    qf = q.reshape(frames, rows, cols, d)
+    qf[0] = qf[0, 2][None]                                        # frame 0: all rows = row 2
+    sim = O.spatial_similarity(qf.reshape(n, d), k, frames, rows, cols, (2,))
+    assert np.abs(sim[0] - 1.0).max() < 1e-12
+    assert sim[1].min() < 0.999                                   # frame 1 keeps its own rows
+
+
+def test_spatial_similarity_disjoint_attention_scores_zero():
+    """Non-anchor rows attend (almost) only to keys of one kind and the anchor
+    row only to keys of another: the flattened distributions are orthogonal."""
+    frames, rows, cols = 1, 3, 4
+    n = frames * rows * cols
+    k = np.zeros((n, 2))
+    k[: n // 2, 0] = 1.0                                          # keys of kind A
+    k[n // 2:, 1] = 1.0                                           # keys of kind B
+    q = np.zeros((n, 2))
+    for rho in range(rows):
+        q[rho * cols:(rho + 1) * cols, 0 if rho != 1 else 1] = 60.0
+    sim = O.spatial_similarity(q, k, frames, rows, cols, (1,), scale=1.0)
+    assert abs(sim[0, 1] - 1.0) < 1e-12
+    assert sim[0, 0] < 1e-20 and sim[0, 2] < 1e-20
+
+
+def test_spatial_similarity_two_token_closed_form():
+    """Two tokens (one frame, two rows of one column, anchor row 0): each
+    attention row is a two-point distribution [sigma(x), 1 - sigma(x)] with x
+    the scaled score difference, so the cosine has a closed form."""
+    q = np.array([[0.7], [-1.3]])
+    k = np.array([[1.1], [-0.4]])
+    scale = 0.9
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    a, b = sig(scale * 0.7 * 1.5), sig(scale * -1.3 * 1.5)
+    cos = (a * b + (1 - a) * (1 - b)) / math.sqrt((a * a + (1 - a) ** 2) * (b * b + (1 - b) ** 2))
+    sim = O.spatial_similarity(q, k, 1, 2, 1, (0,), scale=scale)
+    assert abs(sim[0, 1] - cos) < 1e-14 and abs(sim[0, 0] - 1.0) < 1e-14
+
+
+def test_spatial_similarity_double_loop():
+    """Brute force: explicit loops over columns and keys with math.exp."""
+    rng = np.random.default_rng(33)
+    frames, rows, cols, d = 2, 3, 2, 3
+    n = frames * rows * cols
+    q, k = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    scale = 0.6
+    near = {0: 0, 1: 0, 2: 2}                                     # anchors {0, 2}; row 1 ties -> lower
+    got = O.spatial_similarity(q, k, frames, rows, cols, (0, 2), scale=scale)
+
+    def prob_row(i):
+        e = [math.exp(scale * sum(q[i, t] * k[j, t] for t in range(d))) for j in range(n)]
+        z = sum(e)
+        return [x / z for x in e]
+
+    for f in range(frames):
+        for rho in range(rows):
+            num = na = nb = 0.0
+            for w in range(cols):
+                pr = prob_row(f * rows * cols + rho * cols + w)
+                pa = prob_row(f * rows * cols + near[rho] * cols + w)
+                for j in range(n):
+                    num += pr[j] * pa[j]
+                    na += pr[j] * pr[j]
+                    nb += pa[j] * pa[j]
+            assert abs(got[f, rho] - num / math.sqrt(na * nb)) < 1e-13
+
+
+def test_repetition_flags_mean_and_strict_threshold():
+    sims = np.full((3, 2, 2, 4), 0.87)
+    sims[:, 1] += 0.01                                            # head 1 above the threshold
+    mean, flag = O.repetition_flags(sims, 0.87)
+    assert abs(mean[0] - 0.87) < 1e-15 and not flag[0]            # equal is not "exceeds"
+    assert flag[1]
+    sims[2, 0, 1, 3] = 0.87 + 24 * 0.001                          # one of 24 entries raises the mean by 0.001
+    mean, flag = O.repetition_flags(sims, 0.87)
+    assert abs(mean[0] - 0.871) < 1e-12 and flag[0]
