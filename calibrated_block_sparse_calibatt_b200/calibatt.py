@@ -61,6 +61,9 @@ SIGNATURES = {
     "calibatt_dict_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P(_vp)]),
     "calibatt_dict_set_layer": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
     "calibatt_dict_set_anchor_geometry": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32]),
+    "calibatt_spatial_similarity": (_i32, [_vp, _vp, _P(Shape), _i32, _i32, _i32, _vp, _i32, _f32, _vp, _vp,
+                                           ctypes.c_size_t, _vp]),
+    "calibatt_repetition_flags": (_i32, [_vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
     "calibatt_dict_info": (_i32, [_vp, _P(_i64), _P(_i64), _P(_i32)]),
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
@@ -285,6 +288,33 @@ def calibatt_dual_path_attn(q, k, v, o, d: MaskDictionary, t, l, frames, rows, c
     check(LIB.calibatt_dual_path_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shape), block, d.handle, t,
                                       l, frames, rows, cols, _ptr(a), a.size, float(softmax_scale), _ptr(lse),
                                       _stream(stream)))
+
+
+def calibatt_spatial_similarity(q, k, sim, workspace, frames, rows, cols, anchor_rows, softmax_scale=0.0,
+                                stream=None):
+    """Spatial-repetition score of every (batch, head, frame, row) into sim
+    (float32 [batch, heads, frames, rows]); workspace as calibatt_block_energy's."""
+    shape = shape_of(q)
+    a = _i32_array(anchor_rows)
+    nbytes = workspace.numel() * workspace.element_size()
+    check(LIB.calibatt_spatial_similarity(_ptr(q), _ptr(k), ctypes.byref(shape), frames, rows, cols, _ptr(a), a.size,
+                                          float(softmax_scale), _ptr(sim), _ptr(workspace), nbytes,
+                                          _stream(stream)))
+
+
+def calibatt_repetition_flags(sim, threshold=0.87, mean=None, flags=None, stream=None):
+    """Per-head mean over prompts and rows of sim [prompts, heads, rows...] and
+    the flags mean > threshold; returns (mean, flags) device tensors."""
+    import torch
+    n_prompts, n_heads = int(sim.shape[0]), int(sim.shape[1])
+    per_head = int(sim[0, 0].numel()) if n_heads else 1
+    if mean is None:
+        mean = torch.empty(n_heads, dtype=torch.float32, device=sim.device)
+    if flags is None:
+        flags = torch.empty(n_heads, dtype=torch.uint8, device=sim.device)
+    check(LIB.calibatt_repetition_flags(_ptr(sim), n_prompts, n_heads, per_head, float(threshold), _ptr(mean),
+                                        _ptr(flags), _stream(stream)))
+    return mean, flags
 
 
 def calibatt_block_energy_workspace_size(q) -> int:

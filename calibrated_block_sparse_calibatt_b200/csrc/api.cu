@@ -991,6 +991,89 @@ calibatt_status calibatt_block_energy(const void* q, const void* k, const caliba
   return CALIBATT_OK;
 }
 
+calibatt_status calibatt_spatial_similarity(const void* q, const void* k, const calibatt_shape* shape, int32_t frames,
+                                            int32_t rows, int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
+                                            float softmax_scale, float* similarity, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if (!q || !k || !similarity || !workspace)
+    return fail(CALIBATT_ERR_INVALID_ARG, "q, k, similarity and workspace must be non-NULL");
+  if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
+  if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
+    return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
+                shape->seq_len);
+  if (rows > calibatt::kMaxRepetitionRows)
+    return fail(CALIBATT_ERR_UNSUPPORTED, "more than %d spatial rows per frame", calibatt::kMaxRepetitionRows);
+  if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
+  for (int a = 0; a < n_anchors; ++a) {
+    if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
+    if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
+      return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
+  }
+  size_t need = 0;
+  calibatt_block_energy_workspace_size(shape, &need);
+  if (workspace_bytes < need)
+    return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+  const float sl2 = scale_log2_of(softmax_scale, shape->head_dim);
+  calibatt::EnergyParams e;
+  std::memset(&e, 0, sizeof(e));
+  e.q = q;
+  e.k = k;
+  e.lse = static_cast<float*>(workspace);
+  e.sb = shape->stride_b;
+  e.sn = shape->stride_n;
+  e.sh = shape->stride_h;
+  e.batch = shape->batch;
+  e.seq_len = shape->seq_len;
+  e.heads = shape->heads;
+  e.scale_log2 = sl2;
+  cudaError_t ce = calibatt::launch_row_lse(e, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce, "row log-sum-exp launch");
+  calibatt::RepetitionParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.k = k;
+  p.lse = static_cast<const float*>(workspace);
+  p.sim = similarity;
+  p.sb = shape->stride_b;
+  p.sn = shape->stride_n;
+  p.sh = shape->stride_h;
+  p.batch = shape->batch;
+  p.seq_len = shape->seq_len;
+  p.heads = shape->heads;
+  p.frames = frames;
+  p.rows = rows;
+  p.cols = cols;
+  p.scale_log2 = sl2;
+  // nearest anchor of each row, ties to the lower anchor (as the anchor path)
+  for (int32_t rho = 0; rho < rows; ++rho) {
+    int best = 0;
+    for (int a = 1; a < n_anchors; ++a)
+      if (std::abs(rho - anchor_rows[a]) < std::abs(rho - anchor_rows[best])) best = a;
+    p.nearest[rho] = static_cast<int16_t>(anchor_rows[best]);
+  }
+  ce = calibatt::launch_spatial_similarity(p, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce, "spatial similarity launch");
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_prompts, int32_t n_heads,
+                                          int32_t per_head, float threshold, float* mean, uint8_t* flags,
+                                          void* stream) {
+  if (n_prompts < 1 || n_heads < 0 || per_head < 1)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_prompts and per_head must be >= 1, n_heads >= 0");
+  if (n_heads > 0 && (!similarity || !flags))
+    return fail(CALIBATT_ERR_INVALID_ARG, "similarity and flags must be non-NULL");
+  if (!(threshold == threshold)) return fail(CALIBATT_ERR_INVALID_ARG, "threshold is NaN");
+  cudaError_t e = calibatt::launch_repetition_flags(similarity, n_prompts, n_heads, per_head, threshold, mean, flags,
+                                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "repetition flags launch");
+  return CALIBATT_OK;
+}
+
 calibatt_status calibatt_select_blocks(const float* energy, int64_t n_rows, int32_t nk, float tau, uint8_t* mask,
                                        int32_t* count_accum, void* stream) {
   if (n_rows < 0 || nk < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_rows must be >= 0 and nk >= 1");

@@ -17,6 +17,7 @@ namespace calibatt {
 namespace {
 
 constexpr int kKeysPerStage = 32;
+inline unsigned ceil_blocks(int n, int b) { return static_cast<unsigned>((n + b - 1) / b); }
 constexpr int kKeysPerChunk = 8;  // keys scored per register chunk
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -195,6 +196,22 @@ __global__ void aggregate_kernel(const int32_t* __restrict__ counts, int64_t n, 
 }
 
 }  // namespace
+
+// Pass 1 alone (also the first pass of the spatial-repetition score):
+// lse2[b, h, i] for every query, 128 queries per CTA.
+cudaError_t launch_row_lse(const EnergyParams& p, int head_dim, int dtype, cudaStream_t s) {
+  dim3 g(ceil_blocks(p.seq_len, 128), p.heads, p.batch);
+  if (head_dim == 64) {
+    if (dtype == 1) row_lse_kernel<float, 64, 128><<<g, 256, 0, s>>>(p);
+    else row_lse_kernel<__nv_bfloat16, 64, 128><<<g, 256, 0, s>>>(p);
+  } else if (head_dim == 128) {
+    if (dtype == 1) row_lse_kernel<float, 128, 128><<<g, 256, 0, s>>>(p);
+    else row_lse_kernel<__nv_bfloat16, 128, 128><<<g, 256, 0, s>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_energy(const EnergyParams& p, int head_dim, int block, int dtype,
                                 cudaStream_t s) {

@@ -96,6 +96,25 @@ cudaError_t launch_simt_attn(const SimtParams& p, int head_dim, int block, int d
                              int n_items, cudaStream_t s);
 cudaError_t launch_block_energy(const EnergyParams& p, int head_dim, int block, int dtype,
                                 cudaStream_t s);
+cudaError_t launch_row_lse(const EnergyParams& p, int head_dim, int dtype, cudaStream_t s);
+
+// Spatial-repetition score, pass 2 (repetition.cu).
+struct RepetitionParams {
+  const void* q;
+  const void* k;
+  const float* lse;   // pass-1 log2 LSE [batch, heads, seq_len]
+  float* sim;         // [batch, heads, frames, rows]
+  int64_t sb, sn, sh;
+  int32_t batch, seq_len, heads;
+  int32_t frames, rows, cols;
+  float scale_log2;
+  int16_t nearest[256];  // nearest anchor row of each spatial row
+};
+constexpr int kMaxRepetitionRows = 256;
+cudaError_t launch_spatial_similarity(const RepetitionParams& p, int head_dim, int dtype, cudaStream_t s);
+cudaError_t launch_repetition_flags(const float* sim, int32_t n_prompts, int32_t n_heads, int32_t per_head,
+                                    float threshold, float* mean, uint8_t* flags, cudaStream_t s);
+
 cudaError_t launch_select_blocks(const float* energy, int64_t n_rows, int32_t nk, float tau,
                                  uint8_t* mask, int32_t* count_accum, cudaStream_t s);
 cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,

@@ -289,6 +289,39 @@ calibatt_status calibatt_select_blocks(const float* energy, int64_t n_rows, int3
 calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32_t n_prompts,
                                          float rho, uint8_t* mask, void* stream);
 
+/* Spatial-repetition score (Key Designs 3) of every spatial row of every
+ * head: with tokens ordered (frame, row, column), frames * rows * cols ==
+ * seq_len, and a*(rho) the anchor row nearest to row rho (ties to the lower
+ * anchor), the cosine similarity of the flattened post-softmax attention of
+ * the row's cols queries over all keys and that of a*(rho)'s cols queries
+ * (same frame, same columns):
+ *   sim[b, h, f, rho] = sum_w <P[(f,rho,w)], P[(f,a,w)]>
+ *                       / sqrt(sum_w |P[(f,rho,w)]|^2 * sum_w |P[(f,a,w)]|^2)
+ * with P the dense, unmasked softmax of scale * q.k.  Anchor rows score one.
+ * similarity: device float32 [batch, heads, frames, rows].  workspace:
+ * caller-owned device scratch of at least calibatt_block_energy_workspace_size
+ * bytes (each query's log-sum-exp).  anchor_rows: host int32, strictly
+ * ascending in [0, rows), 1..16 of them; rows <= 256.  Computed on CUDA cores
+ * in float32 with fixed summation orders (bitwise repeatable). */
+calibatt_status calibatt_spatial_similarity(const void* q, const void* k,
+                                            const calibatt_shape* shape, int32_t frames,
+                                            int32_t rows, int32_t cols,
+                                            const int32_t* anchor_rows, int32_t n_anchors,
+                                            float softmax_scale, float* similarity,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream);
+
+/* Repetition flags (Key Designs 3): for each of n_heads heads, the mean of
+ * its per_head similarities over n_prompts calibration prompts (similarity:
+ * device float32 [n_prompts][n_heads][per_head], e.g. per_head = frames *
+ * rows of calibatt_spatial_similarity and n_heads = batch * heads), summed in
+ * float64 in a fixed order; flags[h] = 1 when the mean is strictly greater
+ * than threshold (the page's default is 0.87).  mean (nullable): device
+ * float32 [n_heads]; flags: device uint8 [n_heads]. */
+calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_prompts,
+                                          int32_t n_heads, int32_t per_head, float threshold,
+                                          float* mean, uint8_t* flags, void* stream);
+
 /* ------------------------------------------------------- diagnostics */
 
 /* Synchronises `stream`, then reports the device status word that the

@@ -354,7 +354,7 @@ def attention_probability_rows(q_rows, k, seq_len, scale):
     return p / p.sum(axis=1, keepdims=True)
 
 
-def spatial_similarity(q, k, frames, rows_per_frame, cols, anchors, scale=None):
+def spatial_similarity(q, k, frames, rows_per_frame, cols, anchors, scale=None, only=None):
     """Spatial-repetition score of one head (Key Designs 3): for every frame f
     and spatial row rho, the cosine similarity between the flattened attention
     of the row's W = cols queries and that of the nearest anchor row's W
@@ -363,21 +363,20 @@ def spatial_similarity(q, k, frames, rows_per_frame, cols, anchors, scale=None):
         v(f, rho) = [P[(f, rho, 0), :], ..., P[(f, rho, W-1), :]]   (length W*N)
         sim(f, rho) = <v(f, rho), v(f, a*(rho))> / (|v(f, rho)| |v(f, a*(rho))|)
 
-    q, k: [>= N, D] with N = frames * rows * cols.  Returns float64 [frames, rows]."""
+    q, k: [>= N, D] with N = frames * rows * cols.  only: optional list of
+    (f, rho) to evaluate (the others are NaN).  Returns float64 [frames, rows]."""
     n = frames * rows_per_frame * cols
     q = _f64(q)
     scale = default_scale(q.shape[1]) if scale is None else float(scale)
     near = nearest_anchor_rows(rows_per_frame, anchors)
-    out = np.zeros((frames, rows_per_frame))
-    for f in range(frames):
+    pairs = [(f, r) for f in range(frames) for r in range(rows_per_frame)] if only is None else list(only)
+    out = np.full((frames, rows_per_frame), np.nan)
+    for f, rho in pairs:
         base = f * rows_per_frame * cols
-        p_anchor = {}
-        for a in sorted(set(int(x) for x in near)):
-            p_anchor[a] = attention_probability_rows(q[base + a * cols: base + (a + 1) * cols], k, n, scale)
-        for rho in range(rows_per_frame):
-            pr = attention_probability_rows(q[base + rho * cols: base + (rho + 1) * cols], k, n, scale)
-            pa = p_anchor[int(near[rho])]
-            out[f, rho] = float(np.sum(pr * pa) / math.sqrt(float(np.sum(pr * pr)) * float(np.sum(pa * pa))))
+        a = int(near[rho])
+        pr = attention_probability_rows(q[base + rho * cols: base + (rho + 1) * cols], k, n, scale)
+        pa = attention_probability_rows(q[base + a * cols: base + (a + 1) * cols], k, n, scale)
+        out[f, rho] = float(np.sum(pr * pa) / math.sqrt(float(np.sum(pr * pr)) * float(np.sum(pa * pa))))
     return out
 
 

@@ -513,3 +513,72 @@ def test_fused_geometry_rules(C):
         dl.set_layer(0, 0, rp, ci, rep)
         with pytest.raises(C.CalibattError):
             dl.set_anchor_geometry(2, 8, 64, (0, 4))       # after a layer
+
+
+# ------------------------------------------------------- spatial repetition
+
+def _similarity(C, q, k, frames, rows, cols, anchors):
+    b, n, h, _ = q.shape
+    ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, dtype=torch.float32, device=q.device)
+    sim = torch.full((b, h, frames, rows), float("nan"), dtype=torch.float32, device=q.device)
+    C.calibatt_spatial_similarity(q, k, sim, ws, frames, rows, cols, anchors)
+    _check_status(C)
+    return sim
+
+
+@pytest.mark.parametrize("dtype,d,frames,rows,cols,anchors,batch,heads", [
+    ("fp32", 64, 2, 8, 16, (0, 4), 1, 2),              # the tiny layout
+    ("bf16", 128, 3, 9, 40, (1, 4, 7), 2, 3),          # 40 columns, two batches, three anchors
+    ("bf16", 64, 2, 6, 100, (2,), 1, 2),               # 100 columns: two column passes
+])
+def test_spatial_similarity_matches_oracle(C, dtype, d, frames, rows, cols, anchors, batch, heads):
+    n = frames * rows * cols
+    q, k, _ = W.make_qkv(41, batch, n, heads, d, dtype, 1.0, "cuda")
+    sim = _similarity(C, q, k, frames, rows, cols, anchors)
+    again = _similarity(C, q, k, frames, rows, cols, anchors)
+    assert torch.equal(sim, again)                                    # fixed summation orders
+    got = sim.cpu().numpy().astype(np.float64)
+    for bb in range(batch):
+        for hh in range(heads):
+            ref = O.spatial_similarity(_np(q[bb, :, hh]), _np(k[bb, :, hh]), frames, rows, cols, anchors)
+            assert np.abs(got[bb, hh] - ref).max() <= 1e-4, np.abs(got[bb, hh] - ref).max()
+    assert np.abs(got[:, :, :, list(anchors)] - 1.0).max() <= 1e-5
+
+
+def test_spatial_similarity_720p_sampled_and_flags(C):
+    """Two heads of the 720p layout (75,600 tokens), sampled (frame, row)
+    scores against the oracle; then the flags of three prompts' scores
+    against repetition_flags on the same scores (threshold between the heads'
+    means, so both outcomes occur)."""
+    wl = W.WORKLOADS["720p"]
+    heads = 2
+    sims = []
+    for prompt in range(3):
+        q, k, _ = W.make_qkv(500 + prompt, 1, wl.seq_len, heads, wl.head_dim, "bf16", wl.input_std * 2.0, "cuda")
+        if prompt == 0:
+            # make head 1 strongly repetitive: every row of a frame repeats its nearest anchor row's queries
+            near = O.nearest_anchor_rows(wl.rows, wl.anchors)
+            qv = q.view(1, wl.frames, wl.rows, wl.cols, heads, wl.head_dim)
+            qv[:, :, :, :, 1] = qv[:, :, torch.as_tensor(near, device=q.device), :, 1]
+        sim = _similarity(C, q, k, wl.frames, wl.rows, wl.cols, wl.anchors)
+        if prompt == 0:
+            rng = np.random.default_rng(3)
+            pairs = [(0, 0), (int(rng.integers(wl.frames)), int(rng.integers(wl.rows))), (wl.frames - 1, wl.rows - 1)]
+            for hh in range(heads):
+                ref = O.spatial_similarity(_np(q[0, :, hh]), _np(k[0, :, hh]), wl.frames, wl.rows, wl.cols,
+                                           wl.anchors, only=pairs)
+                for f, rho in pairs:
+                    got = float(sim[0, hh, f, rho])
+                    assert abs(got - ref[f, rho]) <= 1e-4, (hh, f, rho, got, ref[f, rho])
+            assert float(sim[0, 1].min()) > 0.999999
+        sims.append(sim[0])
+        del q, k
+    stack = torch.stack(sims)                                          # [prompts, heads, frames, rows]
+    ref_mean, _ = O.repetition_flags(stack.cpu().numpy(), 0.0)
+    thr = float(ref_mean.mean())
+    mean, flags = C.calibatt_repetition_flags(stack, thr)
+    _check_status(C)
+    ref_mean, ref_flags = O.repetition_flags(stack.cpu().numpy(), thr)
+    assert np.abs(mean.cpu().numpy() - ref_mean).max() <= 1e-6
+    assert np.array_equal(flags.cpu().numpy().astype(bool), ref_flags)
+    assert ref_flags.any() and not ref_flags.all()
