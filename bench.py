@@ -516,6 +516,17 @@ def main():
             "anchor_heads": len(rep_heads), "anchor_ms": anchor_ms,
             "anchor_effective_tflops": anchor_tiles * FLOP_PER_TILE / (anchor_ms * 1e-3) / 1e12,
             "anchor_output_bytes": bcast_bytes}
+        # offline calibration: block energies of the dense attention (two Q K^T passes on the tensor cores)
+        e_out = torch.empty((1, wl.heads, wl.num_blocks, wl.num_blocks), device="cuda")
+        e_ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, device="cuda")
+        energy_ms = max_over_ranks(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_block_energy(q, k, e_out, e_ws, wl.block, stream=stream),
+            3, 1, stream)), dist, "cuda")
+        del e_out, e_ws
+        extras["block_energy_720p"] = {
+            "ms_per_call": energy_ms, "heads": wl.heads,
+            "tflops_two_qk_passes": 2 * 2.0 * wl.seq_len ** 2 * wl.head_dim * wl.heads / (energy_ms * 1e-3) / 1e12,
+            "exp2_per_call": 2 * wl.seq_len ** 2 * wl.heads}
         if C.device_status() != 0:
             raise RuntimeError("device wait timed out during the extra legs")
 

@@ -972,6 +972,36 @@ calibatt_status calibatt_block_energy(const void* q, const void* k, const caliba
     return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
   const int nb = ceil_div(shape->seq_len, block);
   if (nb > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
+  if (shape->dtype == CALIBATT_DTYPE_BF16 && block == 128) {
+    // Tensor-core path: the LSE pass, then the energy pass, as persistent
+    // launches of the attention pipeline without V.
+    TcParams t;
+    std::memset(&t, 0, sizeof(t));
+    if ((st = encode_qkv_map(&t.tm_q, q, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+    if ((st = encode_qkv_map(&t.tm_k, k, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+    t.tm_v = t.tm_k;  // no V in these modes
+    t.q = static_cast<const uint16_t*>(q);
+    t.lse = static_cast<float*>(workspace);
+    t.energy = energy;
+    t.sb = shape->stride_b;
+    t.sn = shape->stride_n;
+    t.sh = shape->stride_h;
+    t.batch = shape->batch;
+    t.seq_len = shape->seq_len;
+    t.heads = shape->heads;
+    t.nb = nb;
+    t.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
+    t.status = status_word_ptr();
+    t.timeout_ns = g_timeout_ns.load();
+    const int sms = device_sm_count();
+    if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    const int grid = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(shape->heads) * nb));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeLse, grid, cs);
+    if (e == cudaSuccess) e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeEnergy, grid, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core block energy launch");
+    return CALIBATT_OK;
+  }
   calibatt::EnergyParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = q;

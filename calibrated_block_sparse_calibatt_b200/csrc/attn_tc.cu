@@ -179,6 +179,10 @@ struct Cursor {
       begin = blockIdx.x;
       end = p.anc.n_heads * p.anc.tiles_per_head;
       step = gridDim.x;
+    } else if (MODE == kModeLse || MODE == kModeEnergy) {
+      begin = blockIdx.x;
+      end = p.heads * p.nb;
+      step = gridDim.x;
     } else {
       begin = p.sched.cta_ptr[blockIdx.x];
       end = p.sched.cta_ptr[blockIdx.x + 1];
@@ -191,6 +195,17 @@ struct Cursor {
       if (idx < end) {
         it.b = b;
         uint32_t w = 0;
+        if (MODE == kModeLse || MODE == kModeEnergy) {
+          // every key block of query block (idx mod nb) of head (idx / nb)
+          it.anchor = false;
+          it.h = idx / p.nb;
+          it.tile = idx % p.nb;
+          it.n = p.nb;
+          it.cols = nullptr;
+          it.ragged_last = (p.seq_len % 128) != 0;
+          idx += step;
+          return true;
+        }
         if (MODE != kModeAnchor) w = p.sched.items[idx];
         if (MODE == kModeAnchor || (MODE == kModeFused && (w & kItemAnchorBit))) {
           it.anchor = true;
@@ -261,6 +276,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
   constexpr int kEmpty = V ? L::bVEmpty : L::bKEmpty;
   constexpr int kRing = V ? L::kV : L::kK;
   const CUtensorMap* map = V ? &p.tm_v : &p.tm_k;
+  if (V && (MODE == kModeLse || MODE == kModeEnergy)) return;  // no P.V in the calibration modes
   Cursor<MODE> cur;
   cur.init(p);
   Item it;
@@ -321,7 +337,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
     for (int j = 0; j < it.n; ++j) {
       if ((j & 31) == 0) {
         const int jj = j + lane;
-        my_col = it.anchor ? static_cast<uint32_t>(jj) : (jj < it.n ? it.cols[jj] : 0u);
+        my_col = it.cols == nullptr ? static_cast<uint32_t>(jj) : (jj < it.n ? it.cols[jj] : 0u);
       }
       const int c = static_cast<int>(__shfl_sync(0xFFFFFFFFu, my_col, j & 31));
       const uint32_t slot = kv % kStages, use = kv / kStages;
@@ -411,6 +427,12 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, 1);
+  if (MODE == kModeLse || MODE == kModeEnergy) {
+    // No P.V: only this thread's share of the drain barrier.
+    if (lane == 0) mma_commit(bar(L::bDrain));
+    __syncwarp();
+    return;
+  }
   Cursor<MODE> cur;
   cur.init(p);
   Item it;
@@ -697,6 +719,124 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   }
 }
 
+// ------------------------------------------------- calibration (energy) roles
+// Key Designs 1, Eq. (5) on the tensor-core pipeline.  LSE mode: each stream
+// keeps an exact running maximum and sum of its rows over its key blocks, and
+// the epilogue merges the two streams into lse2 = log2 sum_j 2^(s_ij log2e
+// scale).  Energy mode: per key block c, each thread sums 2^(s log2e scale -
+// lse2) over the block's keys for its query row; the block's rows are summed
+// in a fixed order (warp shuffle tree, then the four warps of the stream in
+// order) and E[r, c] = sum / |I_r| is written by one thread.
+constexpr int kEnergyBarrier = 6;  // named barriers 6 and 7: the two streams' warps
+
+template <int HD, int MODE>
+__device__ void softmax_energy_role(const TcParams& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
+                                    const Waiter& W, int warp, int lane) {
+  using L = Layout<HD>;
+  auto bar = [&](int i) { return base + L::kBar + 8u * i; };
+  const int quarter = warp & 3, s = warp >> 2;
+  const int row = quarter * 32 + lane;
+  const int pair_bar = 1 + quarter;
+  float* xchg = reinterpret_cast<float*>(gbase + L::kXchg);
+  // per-warp partial sums [2 block parity][2 streams][4 warps] (energy mode)
+  float* part = reinterpret_cast<float*>(gbase + L::kMSlot);
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tS = tmem + lane_off + kColS + s * 128;
+  const int ragged_cols = p.seq_len % 128;
+  const float sl2 = p.scale_log2;
+  Cursor<MODE> cur;
+  cur.init(p);
+  Item it;
+  uint32_t item = 0, t_me = 0;
+  bool ok = true;
+  while (cur.next(p, it)) {
+    const int n_s = (it.n + 1 - s) / 2;
+    const int token = it.tile * 128 + row;
+    const bool valid = token < p.seq_len;
+    const int64_t bh = static_cast<int64_t>(it.b) * p.heads + it.h;
+    float lse2 = 0.f;
+    if (MODE == kModeEnergy && valid) lse2 = p.lse[bh * p.seq_len + token];
+    float m = -INFINITY, l = 0.f;
+    for (int k = 0; k < n_s; ++k) {
+      const int j = 2 * k + s;
+      ok = ok && W.wait(bar(L::bSFull + s), t_me & 1, 10);
+      if (ok) tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld_x128(tS, sr);
+      tc_fence_before();
+      if (ok) mbar_arrive(bar(L::bSFree + s));
+      float sc[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) sc[c] = __uint_as_float(sr[c]);
+      if (j == it.n - 1 && it.ragged_last) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= ragged_cols) sc[c] = -INFINITY;
+      }
+      float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
+      float off;
+      if (MODE == kModeLse) {
+        float mx8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(sc[a], sc[a + 8]);
+#pragma unroll
+        for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sc[c + a], sc[c + a + 8]);
+        }
+        const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
+        const float m_new = fmaxf(m, mx);
+        if (m_new != m) {
+          l = (m == -INFINITY) ? 0.f : l * fast_exp2(m - m_new);
+          m = m_new;
+        }
+        off = (m == -INFINITY) ? 0.f : m;
+      } else {
+        off = lse2;
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float x0, x1;
+        fma2(x0, x1, sc[2 * c], sc[2 * c + 1], sl2, sl2, -off, -off);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        if (c & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
+      }
+      const float rs = (la + lb) + (lc + ld);
+      if (MODE == kModeLse) {
+        l += rs;
+      } else {
+        // sum over the block's valid query rows, in a fixed order
+        float v = valid ? rs : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        float* pb = part + ((k & 1) * 2 + s) * 4;
+        if (lane == 0) pb[quarter] = v;
+        cta_bar_sync(kEnergyBarrier + s, 128);
+        if (quarter == 0 && lane == 0) {
+          const int valid_rows = min(128, p.seq_len - it.tile * 128);
+          const float e = (((pb[0] + pb[1]) + pb[2]) + pb[3]) / static_cast<float>(valid_rows);
+          p.energy[(bh * p.nb + it.tile) * p.nb + j] = e;
+        }
+      }
+      ++t_me;
+    }
+    if (MODE == kModeLse) {
+      // merge the two streams' (m, l) of every row; group 0 writes lse2
+      float* xb = xchg + (item & 1) * 512;
+      xb[(s * 2 + 0) * 128 + row] = m;
+      xb[(s * 2 + 1) * 128 + row] = l;
+      if (bar_red_or(pair_bar, 64, !ok)) { ok = false; break; }
+      if (s == 0 && valid) {
+        const float m1 = xb[(2 + 0) * 128 + row], l1 = xb[(2 + 1) * 128 + row];
+        const float mm = fmaxf(m, m1);
+        const float ll = (m == -INFINITY ? 0.f : l * fast_exp2(m - mm)) + (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - mm));
+        p.lse[bh * p.seq_len + token] = mm + __log2f(ll);
+      }
+    }
+    ++item;
+  }
+}
+
 template <int HD, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<HD>;
@@ -775,7 +915,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 #endif
   } else {
     reg_alloc<kSoftmaxRegs>();
-    softmax_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
+    if (MODE == kModeLse || MODE == kModeEnergy)
+      softmax_energy_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
+    else
+      softmax_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
     tc_fence_before();
     cta_bar_sync(kEndBarrier, kThreads);
   }
@@ -858,11 +1001,15 @@ cudaError_t launch_tc_attn(const TcParams& p, int head_dim, int mode, int grid, 
     if (mode == kModeSparse) return launch_one<128, kModeSparse>(p, grid, s);
     if (mode == kModeAnchor) return launch_one<128, kModeAnchor>(p, grid, s);
     if (mode == kModeFused) return launch_one<128, kModeFused>(p, grid, s);
+    if (mode == kModeLse) return launch_one<128, kModeLse>(p, grid, s);
+    if (mode == kModeEnergy) return launch_one<128, kModeEnergy>(p, grid, s);
   }
   if (head_dim == 64) {
     if (mode == kModeSparse) return launch_one<64, kModeSparse>(p, grid, s);
     if (mode == kModeAnchor) return launch_one<64, kModeAnchor>(p, grid, s);
     if (mode == kModeFused) return launch_one<64, kModeFused>(p, grid, s);
+    if (mode == kModeLse) return launch_one<64, kModeLse>(p, grid, s);
+    if (mode == kModeEnergy) return launch_one<64, kModeEnergy>(p, grid, s);
   }
   return cudaErrorInvalidValue;
 }

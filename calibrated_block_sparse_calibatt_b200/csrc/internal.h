@@ -44,7 +44,8 @@ struct TcParams {
   CUtensorMap tm_v;
   const uint16_t* q;  // raw Q (anchor-row gather)
   uint16_t* o;
-  float* lse;  // nullable [batch, heads, seq_len]
+  float* lse;  // nullable [batch, heads, seq_len]; energy modes: log2 LSE workspace
+  float* energy;  // energy mode: [batch, heads, nb, nb]
   int64_t sb, sn, sh;  // element strides shared by Q, K, V, O
   int32_t batch, seq_len, heads, nb;
   int32_t pos_n, pos_h, pos_b;  // which tensor-map dimension (1..3) holds N, H, batch
@@ -86,6 +87,11 @@ struct EnergyParams {
 constexpr int kModeSparse = 0;
 constexpr int kModeAnchor = 1;
 constexpr int kModeFused = 2;
+// Offline calibration on the same pipeline (no V, no P.V): every (head,
+// query block) visits all key blocks; the LSE mode writes each query's log2
+// log-sum-exp, the energy mode the block energies from it.
+constexpr int kModeLse = 3;
+constexpr int kModeEnergy = 4;
 // Work-item word of the dictionary schedules: bit 31 marks an anchor tile
 // (fused schedules only), bits 16-30 the head, bits 0-15 the query block or
 // anchor tile.

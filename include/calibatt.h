@@ -244,8 +244,10 @@ calibatt_status calibatt_block_energy_workspace_size(const calibatt_shape* shape
  * of E sums to one.  energy: device float32 [batch, heads, nb, nb].
  * workspace: caller-owned device scratch of at least
  * calibatt_block_energy_workspace_size() bytes (row log-sum-exp values).
- * Computed on CUDA cores in float32 with a fixed summation order, so repeated
- * calls give bitwise identical energies. */
+ * bf16 inputs with block 128 run on the tensor cores (the attention
+ * pipeline without V: a log-sum-exp pass, then the energy pass); other cases
+ * on CUDA cores in float32.  Both sum in fixed orders, so repeated calls give
+ * bitwise identical energies. */
 calibatt_status calibatt_block_energy(const void* q, const void* k,
                                       const calibatt_shape* shape, int32_t block,
                                       float softmax_scale, float* energy, void* workspace,

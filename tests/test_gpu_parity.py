@@ -294,9 +294,10 @@ def _energy(C, q, k, block):
     return e
 
 
-@pytest.mark.parametrize("dtype,n,block,d,std", [("fp32", 256, 64, 64, 1.0), ("bf16", 300, 128, 128, 1.0),
+@pytest.mark.parametrize("dtype,n,block,d,std", [("fp32", 256, 64, 64, 1.0), ("bf16", 300, 64, 128, 1.0),
                                                   ("fp32", 500, 64, 128, 0.3)])
 def test_block_energy(C, dtype, n, block, d, std):
+    """CUDA-core energy path (float32, or bf16 with 64-token blocks)."""
     q, k, _ = W.make_qkv(20, 1, n, 2, d, dtype, std, "cuda")
     e = _energy(C, q, k, block)
     ref = O.block_energy_bnhd(_np(q), _np(k), block)
@@ -305,6 +306,21 @@ def test_block_energy(C, dtype, n, block, d, std):
     np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-5)
     e2 = _energy(C, q, k, block)
     assert torch.equal(e, e2), "energies are not bitwise repeatable"
+
+
+@pytest.mark.parametrize("b,n,h,d,std", [(1, 300, 2, 128, 1.0), (2, 2000, 3, 128, 0.5), (1, 1100, 2, 64, 2.0)])
+def test_block_energy_tensor_core(C, b, n, h, d, std):
+    """bf16 with 128-token blocks runs on the tensor cores (LSE pass + energy
+    pass): energies within 1e-5 of the oracle (scores accumulate in float32
+    on the tensor core, exponentials are the MUFU's), rows sum to one,
+    bitwise repeatable; ragged last blocks on both axes."""
+    q, k, _ = W.make_qkv(22, b, n, h, d, "bf16", std, "cuda")
+    e = _energy(C, q, k, 128)
+    ref = O.block_energy_bnhd(_np(q), _np(k), 128)
+    got = e.cpu().numpy().astype(np.float64)
+    assert np.abs(got - ref).max() < 1e-5, np.abs(got - ref).max()
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-4)
+    assert torch.equal(e, _energy(C, q, k, 128)), "energies are not bitwise repeatable"
 
 
 def test_select_blocks_bit_exact_on_identical_energies(C):
