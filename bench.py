@@ -134,11 +134,14 @@ def aggregate_tflops(flop_per_rank, world, ms):
     return world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
+DICT_BITMAP = False  # --dict-format bitmap
+
+
 def build_dict(C, masks, heads, nb, block, geometry=None):
     """One-layer dictionary; with geometry = (frames, rows, cols, anchors) the
     dual path of the layer runs as one launch."""
     rp, ci, rep_arr = C.masks_to_layer_csr(masks, heads, nb)
-    d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, ci.size))
+    d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, ci.size), bitmap=DICT_BITMAP)
     if geometry is not None:
         d.set_anchor_geometry(*geometry)
     d.set_layer(0, 0, rp, ci, rep_arr)
@@ -298,7 +301,7 @@ def run_sweep(args, C, torch, stream, pk):
     T, L, H, nb = args.sweep_steps, args.sweep_layers, wl.heads, wl.num_blocks
     t_build = time.time()
     nnz = sum(W.sweep_record_blocks(wl, t, l, h, T) for t in range(T) for l in range(L) for h in range(H))
-    dct = C.MaskDictionary(T, L, H, nb, nb, wl.block, nnz)
+    dct = C.MaskDictionary(T, L, H, nb, nb, wl.block, nnz, bitmap=DICT_BITMAP)
     dct.set_anchor_geometry(wl.frames, wl.rows, wl.cols, wl.anchors)
     for t in range(T):
         for l in range(L):
@@ -368,6 +371,7 @@ def run_sweep(args, C, torch, stream, pk):
         "config": {"workload": "wan2.1-14b-720p schedule sweep, dual path (block-sparse + anchor heads)",
                    "timesteps": T, "layers": L, "heads": H, "repetitive_heads_per_call": W.SWEEP_REPETITIVE,
                    "anchors": list(wl.anchors), "density": "0.60 -> 0.20 over the timesteps",
+                   "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
                    "inputs": "fresh seeded Q/K/V per call (2.32 GB > L2)", "parallelism": "replicas x1"},
         "pct_of_peak": value / pk["bf16_tflops"],
         "clocks": clk.summary(),
@@ -397,6 +401,8 @@ def main():
     ap.add_argument("--workload", default="720p", choices=["720p", "sweep"],
                     help="sweep: the mask-dictionary schedule sweep (one dual-path 720p call per "
                          "timestep and layer), reported as aggregate time against the dense path")
+    ap.add_argument("--dict-format", default="lists", choices=["lists", "bitmap"],
+                    help="mask dictionary storage: 2-byte index lists, or one bit per block pair")
     ap.add_argument("--sweep-steps", type=int, default=W.SWEEP_STEPS)
     ap.add_argument("--sweep-layers", type=int, default=W.SWEEP_LAYERS)
     ap.add_argument("--epilogue-probe", action="store_true",
@@ -406,6 +412,8 @@ def main():
                     help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    global DICT_BITMAP
+    DICT_BITMAP = args.dict_format == "bitmap"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -562,6 +570,7 @@ def main():
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "wan2.1-14b-720p self-attention, block-sparse path", "batch": 1,
+                       "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
                        "heads": wl.heads, "head_dim": wl.head_dim, "seq_len": wl.seq_len, "block": wl.block,
                        "density": round(density, 4), "retained_tiles": tiles,
                        "l2": "inputs 2.32 GB > 126 MB L2, no flush", "parallelism": f"replicas x{world}"},

@@ -60,6 +60,7 @@ SIGNATURES = {
     "calibatt_lpt_schedule": (_i32, [_i32, _vp, _i32, _vp, _vp, _P(_i64)]),
     "calibatt_dict_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P(_vp)]),
     "calibatt_dict_set_layer": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
+    "calibatt_dict_create_bitmap": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _P(_vp)]),
     "calibatt_dict_set_anchor_geometry": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32]),
     "calibatt_spatial_similarity": (_i32, [_vp, _vp, _P(Shape), _i32, _i32, _i32, _vp, _i32, _f32, _vp, _vp,
                                            ctypes.c_size_t, _vp]),
@@ -204,10 +205,16 @@ def device_status(stream=None, clear=True) -> int:
 class MaskDictionary:
     """Owns a calibatt_dict (per (t, l, h) skip lists and repetitive flags on the GPU)."""
 
-    def __init__(self, T, L, H, nq, nk, block, nnz_capacity, num_ctas=0):
+    def __init__(self, T, L, H, nq, nk, block, nnz_capacity=0, num_ctas=0, bitmap=False):
+        """bitmap=True stores one bit per (query block, key block) per record
+        (calibatt_dict_create_bitmap) instead of index lists."""
         self.T, self.L, self.H, self.nq, self.nk, self.block = T, L, H, nq, nk, block
         h = ctypes.c_void_p(None)
-        check(LIB.calibatt_dict_create(T, L, H, nq, nk, block, int(nnz_capacity), int(num_ctas), ctypes.byref(h)))
+        if bitmap:
+            check(LIB.calibatt_dict_create_bitmap(T, L, H, nq, nk, block, int(num_ctas), ctypes.byref(h)))
+        else:
+            check(LIB.calibatt_dict_create(T, L, H, nq, nk, block, int(nnz_capacity), int(num_ctas),
+                                           ctypes.byref(h)))
         self.handle = h
 
     def set_layer(self, t, l, row_ptr, col_idx, repetitive=None):

@@ -309,6 +309,11 @@ struct calibatt_dict {
   std::vector<int64_t> retained;    // [T*L]
   // Anchor geometry of the dual path (calibatt_dict_set_anchor_geometry) and
   // the joint sparse + anchor schedules built with it, one per layer.
+  // Bitmap format (calibatt_dict_create_bitmap): one bit per (query block,
+  // key block) per record instead of index lists.
+  bool bitmap = false;
+  int32_t words = 0;
+  uint32_t* d_bitmap = nullptr;
   bool has_geom = false;
   int32_t g_frames = 0, g_rows = 0, g_cols = 0, g_tiles = 0;
   std::vector<int32_t> g_anchors;
@@ -335,6 +340,8 @@ struct calibatt_dict {
     s.items = d_items + ly * H * nq;
     s.cta_ptr = d_cta_ptr + ly * (G + 1);
     s.nq = nq;
+    s.bitmap = bitmap ? d_bitmap + ly * H * nq * static_cast<int64_t>(words) : nullptr;
+    s.words = words;
     return s;
   }
 
@@ -346,6 +353,8 @@ struct calibatt_dict {
     cudaFree(d_cta_ptr);
     cudaFree(d_fitems);
     cudaFree(d_fcta_ptr);
+    cudaFree(d_bitmap);
+    d_bitmap = nullptr;
     d_fitems = nullptr;
     d_fcta_ptr = nullptr;
     d_row_ptr = nullptr;
@@ -399,6 +408,8 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
     return CALIBATT_OK;
   }
   // CUDA-core path, heads in chunks of kMaxHeadsPerCall.
+  if (d->bitmap)
+    return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries run on the tensor-core path only (bf16, block 128)");
   std::vector<int16_t> heads;
   for (int h = 0; h < d->H; ++h)
     if (!d->rep[ly * d->H + h]) heads.push_back(static_cast<int16_t>(h));
@@ -670,6 +681,54 @@ calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq
   return CALIBATT_OK;
 }
 
+calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk,
+                                            int32_t block, int32_t num_ctas, calibatt_dict** out) {
+  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1)
+    return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1");
+  if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
+  if (nq > calibatt::kMaxBitmapBlocks)
+    return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries hold at most %d blocks per row", calibatt::kMaxBitmapBlocks);
+  if (H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "H must be <= 65535");
+  calibatt_status st = check_block(block);
+  if (st != CALIBATT_OK) return st;
+  int G = num_ctas;
+  if (G <= 0) G = device_sm_count();
+  if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+  auto* d = new calibatt_dict();
+  d->T = T;
+  d->L = L;
+  d->H = H;
+  d->nq = nq;
+  d->nk = nk;
+  d->block = block;
+  d->G = G;
+  d->bitmap = true;
+  d->words = (nk + 31) / 32;
+  cudaGetDevice(&d->device);
+  const int64_t layers = static_cast<int64_t>(T) * L;
+  const size_t b_bm = sizeof(uint32_t) * layers * H * nq * d->words;
+  const size_t b_it = sizeof(uint32_t) * layers * H * nq;
+  const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
+  cudaError_t e = cudaMalloc(&d->d_bitmap, b_bm);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
+  if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+  if (e != cudaSuccess) {
+    d->release();
+    delete d;
+    return cuda_fail(e, "bitmap dictionary allocation");
+  }
+  d->device_bytes = static_cast<int64_t>(b_bm + b_it + b_cta);
+  d->layer_set.assign(layers, 0);
+  d->rep.assign(layers * H, 0);
+  d->n_sparse.assign(layers, 0);
+  d->n_rep.assign(layers, 0);
+  d->retained.assign(layers, 0);
+  *out = d;
+  return CALIBATT_OK;
+}
+
 calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, const int32_t* row_ptr,
                                         const int32_t* col_idx, const uint8_t* repetitive) {
   if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
@@ -691,11 +750,23 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     head_off[h + 1] = head_off[h] + rp[nq];
   }
   const int64_t nnz = head_off[H];
-  if (d->nnz_used + nnz > d->nnz_cap)
+  if (!d->bitmap && d->nnz_used + nnz > d->nnz_cap)
     return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld)",
                 (long long)d->nnz_used, (long long)nnz, (long long)d->nnz_cap);
-  std::vector<uint16_t> col16(nnz);
-  for (int64_t i = 0; i < nnz; ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
+  std::vector<uint16_t> col16(d->bitmap ? 0 : nnz);
+  for (size_t i = 0; i < col16.size(); ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
+  std::vector<uint32_t> bits;
+  if (d->bitmap) {
+    bits.assign(static_cast<size_t>(H) * nq * d->words, 0u);
+    for (int h = 0; h < H; ++h) {
+      const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+      for (int r = 0; r < nq; ++r)
+        for (int32_t x = rp[r]; x < rp[r + 1]; ++x) {
+          const int32_t c = col_idx[head_off[h] + x];
+          bits[(static_cast<size_t>(h) * nq + r) * d->words + (c >> 5)] |= 1u << (c & 31);
+        }
+    }
+  }
   std::vector<int64_t> col_base(H);
   for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + head_off[h];
   // Work items of the sparse heads and their LPT schedule over the grid.
@@ -770,11 +841,18 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
   cudaGetDevice(&prev);
   if (prev != d->device) cudaSetDevice(d->device);
   cudaError_t e = cudaSuccess;
-  if (nnz > 0) e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess)
-    e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess)
-    e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
+  if (d->bitmap) {
+    e = cudaMemcpy(d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words), bits.data(),
+                   sizeof(uint32_t) * bits.size(), cudaMemcpyHostToDevice);
+  } else {
+    if (nnz > 0)
+      e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1),
+                     cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess && !sched.empty())
     e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess)

@@ -154,7 +154,10 @@ struct Layout {
   static constexpr int kXchg = kMisc + 16;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
   // {m bits, stream ordinal + 1} [2 streams][128 rows], 8-byte slots
   static constexpr int kMSlot = kXchg + 2 * 2 * 2 * 128 * 4;
-  static constexpr int kUsed = kMSlot + 2 * 128 * 8;
+  // uint16 lists of kept key blocks decoded from bitmap rows, one per producer
+  static constexpr int kListBytes = kMaxBitmapBlocks * 2;
+  static constexpr int kList = kMSlot + 2 * 128 * 8;
+  static constexpr int kUsed = kList + 2 * kListBytes;
   // +1024 for aligning the base; at least 120 KB so only one CTA fits per SM
   // (each CTA holds all 512 tensor-memory columns).
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
@@ -163,7 +166,8 @@ struct Layout {
 struct Item {
   int b, h, tile;            // batch, head, query block (sparse) or anchor tile
   int n;                     // key blocks to visit
-  const uint16_t* cols;      // retained key blocks (sparse), nullptr = 0..n-1
+  const uint16_t* cols;      // retained key blocks (sparse lists), nullptr = bits or 0..n-1
+  const uint32_t* bits;      // the row's bitmap (bitmap dictionaries), else nullptr
   bool ragged_last;          // last visited key block is the partial one
   bool anchor;               // anchor-row tile (gathered queries, broadcast epilogue)
 };
@@ -202,6 +206,7 @@ struct Cursor {
           it.tile = idx % p.nb;
           it.n = p.nb;
           it.cols = nullptr;
+          it.bits = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
           idx += step;
           return true;
@@ -218,16 +223,35 @@ struct Cursor {
           }
           it.n = p.nb;
           it.cols = nullptr;
+          it.bits = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
         } else {
           it.anchor = false;
           it.h = static_cast<int>(MODE == kModeFused ? (w >> 16) & 0x7FFFu : w >> 16);
           it.tile = static_cast<int>(w & 0xFFFFu);
-          const int32_t* rp = p.sched.row_ptr + static_cast<int64_t>(it.h) * (p.sched.nq + 1);
-          const int s0 = rp[it.tile];
-          it.n = rp[it.tile + 1] - s0;
-          it.cols = p.sched.col + p.sched.col_base[it.h] + s0;
-          it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
+          if (p.sched.bitmap != nullptr) {
+            const uint32_t* bm =
+                p.sched.bitmap + (static_cast<int64_t>(it.h) * p.sched.nq + it.tile) * p.sched.words;
+            // every role calls next() with its whole warp: lane x counts word x
+            const int lane = threadIdx.x & 31;
+            int cnt = 0;
+            for (int w0 = 0; w0 < p.sched.words; w0 += 32) {
+              const int x = w0 + lane;
+              cnt += __reduce_add_sync(0xFFFFFFFFu, x < p.sched.words ? __popc(bm[x]) : 0);
+            }
+            it.n = cnt;
+            it.cols = nullptr;
+            it.bits = bm;
+            const int last = p.nb - 1;
+            it.ragged_last = cnt > 0 && (p.seq_len % 128) != 0 && ((bm[last >> 5] >> (last & 31)) & 1u);
+          } else {
+            const int32_t* rp = p.sched.row_ptr + static_cast<int64_t>(it.h) * (p.sched.nq + 1);
+            const int s0 = rp[it.tile];
+            it.n = rp[it.tile + 1] - s0;
+            it.cols = p.sched.col + p.sched.col_base[it.h] + s0;
+            it.bits = nullptr;
+            it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
+          }
         }
         idx += step;
         return true;
@@ -268,7 +292,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 // Q/K producer (V == false) and V producer (V == true) walk the same items and
 // key blocks; each lets its own in-flight bulk copies land before exiting.
 template <int HD, int MODE, bool V>
-__device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W, int lane) {
+__device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, const Waiter& W, int lane) {
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr int kStages = V ? kVStages : kKStages;
@@ -333,11 +357,38 @@ __device__ void producer_role(const TcParams& p, uint32_t base, const Waiter& W,
       }
       ++q_items;  // every item completes one phase of q_full, whichever way its Q came
     }
+    const uint16_t* cols = it.cols;
+    if (it.bits != nullptr) {
+      // Bitmap row -> this producer's list of kept key blocks, ascending:
+      // lane x takes word x of each 32-word stretch, a prefix sum of the
+      // words' bit counts places its indices.
+      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
+      int offset = 0;
+      for (int w0 = 0; w0 < p.sched.words; w0 += 32) {
+        const int x = w0 + lane;
+        uint32_t word = x < p.sched.words ? it.bits[x] : 0u;
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        int pos = offset + incl - c;
+        while (word) {
+          list[pos++] = static_cast<uint16_t>(x * 32 + __ffs(word) - 1);
+          word &= word - 1u;
+        }
+        offset += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      __syncwarp();
+      cols = list;
+    }
     uint32_t my_col = 0;
     for (int j = 0; j < it.n; ++j) {
       if ((j & 31) == 0) {
         const int jj = j + lane;
-        my_col = it.cols == nullptr ? static_cast<uint32_t>(jj) : (jj < it.n ? it.cols[jj] : 0u);
+        my_col = cols == nullptr ? static_cast<uint32_t>(jj) : (jj < it.n ? cols[jj] : 0u);
       }
       const int c = static_cast<int>(__shfl_sync(0xFFFFFFFFu, my_col, j & 31));
       const uint32_t slot = kv % kStages, use = kv / kStages;
@@ -896,9 +947,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   if (warp >= 8) {
     reg_dealloc<kOtherRegs>();
     if (warp == kProducerWarp) {
-      producer_role<HD, MODE, false>(p, base, W, lane);
+      producer_role<HD, MODE, false>(p, base, gbase, W, lane);
     } else if (warp == kVProducerWarp) {
-      producer_role<HD, MODE, true>(p, base, W, lane);
+      producer_role<HD, MODE, true>(p, base, gbase, W, lane);
     } else if (warp == kMmaWarp) {
       mma_s_role<HD, MODE>(p, base, tmem, W, lane);
     } else if (warp == kPvWarp) {

@@ -20,7 +20,14 @@ struct LayerSchedule {
   const uint32_t* items;    // work items grouped by CTA
   const int32_t* cta_ptr;   // [grid + 1], CTA c runs items[cta_ptr[c] .. cta_ptr[c+1])
   int32_t nq;
+  // Bitmap dictionaries instead: bit c of row r of head h says key block c is
+  // kept, words 32-bit words per row, [H][nq][words]; row_ptr/col unused.
+  const uint32_t* bitmap;
+  int32_t words;
 };
+// Longest skip list a bitmap dictionary may hold per row (the producers decode
+// each row into a shared-memory list of this many 16-bit indices).
+constexpr int kMaxBitmapBlocks = 2048;
 
 // Frame geometry of the anchor path.  Token = (f * rows + row) * cols + col.
 // Packed anchor query p (0 <= p < anchor_tokens) is

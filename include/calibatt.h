@@ -134,6 +134,19 @@ calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq
                                      int32_t block, int64_t nnz_capacity, int32_t num_ctas,
                                      calibatt_dict** out);
 
+/* Like calibatt_dict_create, but each record stores one bit per (query
+ * block, key block) instead of a 2-byte index per kept block: fixed
+ * T*L*H*nq*ceil(nk/32)*4 bytes whatever the density (the 720p schedule of
+ * 50 x 40 x 40 records: 3.6 GB instead of about 17 GB of index lists at
+ * 20-60% density).  The tensor-core kernels decode each row into a list of
+ * kept blocks in shared memory; results equal those of the list format.
+ * Bitmap dictionaries serve the tensor-core path only (bf16, block 128;
+ * otherwise the attention calls return CALIBATT_ERR_UNSUPPORTED) and hold
+ * nq <= 2048.  All other dictionary functions apply unchanged. */
+calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int32_t nq,
+                                            int32_t nk, int32_t block, int32_t num_ctas,
+                                            calibatt_dict** out);
+
 /* Fills the records of layer l at timestep t for all H heads (each layer
  * may be set once).  Host inputs:
  *   row_ptr int32[H][nq + 1]: each head's CSR row pointer, starting at 0;

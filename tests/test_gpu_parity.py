@@ -598,3 +598,68 @@ def test_spatial_similarity_720p_sampled_and_flags(C):
     assert np.abs(mean.cpu().numpy() - ref_mean).max() <= 1e-6
     assert np.array_equal(flags.cpu().numpy().astype(bool), ref_flags)
     assert ref_flags.any() and not ref_flags.all()
+
+
+# ------------------------------------------------------------ bitmap dictionaries
+
+@pytest.mark.parametrize("d,n,h", [(128, 1000, 3), (64, 4100, 2)])  # ragged; 33 blocks -> 2 words per row
+def test_bitmap_dictionary_matches_lists(C, d, n, h):
+    """A bitmap dictionary gives bitwise the results of the index-list one:
+    sparse call with LSE (an empty row included) and the fused dual path."""
+    q, k, v = W.make_qkv(61, 1, n, h, d, "bf16", 1.0, "cuda")
+    nb = O.num_blocks(n, 128)
+    masks = _random_masks(62, h, nb, 0.4, empty_row_head=1)
+    masks[0][:, nb - 1] = True                                  # ragged last key block kept by every row
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    outs, lses = [], []
+    for bitmap in (False, True):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((1, h, n), float("nan"), device="cuda")
+        with C.MaskDictionary(1, 1, h, nb, nb, 128, ci.size, bitmap=bitmap) as dct:
+            dct.set_layer(0, 0, rp, ci, rep)
+            C.calibatt_block_sparse_attn(q, k, v, out, dct, 0, 0, 128, lse=lse)
+            _check_status(C)
+            assert dct.layer_info(0, 0)["retained_tiles"] == sum(int(m.sum()) for m in masks)
+        outs.append(out)
+        lses.append(lse)
+    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(lses[0], lses[1])
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, 128, seq_len=n)
+    _assert_close(_np(outs[1]), ref, "bf16")
+    # fused dual path over a bitmap dictionary
+    frames, rows, cols = (2, 5, n // 10) if n % 10 == 0 else (1, 41, 100)
+    assert frames * rows * cols == n
+    dmasks = [None if i == h - 1 else masks[i] for i in range(h)]
+    rp2, ci2, rep2 = C.masks_to_layer_csr(dmasks, h, nb)
+    res = []
+    for bitmap in (False, True):
+        out = torch.full_like(q, float("nan"))
+        with C.MaskDictionary(1, 1, h, nb, nb, 128, max(1, ci2.size), bitmap=bitmap) as dct:
+            dct.set_anchor_geometry(frames, rows, cols, (1, 3) if rows == 5 else (10, 30))
+            dct.set_layer(0, 0, rp2, ci2, rep2)
+            C.calibatt_dual_path_attn(q, k, v, out, dct, 0, 0, frames, rows, cols, (1, 3) if rows == 5 else (10, 30))
+            _check_status(C)
+        res.append(out)
+    assert torch.equal(res[0], res[1])
+
+
+def test_bitmap_dictionary_size_and_rules(C):
+    """Device bytes of the two formats at the 720p layer, and the bitmap
+    format's limits."""
+    wl = W.WORKLOADS["720p"]
+    nb = wl.num_blocks
+    masks, _ = W.workload_masks(wl, heads=range(4))
+    rp, ci, rep = C.masks_to_layer_csr([masks[i] for i in range(4)], 4, nb)
+    with C.MaskDictionary(2, 2, 4, nb, nb, 128, 4 * ci.size) as dl, \
+            C.MaskDictionary(2, 2, 4, nb, nb, 128, bitmap=True) as db:
+        bl, bb = dl.info()["device_bytes"], db.info()["device_bytes"]
+        assert bb == 4 * 4 * nb * ((nb + 31) // 32) * 4 + 4 * 4 * nb * 4 + 4 * (db.info()["num_ctas"] + 1) * 4
+        db.set_layer(1, 1, rp, ci, rep)
+        assert db.info()["nnz"] == ci.size
+        assert bb < bl
+        # CUDA-core path (fp32) cannot read a bitmap dictionary
+        q = torch.zeros((1, wl.seq_len, 4, 128), dtype=torch.float32, device="cuda")
+        with pytest.raises(C.CalibattError):
+            C.calibatt_block_sparse_attn(q, q, q, q, db, 1, 1, 128)
+    with pytest.raises(C.CalibattError):
+        C.MaskDictionary(1, 1, 1, 4096, 4096, 128, bitmap=True)    # more than 2048 blocks per row
