@@ -166,12 +166,16 @@ struct Layout {
 struct Item {
   int b, h, tile;            // batch, head, query block (sparse) or anchor tile
   int n;                     // key blocks to visit
-  const uint16_t* cols;      // retained key blocks (sparse lists), nullptr = bits or 0..n-1
-  const uint32_t* bits;      // the row's bitmap (bitmap dictionaries), else nullptr
+  const uint16_t* cols;      // retained key blocks (index lists), nullptr = bitmap row or 0..n-1
   bool ragged_last;          // last visited key block is the partial one
   bool anchor;               // anchor-row tile (gathered queries, broadcast epilogue)
 };
 
+
+// Row (head h, query block r) of a bitmap dictionary layer.
+__device__ __forceinline__ const uint32_t* bitmap_row(const TcParams& p, int h, int r) {
+  return p.sched.bitmap + (static_cast<int64_t>(h) * p.sched.nq + r) * p.sched.words;
+}
 
 // Walks this CTA's work items in the same order in every role.
 template <int MODE>
@@ -206,7 +210,6 @@ struct Cursor {
           it.tile = idx % p.nb;
           it.n = p.nb;
           it.cols = nullptr;
-          it.bits = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
           idx += step;
           return true;
@@ -223,15 +226,13 @@ struct Cursor {
           }
           it.n = p.nb;
           it.cols = nullptr;
-          it.bits = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
         } else {
           it.anchor = false;
           it.h = static_cast<int>(MODE == kModeFused ? (w >> 16) & 0x7FFFu : w >> 16);
           it.tile = static_cast<int>(w & 0xFFFFu);
           if (p.sched.bitmap != nullptr) {
-            const uint32_t* bm =
-                p.sched.bitmap + (static_cast<int64_t>(it.h) * p.sched.nq + it.tile) * p.sched.words;
+            const uint32_t* bm = bitmap_row(p, it.h, it.tile);
             // every role calls next() with its whole warp: lane x counts word x
             const int lane = threadIdx.x & 31;
             int cnt = 0;
@@ -241,7 +242,6 @@ struct Cursor {
             }
             it.n = cnt;
             it.cols = nullptr;
-            it.bits = bm;
             const int last = p.nb - 1;
             it.ragged_last = cnt > 0 && (p.seq_len % 128) != 0 && ((bm[last >> 5] >> (last & 31)) & 1u);
           } else {
@@ -249,7 +249,6 @@ struct Cursor {
             const int s0 = rp[it.tile];
             it.n = rp[it.tile + 1] - s0;
             it.cols = p.sched.col + p.sched.col_base[it.h] + s0;
-            it.bits = nullptr;
             it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
           }
         }
@@ -358,7 +357,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
       ++q_items;  // every item completes one phase of q_full, whichever way its Q came
     }
     const uint16_t* cols = it.cols;
-    if (it.bits != nullptr) {
+    if (p.sched.bitmap != nullptr && !it.anchor) {
       // Bitmap row -> this producer's list of kept key blocks, ascending:
       // lane x takes word x of each 32-word stretch, a prefix sum of the
       // words' bit counts places its indices.
@@ -366,7 +365,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
       int offset = 0;
       for (int w0 = 0; w0 < p.sched.words; w0 += 32) {
         const int x = w0 + lane;
-        uint32_t word = x < p.sched.words ? it.bits[x] : 0u;
+        uint32_t word = x < p.sched.words ? bitmap_row(p, it.h, it.tile)[x] : 0u;
         const int c = __popc(word);
         int incl = c;
 #pragma unroll
