@@ -539,47 +539,32 @@ def main():
             raise RuntimeError("device wait timed out during the extra legs")
 
     # -------------------------------------------------------- end to end (host buffers)
-    # Every step copies its Q, K, V from pinned host memory to the device,
-    # runs the attention call and copies O back to pinned host memory.  Steps
-    # are pipelined on three streams with two device buffer sets: the copy-in
-    # of step i + 1 and the copy-out of step i - 1 overlap the attention of
-    # step i (buffer reuse is ordered by events).
+    # Every step is one calibatt_block_sparse_attn_host call: its Q, K, V are
+    # copied from pinned host memory into a device buffer set, the attention
+    # runs, and O is copied back to pinned host memory, in stream order.
+    # Consecutive steps alternate between two streams and two buffer sets, so
+    # the copies of one step overlap the attention of the neighbouring ones.
     e2e = None
     if not args.no_extras:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         hos = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(2)]
-        dsets = [[torch.empty_like(q) for _ in range(3)] for _ in range(2)]
-        douts = [torch.empty_like(o) for _ in range(2)]
-        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        dsets = [[torch.empty_like(q) for _ in range(4)] for _ in range(2)]
+        streams = [torch.cuda.Stream(), torch.cuda.Stream()]
         e2e_steps = max(4, args.steps // 2)
 
         def run_pipeline(n_steps):
-            ev_in = [torch.cuda.Event() for _ in range(n_steps)]
-            ev_cmp = [torch.cuda.Event() for _ in range(n_steps)]
-            ev_out = [torch.cuda.Event() for _ in range(n_steps)]
             t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            t0.record(s_in)
+            t0.record(streams[0])
+            streams[1].wait_event(t0)
             for i in range(n_steps):
                 b = i % 2
-                with torch.cuda.stream(s_in):
-                    if i >= 2:
-                        s_in.wait_event(ev_cmp[i - 2])       # the attention of step i - 2 read this set
-                    for dst, src in zip(dsets[b], (hq, hk, hv)):
-                        dst.copy_(src, non_blocking=True)
-                    ev_in[i].record(s_in)
-                with torch.cuda.stream(s_cmp):
-                    s_cmp.wait_event(ev_in[i])
-                    if i >= 2:
-                        s_cmp.wait_event(ev_out[i - 2])      # step i - 2's output has left this buffer
-                    C.calibatt_block_sparse_attn(dsets[b][0], dsets[b][1], dsets[b][2], douts[b], d_sparse, 0, 0,
-                                                 wl.block, stream=s_cmp)
-                    ev_cmp[i].record(s_cmp)
-                with torch.cuda.stream(s_out):
-                    s_out.wait_event(ev_cmp[i])
-                    hos[b].copy_(douts[b], non_blocking=True)
-                    ev_out[i].record(s_out)
-            s_out.wait_event(ev_in[n_steps - 1])
-            t1.record(s_out)
+                dq, dk, dv, do = dsets[b]
+                C.calibatt_block_sparse_attn_host(hq, hk, hv, hos[b], dq, dk, dv, do, d_sparse, 0, 0, wl.block,
+                                                  stream=streams[b])
+            end1 = torch.cuda.Event()
+            end1.record(streams[1])
+            streams[0].wait_event(end1)
+            t1.record(streams[0])
             torch.cuda.synchronize()
             return t0.elapsed_time(t1)
 
@@ -588,10 +573,10 @@ def main():
         nbytes = 3 * q.numel() * q.element_size()
         e2e = {"value": aggregate_tflops(flop, world, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": o.numel() * o.element_size(),
-               "steps": e2e_steps, "pipelined": "copy-in, attention and copy-out of consecutive steps overlap"}
+               "steps": e2e_steps, "api": "calibatt_block_sparse_attn_host, steps alternating over two streams"}
         if C.device_status() != 0:
             raise RuntimeError("device wait timed out during the end-to-end leg")
-        del hq, hk, hv, hos, dsets, douts
+        del hq, hk, hv, hos, dsets
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

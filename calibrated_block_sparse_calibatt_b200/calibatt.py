@@ -69,6 +69,8 @@ SIGNATURES = {
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
     "calibatt_block_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32, _i32, _f32, _vp, _vp]),
+    "calibatt_block_sparse_attn_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32,
+                                               _i32, _f32, _vp, _vp]),
     "calibatt_anchor_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _i32, _i32, _i32, _vp, _i32, _vp,
                                     _i32, _f32, _vp]),
     "calibatt_dual_path_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32, _i32, _i32, _i32, _i32,
@@ -276,6 +278,16 @@ def calibatt_block_sparse_attn(q, k, v, o, d: MaskDictionary, t=0, l=0, block=12
     shape = shape_of(q)
     check(LIB.calibatt_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shape), block,
                                          d.handle, t, l, float(softmax_scale), _ptr(lse), _stream(stream)))
+
+
+def calibatt_block_sparse_attn_host(hq, hk, hv, ho, q, k, v, o, d: MaskDictionary, t, l, block=128,
+                                    softmax_scale=0.0, lse=None, stream=None):
+    """Copies host hq/hk/hv into device q/k/v, runs the block-sparse attention
+    into o and copies o to host ho, all enqueued on `stream` (no sync)."""
+    shape = shape_of(q)
+    check(LIB.calibatt_block_sparse_attn_host(_ptr(hq), _ptr(hk), _ptr(hv), _ptr(ho), _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(o), ctypes.byref(shape), block, d.handle, t, l,
+                                              float(softmax_scale), _ptr(lse), _stream(stream)))
 
 
 def calibatt_anchor_attn(q, k, v, o, frames, rows, cols, anchor_rows, head_ids, block=128, softmax_scale=0.0,

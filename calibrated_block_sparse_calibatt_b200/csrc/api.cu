@@ -972,6 +972,35 @@ calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const v
   return launch_sparse(q, k, v, o, *shape, block, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
 }
 
+calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* k_host, const void* v_host,
+                                                void* o_host, void* q, void* k, void* v, void* o,
+                                                const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
+                                                int32_t t, int32_t l, float softmax_scale, float* lse,
+                                                void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if (!q_host || !k_host || !v_host || !o_host)
+    return fail(CALIBATT_ERR_INVALID_ARG, "host buffers must be non-NULL");
+  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+  // bytes from each tensor's base to one past its last element
+  const int64_t elt = shape->dtype == CALIBATT_DTYPE_BF16 ? 2 : 4;
+  const int64_t extent = ((static_cast<int64_t>(shape->batch) - 1) * shape->stride_b +
+                          (static_cast<int64_t>(shape->seq_len) - 1) * shape->stride_n +
+                          (static_cast<int64_t>(shape->heads) - 1) * shape->stride_h + shape->head_dim) * elt;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const void* src[3] = {q_host, k_host, v_host};
+  void* dst[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    cudaError_t e = cudaMemcpyAsync(dst[i], src[i], static_cast<size_t>(extent), cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  }
+  st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
+  if (st != CALIBATT_OK) return st;
+  cudaError_t e = cudaMemcpyAsync(o_host, o, static_cast<size_t>(extent), cudaMemcpyDeviceToHost, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return CALIBATT_OK;
+}
+
 calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
                                      const calibatt_shape* shape, int32_t block, int32_t frames, int32_t rows,
                                      int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,

@@ -214,6 +214,23 @@ calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const v
                                            const calibatt_dict* dict, int32_t t, int32_t l,
                                            float softmax_scale, float* lse, void* stream);
 
+/* End-to-end form of calibatt_block_sparse_attn for inputs in host memory:
+ * enqueues on `stream` the copies of q_host, k_host, v_host into the
+ * caller-owned device buffers q, k, v, the attention (into device o), and the
+ * copy of o into o_host; it does not synchronise.  Host and device tensors
+ * share `shape` (dtype, strides); each copy moves the bytes from the tensor's
+ * base to one past its last element.  Host buffers should be page-locked for
+ * the copies to be asynchronous (they are then ordered on `stream` only);
+ * callers may alternate streams and device buffer sets so that the copies of
+ * one call overlap the attention of another.  Other arguments and errors as
+ * calibatt_block_sparse_attn; a copy failure returns CALIBATT_ERR_CUDA. */
+calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* k_host,
+                                                const void* v_host, void* o_host, void* q,
+                                                void* k, void* v, void* o,
+                                                const calibatt_shape* shape, int32_t block,
+                                                const calibatt_dict* dict, int32_t t, int32_t l,
+                                                float softmax_scale, float* lse, void* stream);
+
 /* Anchor-row attention with broadcast for the given heads (Key Designs 3):
  * only queries of the anchor rows of every frame attend, densely over all N
  * keys and values; every token (f, row, col) takes the output of the anchor

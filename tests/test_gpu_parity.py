@@ -663,3 +663,26 @@ def test_bitmap_dictionary_size_and_rules(C):
             C.calibatt_block_sparse_attn(q, q, q, q, db, 1, 1, 128)
     with pytest.raises(C.CalibattError):
         C.MaskDictionary(1, 1, 1, 4096, 4096, 128, bitmap=True)    # more than 2048 blocks per row
+
+
+def test_host_buffer_entry_point(C):
+    """calibatt_block_sparse_attn_host: host inputs copied in, attention, output
+    copied out, in stream order; equal to the device-buffer call."""
+    n, h, d = 1000, 2, 128
+    q, k, v = W.make_qkv(71, 1, n, h, d, "bf16", 1.0, "cuda")
+    nb = O.num_blocks(n, 128)
+    masks = _random_masks(72, h, nb, 0.5)
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.full_like(q, float("nan"), device="cpu").pin_memory()
+    dq, dk, dv, do = (torch.empty_like(q) for _ in range(4))
+    ref_out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    with C.MaskDictionary(1, 1, h, nb, nb, 128, ci.size) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_block_sparse_attn_host(hq, hk, hv, ho, dq, dk, dv, do, dct, 0, 0, 128, stream=s)
+        s.synchronize()
+        C.calibatt_block_sparse_attn(q, k, v, ref_out, dct, 0, 0, 128)
+        _check_status(C)
+    assert torch.equal(ho, ref_out.cpu())
+    assert torch.equal(dq, q)
