@@ -242,8 +242,11 @@ def test_full_size_sparse_sampled(C, name):
 
 
 def test_full_size_dual_path_sampled(C):
-    """The dual-path 720p layer: every anchor head on sampled rows of two frames,
-    every sparse head on 8 sampled q-blocks, broadcast rows bitwise equal."""
+    """The dual-path 720p layer as ONE fused launch (the dictionary carries the
+    anchor geometry; a bitmap dictionary): every anchor head on sampled rows
+    of two frames, every sparse head on 8 sampled q-blocks, broadcast rows
+    bitwise equal; and bitwise the output of the two-launch path over an
+    index-list dictionary."""
     import _oracle_jobs as J
 
     wl = W.WORKLOADS["720p_dual"]
@@ -252,11 +255,19 @@ def test_full_size_dual_path_sampled(C):
     assert len(rep_heads) == 12
     rp, ci, rep = C.masks_to_layer_csr([masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks)
     out = torch.full_like(q, float("nan"))
-    with C.MaskDictionary(1, 1, wl.heads, wl.num_blocks, wl.num_blocks, wl.block, ci.size) as dct:
+    with C.MaskDictionary(1, 1, wl.heads, wl.num_blocks, wl.num_blocks, wl.block, ci.size, bitmap=True) as dct:
+        dct.set_anchor_geometry(wl.frames, wl.rows, wl.cols, wl.anchors)
         dct.set_layer(0, 0, rp, ci, rep)
         C.calibatt_dual_path_attn(q, k, v, out, dct, 0, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
         _check_status(C)
     assert not torch.isnan(out).any()
+    two = torch.full_like(q, float("nan"))
+    with C.MaskDictionary(1, 1, wl.heads, wl.num_blocks, wl.num_blocks, wl.block, ci.size) as dct:
+        dct.set_layer(0, 0, rp, ci, rep)
+        C.calibatt_dual_path_attn(q, k, v, two, dct, 0, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
+        _check_status(C)
+    assert torch.equal(out, two)
+    del two
     rng = np.random.default_rng(2)
     # anchor heads: rows of two frames, including the last frame's last row
     f_rows = np.concatenate([np.arange(f * wl.tokens_per_frame, (f + 1) * wl.tokens_per_frame)
@@ -407,17 +418,21 @@ def test_fma_exp2_error_bound(C):
     assert (yl >= 0).all() and (yl < 1e-37).all()
 
 
-def test_sweep_records_sampled(C):
+@pytest.mark.parametrize("fmt", ["lists", "bitmap"])
+def test_sweep_records_sampled(C, fmt):
     """Records of the schedule sweep in one dictionary spanning all 50 x 40
-    (timestep, layer) slots: the dual-path call of (t, l) must use that
-    record's masks and anchor heads (checked against the oracle on sampled
-    rows), and retained-tile counts must match the recipe."""
+    (timestep, layer) slots, with the anchor geometry (one fused launch per
+    call): the dual-path call of (t, l) must use that record's masks and
+    anchor heads (checked against the oracle on sampled rows), and
+    retained-tile counts must match the recipe."""
     wl = W.WORKLOADS["720p_sweep"]
     nb = wl.num_blocks
     records = [(0, 0), (25, 17), (49, 39)]
     nnz = sum(W.sweep_record_blocks(wl, t, l, h) for t, l in records for h in range(wl.heads))
     rng = np.random.default_rng(5)
-    with C.MaskDictionary(W.SWEEP_STEPS, W.SWEEP_LAYERS, wl.heads, nb, nb, wl.block, nnz) as dct:
+    with C.MaskDictionary(W.SWEEP_STEPS, W.SWEEP_LAYERS, wl.heads, nb, nb, wl.block, nnz,
+                          bitmap=fmt == "bitmap") as dct:
+        dct.set_anchor_geometry(wl.frames, wl.rows, wl.cols, wl.anchors)
         host = {}
         for t, l in records:
             masks, rep = W.sweep_layer_masks(wl, t, l, "cuda")
