@@ -25,7 +25,8 @@ BUILD = os.path.join(ROOT, "_build")
 # epilogue timers compiled in); never loaded by the product path.
 LIB_TRACE = os.path.join(LIBDIR, "libcalibatt_trace.so")
 
-SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu", "energy_noalloc.cu", "repetition.cu"]
+SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu", "energy_noalloc.cu", "repetition.cu",
+           "diagnostics.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -60,6 +60,7 @@ SIGNATURES = {
     "calibatt_lpt_schedule": (_i32, [_i32, _vp, _i32, _vp, _vp, _P(_i64)]),
     "calibatt_dict_create": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P(_vp)]),
     "calibatt_dict_set_layer": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
+    "calibatt_debug_bounded_wait": (_i32, [_vp]),
     "calibatt_dict_create_bitmap": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _P(_vp)]),
     "calibatt_dict_set_anchor_geometry": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32]),
     "calibatt_spatial_similarity": (_i32, [_vp, _vp, _P(Shape), _i32, _i32, _i32, _vp, _i32, _f32, _vp, _vp,
@@ -192,6 +193,11 @@ def device_sm_count() -> int:
     n = ctypes.c_int32(0)
     check(LIB.calibatt_device_sm_count(ctypes.byref(n)))
     return n.value
+
+
+def debug_bounded_wait(stream=None):
+    """Launches the failure-path check of the bounded waits (see the header)."""
+    check(LIB.calibatt_debug_bounded_wait(_stream(stream)))
 
 
 def device_status(stream=None, clear=True) -> int:

@@ -1241,6 +1241,14 @@ calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, voi
   return CALIBATT_OK;
 }
 
+calibatt_status calibatt_debug_bounded_wait(void* stream) {
+  int32_t* p = status_word_ptr();
+  if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+  cudaError_t e = calibatt::launch_bounded_wait(p, g_timeout_ns.load(), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounded wait launch");
+  return CALIBATT_OK;
+}
+
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear) {
   if (!code) return fail(CALIBATT_ERR_INVALID_ARG, "code is NULL");
   int32_t* p = status_word_ptr();

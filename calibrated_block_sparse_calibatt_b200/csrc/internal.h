@@ -134,6 +134,7 @@ cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts
                              uint8_t* mask, cudaStream_t s);
 
 cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s);
+cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns, cudaStream_t s);
 
 // Records a failure message for calibatt_last_error() on the calling thread.
 void set_last_error(const char* fmt, ...);

@@ -362,6 +362,14 @@ calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_pro
  * Returns CALIBATT_ERR_TIMEOUT when the word is non-zero. */
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);
 
+/* Failure-path check of the bounded waits: launches one warp that waits on
+ * an mbarrier nothing arrives on, through the same bounded wait the kernels
+ * use, with the current calibatt_set_wait_timeout_ms limit.  When the limit
+ * passes it sets the status word (CALIBATT_ERR_TIMEOUT, wait point 15 in the
+ * byte above it) and returns; no fault, no hang, the context stays usable.
+ * Read the result with calibatt_device_status. */
+calibatt_status calibatt_debug_bounded_wait(void* stream);
+
 /* Evaluates, on the device, the FMA-pipe base-2 exponential that the
  * tensor-core softmax uses for part of its probabilities (no counterpart in
  * the paper; exposed so its error bound can be tested): y[i] = 2^x[i] with

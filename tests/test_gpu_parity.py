@@ -701,3 +701,26 @@ def test_host_buffer_entry_point(C):
         _check_status(C)
     assert torch.equal(ho, ref_out.cpu())
     assert torch.equal(dq, q)
+
+
+def test_bounded_wait_runs_out_and_context_survives(C):
+    """A wait that nothing satisfies ends after the configured limit with the
+    timeout status (wait point 15), no fault and no hang; the status clears
+    and the next attention call runs normally."""
+    import time
+    C.set_wait_timeout_ms(50)
+    try:
+        t0 = time.time()
+        C.debug_bounded_wait()
+        code = C.device_status()                       # synchronises, reads and clears
+        assert code & 0xFF == 4 and (code >> 8) == 15, hex(code)
+        assert time.time() - t0 < 5.0
+        assert C.device_status() == 0
+    finally:
+        C.set_wait_timeout_ms(4000)
+    n, h, d = 512, 2, 128
+    q, k, v = W.make_qkv(81, 1, n, h, d, "bf16", 1.0, "cuda")
+    masks = _random_masks(82, h, O.num_blocks(n, 128), 0.5)
+    out, _ = _run_sparse(C, q, k, v, masks, 128)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, 128)
+    _assert_close(_np(out), ref, "bf16")
