@@ -473,12 +473,12 @@ def test_sweep_records_sampled(C, fmt):
 
 # ------------------------------------------------------- fused dual path (one launch)
 
-@pytest.mark.parametrize("d,frames,rows,cols,anchors", [
-    (128, 2, 8, 64, (0, 4)),          # N = 1024: 8 full blocks, 2 anchor tiles per head
-    (128, 3, 9, 40, (1, 4, 7)),       # N = 1080: ragged last block (56 tokens), ragged anchor tile
-    (64, 3, 9, 40, (2, 6)),           # head_dim 64, ties broken to the lower anchor
+@pytest.mark.parametrize("d,frames,rows,cols,anchors,batch", [
+    (128, 2, 8, 64, (0, 4), 1),          # N = 1024: 8 full blocks, 2 anchor tiles per head
+    (128, 3, 9, 40, (1, 4, 7), 2),       # N = 1080: ragged last block (56 tokens), ragged anchor tile; 2 batches
+    (64, 3, 9, 40, (2, 6), 1),           # head_dim 64, ties broken to the lower anchor
 ])
-def test_fused_dual_path(C, d, frames, rows, cols, anchors):
+def test_fused_dual_path(C, d, frames, rows, cols, anchors, batch):
     """A dictionary carrying the anchor geometry runs the dual path in one
     launch over a joint schedule: every row matches the oracle (block-sparse
     heads with their LSE, anchor heads with the broadcast), and the result is
@@ -486,15 +486,15 @@ def test_fused_dual_path(C, d, frames, rows, cols, anchors):
     same way whatever CTA runs it)."""
     n, h, block = frames * rows * cols, 5, 128
     nb = O.num_blocks(n, block)
-    q, k, v = W.make_qkv(21, 1, n, h, d, "bf16", 1.0, "cuda")
+    q, k, v = W.make_qkv(21, batch, n, h, d, "bf16", 1.0, "cuda")
     rep_heads = (1, 3)
     masks = _random_masks(9, h, nb, 0.45)
     masks = [None if i in rep_heads else masks[i] for i in range(h)]
     rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
     fused = torch.full_like(q, float("nan"))
     two = torch.full_like(q, float("nan"))
-    lse_f = torch.full((1, h, n), float("nan"), device="cuda")
-    lse_t = torch.full((1, h, n), float("nan"), device="cuda")
+    lse_f = torch.full((batch, h, n), float("nan"), device="cuda")
+    lse_t = torch.full((batch, h, n), float("nan"), device="cuda")
     with C.MaskDictionary(2, 1, h, nb, nb, block, 2 * max(1, ci.size)) as dg, \
             C.MaskDictionary(1, 1, h, nb, nb, block, max(1, ci.size)) as dp:
         dg.set_anchor_geometry(frames, rows, cols, anchors)
@@ -506,15 +506,16 @@ def test_fused_dual_path(C, d, frames, rows, cols, anchors):
     assert torch.equal(fused, two)
     sparse = [i for i in range(h) if i not in rep_heads]
     assert torch.equal(lse_f[:, sparse], lse_t[:, sparse])
-    qn, kn, vn = _np(q)[0], _np(k)[0], _np(v)[0]
-    got = _np(fused)[0]
-    for i in range(h):
-        if i in rep_heads:
-            ref, _ = O.anchor_attention(qn[:, i], kn[:, i], vn[:, i], frames, rows, cols, anchors)
-        else:
-            ref, ref_lse = O.block_sparse_attention(qn[:, i], kn[:, i], vn[:, i], masks[i], block)
-            np.testing.assert_allclose(lse_f[0, i].cpu().numpy(), ref_lse, atol=2e-2)
-        _assert_close(got[:, i], ref, "bf16")
+    for bb in range(batch):
+        qn, kn, vn = _np(q)[bb], _np(k)[bb], _np(v)[bb]
+        got = _np(fused)[bb]
+        for i in range(h):
+            if i in rep_heads:
+                ref, _ = O.anchor_attention(qn[:, i], kn[:, i], vn[:, i], frames, rows, cols, anchors)
+            else:
+                ref, ref_lse = O.block_sparse_attention(qn[:, i], kn[:, i], vn[:, i], masks[i], block)
+                np.testing.assert_allclose(lse_f[bb, i].cpu().numpy(), ref_lse, atol=2e-2)
+            _assert_close(got[:, i], ref, "bf16")
 
 
 def test_fused_geometry_rules(C):
