@@ -484,17 +484,24 @@ def main():
 
     extras = {}
     if not args.no_extras:
-        # dense all-ones-mask path on the same inputs
-        ones = [np.ones((wl.num_blocks, wl.num_blocks), bool)] * wl.heads
-        d_dense = build_dict(C, ones, wl.heads, wl.num_blocks, wl.block)
-        dense_tiles = d_dense.layer_info(0, 0)["retained_tiles"]
+        # dense path on the same inputs: all-ones skip lists held on the device,
+        # through the direct-CSR call (no dictionary)
+        nbk, hh = wl.num_blocks, wl.heads
+        rp = np.tile((np.arange(nbk + 1) * nbk).astype(np.int32), (hh, 1))
+        items, cta_ptr = C.csr_schedule(rp, list(range(hh)), C.device_sm_count())
+        dense_args = (torch.from_numpy(rp).cuda(), torch.arange(nbk, dtype=torch.int16, device="cuda").repeat(hh * nbk),
+                      torch.arange(hh, dtype=torch.int64, device="cuda") * nbk * nbk, list(range(hh)),
+                      torch.from_numpy(items.view(np.int32)).cuda(), torch.from_numpy(cta_ptr).cuda(),
+                      cta_ptr.size - 1)
+        dense_tiles = q.shape[0] * hh * nbk * nbk
         dense_ms = max_over_ranks(statistics.mean(time_calls(
-            torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d_dense, 0, 0, wl.block, stream=stream),
+            torch, lambda: C.calibatt_block_sparse_attn_csr(q, k, v, o, *dense_args, block=wl.block, stream=stream),
             max(3, args.steps // 4), 2, stream)), dist, "cuda")
-        d_dense.close()
+        del dense_args
         extras["dense"] = {"ms_per_call": dense_ms,
                            "tflops": dense_tiles * FLOP_PER_TILE / (dense_ms * 1e-3) / 1e12,
-                           "speedup_sparse_vs_dense": dense_ms / ms}
+                           "speedup_sparse_vs_dense": dense_ms / ms,
+                           "api": "calibatt_block_sparse_attn_csr, all-ones lists"}
         # dual-path 720p layer: 12 anchor heads + 28 sparse heads
         wd = W.WORKLOADS["720p_dual"]
         dmasks, rep_heads = W.workload_masks(wd)

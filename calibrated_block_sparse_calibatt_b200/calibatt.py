@@ -70,6 +70,9 @@ SIGNATURES = {
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
     "calibatt_block_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32, _i32, _f32, _vp, _vp]),
+    "calibatt_csr_schedule": (_i32, [_i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "calibatt_block_sparse_attn_csr": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _vp, _vp, _vp, _i32, _vp,
+                                              _vp, _i32, _f32, _vp, _vp]),
     "calibatt_block_sparse_attn_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32,
                                                _i32, _f32, _vp, _vp]),
     "calibatt_anchor_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _i32, _i32, _i32, _vp, _i32, _vp,
@@ -179,6 +182,19 @@ def lpt_schedule(cost, n_bins):
     mk = ctypes.c_int64(0)
     check(LIB.calibatt_lpt_schedule(c.size, _ptr(c), n_bins, _ptr(bin_ptr), _ptr(order), ctypes.byref(mk)))
     return bin_ptr, order[:c.size], mk.value
+
+
+def csr_schedule(row_ptr, head_ids, grid):
+    """Host schedule of a direct-CSR call for row_ptr [heads, nq + 1]:
+    (items uint32 [len(head_ids) * nq], cta_ptr int32 [grid + 1])."""
+    rp = _i32_array(row_ptr)
+    heads, nq = rp.shape[0], rp.shape[1] - 1
+    hid = _i32_array(head_ids)
+    items = np.zeros(max(1, hid.size * nq), np.uint32)
+    cta_ptr = np.zeros(grid + 1, np.int32)
+    check(LIB.calibatt_csr_schedule(heads, nq, _ptr(rp), _ptr(hid) if hid.size else None, hid.size, grid,
+                                    _ptr(items), _ptr(cta_ptr)))
+    return items[:hid.size * nq], cta_ptr
 
 
 def calibatt_debug_exp2_fma(x, y, stream=None):
@@ -294,6 +310,20 @@ def calibatt_block_sparse_attn_host(hq, hk, hv, ho, q, k, v, o, d: MaskDictionar
     check(LIB.calibatt_block_sparse_attn_host(_ptr(hq), _ptr(hk), _ptr(hv), _ptr(ho), _ptr(q), _ptr(k), _ptr(v),
                                               _ptr(o), ctypes.byref(shape), block, d.handle, t, l,
                                               float(softmax_scale), _ptr(lse), _stream(stream)))
+
+
+def calibatt_block_sparse_attn_csr(q, k, v, o, row_ptr, col_idx, col_base, head_ids, items=None, cta_ptr=None,
+                                   grid=0, block=128, softmax_scale=0.0, lse=None, stream=None):
+    """Block-sparse attention from device skip lists without a dictionary:
+    row_ptr int32 [heads, nq + 1], col_idx 16-bit, col_base int64 [heads] (all
+    device tensors); items / cta_ptr: the device copy of csr_schedule's result
+    (tensor-core path)."""
+    shape = shape_of(q)
+    hid = _i32_array(head_ids)
+    check(LIB.calibatt_block_sparse_attn_csr(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shape), block,
+                                             _ptr(row_ptr), _ptr(col_idx), _ptr(col_base),
+                                             _ptr(hid) if hid.size else None, hid.size, _ptr(items), _ptr(cta_ptr),
+                                             int(grid), float(softmax_scale), _ptr(lse), _stream(stream)))
 
 
 def calibatt_anchor_attn(q, k, v, o, frames, rows, cols, anchor_rows, head_ids, block=128, softmax_scale=0.0,

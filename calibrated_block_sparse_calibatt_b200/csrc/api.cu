@@ -375,13 +375,13 @@ calibatt_status check_dict_layer(const calibatt_dict* d, int32_t t, int32_t l) {
   return CALIBATT_OK;
 }
 
-calibatt_status launch_sparse(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
-                              int32_t block, const calibatt_dict* d, int32_t t, int32_t l, float softmax_scale,
-                              float* lse, cudaStream_t stream) {
-  const int64_t ly = d->layer(t, l);
-  if (d->n_sparse[ly] == 0) return CALIBATT_OK;
+// Block-sparse attention over one set of skip lists, shared by the dictionary
+// and direct-CSR calls: the tensor-core kernel runs the schedule's items on
+// `grid` persistent CTAs, the CUDA-core kernel walks `heads`.
+calibatt_status run_sparse(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
+                           int32_t block, const LayerSchedule& sch, int32_t grid, const std::vector<int16_t>& heads,
+                           float softmax_scale, float* lse, cudaStream_t stream) {
   const float sl2 = scale_log2_of(softmax_scale, s.head_dim);
-  const LayerSchedule sch = d->schedule(t, l);
   if (s.dtype == CALIBATT_DTYPE_BF16 && block == 128) {
     TcParams p;
     std::memset(&p, 0, sizeof(p));
@@ -403,16 +403,13 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
     p.sched = sch;
     p.status = status_word_ptr();
     p.timeout_ns = g_timeout_ns.load();
-    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeSparse, d->G, stream);
+    cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeSparse, grid, stream);
     if (e != cudaSuccess) return cuda_fail(e, "block-sparse tensor-core launch");
     return CALIBATT_OK;
   }
   // CUDA-core path, heads in chunks of kMaxHeadsPerCall.
-  if (d->bitmap)
+  if (sch.bitmap)
     return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries run on the tensor-core path only (bf16, block 128)");
-  std::vector<int16_t> heads;
-  for (int h = 0; h < d->H; ++h)
-    if (!d->rep[ly * d->H + h]) heads.push_back(static_cast<int16_t>(h));
   for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
     SimtParams p;
     std::memset(&p, 0, sizeof(p));
@@ -433,11 +430,22 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
     const size_t nh = std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0);
     p.n_heads = static_cast<int32_t>(nh);
     for (size_t i = 0; i < nh; ++i) p.head_ids[i] = heads[h0 + i];
-    const int64_t n_items = static_cast<int64_t>(s.batch) * nh * d->nq;
+    const int64_t n_items = static_cast<int64_t>(s.batch) * nh * sch.nq;
     cudaError_t e = calibatt::launch_simt_attn(p, s.head_dim, block, s.dtype, false, static_cast<int>(n_items), stream);
     if (e != cudaSuccess) return cuda_fail(e, "block-sparse CUDA-core launch");
   }
   return CALIBATT_OK;
+}
+
+calibatt_status launch_sparse(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
+                              int32_t block, const calibatt_dict* d, int32_t t, int32_t l, float softmax_scale,
+                              float* lse, cudaStream_t stream) {
+  const int64_t ly = d->layer(t, l);
+  if (d->n_sparse[ly] == 0) return CALIBATT_OK;
+  std::vector<int16_t> heads;
+  for (int h = 0; h < d->H; ++h)
+    if (!d->rep[ly * d->H + h]) heads.push_back(static_cast<int16_t>(h));
+  return run_sparse(q, k, v, o, s, block, d->schedule(t, l), d->G, heads, softmax_scale, lse, stream);
 }
 
 calibatt_status launch_anchor(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
@@ -629,6 +637,45 @@ calibatt_status calibatt_lpt_schedule(int32_t n_items, const int64_t* cost, int3
   for (int32_t i = 0; i < n_items; ++i)
     if (cost[i] < 0) return fail(CALIBATT_ERR_INVALID_ARG, "negative cost at item %d", i);
   lpt(n_items, cost, n_bins, bin_ptr, item_order, makespan);
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* row_ptr, const int32_t* head_ids,
+                                      int32_t n_heads, int32_t grid, uint32_t* items, int32_t* cta_ptr) {
+  if (heads < 1 || heads > 65535 || nq < 1 || nq > 65535)
+    return fail(CALIBATT_ERR_INVALID_ARG, "heads and nq must be in [1, 65535]");
+  if (grid < 1) return fail(CALIBATT_ERR_INVALID_ARG, "grid must be >= 1");
+  if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
+  if (!row_ptr || !cta_ptr || (n_heads > 0 && (!head_ids || !items)))
+    return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+  std::vector<uint8_t> seen(heads, 0);
+  for (int i = 0; i < n_heads; ++i) {
+    const int32_t h = head_ids[i];
+    if (h < 0 || h >= heads) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", h, heads);
+    if (seen[h]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", h);
+    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+    if (rp[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row_ptr[0] != 0", h);
+    for (int r = 0; r < nq; ++r)
+      if (rp[r + 1] < rp[r] || rp[r + 1] - rp[r] > nq)
+        return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row %d has %d blocks", h, r, rp[r + 1] - rp[r]);
+  }
+  // The dictionary's cost model and L2 head groups (calibatt_dict_set_layer).
+  std::vector<uint32_t> all;
+  std::vector<int64_t> cost;
+  std::vector<int32_t> group;
+  const int32_t hpg = heads_per_group(nq);
+  for (int i = 0; i < n_heads; ++i) {
+    const int32_t* rp = row_ptr + static_cast<int64_t>(head_ids[i]) * (nq + 1);
+    for (int r = 0; r < nq; ++r) {
+      all.push_back((static_cast<uint32_t>(head_ids[i]) << 16) | static_cast<uint32_t>(r));
+      cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
+      group.push_back(i / hpg);
+    }
+  }
+  std::vector<int32_t> order(all.size());
+  lpt_grouped(static_cast<int32_t>(all.size()), cost.data(), group.data(), grid, cta_ptr, order.data());
+  for (size_t i = 0; i < all.size(); ++i) items[i] = all[order[i]];
   return CALIBATT_OK;
 }
 
@@ -999,6 +1046,47 @@ calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* 
   cudaError_t e = cudaMemcpyAsync(o_host, o, static_cast<size_t>(extent), cudaMemcpyDeviceToHost, cs);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
   return CALIBATT_OK;
+}
+
+calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, const void* v, void* o,
+                                               const calibatt_shape* shape, int32_t block, const int32_t* row_ptr,
+                                               const uint16_t* col_idx, const int64_t* col_base,
+                                               const int32_t* head_ids, int32_t n_heads, const uint32_t* items,
+                                               const int32_t* cta_ptr, int32_t grid, float softmax_scale, float* lse,
+                                               void* stream) {
+  calibatt_status st;
+  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+  if ((st = check_block(block)) != CALIBATT_OK) return st;
+  if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
+    return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
+  if (n_heads == 0) return CALIBATT_OK;
+  if (!head_ids || !row_ptr || !col_idx || !col_base)
+    return fail(CALIBATT_ERR_INVALID_ARG, "head_ids, row_ptr, col_idx and col_base must be non-NULL");
+  const int32_t nq = ceil_div(shape->seq_len, block);
+  if (nq > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
+  std::vector<uint8_t> seen(shape->heads, 0);
+  std::vector<int16_t> heads;
+  for (int i = 0; i < n_heads; ++i) {
+    if (head_ids[i] < 0 || head_ids[i] >= shape->heads)
+      return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", head_ids[i], shape->heads);
+    if (seen[head_ids[i]]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", head_ids[i]);
+    heads.push_back(static_cast<int16_t>(head_ids[i]));
+  }
+  const bool tc = shape->dtype == CALIBATT_DTYPE_BF16 && block == 128;
+  if (tc && (!items || !cta_ptr || grid < 1))
+    return fail(CALIBATT_ERR_INVALID_ARG, "the tensor-core path needs a device schedule (items, cta_ptr, grid >= 1)");
+  if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  LayerSchedule sch;
+  std::memset(&sch, 0, sizeof(sch));
+  sch.row_ptr = row_ptr;
+  sch.col_base = col_base;
+  sch.col = col_idx;
+  sch.items = items;
+  sch.cta_ptr = cta_ptr;
+  sch.nq = nq;
+  return run_sparse(q, k, v, o, *shape, block, sch, tc ? grid : 1, heads, softmax_scale, lse,
+                    static_cast<cudaStream_t>(stream));
 }
 
 calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,

@@ -231,6 +231,47 @@ calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* 
                                                 const calibatt_dict* dict, int32_t t, int32_t l,
                                                 float softmax_scale, float* lse, void* stream);
 
+/* Work schedule of a direct-CSR call (calibatt_block_sparse_attn_csr), on the
+ * host: one item (head << 16) | query_block per query block of every listed
+ * head, placed on `grid` bins by longest-processing-time first (cost: the
+ * block's retained key blocks + 2), heads taken in list order in groups whose
+ * keys and values fit in L2 together, as the dictionary does per record.
+ *   row_ptr: host int32[heads][nq + 1], each head's offsets starting at 0;
+ *   head_ids: host int32[n_heads], distinct, in [0, heads), n_heads <= 128;
+ *   items: host uint32[n_heads * nq]; cta_ptr: host int32[grid + 1], the
+ *     items of CTA c are items[cta_ptr[c] .. cta_ptr[c+1]).
+ * nq <= 65535, heads <= 65535.  CALIBATT_ERR_INVALID_ARG on a bad argument
+ * or a decreasing row_ptr; column indices are not read. */
+calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* row_ptr,
+                                      const int32_t* head_ids, int32_t n_heads, int32_t grid,
+                                      uint32_t* items, int32_t* cta_ptr);
+
+/* Block-sparse attention from skip lists the caller holds in device memory,
+ * without a dictionary (same operation and outputs as
+ * calibatt_block_sparse_attn, for the listed heads only; an all-ones list
+ * gives dense attention):
+ *   row_ptr: device int32[shape->heads][nq + 1], nq = ceil(seq_len / block),
+ *     each head's offsets starting at 0;
+ *   col_idx: device uint16, head h's list at col_idx + col_base[h], each row
+ *     strictly ascending in [0, nq) (the rules calibatt_csr_validate checks;
+ *     the call does not read device lists on the host, so an index outside
+ *     [0, nq) is undefined behaviour);
+ *   col_base: device int64[shape->heads];
+ *   head_ids: host int32[n_heads], distinct, in [0, heads), n_heads <= 128;
+ *   items, cta_ptr, grid: the device copy of a calibatt_csr_schedule result
+ *     for the same row_ptr and head_ids (used by the tensor-core kernel, BF16
+ *     with block 128, which runs `grid` persistent CTAs; the CUDA-core
+ *     kernel walks head_ids and ignores them, and they may then be NULL).
+ * All device arrays are caller-owned and must stay valid until the call's
+ * work on `stream` completes.  n_heads == 0 is a no-op. */
+calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, const void* v, void* o,
+                                               const calibatt_shape* shape, int32_t block,
+                                               const int32_t* row_ptr, const uint16_t* col_idx,
+                                               const int64_t* col_base, const int32_t* head_ids,
+                                               int32_t n_heads, const uint32_t* items,
+                                               const int32_t* cta_ptr, int32_t grid,
+                                               float softmax_scale, float* lse, void* stream);
+
 /* Anchor-row attention with broadcast for the given heads (Key Designs 3):
  * only queries of the anchor rows of every frame attend, densely over all N
  * keys and values; every token (f, row, col) takes the output of the anchor

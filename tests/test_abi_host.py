@@ -130,3 +130,49 @@ def test_hot_path_rejects_bad_arguments_before_any_gpu_work(calibatt_lib):
     assert L.calibatt_select_blocks(buf, 1, 5000, ctypes.c_float(0.9), buf, None, None) == C.ERR_UNSUPPORTED
     assert L.calibatt_aggregate_masks(buf, 4, 0, ctypes.c_float(0.5), buf, None) == C.ERR_INVALID_ARG
     assert L.calibatt_set_wait_timeout_ms(0) == C.ERR_INVALID_ARG
+
+
+def test_csr_schedule_covers_listed_heads_in_l2_groups(calibatt_lib):
+    C = calibatt_lib
+    rng = np.random.default_rng(3)
+    heads, nq, grid = 6, 1300, 7       # keys and values of one head (85 MB) fill an L2 group
+    lengths = rng.integers(0, nq + 1, (heads, nq))
+    row_ptr = np.zeros((heads, nq + 1), np.int32)
+    row_ptr[:, 1:] = np.cumsum(lengths, axis=1)
+    head_ids = [4, 0, 2]
+    items, cta_ptr = C.csr_schedule(row_ptr, head_ids, grid)
+    assert cta_ptr[0] == 0 and cta_ptr[-1] == len(head_ids) * nq and (np.diff(cta_ptr) >= 0).all()
+    want = sorted((h << 16) | r for h in head_ids for r in range(nq))
+    assert sorted(items.tolist()) == want
+    rank = {h: i for i, h in enumerate(head_ids)}
+    for c in range(grid):
+        mine = items[cta_ptr[c]:cta_ptr[c + 1]]
+        groups = [rank[int(x) >> 16] for x in mine]
+        assert groups == sorted(groups)      # each CTA walks the heads in list order
+        for g in set(groups):                 # inside a group, costs do not increase
+            cost = [lengths[head_ids[g], int(x) & 0xFFFF] for x in mine if rank[int(x) >> 16] == g]
+            assert (np.diff(cost) <= 0).all()
+    # rejected: a head listed twice, a head out of range, a decreasing row_ptr
+    for hid, rp in (([1, 1], row_ptr), ([6], row_ptr), ([0], row_ptr[:, ::-1].copy())):
+        with pytest.raises(C.CalibattError) as e:
+            C.csr_schedule(rp, hid, grid)
+        assert e.value.status == C.ERR_INVALID_ARG
+    items, cta_ptr = C.csr_schedule(row_ptr, [], grid)
+    assert items.size == 0 and (cta_ptr == 0).all()
+
+
+def test_csr_attention_rejects_bad_arguments(calibatt_lib):
+    C = calibatt_lib
+    L = C.LIB
+    buf = ctypes.c_void_p(4096)
+    heads = (ctypes.c_int32 * 2)(0, 0)
+    shape = C.Shape(1, 256, 2, 128, 256 * 2 * 128, 2 * 128, 128, C.DTYPE_BF16, 0)
+    args = lambda hid, n, items, grid: (buf, buf, buf, buf, ctypes.byref(shape), 128, buf, buf, buf, hid, n,
+                                        items, buf, grid, 0.0, None, None)
+    assert L.calibatt_block_sparse_attn_csr(*args(heads, 2, buf, 1)) == C.ERR_INVALID_ARG       # head twice
+    assert "twice" in C.last_error()
+    one = (ctypes.c_int32 * 1)(1)
+    assert L.calibatt_block_sparse_attn_csr(*args(one, 1, None, 1)) == C.ERR_INVALID_ARG        # no schedule
+    assert "schedule" in C.last_error()
+    assert L.calibatt_block_sparse_attn_csr(*args(one, 1, buf, 0)) == C.ERR_INVALID_ARG         # grid 0
+    assert L.calibatt_block_sparse_attn_csr(*args(None, 0, None, 0)) == C.OK                    # no heads

@@ -203,6 +203,60 @@ def test_simt_sparse_bf16_block64_and_fp32_block128(C):
         _assert_close(_np(out), ref, dtype)
 
 
+# ------------------------------------------------------ direct CSR (no dictionary)
+
+def _device_csr(C, masks, h, nb):
+    """Device row_ptr / 16-bit col_idx / col_base of per-head masks, and the host row_ptr."""
+    rp, ci, _ = C.masks_to_layer_csr(masks, h, nb)
+    base = np.zeros(h, np.int64)
+    base[1:] = np.cumsum(rp[:, -1].astype(np.int64))[:-1]
+    col = ci.astype(np.uint16).view(np.int16) if ci.size else np.zeros(1, np.int16)
+    return (torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(), torch.from_numpy(base).cuda(), rp)
+
+
+@pytest.mark.parametrize("d,density", [(128, 0.4), (64, 0.4), (128, 1.0)])   # 1.0: all-ones lists, dense
+def test_csr_call_matches_dictionary_and_oracle(C, d, density):
+    b, n, h, block, grid = 2, 1000, 4, 128, 11
+    q, k, v = W.make_qkv(31, b, n, h, d, "bf16", 1.0, "cuda")
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(9, h, nb, density, empty_row_head=3 if density < 1 else None)
+    rp_d, col_d, base_d, rp = _device_csr(C, masks, h, nb)
+    heads = [3, 0, 2]
+    items, cta_ptr = C.csr_schedule(rp, heads, grid)
+    items_d = torch.from_numpy(items.view(np.int32)).cuda()
+    cta_d = torch.from_numpy(cta_ptr).cuda()
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full((b, h, n), float("nan"), device="cuda")
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, heads, items_d, cta_d, grid, block,
+                                     lse=lse)
+    _check_status(C)
+    assert torch.isnan(out[:, :, 1]).all() and torch.isnan(lse[:, 1]).all(), "a head not listed was written"
+    # the dictionary call on the same lists (head 1 routed to the other path) gives the same bits
+    ref_out, ref_lse = _run_sparse(C, q, k, v, [m if i in heads else None for i, m in enumerate(masks)], block,
+                                   lse=True)
+    assert torch.equal(out[:, :, heads], ref_out[:, :, heads])
+    assert torch.equal(lse[:, heads], ref_lse[:, heads])
+    ref, _ = O.block_sparse_attention_bnhd(_np(q)[:, :, heads], _np(k)[:, :, heads], _np(v)[:, :, heads],
+                                           [masks[i] for i in heads], block)
+    _assert_close(_np(out)[:, :, heads], ref, "bf16")
+
+
+def test_csr_call_cuda_core_paths(C):
+    for dtype, block, d in (("fp32", 64, 64), ("bf16", 64, 128), ("fp32", 128, 128)):
+        b, n, h = 1, 700, 3
+        q, k, v = W.make_qkv(32, b, n, h, d, dtype, 1.0, "cuda")
+        nb = O.num_blocks(n, block)
+        masks = _random_masks(10, h, nb, 0.5, empty_row_head=2)
+        rp_d, col_d, base_d, _ = _device_csr(C, masks, h, nb)
+        out = torch.full_like(q, float("nan"))
+        C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [2, 0], block=block)   # no schedule
+        _check_status(C)
+        assert torch.isnan(out[:, :, 1]).all()
+        ref, _ = O.block_sparse_attention_bnhd(_np(q)[:, :, [0, 2]], _np(k)[:, :, [0, 2]], _np(v)[:, :, [0, 2]],
+                                               [masks[0], masks[2]], block)
+        _assert_close(_np(out)[:, :, [0, 2]], ref, dtype)
+
+
 # ------------------------------------------------------ full-size sampled parity
 
 def _sampled_blocks(rng, nb, k):
