@@ -713,6 +713,86 @@ def test_bitmap_dictionary_matches_lists(C, d, n, h):
     assert torch.equal(res[0], res[1])
 
 
+def _compact_reference(q, k, v, n, r, cols, block=128):
+    """Oracle output and LSE of query block r whose skip list is `cols`: plain
+    attention of its rows over exactly the keys of the listed blocks (the
+    retained key set; gathering it is index selection only)."""
+    rows = np.arange(r * block, min(n, (r + 1) * block))
+    keys = np.concatenate([np.arange(c * block, min(n, (c + 1) * block)) for c in cols])
+    kt = torch.as_tensor(keys, device=k.device)
+    qr = _f32(q[0, torch.as_tensor(rows, device=q.device), 0])
+    ref, lse = O.attention_rows(qr, _f32(k[0, kt, 0]), _f32(v[0, kt, 0]), len(keys), O.default_scale(q.shape[-1]))
+    return rows, ref, lse
+
+
+def _check_rows(C, out, lse, q, k, v, n, lists, sample):
+    for r in sample:
+        rows, ref, ref_lse = _compact_reference(q, k, v, n, r, lists[r])
+        rt = torch.as_tensor(rows, device=out.device)
+        _assert_close(_np(out[0, rt, 0]), ref, "bf16")
+        assert np.abs(lse[0, 0, rt].cpu().numpy() - ref_lse).max() < 2e-2
+
+
+def test_longest_sequence_of_index_lists(C):
+    """The largest problem the index-list dictionary takes: 65,535 blocks of 128
+    (16-bit block indices), N = 8,388,429 tokens with a ragged last block of 77
+    tokens and NaN rows behind it, one head; sampled query blocks against the
+    oracle over exactly their retained keys."""
+    nb, block = 65535, 128
+    n = (nb - 1) * block + 77
+    qa, ka, va = W.make_qkv(41, 1, n, 1, 128, "bf16", 1.0, "cuda", seq_alloc=nb * block)
+    q, k, v = qa[:, :n], ka[:, :n], va[:, :n]
+    rng = np.random.default_rng(7)
+    extra = rng.integers(0, nb, (nb, 5))
+    lists = []
+    for r in range(nb):
+        c = [r, 0, *extra[r].tolist()] + ([nb - 1] if r % 1000 == 0 else [])
+        lists.append(np.unique(np.asarray(c, np.int32)))
+    row_ptr = np.zeros((1, nb + 1), np.int32)
+    row_ptr[0, 1:] = np.cumsum([len(c) for c in lists])
+    col = np.concatenate(lists)
+    out = torch.full_like(qa, float("nan"))
+    lse = torch.full((1, 1, n), float("nan"), device="cuda")
+    with C.MaskDictionary(1, 1, 1, nb, nb, block, col.size) as dct:
+        dct.set_layer(0, 0, row_ptr, col, None)
+        C.calibatt_block_sparse_attn(q, k, v, out[:, :n], dct, 0, 0, block, lse=lse)
+        _check_status(C)
+    assert torch.isnan(out[:, n:]).all(), "padding rows of the output were written"
+    _check_rows(C, out, lse, q, k, v, n, lists, [0, 1, 31000, nb - 2, nb - 1])
+    del qa, ka, va, q, k, v, out
+    torch.cuda.empty_cache()
+
+
+def test_longest_bitmap_row(C):
+    """The largest bitmap dictionary row: 2,048 key blocks, N = 262,066 (ragged
+    last block of 50 tokens), one query block keeping every key block and others
+    keeping few; bitwise equal to the index-list dictionary and against the
+    oracle."""
+    nb, block = 2048, 128
+    n = (nb - 1) * block + 50
+    q, k, v = W.make_qkv(42, 1, n, 1, 128, "bf16", 1.0, "cuda")
+    rng = np.random.default_rng(8)
+    masks = rng.random((nb, nb)) < 0.01
+    masks[np.arange(nb), np.arange(nb)] = True
+    masks[777, :] = True                      # the longest row: all 2,048 key blocks
+    masks[5, :] = False                       # an empty row
+    rp, ci, rep = C.masks_to_layer_csr([masks], 1, nb)
+    outs, lses = [], []
+    for bitmap in (False, True):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((1, 1, n), float("nan"), device="cuda")
+        with C.MaskDictionary(1, 1, 1, nb, nb, block, 0 if bitmap else ci.size, bitmap=bitmap) as dct:
+            dct.set_layer(0, 0, rp, ci, rep)
+            C.calibatt_block_sparse_attn(q, k, v, out, dct, 0, 0, block, lse=lse)
+            _check_status(C)
+        outs.append(out)
+        lses.append(lse)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(lses[0], lses[1])
+    lists = [np.nonzero(masks[r])[0] for r in range(nb)]
+    _check_rows(C, outs[1], lses[1], q, k, v, n, lists, [0, 777, 1500, nb - 1])
+    assert (outs[1][0, 5 * 128:6 * 128].float() == 0).all() and torch.isneginf(lses[1][0, 0, 5 * 128:6 * 128]).all()
+
+
 def test_bitmap_dictionary_size_and_rules(C):
     """Device bytes of the two formats at the 720p layer, and the bitmap
     format's limits."""
