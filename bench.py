@@ -241,6 +241,30 @@ def run_reference(args, rank, world):
     del torch
 
 
+def run_anchor_case(args, torch, C, pk):
+    """The anchor path alone: the 12 repetitive heads of the dual-path 720p
+    layer (anchor rows attend to all keys, the output is broadcast to every
+    row), timed with CUDA events; a case of its own for profiling the anchor
+    kernel.  Prints effective TFLOP/s (8.39 MFLOP per anchor tile x key block)."""
+    wd = W.WORKLOADS["720p_dual"]
+    _, rep_heads = W.workload_masks(wd)
+    q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    tiles = len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128) * wd.num_blocks
+    per_call = time_calls(torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols,
+                                                                wd.anchors, list(rep_heads), stream=stream),
+                          args.steps, args.warmup, stream)
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the anchor case")
+    ms = statistics.mean(per_call)
+    tf = tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12
+    print(json.dumps({"anchor_case": {
+        "heads": len(rep_heads), "anchor_tiles_x_key_blocks": tiles, "ms_per_call": ms,
+        "effective_tflops": tf, "frac_of_burst_peak": tf / pk["bf16_tflops"],
+        "output_bytes": len(rep_heads) * wd.seq_len * wd.head_dim * 2}}), flush=True)
+
+
 def run_epilogue_probe(torch, B, C):
     """Store rate of the anchor broadcast epilogue (the 12 repetitive heads of
     the dual-path 720p layer).  The measurement build records, per CTA, the
@@ -408,6 +432,8 @@ def main():
     ap.add_argument("--epilogue-probe", action="store_true",
                     help="time the anchor broadcast epilogue with the library's measurement build "
                          "(-DCALIBATT_TRACE) and print its store rate")
+    ap.add_argument("--anchor-case", action="store_true",
+                    help="time the anchor path alone (the 12 repetitive heads of the dual-path 720p layer)")
     ap.add_argument("--dense-sample", type=int, default=50,
                     help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
@@ -440,6 +466,9 @@ def main():
     stream = torch.cuda.current_stream()
     if args.epilogue_probe:
         run_epilogue_probe(torch, B, C)
+        return
+    if args.anchor_case:
+        run_anchor_case(args, torch, C, pk)
         return
     if args.workload == "sweep":
         if world > 1:
