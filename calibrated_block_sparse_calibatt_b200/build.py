@@ -9,6 +9,7 @@ library also loads on a machine without a GPU).
 from __future__ import annotations
 
 import concurrent.futures
+import fcntl
 import os
 import shutil
 import subprocess
@@ -63,19 +64,30 @@ def _stale(lib: str = LIB) -> bool:
 
 def build(force: bool = False, verbose_ptxas: bool = False, trace: bool = False) -> str:
     """Compiles the library (or, with trace=True, its measurement variant) if
-    any source is newer than it; returns its path."""
+    any source is newer than it; returns its path.
+
+    Safe to call from several processes at once (the ranks of a multi-GPU
+    run): one builds under an exclusive file lock while the others wait, then
+    find the library current; the new file replaces the old one atomically."""
     lib = LIB_TRACE if trace else LIB
     if not force and not verbose_ptxas and not _stale(lib):
         return lib
-    os.makedirs(os.path.join(BUILD, "trace") if trace else BUILD, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
-    with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, trace), SOURCES))
-    tmp = lib + ".tmp"
-    r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, lib)
+    with open(os.path.join(LIBDIR, ".build.lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            if not force and not verbose_ptxas and not _stale(lib):
+                return lib                                   # built by another process meanwhile
+            os.makedirs(os.path.join(BUILD, "trace") if trace else BUILD, exist_ok=True)
+            with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+                objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, trace), SOURCES))
+            tmp = f"{lib}.{os.getpid()}.tmp"
+            r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], capture_output=True, text=True)
+            if r.returncode != 0:
+                raise RuntimeError(f"link failed:\n{r.stderr}")
+            os.replace(tmp, lib)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
     return lib
 
 
