@@ -54,13 +54,22 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # nvidia-smi numbers GPUs physically, CUDA by CUDA_VISIBLE_DEVICES:
+        # name the device by its UUID so that each rank samples its own GPU
+        self.smi_id = str(index)
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(index).uuid)
+            self.smi_id = u if u.startswith("GPU-") else f"GPU-{u}"
+        except Exception:
+            pass
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}",
+                ["nvidia-smi", f"--id={self.smi_id}",
                  "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
