@@ -69,6 +69,8 @@ SIGNATURES = {
     "calibatt_dict_info": (_i32, [_vp, _P(_i64), _P(_i64), _P(_i32)]),
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
+    "calibatt_dict_save": (_i32, [_vp, ctypes.c_char_p]),
+    "calibatt_dict_load": (_i32, [ctypes.c_char_p, _i32, _P(_vp)]),
     "calibatt_block_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32, _i32, _f32, _vp, _vp]),
     "calibatt_csr_schedule": (_i32, [_i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp]),
     "calibatt_block_sparse_attn_csr": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _vp, _vp, _vp, _i32, _vp,
@@ -240,6 +242,19 @@ class MaskDictionary:
             check(LIB.calibatt_dict_create(T, L, H, nq, nk, block, int(nnz_capacity), int(num_ctas),
                                            ctypes.byref(h)))
         self.handle = h
+
+    @classmethod
+    def load(cls, path, num_ctas=0):
+        """A dictionary read from a file written by save() (calibatt_dict_load)."""
+        h = ctypes.c_void_p(None)
+        check(LIB.calibatt_dict_load(os.fsencode(path), int(num_ctas), ctypes.byref(h)))
+        self = cls.__new__(cls)
+        self.handle = h
+        return self
+
+    def save(self, path):
+        """Writes the dictionary's records to `path` (calibatt_dict_save)."""
+        check(LIB.calibatt_dict_save(self.handle, os.fsencode(path)))
 
     def set_layer(self, t, l, row_ptr, col_idx, repetitive=None):
         rp = _i32_array(row_ptr).reshape(-1)

@@ -1002,6 +1002,293 @@ calibatt_status calibatt_dict_destroy(calibatt_dict* d) {
   return CALIBATT_OK;
 }
 
+// ------------------------------------------------------------ dictionary file
+
+namespace {
+
+constexpr char kDictMagic[8] = {'C', 'A', 'L', 'I', 'B', 'D', 'C', 'T'};
+constexpr char kDictEnd[8] = {'C', 'A', 'L', 'I', 'B', 'E', 'N', 'D'};
+constexpr uint32_t kDictFileVersion = 1;
+
+struct DictFileHeader {
+  char magic[8];
+  uint32_t version;
+  uint32_t format;  // 0 index lists, 1 bitmap
+  int32_t T, L, H, nq, nk, block;
+  int32_t has_geom, frames, rows, cols, n_anchors;
+  int32_t anchors[calibatt::kMaxAnchors];
+  int32_t reserved;
+  int64_t records;
+  int64_t nnz_total;
+};
+static_assert(sizeof(DictFileHeader) == 144, "dictionary file header layout");
+
+struct DictFileRecord {
+  int32_t t, l;
+  int64_t nnz;
+};
+
+// 64-bit FNV-1a over the file's 8-byte little-endian words.
+struct WordHash {
+  uint64_t h = 0xcbf29ce484222325ull;
+  void add(const unsigned char* p, size_t n) {  // n is a multiple of 8
+    for (size_t i = 0; i < n; i += 8) {
+      uint64_t w;
+      std::memcpy(&w, p + i, 8);
+      h = (h ^ w) * 0x100000001b3ull;
+    }
+  }
+};
+
+size_t padded8(size_t n) { return (n + 7) & ~static_cast<size_t>(7); }
+
+struct DictWriter {
+  FILE* f = nullptr;
+  WordHash hash;
+  bool ok = true;
+  std::vector<unsigned char> buf;
+  // Writes n bytes followed by zeros up to the next multiple of 8.
+  void put(const void* p, size_t n) {
+    if (!ok) return;
+    buf.assign(padded8(n), 0);
+    if (n) std::memcpy(buf.data(), p, n);
+    hash.add(buf.data(), buf.size());
+    ok = std::fwrite(buf.data(), 1, buf.size(), f) == buf.size();
+  }
+};
+
+struct DictReader {
+  FILE* f = nullptr;
+  WordHash hash;
+  std::vector<unsigned char> buf;
+  // Reads n bytes and their zero padding; false on a short read or a non-zero pad.
+  bool get(void* p, size_t n) {
+    buf.resize(padded8(n));
+    if (std::fread(buf.data(), 1, buf.size(), f) != buf.size()) return false;
+    for (size_t i = n; i < buf.size(); ++i)
+      if (buf[i] != 0) return false;
+    hash.add(buf.data(), buf.size());
+    if (n) std::memcpy(p, buf.data(), n);
+    return true;
+  }
+};
+
+}  // namespace
+
+calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
+  if (!d || !path) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary and path must be non-NULL");
+  const int H = d->H, nq = d->nq;
+  const int64_t layers = static_cast<int64_t>(d->T) * d->L;
+  DictFileHeader hd;
+  std::memset(&hd, 0, sizeof(hd));
+  std::memcpy(hd.magic, kDictMagic, 8);
+  hd.version = kDictFileVersion;
+  hd.format = d->bitmap ? 1u : 0u;
+  hd.T = d->T;
+  hd.L = d->L;
+  hd.H = H;
+  hd.nq = nq;
+  hd.nk = d->nk;
+  hd.block = d->block;
+  if (d->has_geom) {
+    hd.has_geom = 1;
+    hd.frames = d->g_frames;
+    hd.rows = d->g_rows;
+    hd.cols = d->g_cols;
+    hd.n_anchors = static_cast<int32_t>(d->g_anchors.size());
+    for (size_t a = 0; a < d->g_anchors.size(); ++a) hd.anchors[a] = d->g_anchors[a];
+  }
+  for (uint8_t set : d->layer_set) hd.records += set;
+  hd.nnz_total = d->nnz_used;
+  const std::string tmp = std::string(path) + ".tmp";
+  DictWriter w;
+  w.f = std::fopen(tmp.c_str(), "wb");
+  if (!w.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s for writing", tmp.c_str());
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != d->device) cudaSetDevice(d->device);
+  cudaError_t e = cudaSuccess;
+  w.put(&hd, sizeof(hd));
+  std::vector<int32_t> rp;
+  std::vector<int64_t> cb;
+  std::vector<uint16_t> col;
+  std::vector<uint32_t> bits;
+  for (int64_t ly = 0; ly < layers && w.ok && e == cudaSuccess; ++ly) {
+    if (!d->layer_set[ly]) continue;
+    DictFileRecord rec{static_cast<int32_t>(ly / d->L), static_cast<int32_t>(ly % d->L), 0};
+    if (d->bitmap) {
+      bits.resize(static_cast<size_t>(H) * nq * d->words);
+      e = cudaMemcpy(bits.data(), d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words),
+                     sizeof(uint32_t) * bits.size(), cudaMemcpyDeviceToHost);
+      for (uint32_t x : bits) rec.nnz += __builtin_popcount(x);
+    } else {
+      rp.resize(static_cast<size_t>(H) * (nq + 1));
+      cb.resize(H);
+      e = cudaMemcpy(rp.data(), d->d_row_ptr + ly * H * (nq + 1), sizeof(int32_t) * rp.size(),
+                     cudaMemcpyDeviceToHost);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(cb.data(), d->d_col_base + ly * H, sizeof(int64_t) * H, cudaMemcpyDeviceToHost);
+      for (int h = 0; h < H; ++h) rec.nnz += rp[static_cast<size_t>(h) * (nq + 1) + nq];
+      col.resize(rec.nnz);
+      // a layer's lists are stored contiguously, head after head, from head 0's offset
+      if (e == cudaSuccess && rec.nnz > 0)
+        e = cudaMemcpy(col.data(), d->d_col + cb[0], sizeof(uint16_t) * rec.nnz, cudaMemcpyDeviceToHost);
+    }
+    if (e != cudaSuccess) break;
+    w.put(&rec, sizeof(rec));
+    w.put(d->rep.data() + ly * H, H);
+    if (d->bitmap) {
+      w.put(bits.data(), sizeof(uint32_t) * bits.size());
+    } else {
+      w.put(rp.data(), sizeof(int32_t) * rp.size());
+      w.put(col.data(), sizeof(uint16_t) * col.size());
+    }
+  }
+  if (prev != d->device) cudaSetDevice(prev);
+  if (w.ok && e == cudaSuccess) {
+    unsigned char trailer[16];
+    std::memcpy(trailer, kDictEnd, 8);
+    const uint64_t hv = w.hash.h;
+    std::memcpy(trailer + 8, &hv, 8);
+    w.ok = std::fwrite(trailer, 1, 16, w.f) == 16;
+  }
+  const bool closed = std::fclose(w.f) == 0;
+  if (e != cudaSuccess || !w.ok || !closed) {
+    std::remove(tmp.c_str());
+    if (e != cudaSuccess) return cuda_fail(e, "dictionary copy to host");
+    return fail(CALIBATT_ERR_INVALID_ARG, "writing %s failed", tmp.c_str());
+  }
+  if (std::rename(tmp.c_str(), path) != 0) {
+    std::remove(tmp.c_str());
+    return fail(CALIBATT_ERR_INVALID_ARG, "cannot rename %s to %s", tmp.c_str(), path);
+  }
+  return CALIBATT_OK;
+}
+
+namespace {
+
+calibatt_status load_records(DictReader& r, const DictFileHeader& hd, calibatt_dict* d, const char* path) {
+  const int H = hd.H, nq = hd.nq;
+  const int32_t words = (hd.nk + 31) / 32;
+  const int64_t per_record_max = static_cast<int64_t>(H) * nq * hd.nk;
+  int64_t prev_ly = -1, nnz_seen = 0;
+  std::vector<uint8_t> rep(H);
+  std::vector<int32_t> rp(static_cast<size_t>(H) * (nq + 1)), col32;
+  std::vector<uint16_t> col;
+  std::vector<uint32_t> bits;
+  for (int64_t i = 0; i < hd.records; ++i) {
+    DictFileRecord rec;
+    if (!r.get(&rec, sizeof(rec))) return fail(CALIBATT_ERR_INVALID_ARG, "%s: record %lld is cut short", path, (long long)i);
+    if (rec.t < 0 || rec.t >= hd.T || rec.l < 0 || rec.l >= hd.L)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) outside %d x %d", path, rec.t, rec.l, hd.T, hd.L);
+    const int64_t ly = static_cast<int64_t>(rec.t) * hd.L + rec.l;
+    if (ly <= prev_ly) return fail(CALIBATT_ERR_INVALID_ARG, "%s: records out of order", path);
+    prev_ly = ly;
+    if (rec.nnz < 0 || rec.nnz > per_record_max || nnz_seen + rec.nnz > hd.nnz_total)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) has %lld blocks", path, rec.t, rec.l, (long long)rec.nnz);
+    nnz_seen += rec.nnz;
+    if (!r.get(rep.data(), H)) return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
+    if (hd.format == 1) {
+      bits.resize(static_cast<size_t>(H) * nq * words);
+      if (!r.get(bits.data(), sizeof(uint32_t) * bits.size()))
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
+      // decode into per-head CSR: row pointers counted from each head's first block
+      col32.clear();
+      for (int h = 0; h < H; ++h) {
+        int32_t* hp = rp.data() + static_cast<size_t>(h) * (nq + 1);
+        const size_t head_start = col32.size();
+        for (int q = 0; q < nq; ++q) {
+          hp[q] = static_cast<int32_t>(col32.size() - head_start);
+          const uint32_t* row = bits.data() + (static_cast<size_t>(h) * nq + q) * words;
+          for (int32_t wd = 0; wd < words; ++wd) {
+            for (uint32_t x = row[wd]; x; x &= x - 1) {
+              const int c = wd * 32 + __builtin_ctz(x);
+              if (c >= hd.nk) return fail(CALIBATT_ERR_INVALID_ARG, "%s: bit beyond the last key block", path);
+              col32.push_back(c);
+            }
+          }
+        }
+        hp[nq] = static_cast<int32_t>(col32.size() - head_start);
+      }
+    } else {
+      if (!r.get(rp.data(), sizeof(int32_t) * rp.size()))
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
+      col.resize(rec.nnz);
+      if (!r.get(col.data(), sizeof(uint16_t) * col.size()))
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
+      col32.assign(col.begin(), col.end());
+    }
+    // every head's row pointers start at 0 and never decrease, and together
+    // they cover exactly the record's blocks, so each head's list lies inside col32
+    int64_t total = 0;
+    for (int h = 0; h < H; ++h) {
+      const int32_t* hp = rp.data() + static_cast<size_t>(h) * (nq + 1);
+      if (hp[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d row_ptr[0] != 0", path, rec.t, rec.l, h);
+      for (int q = 0; q < nq; ++q)
+        if (hp[q + 1] < hp[q])
+          return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d row_ptr decreases", path, rec.t, rec.l, h);
+      total += hp[nq];
+    }
+    if (total != rec.nnz || static_cast<int64_t>(col32.size()) != rec.nnz)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) block count mismatch", path, rec.t, rec.l);
+    calibatt_status st = calibatt_dict_set_layer(d, rec.t, rec.l, rp.data(), col32.empty() ? nullptr : col32.data(), rep.data());
+    if (st != CALIBATT_OK) return st;
+  }
+  if (nnz_seen != hd.nnz_total) return fail(CALIBATT_ERR_INVALID_ARG, "%s: total block count mismatch", path);
+  return CALIBATT_OK;
+}
+
+}  // namespace
+
+calibatt_status calibatt_dict_load(const char* path, int32_t num_ctas, calibatt_dict** out) {
+  if (!out || !path) return fail(CALIBATT_ERR_INVALID_ARG, "path and out must be non-NULL");
+  *out = nullptr;
+  DictReader r;
+  r.f = std::fopen(path, "rb");
+  if (!r.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s", path);
+  struct Closer {
+    FILE* f;
+    ~Closer() { std::fclose(f); }
+  } closer{r.f};
+  DictFileHeader hd;
+  if (!r.get(&hd, sizeof(hd)) || std::memcmp(hd.magic, kDictMagic, 8) != 0)
+    return fail(CALIBATT_ERR_INVALID_ARG, "%s is not a dictionary file", path);
+  if (hd.version != kDictFileVersion || hd.format > 1 || hd.reserved != 0)
+    return fail(CALIBATT_ERR_INVALID_ARG, "%s: unsupported version %u / format %u", path, hd.version, hd.format);
+  if (hd.T < 1 || hd.L < 1 || hd.H < 1 || hd.nq < 1 || hd.nk != hd.nq || hd.H > 65535 || hd.nq > 65535 ||
+      (hd.block != 64 && hd.block != 128) || hd.records < 0 || hd.records > static_cast<int64_t>(hd.T) * hd.L ||
+      hd.nnz_total < 0 || (hd.format == 1 && hd.nq > calibatt::kMaxBitmapBlocks) || hd.n_anchors < 0 ||
+      hd.n_anchors > calibatt::kMaxAnchors || (hd.has_geom != 0 && hd.has_geom != 1))
+    return fail(CALIBATT_ERR_INVALID_ARG, "%s: header fields out of range", path);
+  calibatt_dict* d = nullptr;
+  calibatt_status st = hd.format == 1
+      ? calibatt_dict_create_bitmap(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, num_ctas, &d)
+      : calibatt_dict_create(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d);
+  if (st != CALIBATT_OK) return st;
+  if (hd.has_geom) st = calibatt_dict_set_anchor_geometry(d, hd.frames, hd.rows, hd.cols, hd.anchors, hd.n_anchors);
+  if (st == CALIBATT_OK) st = load_records(r, hd, d, path);
+  if (st == CALIBATT_OK) {
+    const uint64_t want = r.hash.h;
+    unsigned char trailer[16];
+    uint64_t got = 0;
+    if (std::fread(trailer, 1, 16, r.f) != 16 || std::memcmp(trailer, kDictEnd, 8) != 0) {
+      st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailer missing", path);
+    } else {
+      std::memcpy(&got, trailer + 8, 8);
+      if (got != want) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: checksum mismatch", path);
+      else if (std::fgetc(r.f) != EOF) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailing bytes", path);
+    }
+  }
+  if (st != CALIBATT_OK) {
+    const std::string msg = g_last_error;
+    calibatt_dict_destroy(d);
+    g_last_error = msg;
+    return st;
+  }
+  *out = d;
+  return CALIBATT_OK;
+}
+
 calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const void* v, void* o,
                                            const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
                                            int32_t t, int32_t l, float softmax_scale, float* lse, void* stream) {

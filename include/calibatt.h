@@ -194,6 +194,34 @@ calibatt_status calibatt_dict_layer_info(const calibatt_dict* dict, int32_t t, i
 /* Frees the dictionary's device and host memory (synchronises the device). */
 calibatt_status calibatt_dict_destroy(calibatt_dict* dict);
 
+/* Checkpoint of the calibration output (the dictionary is the method's only
+ * persistent artefact, computed offline and loaded before generation, Key
+ * Designs 4).  Writes to `path` (replaced atomically: written to a temporary
+ * name, then renamed) a little-endian file:
+ *   header: "CALIBDCT", version 1, format (0 index lists, 1 bitmap), T, L,
+ *     H, nq, nk, block, the anchor geometry if set, records stored, total
+ *     retained blocks (144 bytes);
+ *   one entry per set record (t, l) in (t, l) order: t, l, retained blocks,
+ *     the H repetitive flags, then the H CSR row pointers and the 16-bit
+ *     block indices (index lists) or the H*nq*ceil(nk/32) bitmap words, each
+ *     part zero-padded to 8 bytes;
+ *   trailer: "CALIBEND" and a 64-bit FNV-1a hash of every 8-byte word before
+ *     it.
+ * Schedules are not stored.  Copies the records from the device
+ * (synchronously).  CALIBATT_ERR_INVALID_ARG if the file cannot be written
+ * (the message names the cause). */
+calibatt_status calibatt_dict_save(const calibatt_dict* dict, const char* path);
+
+/* Reads a file written by calibatt_dict_save into a new dictionary of the
+ * same format on the current device, rebuilding every record's schedules
+ * for num_ctas persistent CTAs (<= 0: the device's SM count).  The header,
+ * every record (through calibatt_dict_set_layer's validation), the record
+ * order and counts, the padding and the trailing hash are checked;
+ * CALIBATT_ERR_INVALID_ARG on any mismatch, a short file or trailing bytes,
+ * and then no dictionary is returned.  Allocation failures as
+ * calibatt_dict_create. */
+calibatt_status calibatt_dict_load(const char* path, int32_t num_ctas, calibatt_dict** out);
+
 /* ------------------------------------------------------- hot path */
 
 /* Block-sparse attention for every non-repetitive head of record (t, l)

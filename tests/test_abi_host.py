@@ -176,3 +176,35 @@ def test_csr_attention_rejects_bad_arguments(calibatt_lib):
     assert "schedule" in C.last_error()
     assert L.calibatt_block_sparse_attn_csr(*args(one, 1, buf, 0)) == C.ERR_INVALID_ARG         # grid 0
     assert L.calibatt_block_sparse_attn_csr(*args(None, 0, None, 0)) == C.OK                    # no heads
+
+
+def test_dict_load_rejects_bad_files_before_touching_the_device(calibatt_lib, tmp_path):
+    C = calibatt_lib
+    L = C.LIB
+    h = ctypes.c_void_p(None)
+    missing = tmp_path / "missing.dict"
+    assert L.calibatt_dict_load(os.fsencode(missing), 4, ctypes.byref(h)) == C.ERR_INVALID_ARG
+    assert "cannot open" in C.last_error() and not h.value
+    bad = tmp_path / "bad.dict"
+    bad.write_bytes(b"NOTADICT" + bytes(200))
+    assert L.calibatt_dict_load(os.fsencode(bad), 4, ctypes.byref(h)) == C.ERR_INVALID_ARG
+    assert "not a dictionary file" in C.last_error()
+
+    def header(**kw):
+        f = dict(version=1, format=0, T=1, L=1, H=2, nq=4, nk=4, block=128, has_geom=0, records=0, nnz=0)
+        f.update(kw)
+        return (b"CALIBDCT" + np.array([f["version"], f["format"]], np.uint32).tobytes()
+                + np.array([f["T"], f["L"], f["H"], f["nq"], f["nk"], f["block"], f["has_geom"], 0, 0, 0, 0],
+                           np.int32).tobytes()
+                + np.zeros(16 + 1, np.int32).tobytes() + np.array([f["records"], f["nnz"]], np.int64).tobytes())
+
+    assert len(header()) == 144
+    for kw, words in (({"version": 2}, "unsupported"), ({"format": 3}, "unsupported"),
+                      ({"nk": 5}, "out of range"), ({"block": 96}, "out of range"),
+                      ({"records": 2}, "out of range"), ({"nnz": -1}, "out of range"),
+                      ({"format": 1, "nq": 4096, "nk": 4096}, "out of range")):
+        bad.write_bytes(header(**kw))
+        assert L.calibatt_dict_load(os.fsencode(bad), 4, ctypes.byref(h)) == C.ERR_INVALID_ARG, kw
+        assert words in C.last_error(), (kw, C.last_error())
+    bad.write_bytes(header()[:100])                                  # cut inside the header
+    assert L.calibatt_dict_load(os.fsencode(bad), 4, ctypes.byref(h)) == C.ERR_INVALID_ARG

@@ -815,6 +815,62 @@ def test_bitmap_dictionary_size_and_rules(C):
         C.MaskDictionary(1, 1, 1, 4096, 4096, 128, bitmap=True)    # more than 2048 blocks per row
 
 
+@pytest.mark.parametrize("bitmap", [False, True])
+def test_dictionary_save_load_round_trip(C, tmp_path, bitmap):
+    """calibatt_dict_save / calibatt_dict_load: a dictionary with the anchor
+    geometry, three of its four records set (repetitive heads included), written
+    and read back with another persistent grid; every record's counts match and
+    its single-path and dual-path outputs are bitwise those of the original;
+    damaged files are refused."""
+    frames, rows, cols, anchors = 3, 10, 100, (2, 7)
+    n, h, d, block = frames * rows * cols, 4, 128, 128
+    nb = O.num_blocks(n, block)
+    q, k, v = W.make_qkv(51, 1, n, h, d, "bf16", 1.0, "cuda")
+    path = tmp_path / "masks.dict"
+    records = {(0, 0): (0, 3), (0, 1): (), (1, 1): (1,)}           # (t, l) -> repetitive heads
+    with C.MaskDictionary(2, 2, h, nb, nb, block, 4 * h * nb * nb, bitmap=bitmap) as dct:
+        dct.set_anchor_geometry(frames, rows, cols, anchors)
+        for i, ((t, l), rep) in enumerate(records.items()):
+            masks = _random_masks(60 + i, h, nb, 0.4)
+            masks = [None if hh in rep else masks[hh] for hh in range(h)]
+            rp, ci, rf = C.masks_to_layer_csr(masks, h, nb)
+            dct.set_layer(t, l, rp, ci, rf)
+        dct.save(path)
+        ref = {}
+        for (t, l) in records:
+            o1, o2 = torch.zeros_like(q), torch.zeros_like(q)
+            C.calibatt_block_sparse_attn(q, k, v, o1, dct, t, l, block)
+            C.calibatt_dual_path_attn(q, k, v, o2, dct, t, l, frames, rows, cols, anchors, block)
+            ref[t, l] = (o1, o2, dct.layer_info(t, l))
+        info = dct.info()
+        _check_status(C)
+    loaded = C.MaskDictionary.load(path, num_ctas=11)
+    try:
+        assert loaded.info()["nnz"] == info["nnz"] and loaded.info()["num_ctas"] == 11
+        for (t, l), (o1, o2, li) in ref.items():
+            g1, g2 = torch.zeros_like(q), torch.zeros_like(q)
+            C.calibatt_block_sparse_attn(q, k, v, g1, loaded, t, l, block)
+            C.calibatt_dual_path_attn(q, k, v, g2, loaded, t, l, frames, rows, cols, anchors, block)
+            _check_status(C)
+            assert loaded.layer_info(t, l) == li
+            assert torch.equal(g1, o1) and torch.equal(g2, o2)
+        with pytest.raises(C.CalibattError):
+            loaded.layer_info(1, 0)                                 # the record never set stays unset
+    finally:
+        loaded.close()
+    raw = path.read_bytes()
+    damaged = tmp_path / "damaged.dict"
+    for blob in (raw[:-1], raw + b"\0", raw[:len(raw) // 2],
+                 raw[:len(raw) // 2] + bytes([raw[len(raw) // 2] ^ 0x10]) + raw[len(raw) // 2 + 1:]):
+        damaged.write_bytes(blob)
+        with pytest.raises(C.CalibattError) as e:
+            C.MaskDictionary.load(damaged)
+        assert e.value.status == C.ERR_INVALID_ARG
+    with pytest.raises(C.CalibattError):
+        with C.MaskDictionary(1, 1, 1, 4, 4, 128, 16) as small:
+            small.save(tmp_path / "no_such_dir" / "x.dict")
+
+
 def test_host_buffer_entry_point(C):
     """calibatt_block_sparse_attn_host: host inputs copied in, attention, output
     copied out, in stream order; equal to the device-buffer call."""
