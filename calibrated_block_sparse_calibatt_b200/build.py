@@ -27,7 +27,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB_TRACE = os.path.join(LIBDIR, "libcalibatt_trace.so")
 
 SOURCES = ["api.cu", "attn_tc.cu", "attn_simt.cu", "energy.cu", "energy_noalloc.cu", "repetition.cu",
-           "diagnostics.cu"]
+           "diagnostics.cu", "csr_check.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -221,7 +221,7 @@ def debug_bounded_wait(stream=None):
 def device_status(stream=None, clear=True) -> int:
     code = ctypes.c_int32(0)
     st = LIB.calibatt_device_status(_stream(stream), ctypes.byref(code), int(clear))
-    if st not in (OK, ERR_TIMEOUT):
+    if st not in (OK, ERR_TIMEOUT, ERR_INVALID_ARG):
         check(st)
     return code.value
 

@@ -426,6 +426,7 @@ calibatt_status run_sparse(const void* q, const void* k, const void* v, void* o,
     p.heads = s.heads;
     p.nb = ceil_div(s.seq_len, block);
     p.scale_log2 = sl2;
+    p.status = status_word_ptr();
     p.sched = sch;
     const size_t nh = std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0);
     p.n_heads = static_cast<int32_t>(nh);
@@ -528,6 +529,7 @@ calibatt_status launch_anchor(const void* q, const void* k, const void* v, void*
   p.heads = s.heads;
   p.nb = ceil_div(s.seq_len, block);
   p.scale_log2 = sl2;
+  p.status = status_word_ptr();
   g.tiles_per_head = ceil_div(g.anchor_tokens, block);
   p.anc = g;
   const int64_t n_items = static_cast<int64_t>(s.batch) * n_heads * g.tiles_per_head;
@@ -1364,6 +1366,19 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
   if (tc && (!items || !cta_ptr || grid < 1))
     return fail(CALIBATT_ERR_INVALID_ARG, "the tensor-core path needs a device schedule (items, cta_ptr, grid >= 1)");
   if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  // the lists were never read on the host: check them on the device first
+  calibatt::CsrCheckParams chk;
+  std::memset(&chk, 0, sizeof(chk));
+  chk.row_ptr = row_ptr;
+  chk.col = col_idx;
+  chk.col_base = col_base;
+  chk.nq = nq;
+  chk.n_heads = n_heads;
+  for (int i = 0; i < n_heads; ++i) chk.head_ids[i] = heads[i];
+  chk.status = status_word_ptr();
+  if (!chk.status) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+  cudaError_t e = calibatt::launch_csr_check(chk, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "skip-list check launch");
   LayerSchedule sch;
   std::memset(&sch, 0, sizeof(sch));
   sch.row_ptr = row_ptr;
@@ -1636,7 +1651,12 @@ calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clea
     e = cudaMemset(p, 0, sizeof(int32_t));
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
   }
-  if (*code != 0) return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
+  if (*code != 0) {
+    if ((*code & 0xFF) == CALIBATT_ERR_INVALID_ARG)
+      return fail(CALIBATT_ERR_INVALID_ARG, "a kernel met a key-block index outside the key range (code 0x%x)",
+                  *code);
+    return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
+  }
   return CALIBATT_OK;
 }
 

@@ -90,6 +90,12 @@ __global__ void __launch_bounds__(2 * BLK) simt_attn_kernel(const __grid_constan
   const float sl2 = p.scale_log2;
   for (int j = 0; j < n; ++j) {
     const int c = ANCHOR ? j : static_cast<int>(cols[j]);
+    if (c >= p.nb) {
+      // a block index outside the key range (device lists the host never
+      // checked): record it and skip the block rather than read past N
+      if (tid == 0 && p.status) atomicCAS(p.status, 0, 1 | (22 << 8));
+      continue;
+    }
     for (int k0 = c * BLK; k0 < c * BLK + BLK; k0 += kKeysPerStage) {
       __syncthreads();
       for (int idx = tid; idx < kKeysPerStage * HD; idx += 2 * BLK) {

@@ -77,6 +77,7 @@ struct SimtParams {
   int32_t n_heads;               // sparse mode: number of heads in head_ids
   int16_t head_ids[kMaxHeadsPerCall];
   AnchorGeom anc;
+  int32_t* status;               // device status word (a block index out of range is recorded)
 };
 
 struct EnergyParams {
@@ -132,6 +133,18 @@ cudaError_t launch_select_blocks(const float* energy, int64_t n_rows, int32_t nk
                                  uint8_t* mask, int32_t* count_accum, cudaStream_t s);
 cudaError_t launch_aggregate(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,
                              uint8_t* mask, cudaStream_t s);
+
+// Device-side check of caller-held skip lists (csr_check.cu).
+struct CsrCheckParams {
+  const int32_t* row_ptr;   // [heads][nq + 1]
+  const uint16_t* col;
+  const int64_t* col_base;  // [heads]
+  int32_t nq;
+  int32_t n_heads;
+  int16_t head_ids[kMaxHeadsPerCall];
+  int32_t* status;
+};
+cudaError_t launch_csr_check(const CsrCheckParams& p, cudaStream_t s);
 
 cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s);
 cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns, cudaStream_t s);

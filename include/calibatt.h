@@ -282,8 +282,13 @@ calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* 
  *     each head's offsets starting at 0;
  *   col_idx: device uint16, head h's list at col_idx + col_base[h], each row
  *     strictly ascending in [0, nq) (the rules calibatt_csr_validate checks;
- *     the call does not read device lists on the host, so an index outside
- *     [0, nq) is undefined behaviour);
+ *     the call does not read device lists on the host: a small kernel checks
+ *     them on `stream` before the attention and records the first violation
+ *     in the device status word (calibatt_device_status); the attention
+ *     kernels never read outside Q, K, V for a block index >= nq (the
+ *     tensor-core kernel's copies are bounded by its tensor maps, the
+ *     CUDA-core kernel skips the block), but that call's output is then
+ *     meaningless);
  *   col_base: device int64[shape->heads];
  *   head_ids: host int32[n_heads], distinct, in [0, heads), n_heads <= 128;
  *   items, cta_ptr, grid: the device copy of a calibatt_csr_schedule result
@@ -425,10 +430,14 @@ calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_pro
 
 /* ------------------------------------------------------- diagnostics */
 
-/* Synchronises `stream`, then reports the device status word that the
- * kernels set when a bounded wait runs out (CALIBATT_ERR_TIMEOUT in the low
- * byte, the waiting role and barrier above it) and optionally clears it.
- * Returns CALIBATT_ERR_TIMEOUT when the word is non-zero. */
+/* Synchronises `stream`, then reports the device status word and optionally
+ * clears it.  The kernels set it (first event wins) when a bounded wait runs
+ * out (CALIBATT_ERR_TIMEOUT in the low byte, the waiting role and barrier
+ * above it) or when a skip list the host never read breaks the list rules
+ * (CALIBATT_ERR_INVALID_ARG in the low byte; 23: the device-side check that
+ * calibatt_block_sparse_attn_csr runs before its attention kernel; 22: the
+ * CUDA-core kernel met a block index >= nq and skipped that block).  Returns
+ * the low byte's status when the word is non-zero. */
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);
 
 /* Failure-path check of the bounded waits: launches one warp that waits on

@@ -241,6 +241,43 @@ def test_csr_call_matches_dictionary_and_oracle(C, d, density):
     _assert_close(_np(out)[:, :, heads], ref, "bf16")
 
 
+@pytest.mark.parametrize("dtype,block,d", [("bf16", 128, 128), ("fp32", 64, 64)])
+def test_csr_call_flags_block_index_out_of_range(C, dtype, block, d):
+    """Device lists are not read on the host: an index >= nq in one row is
+    caught on the device (the list check ahead of the attention, code 23; no
+    kernel reads outside the tensors), recorded in the status word (low byte
+    CALIBATT_ERR_INVALID_ARG) and cleared by the read; the next valid call is
+    unaffected."""
+    b, n, h = 1, 1000, 2
+    q, k, v = W.make_qkv(33, b, n, h, d, dtype, 1.0, "cuda")
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(11, h, nb, 0.5)
+    rp_d, col_d, base_d, rp = _device_csr(C, masks, h, nb)
+    bad = col_d.clone()
+    bad[int(rp[0, 3])] = nb + 5                # first block of head 0, row 3
+    bad[int(rp[0, nb] - 1)] = 0x7FFF           # last block of head 0's last row
+    items, cta_ptr = C.csr_schedule(rp, [0, 1], 5)
+    sched = (torch.from_numpy(items.view(np.int32)).cuda(), torch.from_numpy(cta_ptr).cuda(), 5)
+    out = torch.zeros_like(q)
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, bad, base_d, [0, 1], *sched, block=block)
+    code = C.device_status()
+    assert code & 0xFF == C.ERR_INVALID_ARG and code >> 8 == 23, hex(code)
+    assert "key-block index" in C.last_error()
+    assert C.device_status() == 0                                   # the read cleared it
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [0, 1], *sched, block=block)
+    _check_status(C)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block)
+    _assert_close(_np(out), ref, dtype)
+    # indices in range but out of order (head 1, the first row with two blocks) are flagged too
+    r = next(r for r in range(nb) if rp[1, r + 1] - rp[1, r] >= 2)
+    i = int(rp[0, nb] + rp[1, r])
+    swapped = col_d.clone()
+    swapped[i], swapped[i + 1] = col_d[i + 1], col_d[i]
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, swapped, base_d, [0, 1], *sched, block=block)
+    code = C.device_status()
+    assert code & 0xFF == C.ERR_INVALID_ARG and code >> 8 == 23, hex(code)
+
+
 def test_csr_call_cuda_core_paths(C):
     for dtype, block, d in (("fp32", 64, 64), ("bf16", 64, 128), ("fp32", 128, 128)):
         b, n, h = 1, 700, 3
