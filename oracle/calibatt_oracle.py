@@ -88,6 +88,9 @@ __all__ = [
     "block_energy_bnhd",
     "select_blocks",
     "aggregate_masks",
+    "attention_probability_rows",
+    "spatial_similarity",
+    "repetition_flags",
     "num_blocks",
 ]
 
