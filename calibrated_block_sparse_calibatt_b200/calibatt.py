@@ -87,6 +87,7 @@ SIGNATURES = {
     "calibatt_select_blocks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp, _vp]),
     "calibatt_aggregate_masks": (_i32, [_vp, _i64, _i32, _f32, _vp, _vp]),
     "calibatt_debug_exp2_fma": (_i32, [_vp, _vp, _i64, _vp]),
+    "calibatt_debug_exp2_fma_quintic": (_i32, [_vp, _vp, _i64, _vp]),
     "calibatt_device_status": (_i32, [_vp, _P(_i32), _i32]),
     "calibatt_set_wait_timeout_ms": (_i32, [_i32]),
     "calibatt_device_sm_count": (_i32, [_P(_i32)]),
@@ -201,6 +202,10 @@ def csr_schedule(row_ptr, head_ids, grid):
 
 def calibatt_debug_exp2_fma(x, y, stream=None):
     check(LIB.calibatt_debug_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def calibatt_debug_exp2_fma_quintic(x, y, stream=None):
+    check(LIB.calibatt_debug_exp2_fma_quintic(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
 def set_wait_timeout_ms(ms: int) -> None:

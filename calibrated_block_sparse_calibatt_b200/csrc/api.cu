@@ -1626,7 +1626,15 @@ calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32
 calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
   if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
   if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
-  cudaError_t e = calibatt::launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream));
+  cudaError_t e = calibatt::launch_exp2_fma(x, y, n, false, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
+  return CALIBATT_OK;
+}
+
+calibatt_status calibatt_debug_exp2_fma_quintic(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
+  if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
+  cudaError_t e = calibatt::launch_exp2_fma(x, y, n, true, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
   return CALIBATT_OK;
 }

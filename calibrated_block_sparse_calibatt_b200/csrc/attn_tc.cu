@@ -127,6 +127,17 @@ constexpr float kRescaleLog2 = 8.0f;
 #define CALIBATT_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
+// The offline energy passes (LSE and energy modes) have half the tensor work
+// of attention per key block but the same 16,384 exponentials, so the MUFU
+// unit is their busiest pipe while the FMA pipe idles: one pair in
+// kEnergyPolyEvery runs on the FMA pipe with the quintic (as accurate as
+// ex2.approx).  Measured on the 720p energy call under the power cap: 1/4 of
+// the pairs is 2% faster than none, 1/3 and 1/2 are 6% and 12% slower (the
+// polynomial spends more energy per result than the MUFU).
+#ifndef CALIBATT_ENERGY_POLY_EVERY
+#define CALIBATT_ENERGY_POLY_EVERY 4
+#endif
+constexpr int kEnergyPolyEvery = CALIBATT_ENERGY_POLY_EVERY;
 
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
 
@@ -848,7 +859,13 @@ __device__ void softmax_energy_role(const TcParams& p, uint32_t base, uint8_t* g
       for (int c = 0; c < 64; ++c) {
         float x0, x1;
         fma2(x0, x1, sc[2 * c], sc[2 * c + 1], sl2, sl2, -off, -off);
-        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        float p0, p1;
+        if (kEnergyPolyEvery > 0 && (c % kEnergyPolyEvery) == kEnergyPolyEvery - 1) {
+          exp2_fma2_quintic(p0, p1, x0, x1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
+        }
         if (c & 1) add2(lc, ld, lc, ld, p0, p1); else add2(la, lb, la, lb, p0, p1);
       }
       const float rs = (la + lb) + (lc + ld);
@@ -992,17 +1009,21 @@ cudaError_t launch_one(const TcParams& p, int grid, cudaStream_t s) {
 
 // Even elements go through the packed pair routine the softmax uses (with their
 // odd neighbour), a trailing odd element through the scalar one.
+template <bool QUINTIC>
 __global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
   for (int64_t i = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); i < n;
        i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    if (i + 1 < n) {
-      float y0, y1;
-      exp2_fma2(y0, y1, x[i], x[i + 1]);
-      y[i] = y0;
-      y[i + 1] = y1;
+    const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+    float y0, y1;
+    if (QUINTIC) {
+      exp2_fma2_quintic(y0, y1, x[i], x1);
+    } else if (i + 1 < n) {
+      exp2_fma2(y0, y1, x[i], x1);
     } else {
-      y[i] = exp2_fma(x[i]);
+      y0 = exp2_fma(x[i]);
     }
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
   }
 }
 
@@ -1035,10 +1056,14 @@ extern "C" void calibatt_trace_reset() {
 }
 #endif
 
-cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s) {
+cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, bool quintic, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   const int64_t blocks = (n + 255) / 256;
-  exp2_fma_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(x, y, n);
+  const unsigned grid = static_cast<unsigned>(blocks < 1024 ? blocks : 1024);
+  if (quintic)
+    exp2_fma_kernel<true><<<grid, 256, 0, s>>>(x, y, n);
+  else
+    exp2_fma_kernel<false><<<grid, 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

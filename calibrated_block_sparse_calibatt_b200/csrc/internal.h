@@ -146,7 +146,7 @@ struct CsrCheckParams {
 };
 cudaError_t launch_csr_check(const CsrCheckParams& p, cudaStream_t s);
 
-cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, cudaStream_t s);
+cudaError_t launch_exp2_fma(const float* x, float* y, int64_t n, bool quintic, cudaStream_t s);
 cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns, cudaStream_t s);
 
 // Records a failure message for calibatt_last_error() on the calling thread.

@@ -302,6 +302,28 @@ __device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float 
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// 2^x for two values on the FMA and integer pipes, the same reduction with a
+// quintic fitted by Remez exchange to the relative error of 2^f on
+// [-1/2, 1/2] (max relative error 7.5e-8, under one float32 ulp, close to
+// the MUFU's ex2.approx; coefficients from
+// csrc/fit_exp2_poly.py).  Serves float32 sums (the offline energy passes),
+// where the cubic's 7.5e-5 would show.  Same input range as exp2_fma.
+__device__ __forceinline__ void exp2_fma2_quintic(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0, t1, u0, u1, f0, f1, p0, p1;
+  add2(t0, t1, x0, x1, 12582912.0f, 12582912.0f);
+  add2(u0, u1, t0, t1, -12582912.0f, -12582912.0f);
+  fma2(f0, f1, u0, u1, -1.0f, -1.0f, x0, x1);
+  fma2(p0, p1, f0, f1, 1.327647199e-03f, 1.327647199e-03f, 9.675541334e-03f, 9.675541334e-03f);
+  fma2(p0, p1, p0, p1, f0, f1, 5.550713273e-02f, 5.550713273e-02f);
+  fma2(p0, p1, p0, p1, f0, f1, 2.402211972e-01f, 2.402211972e-01f);
+  fma2(p0, p1, p0, p1, f0, f1, 6.931469671e-01f, 6.931469671e-01f);
+  fma2(p0, p1, p0, p1, f0, f1, 1.000000072e+00f, 1.000000072e+00f);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

@@ -455,6 +455,12 @@ calibatt_status calibatt_debug_bounded_wait(void* stream);
  * x, y: device float32[n]. */
 calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, void* stream);
 
+/* The same for the quintic FMA-pipe exponential that the offline energy
+ * passes use for a quarter of their exponentials: relative error below 3e-7
+ * (the fit's 7.5e-8 plus float32 evaluation) for -125 <= x <= 126, about
+ * 2^-125 for smaller x.  x, y: device float32[n]. */
+calibatt_status calibatt_debug_exp2_fma_quintic(const float* x, float* y, int64_t n, void* stream);
+
 /* Time limit of every in-kernel barrier wait, in milliseconds (default 4000;
  * applies to launches made after the call). */
 calibatt_status calibatt_set_wait_timeout_ms(int32_t ms);

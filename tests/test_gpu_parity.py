@@ -509,6 +509,27 @@ def test_fma_exp2_error_bound(C):
     assert (yl >= 0).all() and (yl < 1e-37).all()
 
 
+def test_fma_exp2_quintic_error_bound(C):
+    """The quintic FMA-pipe 2^x of the offline energy passes: relative error
+    below 3e-7 against float64 over the whole input range (the fit's 7.5e-8
+    plus float32 evaluation), odd lengths included, tiny values for x < -125."""
+    rng = np.random.default_rng(23)
+    x = np.concatenate([rng.uniform(-125, 126, 200000), rng.uniform(-1, 1, 50001), np.arange(-125, 127, 0.125),
+                        [0.0, -0.5, 0.5, 8.0, -1e-7, 1e-7, -0.4999999, 0.4999999]]).astype(np.float32)
+    assert x.size % 2 == 1
+    xt = torch.from_numpy(x).cuda()
+    y = torch.empty_like(xt)
+    C.calibatt_debug_exp2_fma_quintic(xt, y)
+    _check_status(C)
+    rel = np.abs(y.cpu().numpy().astype(np.float64) / np.exp2(x.astype(np.float64)) - 1.0)
+    assert rel.max() < 3e-7, rel.max()
+    low = torch.tensor([-126.0, -200.0, float("-inf")], device="cuda")
+    yl = torch.empty_like(low)
+    C.calibatt_debug_exp2_fma_quintic(low, yl)
+    _check_status(C)
+    assert (yl >= 0).all() and (yl < 1e-37).all()
+
+
 @pytest.mark.parametrize("fmt", ["lists", "bitmap"])
 def test_sweep_records_sampled(C, fmt):
     """Records of the schedule sweep in one dictionary spanning all 50 x 40
