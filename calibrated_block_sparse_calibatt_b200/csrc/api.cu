@@ -134,10 +134,16 @@ void lpt_grouped(int32_t n, const int64_t* cost, const int32_t* group, int32_t b
   bin_ptr[bins] = pos;
 }
 
-// Heads whose keys and values (at head_dim 128) fit together in about 80 MB of L2.
+// Heads whose keys and values (at head_dim 128) fit together in about 40 MB
+// of L2, a third of it and within one die's half.  On the 720p call (38.7 MB
+// per head) one, two and three heads per group measured 35.4, 36.8 and
+// 38.4 ms in one run: the fewer heads in flight, the fewer K/V re-reads.
+#ifndef CALIBATT_L2_GROUP_MB
+#define CALIBATT_L2_GROUP_MB 40
+#endif
 int32_t heads_per_group(int32_t nq) {
   const int64_t per_head = static_cast<int64_t>(nq) * 128 * 128 * 2 * 2;
-  return static_cast<int32_t>(std::max<int64_t>(1, (80ll << 20) / per_head));
+  return static_cast<int32_t>(std::max<int64_t>(1, (static_cast<int64_t>(CALIBATT_L2_GROUP_MB) << 20) / per_head));
 }
 
 // ------------------------------------------------------------ tensor maps

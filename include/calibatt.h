@@ -157,7 +157,7 @@ calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int
  * converted to 16-bit indices, copied to the device (synchronously), and a
  * longest-processing-time schedule of the layer's (head, query block) work
  * is built for the dictionary's num_ctas: heads are taken in groups whose
- * keys and values fit in about 80 MB of L2, and the schedule keeps one
+ * keys and values fit in about 40 MB of L2, and the schedule keeps one
  * running LPT balance across the groups while listing each CTA's items group
  * by group, so the persistent CTAs work on the same few heads at a time. */
 calibatt_status calibatt_dict_set_layer(calibatt_dict* dict, int32_t t, int32_t l,
