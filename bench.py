@@ -171,8 +171,10 @@ def time_calls(torch, fn, steps, warmup, stream):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def cpu_baseline(wl, masks, q, k, v, budget_s=12.0, seed=0):
-    """The float64 oracle, as it stands, on a bounded seeded sample of query blocks."""
+def cpu_baseline(wl, masks, q, k, v, o=None, budget_s=12.0, seed=0):
+    """The float64 oracle, as it stands, on a bounded seeded sample of query
+    blocks.  With o (the library's output of the same call) the sampled rows
+    are also compared: returns (baseline, parity)."""
     from oracle import calibatt_oracle as O
 
     rng = np.random.default_rng(seed)
@@ -181,8 +183,9 @@ def cpu_baseline(wl, masks, q, k, v, budget_s=12.0, seed=0):
     t_or = 0.0
     tiles = 0
     n_blocks = 0
-    qn = kn = vn = None
+    qn = kn = vn = on = None
     last_h = None
+    err_max, err_sum, err_n = 0.0, 0.0, 0
     while time.perf_counter() - t_start < budget_s:
         h = int(rng.choice(heads))
         r = int(rng.integers(0, wl.num_blocks))
@@ -190,19 +193,31 @@ def cpu_baseline(wl, masks, q, k, v, budget_s=12.0, seed=0):
             qn = q[0, :, h].float().cpu().numpy().astype(np.float64)
             kn = k[0, :, h].float().cpu().numpy().astype(np.float64)
             vn = v[0, :, h].float().cpu().numpy().astype(np.float64)
+            on = o[0, :, h].float().cpu().numpy().astype(np.float64) if o is not None else None
             last_h = h
         rows = np.arange(r * wl.block, min(wl.seq_len, (r + 1) * wl.block))
         ts = time.perf_counter()
-        O.block_sparse_attention(qn, kn, vn, masks[h], wl.block, rows=rows)
+        ref, _ = O.block_sparse_attention(qn, kn, vn, masks[h], wl.block, rows=rows)
         t_or += time.perf_counter() - ts
+        if on is not None:
+            err = np.abs(on[rows] - ref)
+            err_max, err_sum, err_n = max(err_max, float(err.max())), err_sum + float(err.sum()), err_n + err.size
         tiles += int(masks[h][r].sum())
         n_blocks += 1
     tflops = tiles * FLOP_PER_TILE / t_or / 1e12
-    return {"value": tflops, "unit": "TFLOP/s (effective, retained blocks)", "cores": os.cpu_count(),
+    base = {"value": tflops, "unit": "TFLOP/s (effective, retained blocks)", "cores": os.cpu_count(),
             "kind": "oracle",
             "sample": f"{n_blocks} seeded (head, q-block) rows of the 720p layer, {tiles} retained tiles, "
                       f"{t_or:.1f} s of float64 NumPy; ms/call extrapolated to the full call = "
                       f"{t_or / max(tiles, 1) * sum(int(m.sum()) for m in masks.values()) * 1e3:.0f} ms"}
+    if o is None:
+        return base
+    mean = err_sum / max(err_n, 1)
+    parity = {"max_abs": err_max, "mean_abs": mean, "tolerance": {"max_abs": 2e-2, "mean_abs": 2e-3},
+              "within_tolerance": err_max <= 2e-2 and mean <= 2e-3,
+              "sample": f"the same {n_blocks} (head, q-block) rows of this run's block-sparse output "
+                        f"against the float64 oracle"}
+    return base, parity
 
 
 def run_reference(args, rank, world):
@@ -628,9 +643,12 @@ def main():
             raise RuntimeError("device wait timed out during the end-to-end leg")
         del hq, hk, hv, hos, dsets
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, masks, q, k, v)
+        # the block-sparse output of this run's inputs (the extra legs reused o)
+        C.calibatt_block_sparse_attn(q, k, v, o, d_sparse, 0, 0, wl.block, stream=stream)
+        torch.cuda.synchronize()
+        cpu, parity = cpu_baseline(wl, masks, q, k, v, o)
 
     if rank == 0:
         line = {
@@ -653,6 +671,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": args.steps,
             "cpu_baseline": cpu,
+            "parity": parity,
             **extras,
         }
         print(json.dumps(line), flush=True)
