@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <functional>
+#include <memory>
 #include <mutex>
 #include <numeric>
 #include <queue>
@@ -586,6 +587,26 @@ calibatt_status launch_fused(const void* q, const void* k, const void* v, void* 
 
 }  // namespace
 
+namespace {
+
+// Runs an entry point's body so that no C++ exception crosses the C ABI: a
+// failed host allocation (std::bad_alloc from a container or new) becomes
+// CALIBATT_ERR_OOM, anything else CALIBATT_ERR_INVALID_ARG with its message.
+template <typename Body>
+calibatt_status guarded(Body&& body) {
+  try {
+    return body();
+  } catch (const std::bad_alloc&) {
+    return fail(CALIBATT_ERR_OOM, "host memory allocation failed");
+  } catch (const std::exception& e) {
+    return fail(CALIBATT_ERR_INVALID_ARG, "internal error: %s", e.what());
+  } catch (...) {
+    return fail(CALIBATT_ERR_INVALID_ARG, "internal error");
+  }
+}
+
+}  // namespace
+
 // ===================================================================== ABI
 
 extern "C" {
@@ -608,406 +629,430 @@ int32_t calibatt_abi_version(void) { return 1; }
 
 calibatt_status calibatt_csr_validate(int32_t nq, int32_t nk, const int32_t* row_ptr, const int32_t* col_idx,
                                       int32_t require_diagonal) {
-  return validate_csr(nq, nk, row_ptr, col_idx, require_diagonal != 0, "csr");
+  return guarded([&]() -> calibatt_status {
+    return validate_csr(nq, nk, row_ptr, col_idx, require_diagonal != 0, "csr");
+  });
 }
 
 calibatt_status calibatt_csr_to_intervals(int32_t nq, const int32_t* row_ptr, const int32_t* col_idx,
                                           int32_t* interval_ptr, int32_t* interval_start, int32_t* interval_len,
                                           int64_t capacity, int64_t* n_intervals) {
-  if (nq < 0 || !row_ptr || !interval_ptr || !n_intervals) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
-  if (row_ptr[nq] > 0 && !col_idx) return fail(CALIBATT_ERR_INVALID_ARG, "col_idx is NULL");
-  int64_t total = 0;
-  for (int32_t r = 0; r < nq; ++r) {
-    interval_ptr[r] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
-    for (int32_t i = row_ptr[r]; i < row_ptr[r + 1]; ++i) {
-      const bool starts = (i == row_ptr[r]) || (col_idx[i] != col_idx[i - 1] + 1);
-      if (starts) {
-        if (total < capacity && interval_start && interval_len) {
-          interval_start[total] = col_idx[i];
-          interval_len[total] = 1;
+  return guarded([&]() -> calibatt_status {
+    if (nq < 0 || !row_ptr || !interval_ptr || !n_intervals) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+    if (row_ptr[nq] > 0 && !col_idx) return fail(CALIBATT_ERR_INVALID_ARG, "col_idx is NULL");
+    int64_t total = 0;
+    for (int32_t r = 0; r < nq; ++r) {
+      interval_ptr[r] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
+      for (int32_t i = row_ptr[r]; i < row_ptr[r + 1]; ++i) {
+        const bool starts = (i == row_ptr[r]) || (col_idx[i] != col_idx[i - 1] + 1);
+        if (starts) {
+          if (total < capacity && interval_start && interval_len) {
+            interval_start[total] = col_idx[i];
+            interval_len[total] = 1;
+          }
+          ++total;
+        } else if (total - 1 < capacity && interval_len) {
+          interval_len[total - 1] += 1;
         }
-        ++total;
-      } else if (total - 1 < capacity && interval_len) {
-        interval_len[total - 1] += 1;
       }
     }
-  }
-  interval_ptr[nq] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
-  *n_intervals = total;
-  if (total > capacity) return fail(CALIBATT_ERR_INVALID_ARG, "capacity %lld < %lld intervals", (long long)capacity, (long long)total);
-  return CALIBATT_OK;
+    interval_ptr[nq] = static_cast<int32_t>(std::min<int64_t>(total, INT32_MAX));
+    *n_intervals = total;
+    if (total > capacity) return fail(CALIBATT_ERR_INVALID_ARG, "capacity %lld < %lld intervals", (long long)capacity, (long long)total);
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_lpt_schedule(int32_t n_items, const int64_t* cost, int32_t n_bins, int32_t* bin_ptr,
                                       int32_t* item_order, int64_t* makespan) {
-  if (n_items < 0 || n_bins < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_items must be >= 0 and n_bins >= 1");
-  if (!bin_ptr || (n_items > 0 && (!cost || !item_order))) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
-  for (int32_t i = 0; i < n_items; ++i)
-    if (cost[i] < 0) return fail(CALIBATT_ERR_INVALID_ARG, "negative cost at item %d", i);
-  lpt(n_items, cost, n_bins, bin_ptr, item_order, makespan);
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n_items < 0 || n_bins < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_items must be >= 0 and n_bins >= 1");
+    if (!bin_ptr || (n_items > 0 && (!cost || !item_order))) return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+    for (int32_t i = 0; i < n_items; ++i)
+      if (cost[i] < 0) return fail(CALIBATT_ERR_INVALID_ARG, "negative cost at item %d", i);
+    lpt(n_items, cost, n_bins, bin_ptr, item_order, makespan);
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* row_ptr, const int32_t* head_ids,
                                       int32_t n_heads, int32_t grid, uint32_t* items, int32_t* cta_ptr) {
-  if (heads < 1 || heads > 65535 || nq < 1 || nq > 65535)
-    return fail(CALIBATT_ERR_INVALID_ARG, "heads and nq must be in [1, 65535]");
-  if (grid < 1) return fail(CALIBATT_ERR_INVALID_ARG, "grid must be >= 1");
-  if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
-    return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
-  if (!row_ptr || !cta_ptr || (n_heads > 0 && (!head_ids || !items)))
-    return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
-  std::vector<uint8_t> seen(heads, 0);
-  for (int i = 0; i < n_heads; ++i) {
-    const int32_t h = head_ids[i];
-    if (h < 0 || h >= heads) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", h, heads);
-    if (seen[h]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", h);
-    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
-    if (rp[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row_ptr[0] != 0", h);
-    for (int r = 0; r < nq; ++r)
-      if (rp[r + 1] < rp[r] || rp[r + 1] - rp[r] > nq)
-        return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row %d has %d blocks", h, r, rp[r + 1] - rp[r]);
-  }
-  // The dictionary's cost model and L2 head groups (calibatt_dict_set_layer).
-  std::vector<uint32_t> all;
-  std::vector<int64_t> cost;
-  std::vector<int32_t> group;
-  const int32_t hpg = heads_per_group(nq);
-  for (int i = 0; i < n_heads; ++i) {
-    const int32_t* rp = row_ptr + static_cast<int64_t>(head_ids[i]) * (nq + 1);
-    for (int r = 0; r < nq; ++r) {
-      all.push_back((static_cast<uint32_t>(head_ids[i]) << 16) | static_cast<uint32_t>(r));
-      cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
-      group.push_back(i / hpg);
+  return guarded([&]() -> calibatt_status {
+    if (heads < 1 || heads > 65535 || nq < 1 || nq > 65535)
+      return fail(CALIBATT_ERR_INVALID_ARG, "heads and nq must be in [1, 65535]");
+    if (grid < 1) return fail(CALIBATT_ERR_INVALID_ARG, "grid must be >= 1");
+    if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
+      return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
+    if (!row_ptr || !cta_ptr || (n_heads > 0 && (!head_ids || !items)))
+      return fail(CALIBATT_ERR_INVALID_ARG, "NULL argument");
+    std::vector<uint8_t> seen(heads, 0);
+    for (int i = 0; i < n_heads; ++i) {
+      const int32_t h = head_ids[i];
+      if (h < 0 || h >= heads) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", h, heads);
+      if (seen[h]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", h);
+      const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+      if (rp[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row_ptr[0] != 0", h);
+      for (int r = 0; r < nq; ++r)
+        if (rp[r + 1] < rp[r] || rp[r + 1] - rp[r] > nq)
+          return fail(CALIBATT_ERR_INVALID_ARG, "head %d: row %d has %d blocks", h, r, rp[r + 1] - rp[r]);
     }
-  }
-  std::vector<int32_t> order(all.size());
-  lpt_grouped(static_cast<int32_t>(all.size()), cost.data(), group.data(), grid, cta_ptr, order.data());
-  for (size_t i = 0; i < all.size(); ++i) items[i] = all[order[i]];
-  return CALIBATT_OK;
+    // The dictionary's cost model and L2 head groups (calibatt_dict_set_layer).
+    std::vector<uint32_t> all;
+    std::vector<int64_t> cost;
+    std::vector<int32_t> group;
+    const int32_t hpg = heads_per_group(nq);
+    for (int i = 0; i < n_heads; ++i) {
+      const int32_t* rp = row_ptr + static_cast<int64_t>(head_ids[i]) * (nq + 1);
+      for (int r = 0; r < nq; ++r) {
+        all.push_back((static_cast<uint32_t>(head_ids[i]) << 16) | static_cast<uint32_t>(r));
+        cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
+        group.push_back(i / hpg);
+      }
+    }
+    std::vector<int32_t> order(all.size());
+    lpt_grouped(static_cast<int32_t>(all.size()), cost.data(), group.data(), grid, cta_ptr, order.data());
+    for (size_t i = 0; i < all.size(); ++i) items[i] = all[order[i]];
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk, int32_t block,
                                      int64_t nnz_capacity, int32_t num_ctas, calibatt_dict** out) {
-  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
-  *out = nullptr;
-  if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1 || nnz_capacity < 0)
-    return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1 and nnz_capacity >= 0");
-  if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
-  if (nq > 65535 || H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "nq and H must be <= 65535");
-  calibatt_status st = check_block(block);
-  if (st != CALIBATT_OK) return st;
-  int G = num_ctas;
-  if (G <= 0) G = device_sm_count();
-  if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
-  auto* d = new calibatt_dict();
-  d->T = T;
-  d->L = L;
-  d->H = H;
-  d->nq = nq;
-  d->nk = nk;
-  d->block = block;
-  d->G = G;
-  cudaGetDevice(&d->device);
-  d->nnz_cap = nnz_capacity;
-  const int64_t layers = static_cast<int64_t>(T) * L;
-  const size_t b_rp = sizeof(int32_t) * layers * H * (nq + 1);
-  const size_t b_cb = sizeof(int64_t) * layers * H;
-  const size_t b_col = sizeof(uint16_t) * std::max<int64_t>(1, nnz_capacity);
-  const size_t b_it = sizeof(uint32_t) * layers * H * nq;
-  const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
-  cudaError_t e = cudaMalloc(&d->d_row_ptr, b_rp);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_col_base, b_cb);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_col, b_col);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
-  if (e != cudaSuccess) {
-    d->release();
-    delete d;
-    return cuda_fail(e, "dictionary allocation");
-  }
-  d->device_bytes = static_cast<int64_t>(b_rp + b_cb + b_col + b_it + b_cta);
-  d->layer_set.assign(layers, 0);
-  d->rep.assign(layers * H, 0);
-  d->n_sparse.assign(layers, 0);
-  d->n_rep.assign(layers, 0);
-  d->retained.assign(layers, 0);
-  *out = d;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1 || nnz_capacity < 0)
+      return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1 and nnz_capacity >= 0");
+    if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
+    if (nq > 65535 || H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "nq and H must be <= 65535");
+    calibatt_status st = check_block(block);
+    if (st != CALIBATT_OK) return st;
+    int G = num_ctas;
+    if (G <= 0) G = device_sm_count();
+    if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    // owned here until returned, so an exception frees it (host vectors are
+    // sized before any device allocation)
+    std::unique_ptr<calibatt_dict> holder(new calibatt_dict());
+    calibatt_dict* d = holder.get();
+    d->T = T;
+    d->L = L;
+    d->H = H;
+    d->nq = nq;
+    d->nk = nk;
+    d->block = block;
+    d->G = G;
+    cudaGetDevice(&d->device);
+    d->nnz_cap = nnz_capacity;
+    const int64_t layers = static_cast<int64_t>(T) * L;
+    d->layer_set.assign(layers, 0);
+    d->rep.assign(layers * H, 0);
+    d->n_sparse.assign(layers, 0);
+    d->n_rep.assign(layers, 0);
+    d->retained.assign(layers, 0);
+    const size_t b_rp = sizeof(int32_t) * layers * H * (nq + 1);
+    const size_t b_cb = sizeof(int64_t) * layers * H;
+    const size_t b_col = sizeof(uint16_t) * std::max<int64_t>(1, nnz_capacity);
+    const size_t b_it = sizeof(uint32_t) * layers * H * nq;
+    const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
+    cudaError_t e = cudaMalloc(&d->d_row_ptr, b_rp);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_col_base, b_cb);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_col, b_col);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e != cudaSuccess) {
+      d->release();
+      return cuda_fail(e, "dictionary allocation");
+    }
+    d->device_bytes = static_cast<int64_t>(b_rp + b_cb + b_col + b_it + b_cta);
+    *out = holder.release();
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk,
                                             int32_t block, int32_t num_ctas, calibatt_dict** out) {
-  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
-  *out = nullptr;
-  if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1)
-    return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1");
-  if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
-  if (nq > calibatt::kMaxBitmapBlocks)
-    return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries hold at most %d blocks per row", calibatt::kMaxBitmapBlocks);
-  if (H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "H must be <= 65535");
-  calibatt_status st = check_block(block);
-  if (st != CALIBATT_OK) return st;
-  int G = num_ctas;
-  if (G <= 0) G = device_sm_count();
-  if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
-  auto* d = new calibatt_dict();
-  d->T = T;
-  d->L = L;
-  d->H = H;
-  d->nq = nq;
-  d->nk = nk;
-  d->block = block;
-  d->G = G;
-  d->bitmap = true;
-  d->words = (nk + 31) / 32;
-  cudaGetDevice(&d->device);
-  const int64_t layers = static_cast<int64_t>(T) * L;
-  const size_t b_bm = sizeof(uint32_t) * layers * H * nq * d->words;
-  const size_t b_it = sizeof(uint32_t) * layers * H * nq;
-  const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
-  cudaError_t e = cudaMalloc(&d->d_bitmap, b_bm);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
-  if (e != cudaSuccess) {
-    d->release();
-    delete d;
-    return cuda_fail(e, "bitmap dictionary allocation");
-  }
-  d->device_bytes = static_cast<int64_t>(b_bm + b_it + b_cta);
-  d->layer_set.assign(layers, 0);
-  d->rep.assign(layers * H, 0);
-  d->n_sparse.assign(layers, 0);
-  d->n_rep.assign(layers, 0);
-  d->retained.assign(layers, 0);
-  *out = d;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1)
+      return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1");
+    if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
+    if (nq > calibatt::kMaxBitmapBlocks)
+      return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries hold at most %d blocks per row", calibatt::kMaxBitmapBlocks);
+    if (H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "H must be <= 65535");
+    calibatt_status st = check_block(block);
+    if (st != CALIBATT_OK) return st;
+    int G = num_ctas;
+    if (G <= 0) G = device_sm_count();
+    if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    std::unique_ptr<calibatt_dict> holder(new calibatt_dict());
+    calibatt_dict* d = holder.get();
+    d->T = T;
+    d->L = L;
+    d->H = H;
+    d->nq = nq;
+    d->nk = nk;
+    d->block = block;
+    d->G = G;
+    d->bitmap = true;
+    d->words = (nk + 31) / 32;
+    cudaGetDevice(&d->device);
+    const int64_t layers = static_cast<int64_t>(T) * L;
+    d->layer_set.assign(layers, 0);
+    d->rep.assign(layers * H, 0);
+    d->n_sparse.assign(layers, 0);
+    d->n_rep.assign(layers, 0);
+    d->retained.assign(layers, 0);
+    const size_t b_bm = sizeof(uint32_t) * layers * H * nq * d->words;
+    const size_t b_it = sizeof(uint32_t) * layers * H * nq;
+    const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
+    cudaError_t e = cudaMalloc(&d->d_bitmap, b_bm);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e != cudaSuccess) {
+      d->release();
+      return cuda_fail(e, "bitmap dictionary allocation");
+    }
+    d->device_bytes = static_cast<int64_t>(b_bm + b_it + b_cta);
+    *out = holder.release();
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, const int32_t* row_ptr,
                                         const int32_t* col_idx, const uint8_t* repetitive) {
-  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
-  if (t < 0 || t >= d->T || l < 0 || l >= d->L)
-    return fail(CALIBATT_ERR_INVALID_ARG, "record (t=%d, l=%d) outside the dictionary", t, l);
-  const int64_t ly = d->layer(t, l);
-  if (d->layer_set[ly]) return fail(CALIBATT_ERR_INVALID_ARG, "layer (t=%d, l=%d) is already set", t, l);
-  if (!row_ptr) return fail(CALIBATT_ERR_INVALID_ARG, "row_ptr is NULL");
-  const int H = d->H, nq = d->nq;
-  std::vector<int64_t> head_off(H + 1, 0);
-  char what[64];
-  for (int h = 0; h < H; ++h) {
-    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
-    snprintf(what, sizeof(what), "layer (%d, %d) head %d", t, l, h);
-    calibatt_status st = validate_csr(nq, d->nk, rp, col_idx ? col_idx + head_off[h] : nullptr, false, what);
-    if (st != CALIBATT_OK) return st;
-    if (repetitive && repetitive[h] && rp[nq] != 0)
-      return fail(CALIBATT_ERR_INVALID_ARG, "%s is repetitive but has a non-empty skip list", what);
-    head_off[h + 1] = head_off[h] + rp[nq];
-  }
-  const int64_t nnz = head_off[H];
-  if (!d->bitmap && d->nnz_used + nnz > d->nnz_cap)
-    return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld)",
-                (long long)d->nnz_used, (long long)nnz, (long long)d->nnz_cap);
-  std::vector<uint16_t> col16(d->bitmap ? 0 : nnz);
-  for (size_t i = 0; i < col16.size(); ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
-  std::vector<uint32_t> bits;
-  if (d->bitmap) {
-    bits.assign(static_cast<size_t>(H) * nq * d->words, 0u);
+  return guarded([&]() -> calibatt_status {
+    if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+    if (t < 0 || t >= d->T || l < 0 || l >= d->L)
+      return fail(CALIBATT_ERR_INVALID_ARG, "record (t=%d, l=%d) outside the dictionary", t, l);
+    const int64_t ly = d->layer(t, l);
+    if (d->layer_set[ly]) return fail(CALIBATT_ERR_INVALID_ARG, "layer (t=%d, l=%d) is already set", t, l);
+    if (!row_ptr) return fail(CALIBATT_ERR_INVALID_ARG, "row_ptr is NULL");
+    const int H = d->H, nq = d->nq;
+    std::vector<int64_t> head_off(H + 1, 0);
+    char what[64];
     for (int h = 0; h < H; ++h) {
       const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
-      for (int r = 0; r < nq; ++r)
-        for (int32_t x = rp[r]; x < rp[r + 1]; ++x) {
-          const int32_t c = col_idx[head_off[h] + x];
-          bits[(static_cast<size_t>(h) * nq + r) * d->words + (c >> 5)] |= 1u << (c & 31);
-        }
+      snprintf(what, sizeof(what), "layer (%d, %d) head %d", t, l, h);
+      calibatt_status st = validate_csr(nq, d->nk, rp, col_idx ? col_idx + head_off[h] : nullptr, false, what);
+      if (st != CALIBATT_OK) return st;
+      if (repetitive && repetitive[h] && rp[nq] != 0)
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s is repetitive but has a non-empty skip list", what);
+      head_off[h + 1] = head_off[h] + rp[nq];
     }
-  }
-  std::vector<int64_t> col_base(H);
-  for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + head_off[h];
-  // Work items of the sparse heads and their LPT schedule over the grid.
-  std::vector<uint32_t> items;
-  std::vector<int64_t> cost;
-  std::vector<int32_t> group;
-  int32_t n_sparse = 0, n_rep = 0;
-  int64_t retained = 0;
-  const int32_t hpg = heads_per_group(nq);
-  for (int h = 0; h < H; ++h) {
-    if (repetitive && repetitive[h]) {
-      ++n_rep;
-      continue;
-    }
-    const int32_t g = n_sparse / hpg;
-    ++n_sparse;
-    const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
-    for (int r = 0; r < nq; ++r) {
-      items.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
-      cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);  // +2: Q load and epilogue
-      group.push_back(g);
-      retained += rp[r + 1] - rp[r];
-    }
-  }
-  std::vector<int32_t> cta_ptr(d->G + 1), order(items.size());
-  lpt_grouped(static_cast<int32_t>(items.size()), cost.data(), group.data(), d->G, cta_ptr.data(), order.data());
-  std::vector<uint32_t> sched(items.size());
-  for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
-  // Joint schedule of the dual path.  All anchor tiles of the repetitive
-  // heads come first, as one group in head order (a tile visits all nq key
-  // blocks; its epilogue writes about rows / n_anchors output rows per query,
-  // counted as that many extra blocks): the equal-cost tiles go round-robin
-  // over the CTAs, so the grid works on two or three heads at a time.  The
-  // sparse items follow in the L2 groups of the sparse-only schedule, with the
-  // running balance starting from the anchor loads.  (Interleaving both kinds
-  // in head-order groups let CTAs drift several groups apart behind the large
-  // anchor tiles, and the keys and values of the heads in flight no longer
-  // fitted in L2.)
-  std::vector<uint32_t> fsched;
-  std::vector<int32_t> fcta_ptr;
-  if (d->has_geom) {
-    std::vector<uint32_t> fitems;
-    std::vector<int64_t> fcost;
-    std::vector<int32_t> fgroup;
-    const int64_t bcast = std::max<int64_t>(1, d->g_rows / static_cast<int64_t>(d->g_anchors.size()));
-    int32_t sparse_rank = 0;
-    for (int h = 0; h < H; ++h) {
-      if (repetitive && repetitive[h]) {
-        for (int tile = 0; tile < d->g_tiles; ++tile) {
-          fitems.push_back(calibatt::kItemAnchorBit | (static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(tile));
-          fcost.push_back(static_cast<int64_t>(nq) + 2 + bcast);
-          fgroup.push_back(0);
-        }
-      } else {
-        const int32_t g = 1 + sparse_rank++ / hpg;
+    const int64_t nnz = head_off[H];
+    if (!d->bitmap && d->nnz_used + nnz > d->nnz_cap)
+      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld)",
+                  (long long)d->nnz_used, (long long)nnz, (long long)d->nnz_cap);
+    std::vector<uint16_t> col16(d->bitmap ? 0 : nnz);
+    for (size_t i = 0; i < col16.size(); ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
+    std::vector<uint32_t> bits;
+    if (d->bitmap) {
+      bits.assign(static_cast<size_t>(H) * nq * d->words, 0u);
+      for (int h = 0; h < H; ++h) {
         const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
-        for (int r = 0; r < nq; ++r) {
-          fitems.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
-          fcost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
-          fgroup.push_back(g);
-        }
+        for (int r = 0; r < nq; ++r)
+          for (int32_t x = rp[r]; x < rp[r + 1]; ++x) {
+            const int32_t c = col_idx[head_off[h] + x];
+            bits[(static_cast<size_t>(h) * nq + r) * d->words + (c >> 5)] |= 1u << (c & 31);
+          }
       }
     }
-    fcta_ptr.assign(d->G + 1, 0);
-    std::vector<int32_t> forder(fitems.size());
-    lpt_grouped(static_cast<int32_t>(fitems.size()), fcost.data(), fgroup.data(), d->G, fcta_ptr.data(),
-                forder.data());
-    fsched.resize(fitems.size());
-    for (size_t i = 0; i < fitems.size(); ++i) fsched[i] = fitems[forder[i]];
-  }
-  int prev = 0;
-  cudaGetDevice(&prev);
-  if (prev != d->device) cudaSetDevice(d->device);
-  cudaError_t e = cudaSuccess;
-  if (d->bitmap) {
-    e = cudaMemcpy(d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words), bits.data(),
-                   sizeof(uint32_t) * bits.size(), cudaMemcpyHostToDevice);
-  } else {
-    if (nnz > 0)
-      e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    std::vector<int64_t> col_base(H);
+    for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + head_off[h];
+    // Work items of the sparse heads and their LPT schedule over the grid.
+    std::vector<uint32_t> items;
+    std::vector<int64_t> cost;
+    std::vector<int32_t> group;
+    int32_t n_sparse = 0, n_rep = 0;
+    int64_t retained = 0;
+    const int32_t hpg = heads_per_group(nq);
+    for (int h = 0; h < H; ++h) {
+      if (repetitive && repetitive[h]) {
+        ++n_rep;
+        continue;
+      }
+      const int32_t g = n_sparse / hpg;
+      ++n_sparse;
+      const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+      for (int r = 0; r < nq; ++r) {
+        items.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
+        cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);  // +2: Q load and epilogue
+        group.push_back(g);
+        retained += rp[r + 1] - rp[r];
+      }
+    }
+    std::vector<int32_t> cta_ptr(d->G + 1), order(items.size());
+    lpt_grouped(static_cast<int32_t>(items.size()), cost.data(), group.data(), d->G, cta_ptr.data(), order.data());
+    std::vector<uint32_t> sched(items.size());
+    for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
+    // Joint schedule of the dual path.  All anchor tiles of the repetitive
+    // heads come first, as one group in head order (a tile visits all nq key
+    // blocks; its epilogue writes about rows / n_anchors output rows per query,
+    // counted as that many extra blocks): the equal-cost tiles go round-robin
+    // over the CTAs, so the grid works on two or three heads at a time.  The
+    // sparse items follow in the L2 groups of the sparse-only schedule, with the
+    // running balance starting from the anchor loads.  (Interleaving both kinds
+    // in head-order groups let CTAs drift several groups apart behind the large
+    // anchor tiles, and the keys and values of the heads in flight no longer
+    // fitted in L2.)
+    std::vector<uint32_t> fsched;
+    std::vector<int32_t> fcta_ptr;
+    if (d->has_geom) {
+      std::vector<uint32_t> fitems;
+      std::vector<int64_t> fcost;
+      std::vector<int32_t> fgroup;
+      const int64_t bcast = std::max<int64_t>(1, d->g_rows / static_cast<int64_t>(d->g_anchors.size()));
+      int32_t sparse_rank = 0;
+      for (int h = 0; h < H; ++h) {
+        if (repetitive && repetitive[h]) {
+          for (int tile = 0; tile < d->g_tiles; ++tile) {
+            fitems.push_back(calibatt::kItemAnchorBit | (static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(tile));
+            fcost.push_back(static_cast<int64_t>(nq) + 2 + bcast);
+            fgroup.push_back(0);
+          }
+        } else {
+          const int32_t g = 1 + sparse_rank++ / hpg;
+          const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+          for (int r = 0; r < nq; ++r) {
+            fitems.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
+            fcost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
+            fgroup.push_back(g);
+          }
+        }
+      }
+      fcta_ptr.assign(d->G + 1, 0);
+      std::vector<int32_t> forder(fitems.size());
+      lpt_grouped(static_cast<int32_t>(fitems.size()), fcost.data(), fgroup.data(), d->G, fcta_ptr.data(),
+                  forder.data());
+      fsched.resize(fitems.size());
+      for (size_t i = 0; i < fitems.size(); ++i) fsched[i] = fitems[forder[i]];
+    }
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != d->device) cudaSetDevice(d->device);
+    cudaError_t e = cudaSuccess;
+    if (d->bitmap) {
+      e = cudaMemcpy(d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words), bits.data(),
+                     sizeof(uint32_t) * bits.size(), cudaMemcpyHostToDevice);
+    } else {
+      if (nnz > 0)
+        e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1),
+                       cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
+    }
+    if (e == cudaSuccess && !sched.empty())
+      e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
-      e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1),
+      e = cudaMemcpy(d->d_cta_ptr + ly * (d->G + 1), cta_ptr.data(), sizeof(int32_t) * (d->G + 1), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && d->has_geom && !fsched.empty())
+      e = cudaMemcpy(d->d_fitems + ly * d->f_stride, fsched.data(), sizeof(uint32_t) * fsched.size(),
                      cudaMemcpyHostToDevice);
-    if (e == cudaSuccess)
-      e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
-  }
-  if (e == cudaSuccess && !sched.empty())
-    e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess)
-    e = cudaMemcpy(d->d_cta_ptr + ly * (d->G + 1), cta_ptr.data(), sizeof(int32_t) * (d->G + 1), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess && d->has_geom && !fsched.empty())
-    e = cudaMemcpy(d->d_fitems + ly * d->f_stride, fsched.data(), sizeof(uint32_t) * fsched.size(),
-                   cudaMemcpyHostToDevice);
-  if (e == cudaSuccess && d->has_geom)
-    e = cudaMemcpy(d->d_fcta_ptr + ly * (d->G + 1), fcta_ptr.data(), sizeof(int32_t) * (d->G + 1),
-                   cudaMemcpyHostToDevice);
-  if (prev != d->device) cudaSetDevice(prev);
-  if (e != cudaSuccess) return cuda_fail(e, "dictionary upload");
-  d->nnz_used += nnz;
-  for (int h = 0; h < H; ++h) d->rep[ly * H + h] = (repetitive && repetitive[h]) ? 1 : 0;
-  d->n_sparse[ly] = n_sparse;
-  d->n_rep[ly] = n_rep;
-  d->retained[ly] = retained;
-  d->layer_set[ly] = 1;
-  return CALIBATT_OK;
+    if (e == cudaSuccess && d->has_geom)
+      e = cudaMemcpy(d->d_fcta_ptr + ly * (d->G + 1), fcta_ptr.data(), sizeof(int32_t) * (d->G + 1),
+                     cudaMemcpyHostToDevice);
+    if (prev != d->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) return cuda_fail(e, "dictionary upload");
+    d->nnz_used += nnz;
+    for (int h = 0; h < H; ++h) d->rep[ly * H + h] = (repetitive && repetitive[h]) ? 1 : 0;
+    d->n_sparse[ly] = n_sparse;
+    d->n_rep[ly] = n_rep;
+    d->retained[ly] = retained;
+    d->layer_set[ly] = 1;
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* d, int32_t frames, int32_t rows, int32_t cols,
                                                   const int32_t* anchor_rows, int32_t n_anchors) {
-  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
-  if (d->has_geom) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry is already set");
-  for (uint8_t set : d->layer_set)
-    if (set) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry must be set before the first layer");
-  if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
-  const int64_t tokens = static_cast<int64_t>(frames) * rows * cols;
-  if (ceil_div(tokens, d->block) != d->nq)
-    return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld tokens do not make the dictionary's %d blocks",
-                (long long)tokens, d->nq);
-  if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
-    return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
-  for (int a = 0; a < n_anchors; ++a) {
-    if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
-      return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
-    if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
-      return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
-  }
-  if (d->H > 32767) return fail(CALIBATT_ERR_UNSUPPORTED, "joint schedules need H <= 32767");
-  const int64_t tiles = ceil_div(static_cast<int64_t>(frames) * n_anchors * cols, 128);
-  if (tiles > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 anchor tiles per head");
-  const int64_t layers = static_cast<int64_t>(d->T) * d->L;
-  const int64_t stride = static_cast<int64_t>(d->H) * std::max<int64_t>(d->nq, tiles);
-  int prev = 0;
-  cudaGetDevice(&prev);
-  if (prev != d->device) cudaSetDevice(d->device);
-  cudaError_t e = cudaMalloc(&d->d_fitems, sizeof(uint32_t) * layers * stride);
-  if (e == cudaSuccess) e = cudaMalloc(&d->d_fcta_ptr, sizeof(int32_t) * layers * (d->G + 1));
-  if (prev != d->device) cudaSetDevice(prev);
-  if (e != cudaSuccess) {
-    cudaFree(d->d_fitems);
-    cudaFree(d->d_fcta_ptr);
-    d->d_fitems = nullptr;
-    d->d_fcta_ptr = nullptr;
-    return cuda_fail(e, "joint schedule allocation");
-  }
-  d->device_bytes += static_cast<int64_t>(sizeof(uint32_t) * layers * stride + sizeof(int32_t) * layers * (d->G + 1));
-  d->f_stride = stride;
-  d->g_frames = frames;
-  d->g_rows = rows;
-  d->g_cols = cols;
-  d->g_tiles = static_cast<int32_t>(tiles);
-  d->g_anchors.assign(anchor_rows, anchor_rows + n_anchors);
-  d->has_geom = true;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+    if (d->has_geom) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry is already set");
+    for (uint8_t set : d->layer_set)
+      if (set) return fail(CALIBATT_ERR_INVALID_ARG, "the anchor geometry must be set before the first layer");
+    if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
+    const int64_t tokens = static_cast<int64_t>(frames) * rows * cols;
+    if (ceil_div(tokens, d->block) != d->nq)
+      return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld tokens do not make the dictionary's %d blocks",
+                  (long long)tokens, d->nq);
+    if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
+      return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
+    for (int a = 0; a < n_anchors; ++a) {
+      if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
+        return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
+      if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
+        return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
+    }
+    if (d->H > 32767) return fail(CALIBATT_ERR_UNSUPPORTED, "joint schedules need H <= 32767");
+    const int64_t tiles = ceil_div(static_cast<int64_t>(frames) * n_anchors * cols, 128);
+    if (tiles > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 anchor tiles per head");
+    const int64_t layers = static_cast<int64_t>(d->T) * d->L;
+    const int64_t stride = static_cast<int64_t>(d->H) * std::max<int64_t>(d->nq, tiles);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != d->device) cudaSetDevice(d->device);
+    cudaError_t e = cudaMalloc(&d->d_fitems, sizeof(uint32_t) * layers * stride);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_fcta_ptr, sizeof(int32_t) * layers * (d->G + 1));
+    if (prev != d->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) {
+      cudaFree(d->d_fitems);
+      cudaFree(d->d_fcta_ptr);
+      d->d_fitems = nullptr;
+      d->d_fcta_ptr = nullptr;
+      return cuda_fail(e, "joint schedule allocation");
+    }
+    d->device_bytes += static_cast<int64_t>(sizeof(uint32_t) * layers * stride + sizeof(int32_t) * layers * (d->G + 1));
+    d->f_stride = stride;
+    d->g_frames = frames;
+    d->g_rows = rows;
+    d->g_cols = cols;
+    d->g_tiles = static_cast<int32_t>(tiles);
+    d->g_anchors.assign(anchor_rows, anchor_rows + n_anchors);
+    d->has_geom = true;
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_info(const calibatt_dict* d, int64_t* device_bytes, int64_t* nnz_total,
                                    int32_t* num_ctas) {
-  if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
-  if (device_bytes) *device_bytes = d->device_bytes;
-  if (nnz_total) *nnz_total = d->nnz_used;
-  if (num_ctas) *num_ctas = d->G;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
+    if (device_bytes) *device_bytes = d->device_bytes;
+    if (nnz_total) *nnz_total = d->nnz_used;
+    if (num_ctas) *num_ctas = d->G;
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_layer_info(const calibatt_dict* d, int32_t t, int32_t l, int32_t* n_sparse_heads,
                                          int32_t* n_repetitive_heads, int64_t* retained_tiles) {
-  calibatt_status st = check_dict_layer(d, t, l);
-  if (st != CALIBATT_OK) return st;
-  const int64_t ly = d->layer(t, l);
-  if (n_sparse_heads) *n_sparse_heads = d->n_sparse[ly];
-  if (n_repetitive_heads) *n_repetitive_heads = d->n_rep[ly];
-  if (retained_tiles) *retained_tiles = d->retained[ly];
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st = check_dict_layer(d, t, l);
+    if (st != CALIBATT_OK) return st;
+    const int64_t ly = d->layer(t, l);
+    if (n_sparse_heads) *n_sparse_heads = d->n_sparse[ly];
+    if (n_repetitive_heads) *n_repetitive_heads = d->n_rep[ly];
+    if (retained_tiles) *retained_tiles = d->retained[ly];
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_dict_destroy(calibatt_dict* d) {
-  if (!d) return CALIBATT_OK;
-  int prev = 0;
-  cudaGetDevice(&prev);
-  if (prev != d->device) cudaSetDevice(d->device);
-  cudaDeviceSynchronize();
-  d->release();
-  if (prev != d->device) cudaSetDevice(prev);
-  delete d;
-  cudaGetLastError();
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!d) return CALIBATT_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != d->device) cudaSetDevice(d->device);
+    cudaDeviceSynchronize();
+    d->release();
+    if (prev != d->device) cudaSetDevice(prev);
+    delete d;
+    cudaGetLastError();
+    return CALIBATT_OK;
+  });
 }
 
 // ------------------------------------------------------------ dictionary file
@@ -1084,93 +1129,95 @@ struct DictReader {
 }  // namespace
 
 calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
-  if (!d || !path) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary and path must be non-NULL");
-  const int H = d->H, nq = d->nq;
-  const int64_t layers = static_cast<int64_t>(d->T) * d->L;
-  DictFileHeader hd;
-  std::memset(&hd, 0, sizeof(hd));
-  std::memcpy(hd.magic, kDictMagic, 8);
-  hd.version = kDictFileVersion;
-  hd.format = d->bitmap ? 1u : 0u;
-  hd.T = d->T;
-  hd.L = d->L;
-  hd.H = H;
-  hd.nq = nq;
-  hd.nk = d->nk;
-  hd.block = d->block;
-  if (d->has_geom) {
-    hd.has_geom = 1;
-    hd.frames = d->g_frames;
-    hd.rows = d->g_rows;
-    hd.cols = d->g_cols;
-    hd.n_anchors = static_cast<int32_t>(d->g_anchors.size());
-    for (size_t a = 0; a < d->g_anchors.size(); ++a) hd.anchors[a] = d->g_anchors[a];
-  }
-  for (uint8_t set : d->layer_set) hd.records += set;
-  hd.nnz_total = d->nnz_used;
-  const std::string tmp = std::string(path) + ".tmp";
-  DictWriter w;
-  w.f = std::fopen(tmp.c_str(), "wb");
-  if (!w.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s for writing", tmp.c_str());
-  int prev = 0;
-  cudaGetDevice(&prev);
-  if (prev != d->device) cudaSetDevice(d->device);
-  cudaError_t e = cudaSuccess;
-  w.put(&hd, sizeof(hd));
-  std::vector<int32_t> rp;
-  std::vector<int64_t> cb;
-  std::vector<uint16_t> col;
-  std::vector<uint32_t> bits;
-  for (int64_t ly = 0; ly < layers && w.ok && e == cudaSuccess; ++ly) {
-    if (!d->layer_set[ly]) continue;
-    DictFileRecord rec{static_cast<int32_t>(ly / d->L), static_cast<int32_t>(ly % d->L), 0};
-    if (d->bitmap) {
-      bits.resize(static_cast<size_t>(H) * nq * d->words);
-      e = cudaMemcpy(bits.data(), d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words),
-                     sizeof(uint32_t) * bits.size(), cudaMemcpyDeviceToHost);
-      for (uint32_t x : bits) rec.nnz += __builtin_popcount(x);
-    } else {
-      rp.resize(static_cast<size_t>(H) * (nq + 1));
-      cb.resize(H);
-      e = cudaMemcpy(rp.data(), d->d_row_ptr + ly * H * (nq + 1), sizeof(int32_t) * rp.size(),
-                     cudaMemcpyDeviceToHost);
-      if (e == cudaSuccess)
-        e = cudaMemcpy(cb.data(), d->d_col_base + ly * H, sizeof(int64_t) * H, cudaMemcpyDeviceToHost);
-      for (int h = 0; h < H; ++h) rec.nnz += rp[static_cast<size_t>(h) * (nq + 1) + nq];
-      col.resize(rec.nnz);
-      // a layer's lists are stored contiguously, head after head, from head 0's offset
-      if (e == cudaSuccess && rec.nnz > 0)
-        e = cudaMemcpy(col.data(), d->d_col + cb[0], sizeof(uint16_t) * rec.nnz, cudaMemcpyDeviceToHost);
+  return guarded([&]() -> calibatt_status {
+    if (!d || !path) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary and path must be non-NULL");
+    const int H = d->H, nq = d->nq;
+    const int64_t layers = static_cast<int64_t>(d->T) * d->L;
+    DictFileHeader hd;
+    std::memset(&hd, 0, sizeof(hd));
+    std::memcpy(hd.magic, kDictMagic, 8);
+    hd.version = kDictFileVersion;
+    hd.format = d->bitmap ? 1u : 0u;
+    hd.T = d->T;
+    hd.L = d->L;
+    hd.H = H;
+    hd.nq = nq;
+    hd.nk = d->nk;
+    hd.block = d->block;
+    if (d->has_geom) {
+      hd.has_geom = 1;
+      hd.frames = d->g_frames;
+      hd.rows = d->g_rows;
+      hd.cols = d->g_cols;
+      hd.n_anchors = static_cast<int32_t>(d->g_anchors.size());
+      for (size_t a = 0; a < d->g_anchors.size(); ++a) hd.anchors[a] = d->g_anchors[a];
     }
-    if (e != cudaSuccess) break;
-    w.put(&rec, sizeof(rec));
-    w.put(d->rep.data() + ly * H, H);
-    if (d->bitmap) {
-      w.put(bits.data(), sizeof(uint32_t) * bits.size());
-    } else {
-      w.put(rp.data(), sizeof(int32_t) * rp.size());
-      w.put(col.data(), sizeof(uint16_t) * col.size());
+    for (uint8_t set : d->layer_set) hd.records += set;
+    hd.nnz_total = d->nnz_used;
+    const std::string tmp = std::string(path) + ".tmp";
+    DictWriter w;
+    w.f = std::fopen(tmp.c_str(), "wb");
+    if (!w.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s for writing", tmp.c_str());
+    int prev = 0;
+    cudaGetDevice(&prev);
+    if (prev != d->device) cudaSetDevice(d->device);
+    cudaError_t e = cudaSuccess;
+    w.put(&hd, sizeof(hd));
+    std::vector<int32_t> rp;
+    std::vector<int64_t> cb;
+    std::vector<uint16_t> col;
+    std::vector<uint32_t> bits;
+    for (int64_t ly = 0; ly < layers && w.ok && e == cudaSuccess; ++ly) {
+      if (!d->layer_set[ly]) continue;
+      DictFileRecord rec{static_cast<int32_t>(ly / d->L), static_cast<int32_t>(ly % d->L), 0};
+      if (d->bitmap) {
+        bits.resize(static_cast<size_t>(H) * nq * d->words);
+        e = cudaMemcpy(bits.data(), d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words),
+                       sizeof(uint32_t) * bits.size(), cudaMemcpyDeviceToHost);
+        for (uint32_t x : bits) rec.nnz += __builtin_popcount(x);
+      } else {
+        rp.resize(static_cast<size_t>(H) * (nq + 1));
+        cb.resize(H);
+        e = cudaMemcpy(rp.data(), d->d_row_ptr + ly * H * (nq + 1), sizeof(int32_t) * rp.size(),
+                       cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+          e = cudaMemcpy(cb.data(), d->d_col_base + ly * H, sizeof(int64_t) * H, cudaMemcpyDeviceToHost);
+        for (int h = 0; h < H; ++h) rec.nnz += rp[static_cast<size_t>(h) * (nq + 1) + nq];
+        col.resize(rec.nnz);
+        // a layer's lists are stored contiguously, head after head, from head 0's offset
+        if (e == cudaSuccess && rec.nnz > 0)
+          e = cudaMemcpy(col.data(), d->d_col + cb[0], sizeof(uint16_t) * rec.nnz, cudaMemcpyDeviceToHost);
+      }
+      if (e != cudaSuccess) break;
+      w.put(&rec, sizeof(rec));
+      w.put(d->rep.data() + ly * H, H);
+      if (d->bitmap) {
+        w.put(bits.data(), sizeof(uint32_t) * bits.size());
+      } else {
+        w.put(rp.data(), sizeof(int32_t) * rp.size());
+        w.put(col.data(), sizeof(uint16_t) * col.size());
+      }
     }
-  }
-  if (prev != d->device) cudaSetDevice(prev);
-  if (w.ok && e == cudaSuccess) {
-    unsigned char trailer[16];
-    std::memcpy(trailer, kDictEnd, 8);
-    const uint64_t hv = w.hash.h;
-    std::memcpy(trailer + 8, &hv, 8);
-    w.ok = std::fwrite(trailer, 1, 16, w.f) == 16;
-  }
-  const bool closed = std::fclose(w.f) == 0;
-  if (e != cudaSuccess || !w.ok || !closed) {
-    std::remove(tmp.c_str());
-    if (e != cudaSuccess) return cuda_fail(e, "dictionary copy to host");
-    return fail(CALIBATT_ERR_INVALID_ARG, "writing %s failed", tmp.c_str());
-  }
-  if (std::rename(tmp.c_str(), path) != 0) {
-    std::remove(tmp.c_str());
-    return fail(CALIBATT_ERR_INVALID_ARG, "cannot rename %s to %s", tmp.c_str(), path);
-  }
-  return CALIBATT_OK;
+    if (prev != d->device) cudaSetDevice(prev);
+    if (w.ok && e == cudaSuccess) {
+      unsigned char trailer[16];
+      std::memcpy(trailer, kDictEnd, 8);
+      const uint64_t hv = w.hash.h;
+      std::memcpy(trailer + 8, &hv, 8);
+      w.ok = std::fwrite(trailer, 1, 16, w.f) == 16;
+    }
+    const bool closed = std::fclose(w.f) == 0;
+    if (e != cudaSuccess || !w.ok || !closed) {
+      std::remove(tmp.c_str());
+      if (e != cudaSuccess) return cuda_fail(e, "dictionary copy to host");
+      return fail(CALIBATT_ERR_INVALID_ARG, "writing %s failed", tmp.c_str());
+    }
+    if (std::rename(tmp.c_str(), path) != 0) {
+      std::remove(tmp.c_str());
+      return fail(CALIBATT_ERR_INVALID_ARG, "cannot rename %s to %s", tmp.c_str(), path);
+    }
+    return CALIBATT_OK;
+  });
 }
 
 namespace {
@@ -1249,69 +1296,80 @@ calibatt_status load_records(DictReader& r, const DictFileHeader& hd, calibatt_d
 }  // namespace
 
 calibatt_status calibatt_dict_load(const char* path, int32_t num_ctas, calibatt_dict** out) {
-  if (!out || !path) return fail(CALIBATT_ERR_INVALID_ARG, "path and out must be non-NULL");
-  *out = nullptr;
-  DictReader r;
-  r.f = std::fopen(path, "rb");
-  if (!r.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s", path);
-  struct Closer {
-    FILE* f;
-    ~Closer() { std::fclose(f); }
-  } closer{r.f};
-  DictFileHeader hd;
-  if (!r.get(&hd, sizeof(hd)) || std::memcmp(hd.magic, kDictMagic, 8) != 0)
-    return fail(CALIBATT_ERR_INVALID_ARG, "%s is not a dictionary file", path);
-  if (hd.version != kDictFileVersion || hd.format > 1 || hd.reserved != 0)
-    return fail(CALIBATT_ERR_INVALID_ARG, "%s: unsupported version %u / format %u", path, hd.version, hd.format);
-  if (hd.T < 1 || hd.L < 1 || hd.H < 1 || hd.nq < 1 || hd.nk != hd.nq || hd.H > 65535 || hd.nq > 65535 ||
-      (hd.block != 64 && hd.block != 128) || hd.records < 0 || hd.records > static_cast<int64_t>(hd.T) * hd.L ||
-      hd.nnz_total < 0 || (hd.format == 1 && hd.nq > calibatt::kMaxBitmapBlocks) || hd.n_anchors < 0 ||
-      hd.n_anchors > calibatt::kMaxAnchors || (hd.has_geom != 0 && hd.has_geom != 1))
-    return fail(CALIBATT_ERR_INVALID_ARG, "%s: header fields out of range", path);
-  calibatt_dict* d = nullptr;
-  calibatt_status st = hd.format == 1
-      ? calibatt_dict_create_bitmap(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, num_ctas, &d)
-      : calibatt_dict_create(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d);
-  if (st != CALIBATT_OK) return st;
-  if (hd.has_geom) st = calibatt_dict_set_anchor_geometry(d, hd.frames, hd.rows, hd.cols, hd.anchors, hd.n_anchors);
-  if (st == CALIBATT_OK) st = load_records(r, hd, d, path);
-  if (st == CALIBATT_OK) {
-    const uint64_t want = r.hash.h;
-    unsigned char trailer[16];
-    uint64_t got = 0;
-    if (std::fread(trailer, 1, 16, r.f) != 16 || std::memcmp(trailer, kDictEnd, 8) != 0) {
-      st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailer missing", path);
-    } else {
-      std::memcpy(&got, trailer + 8, 8);
-      if (got != want) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: checksum mismatch", path);
-      else if (std::fgetc(r.f) != EOF) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailing bytes", path);
+  return guarded([&]() -> calibatt_status {
+    if (!out || !path) return fail(CALIBATT_ERR_INVALID_ARG, "path and out must be non-NULL");
+    *out = nullptr;
+    DictReader r;
+    r.f = std::fopen(path, "rb");
+    if (!r.f) return fail(CALIBATT_ERR_INVALID_ARG, "cannot open %s", path);
+    struct Closer {
+      FILE* f;
+      ~Closer() { std::fclose(f); }
+    } closer{r.f};
+    DictFileHeader hd;
+    if (!r.get(&hd, sizeof(hd)) || std::memcmp(hd.magic, kDictMagic, 8) != 0)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s is not a dictionary file", path);
+    if (hd.version != kDictFileVersion || hd.format > 1 || hd.reserved != 0)
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: unsupported version %u / format %u", path, hd.version, hd.format);
+    if (hd.T < 1 || hd.L < 1 || hd.H < 1 || hd.nq < 1 || hd.nk != hd.nq || hd.H > 65535 || hd.nq > 65535 ||
+        (hd.block != 64 && hd.block != 128) || hd.records < 0 || hd.records > static_cast<int64_t>(hd.T) * hd.L ||
+        hd.nnz_total < 0 || (hd.format == 1 && hd.nq > calibatt::kMaxBitmapBlocks) || hd.n_anchors < 0 ||
+        hd.n_anchors > calibatt::kMaxAnchors || (hd.has_geom != 0 && hd.has_geom != 1))
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: header fields out of range", path);
+    calibatt_dict* d = nullptr;
+    calibatt_status st = hd.format == 1
+        ? calibatt_dict_create_bitmap(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, num_ctas, &d)
+        : calibatt_dict_create(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d);
+    if (st != CALIBATT_OK) return st;
+    if (hd.has_geom) st = calibatt_dict_set_anchor_geometry(d, hd.frames, hd.rows, hd.cols, hd.anchors, hd.n_anchors);
+    if (st == CALIBATT_OK) {
+      try {
+        st = load_records(r, hd, d, path);
+      } catch (...) {
+        calibatt_dict_destroy(d);  // then the guard reports the exception
+        throw;
+      }
     }
-  }
-  if (st != CALIBATT_OK) {
-    const std::string msg = g_last_error;
-    calibatt_dict_destroy(d);
-    g_last_error = msg;
-    return st;
-  }
-  *out = d;
-  return CALIBATT_OK;
+    if (st == CALIBATT_OK) {
+      const uint64_t want = r.hash.h;
+      unsigned char trailer[16];
+      uint64_t got = 0;
+      if (std::fread(trailer, 1, 16, r.f) != 16 || std::memcmp(trailer, kDictEnd, 8) != 0) {
+        st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailer missing", path);
+      } else {
+        std::memcpy(&got, trailer + 8, 8);
+        if (got != want) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: checksum mismatch", path);
+        else if (std::fgetc(r.f) != EOF) st = fail(CALIBATT_ERR_INVALID_ARG, "%s: trailing bytes", path);
+      }
+    }
+    if (st != CALIBATT_OK) {
+      const std::string msg = g_last_error;
+      calibatt_dict_destroy(d);
+      g_last_error = msg;
+      return st;
+    }
+    *out = d;
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const void* v, void* o,
                                            const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
                                            int32_t t, int32_t l, float softmax_scale, float* lse, void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
-  if ((st = check_block(block)) != CALIBATT_OK) return st;
-  if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
-  if (dict->H != shape->heads) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
-  if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
-  if (dict->nq != ceil_div(shape->seq_len, block))
-    return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq, shape->seq_len,
-                ceil_div(shape->seq_len, block));
-  if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-  return launch_sparse(q, k, v, o, *shape, block, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+    if ((st = check_block(block)) != CALIBATT_OK) return st;
+    if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
+    if (dict->H != shape->heads) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
+    if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
+    if (dict->nq != ceil_div(shape->seq_len, block))
+      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq, shape->seq_len,
+                  ceil_div(shape->seq_len, block));
+    if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    return launch_sparse(q, k, v, o, *shape, block, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
+  });
 }
 
 calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* k_host, const void* v_host,
@@ -1319,28 +1377,30 @@ calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* 
                                                 const calibatt_shape* shape, int32_t block, const calibatt_dict* dict,
                                                 int32_t t, int32_t l, float softmax_scale, float* lse,
                                                 void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if (!q_host || !k_host || !v_host || !o_host)
-    return fail(CALIBATT_ERR_INVALID_ARG, "host buffers must be non-NULL");
-  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
-  // bytes from each tensor's base to one past its last element
-  const int64_t elt = shape->dtype == CALIBATT_DTYPE_BF16 ? 2 : 4;
-  const int64_t extent = ((static_cast<int64_t>(shape->batch) - 1) * shape->stride_b +
-                          (static_cast<int64_t>(shape->seq_len) - 1) * shape->stride_n +
-                          (static_cast<int64_t>(shape->heads) - 1) * shape->stride_h + shape->head_dim) * elt;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const void* src[3] = {q_host, k_host, v_host};
-  void* dst[3] = {q, k, v};
-  for (int i = 0; i < 3; ++i) {
-    cudaError_t e = cudaMemcpyAsync(dst[i], src[i], static_cast<size_t>(extent), cudaMemcpyHostToDevice, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  }
-  st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
-  if (st != CALIBATT_OK) return st;
-  cudaError_t e = cudaMemcpyAsync(o_host, o, static_cast<size_t>(extent), cudaMemcpyDeviceToHost, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if (!q_host || !k_host || !v_host || !o_host)
+      return fail(CALIBATT_ERR_INVALID_ARG, "host buffers must be non-NULL");
+    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+    // bytes from each tensor's base to one past its last element
+    const int64_t elt = shape->dtype == CALIBATT_DTYPE_BF16 ? 2 : 4;
+    const int64_t extent = ((static_cast<int64_t>(shape->batch) - 1) * shape->stride_b +
+                            (static_cast<int64_t>(shape->seq_len) - 1) * shape->stride_n +
+                            (static_cast<int64_t>(shape->heads) - 1) * shape->stride_h + shape->head_dim) * elt;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const void* src[3] = {q_host, k_host, v_host};
+    void* dst[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i) {
+      cudaError_t e = cudaMemcpyAsync(dst[i], src[i], static_cast<size_t>(extent), cudaMemcpyHostToDevice, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    }
+    st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
+    if (st != CALIBATT_OK) return st;
+    cudaError_t e = cudaMemcpyAsync(o_host, o, static_cast<size_t>(extent), cudaMemcpyDeviceToHost, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, const void* v, void* o,
@@ -1349,64 +1409,68 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
                                                const int32_t* head_ids, int32_t n_heads, const uint32_t* items,
                                                const int32_t* cta_ptr, int32_t grid, float softmax_scale, float* lse,
                                                void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
-  if ((st = check_block(block)) != CALIBATT_OK) return st;
-  if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
-    return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
-  if (n_heads == 0) return CALIBATT_OK;
-  if (!head_ids || !row_ptr || !col_idx || !col_base)
-    return fail(CALIBATT_ERR_INVALID_ARG, "head_ids, row_ptr, col_idx and col_base must be non-NULL");
-  const int32_t nq = ceil_div(shape->seq_len, block);
-  if (nq > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
-  std::vector<uint8_t> seen(shape->heads, 0);
-  std::vector<int16_t> heads;
-  for (int i = 0; i < n_heads; ++i) {
-    if (head_ids[i] < 0 || head_ids[i] >= shape->heads)
-      return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", head_ids[i], shape->heads);
-    if (seen[head_ids[i]]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", head_ids[i]);
-    heads.push_back(static_cast<int16_t>(head_ids[i]));
-  }
-  const bool tc = shape->dtype == CALIBATT_DTYPE_BF16 && block == 128;
-  if (tc && (!items || !cta_ptr || grid < 1))
-    return fail(CALIBATT_ERR_INVALID_ARG, "the tensor-core path needs a device schedule (items, cta_ptr, grid >= 1)");
-  if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-  // the lists were never read on the host: check them on the device first
-  calibatt::CsrCheckParams chk;
-  std::memset(&chk, 0, sizeof(chk));
-  chk.row_ptr = row_ptr;
-  chk.col = col_idx;
-  chk.col_base = col_base;
-  chk.nq = nq;
-  chk.n_heads = n_heads;
-  for (int i = 0; i < n_heads; ++i) chk.head_ids[i] = heads[i];
-  chk.status = status_word_ptr();
-  if (!chk.status) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
-  cudaError_t e = calibatt::launch_csr_check(chk, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "skip-list check launch");
-  LayerSchedule sch;
-  std::memset(&sch, 0, sizeof(sch));
-  sch.row_ptr = row_ptr;
-  sch.col_base = col_base;
-  sch.col = col_idx;
-  sch.items = items;
-  sch.cta_ptr = cta_ptr;
-  sch.nq = nq;
-  return run_sparse(q, k, v, o, *shape, block, sch, tc ? grid : 1, heads, softmax_scale, lse,
-                    static_cast<cudaStream_t>(stream));
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+    if ((st = check_block(block)) != CALIBATT_OK) return st;
+    if (n_heads < 0 || n_heads > calibatt::kMaxHeadsPerCall)
+      return fail(CALIBATT_ERR_INVALID_ARG, "n_heads must be in [0, %d]", calibatt::kMaxHeadsPerCall);
+    if (n_heads == 0) return CALIBATT_OK;
+    if (!head_ids || !row_ptr || !col_idx || !col_base)
+      return fail(CALIBATT_ERR_INVALID_ARG, "head_ids, row_ptr, col_idx and col_base must be non-NULL");
+    const int32_t nq = ceil_div(shape->seq_len, block);
+    if (nq > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
+    std::vector<uint8_t> seen(shape->heads, 0);
+    std::vector<int16_t> heads;
+    for (int i = 0; i < n_heads; ++i) {
+      if (head_ids[i] < 0 || head_ids[i] >= shape->heads)
+        return fail(CALIBATT_ERR_INVALID_ARG, "head id %d outside [0, %d)", head_ids[i], shape->heads);
+      if (seen[head_ids[i]]++) return fail(CALIBATT_ERR_INVALID_ARG, "head id %d listed twice", head_ids[i]);
+      heads.push_back(static_cast<int16_t>(head_ids[i]));
+    }
+    const bool tc = shape->dtype == CALIBATT_DTYPE_BF16 && block == 128;
+    if (tc && (!items || !cta_ptr || grid < 1))
+      return fail(CALIBATT_ERR_INVALID_ARG, "the tensor-core path needs a device schedule (items, cta_ptr, grid >= 1)");
+    if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    // the lists were never read on the host: check them on the device first
+    calibatt::CsrCheckParams chk;
+    std::memset(&chk, 0, sizeof(chk));
+    chk.row_ptr = row_ptr;
+    chk.col = col_idx;
+    chk.col_base = col_base;
+    chk.nq = nq;
+    chk.n_heads = n_heads;
+    for (int i = 0; i < n_heads; ++i) chk.head_ids[i] = heads[i];
+    chk.status = status_word_ptr();
+    if (!chk.status) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+    cudaError_t e = calibatt::launch_csr_check(chk, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "skip-list check launch");
+    LayerSchedule sch;
+    std::memset(&sch, 0, sizeof(sch));
+    sch.row_ptr = row_ptr;
+    sch.col_base = col_base;
+    sch.col = col_idx;
+    sch.items = items;
+    sch.cta_ptr = cta_ptr;
+    sch.nq = nq;
+    return run_sparse(q, k, v, o, *shape, block, sch, tc ? grid : 1, heads, softmax_scale, lse,
+                      static_cast<cudaStream_t>(stream));
+  });
 }
 
 calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
                                      const calibatt_shape* shape, int32_t block, int32_t frames, int32_t rows,
                                      int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
                                      const int32_t* head_ids, int32_t n_heads, float softmax_scale, void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
-  if ((st = check_block(block)) != CALIBATT_OK) return st;
-  return launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, head_ids, n_heads,
-                       softmax_scale, static_cast<cudaStream_t>(stream));
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+    if ((st = check_block(block)) != CALIBATT_OK) return st;
+    return launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, head_ids, n_heads,
+                         softmax_scale, static_cast<cudaStream_t>(stream));
+  });
 }
 
 calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void* v, void* o,
@@ -1414,281 +1478,307 @@ calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void
                                         int32_t t, int32_t l, int32_t frames, int32_t rows, int32_t cols,
                                         const int32_t* anchor_rows, int32_t n_anchors, float softmax_scale,
                                         float* lse, void* stream) {
-  // One launch when the dictionary carries this call's anchor geometry and
-  // the tensor-core path applies; otherwise the sparse and anchor launches.
-  if (dict && shape && dict->has_geom && shape->dtype == CALIBATT_DTYPE_BF16 && block == 128 &&
-      frames == dict->g_frames && rows == dict->g_rows && cols == dict->g_cols && anchor_rows &&
-      n_anchors == static_cast<int32_t>(dict->g_anchors.size()) &&
-      std::equal(dict->g_anchors.begin(), dict->g_anchors.end(), anchor_rows)) {
-    calibatt_status st;
-    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-    if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
-    if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
-    if (dict->H != shape->heads)
-      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
-    if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
-    if (dict->nq != ceil_div(shape->seq_len, block))
-      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq,
-                  shape->seq_len, ceil_div(shape->seq_len, block));
-    if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
-      return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
-                  shape->seq_len);
-    if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-    const int64_t ly = dict->layer(t, l);
-    if (dict->n_sparse[ly] + dict->n_rep[ly] == 0) return CALIBATT_OK;
-    return launch_fused(q, k, v, o, *shape, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
-  }
-  calibatt_status st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
-  if (st != CALIBATT_OK) return st;
-  const int64_t ly = dict->layer(t, l);
-  std::vector<int32_t> heads;
-  for (int h = 0; h < dict->H; ++h)
-    if (dict->rep[ly * dict->H + h]) heads.push_back(h);
-  if (heads.empty()) return CALIBATT_OK;
-  for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
-    const int32_t nh = static_cast<int32_t>(std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0));
-    st = launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, heads.data() + h0, nh,
-                       softmax_scale, static_cast<cudaStream_t>(stream));
+  return guarded([&]() -> calibatt_status {
+    // One launch when the dictionary carries this call's anchor geometry and
+    // the tensor-core path applies; otherwise the sparse and anchor launches.
+    if (dict && shape && dict->has_geom && shape->dtype == CALIBATT_DTYPE_BF16 && block == 128 &&
+        frames == dict->g_frames && rows == dict->g_rows && cols == dict->g_cols && anchor_rows &&
+        n_anchors == static_cast<int32_t>(dict->g_anchors.size()) &&
+        std::equal(dict->g_anchors.begin(), dict->g_anchors.end(), anchor_rows)) {
+      calibatt_status st;
+      if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+      if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
+      if ((st = check_dict_layer(dict, t, l)) != CALIBATT_OK) return st;
+      if (dict->H != shape->heads)
+        return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d heads, shape %d", dict->H, shape->heads);
+      if (dict->block != block) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary block %d != %d", dict->block, block);
+      if (dict->nq != ceil_div(shape->seq_len, block))
+        return fail(CALIBATT_ERR_INVALID_ARG, "dictionary has %d blocks, seq_len %d needs %d", dict->nq,
+                    shape->seq_len, ceil_div(shape->seq_len, block));
+      if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
+        return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
+                    shape->seq_len);
+      if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(CALIBATT_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+      const int64_t ly = dict->layer(t, l);
+      if (dict->n_sparse[ly] + dict->n_rep[ly] == 0) return CALIBATT_OK;
+      return launch_fused(q, k, v, o, *shape, dict, t, l, softmax_scale, lse, static_cast<cudaStream_t>(stream));
+    }
+    calibatt_status st = calibatt_block_sparse_attn(q, k, v, o, shape, block, dict, t, l, softmax_scale, lse, stream);
     if (st != CALIBATT_OK) return st;
-  }
-  return CALIBATT_OK;
+    const int64_t ly = dict->layer(t, l);
+    std::vector<int32_t> heads;
+    for (int h = 0; h < dict->H; ++h)
+      if (dict->rep[ly * dict->H + h]) heads.push_back(h);
+    if (heads.empty()) return CALIBATT_OK;
+    for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
+      const int32_t nh = static_cast<int32_t>(std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0));
+      st = launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, heads.data() + h0, nh,
+                         softmax_scale, static_cast<cudaStream_t>(stream));
+      if (st != CALIBATT_OK) return st;
+    }
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_block_energy_workspace_size(const calibatt_shape* shape, size_t* bytes) {
-  calibatt_status st = check_shape(shape);
-  if (st != CALIBATT_OK) return st;
-  if (!bytes) return fail(CALIBATT_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = sizeof(float) * static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st = check_shape(shape);
+    if (st != CALIBATT_OK) return st;
+    if (!bytes) return fail(CALIBATT_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = sizeof(float) * static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len;
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_block_energy(const void* q, const void* k, const calibatt_shape* shape, int32_t block,
                                       float softmax_scale, float* energy, void* workspace, size_t workspace_bytes,
                                       void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if ((st = check_block(block)) != CALIBATT_OK) return st;
-  if (!q || !k || !energy || !workspace) return fail(CALIBATT_ERR_INVALID_ARG, "q, k, energy and workspace must be non-NULL");
-  size_t need = 0;
-  calibatt_block_energy_workspace_size(shape, &need);
-  if (workspace_bytes < need)
-    return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
-  const int nb = ceil_div(shape->seq_len, block);
-  if (nb > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
-  if (shape->dtype == CALIBATT_DTYPE_BF16 && block == 128) {
-    // Tensor-core path: the LSE pass, then the energy pass, as persistent
-    // launches of the attention pipeline without V.
-    TcParams t;
-    std::memset(&t, 0, sizeof(t));
-    if ((st = encode_qkv_map(&t.tm_q, q, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
-    if ((st = encode_qkv_map(&t.tm_k, k, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
-    t.tm_v = t.tm_k;  // no V in these modes
-    t.q = static_cast<const uint16_t*>(q);
-    t.lse = static_cast<float*>(workspace);
-    t.energy = energy;
-    t.sb = shape->stride_b;
-    t.sn = shape->stride_n;
-    t.sh = shape->stride_h;
-    t.batch = shape->batch;
-    t.seq_len = shape->seq_len;
-    t.heads = shape->heads;
-    t.nb = nb;
-    t.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
-    t.status = status_word_ptr();
-    t.timeout_ns = g_timeout_ns.load();
-    const int sms = device_sm_count();
-    if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
-    const int grid = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(shape->heads) * nb));
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    cudaError_t e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeLse, grid, cs);
-    if (e == cudaSuccess) e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeEnergy, grid, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core block energy launch");
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if ((st = check_block(block)) != CALIBATT_OK) return st;
+    if (!q || !k || !energy || !workspace) return fail(CALIBATT_ERR_INVALID_ARG, "q, k, energy and workspace must be non-NULL");
+    size_t need = 0;
+    calibatt_block_energy_workspace_size(shape, &need);
+    if (workspace_bytes < need)
+      return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+    const int nb = ceil_div(shape->seq_len, block);
+    if (nb > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 65535 blocks");
+    if (shape->dtype == CALIBATT_DTYPE_BF16 && block == 128) {
+      // Tensor-core path: the LSE pass, then the energy pass, as persistent
+      // launches of the attention pipeline without V.
+      TcParams t;
+      std::memset(&t, 0, sizeof(t));
+      if ((st = encode_qkv_map(&t.tm_q, q, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+      if ((st = encode_qkv_map(&t.tm_k, k, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+      t.tm_v = t.tm_k;  // no V in these modes
+      t.q = static_cast<const uint16_t*>(q);
+      t.lse = static_cast<float*>(workspace);
+      t.energy = energy;
+      t.sb = shape->stride_b;
+      t.sn = shape->stride_n;
+      t.sh = shape->stride_h;
+      t.batch = shape->batch;
+      t.seq_len = shape->seq_len;
+      t.heads = shape->heads;
+      t.nb = nb;
+      t.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
+      t.status = status_word_ptr();
+      t.timeout_ns = g_timeout_ns.load();
+      const int sms = device_sm_count();
+      if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+      const int grid = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(shape->heads) * nb));
+      cudaStream_t cs = static_cast<cudaStream_t>(stream);
+      cudaError_t e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeLse, grid, cs);
+      if (e == cudaSuccess) e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeEnergy, grid, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "tensor-core block energy launch");
+      return CALIBATT_OK;
+    }
+    calibatt::EnergyParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.energy = energy;
+    p.lse = static_cast<float*>(workspace);
+    p.sb = shape->stride_b;
+    p.sn = shape->stride_n;
+    p.sh = shape->stride_h;
+    p.batch = shape->batch;
+    p.seq_len = shape->seq_len;
+    p.heads = shape->heads;
+    p.nb = nb;
+    p.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
+    cudaError_t e = calibatt::launch_block_energy(p, shape->head_dim, block, shape->dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "block energy launch");
     return CALIBATT_OK;
-  }
-  calibatt::EnergyParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.q = q;
-  p.k = k;
-  p.energy = energy;
-  p.lse = static_cast<float*>(workspace);
-  p.sb = shape->stride_b;
-  p.sn = shape->stride_n;
-  p.sh = shape->stride_h;
-  p.batch = shape->batch;
-  p.seq_len = shape->seq_len;
-  p.heads = shape->heads;
-  p.nb = nb;
-  p.scale_log2 = scale_log2_of(softmax_scale, shape->head_dim);
-  cudaError_t e = calibatt::launch_block_energy(p, shape->head_dim, block, shape->dtype, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "block energy launch");
-  return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_spatial_similarity(const void* q, const void* k, const calibatt_shape* shape, int32_t frames,
                                             int32_t rows, int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
                                             float softmax_scale, float* similarity, void* workspace,
                                             size_t workspace_bytes, void* stream) {
-  calibatt_status st;
-  if ((st = check_shape(shape)) != CALIBATT_OK) return st;
-  if (!q || !k || !similarity || !workspace)
-    return fail(CALIBATT_ERR_INVALID_ARG, "q, k, similarity and workspace must be non-NULL");
-  if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
-  if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
-    return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
-                shape->seq_len);
-  if (rows > calibatt::kMaxRepetitionRows)
-    return fail(CALIBATT_ERR_UNSUPPORTED, "more than %d spatial rows per frame", calibatt::kMaxRepetitionRows);
-  if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
-    return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
-  for (int a = 0; a < n_anchors; ++a) {
-    if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
-      return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
-    if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
-      return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
-  }
-  size_t need = 0;
-  calibatt_block_energy_workspace_size(shape, &need);
-  if (workspace_bytes < need)
-    return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
-  const float sl2 = scale_log2_of(softmax_scale, shape->head_dim);
-  calibatt::EnergyParams e;
-  std::memset(&e, 0, sizeof(e));
-  e.q = q;
-  e.k = k;
-  e.lse = static_cast<float*>(workspace);
-  e.sb = shape->stride_b;
-  e.sn = shape->stride_n;
-  e.sh = shape->stride_h;
-  e.batch = shape->batch;
-  e.seq_len = shape->seq_len;
-  e.heads = shape->heads;
-  e.scale_log2 = sl2;
-  cudaError_t ce = calibatt::launch_row_lse(e, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
-  if (ce != cudaSuccess) return cuda_fail(ce, "row log-sum-exp launch");
-  calibatt::RepetitionParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.q = q;
-  p.k = k;
-  p.lse = static_cast<const float*>(workspace);
-  p.sim = similarity;
-  p.sb = shape->stride_b;
-  p.sn = shape->stride_n;
-  p.sh = shape->stride_h;
-  p.batch = shape->batch;
-  p.seq_len = shape->seq_len;
-  p.heads = shape->heads;
-  p.frames = frames;
-  p.rows = rows;
-  p.cols = cols;
-  p.scale_log2 = sl2;
-  // nearest anchor of each row, ties to the lower anchor (as the anchor path)
-  for (int32_t rho = 0; rho < rows; ++rho) {
-    int best = 0;
-    for (int a = 1; a < n_anchors; ++a)
-      if (std::abs(rho - anchor_rows[a]) < std::abs(rho - anchor_rows[best])) best = a;
-    p.nearest[rho] = static_cast<int16_t>(anchor_rows[best]);
-  }
-  ce = calibatt::launch_spatial_similarity(p, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
-  if (ce != cudaSuccess) return cuda_fail(ce, "spatial similarity launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if (!q || !k || !similarity || !workspace)
+      return fail(CALIBATT_ERR_INVALID_ARG, "q, k, similarity and workspace must be non-NULL");
+    if (frames < 1 || rows < 1 || cols < 1) return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
+    if (static_cast<int64_t>(frames) * rows * cols != shape->seq_len)
+      return fail(CALIBATT_ERR_INVALID_ARG, "frames*rows*cols = %lld != seq_len %d", (long long)frames * rows * cols,
+                  shape->seq_len);
+    if (rows > calibatt::kMaxRepetitionRows)
+      return fail(CALIBATT_ERR_UNSUPPORTED, "more than %d spatial rows per frame", calibatt::kMaxRepetitionRows);
+    if (!anchor_rows || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors)
+      return fail(CALIBATT_ERR_INVALID_ARG, "n_anchors must be in [1, %d] with a non-NULL list", calibatt::kMaxAnchors);
+    for (int a = 0; a < n_anchors; ++a) {
+      if (anchor_rows[a] < 0 || anchor_rows[a] >= rows)
+        return fail(CALIBATT_ERR_INVALID_ARG, "anchor row %d outside [0, %d)", anchor_rows[a], rows);
+      if (a > 0 && anchor_rows[a] <= anchor_rows[a - 1])
+        return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
+    }
+    size_t need = 0;
+    calibatt_block_energy_workspace_size(shape, &need);
+    if (workspace_bytes < need)
+      return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+    const float sl2 = scale_log2_of(softmax_scale, shape->head_dim);
+    calibatt::EnergyParams e;
+    std::memset(&e, 0, sizeof(e));
+    e.q = q;
+    e.k = k;
+    e.lse = static_cast<float*>(workspace);
+    e.sb = shape->stride_b;
+    e.sn = shape->stride_n;
+    e.sh = shape->stride_h;
+    e.batch = shape->batch;
+    e.seq_len = shape->seq_len;
+    e.heads = shape->heads;
+    e.scale_log2 = sl2;
+    cudaError_t ce = calibatt::launch_row_lse(e, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) return cuda_fail(ce, "row log-sum-exp launch");
+    calibatt::RepetitionParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.lse = static_cast<const float*>(workspace);
+    p.sim = similarity;
+    p.sb = shape->stride_b;
+    p.sn = shape->stride_n;
+    p.sh = shape->stride_h;
+    p.batch = shape->batch;
+    p.seq_len = shape->seq_len;
+    p.heads = shape->heads;
+    p.frames = frames;
+    p.rows = rows;
+    p.cols = cols;
+    p.scale_log2 = sl2;
+    // nearest anchor of each row, ties to the lower anchor (as the anchor path)
+    for (int32_t rho = 0; rho < rows; ++rho) {
+      int best = 0;
+      for (int a = 1; a < n_anchors; ++a)
+        if (std::abs(rho - anchor_rows[a]) < std::abs(rho - anchor_rows[best])) best = a;
+      p.nearest[rho] = static_cast<int16_t>(anchor_rows[best]);
+    }
+    ce = calibatt::launch_spatial_similarity(p, shape->head_dim, shape->dtype, static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) return cuda_fail(ce, "spatial similarity launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_prompts, int32_t n_heads,
                                           int32_t per_head, float threshold, float* mean, uint8_t* flags,
                                           void* stream) {
-  if (n_prompts < 1 || n_heads < 0 || per_head < 1)
-    return fail(CALIBATT_ERR_INVALID_ARG, "n_prompts and per_head must be >= 1, n_heads >= 0");
-  if (n_heads > 0 && (!similarity || !flags))
-    return fail(CALIBATT_ERR_INVALID_ARG, "similarity and flags must be non-NULL");
-  if (!(threshold == threshold)) return fail(CALIBATT_ERR_INVALID_ARG, "threshold is NaN");
-  cudaError_t e = calibatt::launch_repetition_flags(similarity, n_prompts, n_heads, per_head, threshold, mean, flags,
-                                                    static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "repetition flags launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n_prompts < 1 || n_heads < 0 || per_head < 1)
+      return fail(CALIBATT_ERR_INVALID_ARG, "n_prompts and per_head must be >= 1, n_heads >= 0");
+    if (n_heads > 0 && (!similarity || !flags))
+      return fail(CALIBATT_ERR_INVALID_ARG, "similarity and flags must be non-NULL");
+    if (!(threshold == threshold)) return fail(CALIBATT_ERR_INVALID_ARG, "threshold is NaN");
+    cudaError_t e = calibatt::launch_repetition_flags(similarity, n_prompts, n_heads, per_head, threshold, mean, flags,
+                                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "repetition flags launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_select_blocks(const float* energy, int64_t n_rows, int32_t nk, float tau, uint8_t* mask,
                                        int32_t* count_accum, void* stream) {
-  if (n_rows < 0 || nk < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_rows must be >= 0 and nk >= 1");
-  if (nk > 4096) return fail(CALIBATT_ERR_UNSUPPORTED, "nk %d > 4096", nk);
-  if (n_rows > 2147483647LL) return fail(CALIBATT_ERR_UNSUPPORTED, "too many rows");
-  if (n_rows > 0 && (!energy || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "energy and mask must be non-NULL");
-  if (!(tau == tau)) return fail(CALIBATT_ERR_INVALID_ARG, "tau is NaN");
-  cudaError_t e = calibatt::launch_select_blocks(energy, n_rows, nk, tau, mask, count_accum, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "select launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n_rows < 0 || nk < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n_rows must be >= 0 and nk >= 1");
+    if (nk > 4096) return fail(CALIBATT_ERR_UNSUPPORTED, "nk %d > 4096", nk);
+    if (n_rows > 2147483647LL) return fail(CALIBATT_ERR_UNSUPPORTED, "too many rows");
+    if (n_rows > 0 && (!energy || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "energy and mask must be non-NULL");
+    if (!(tau == tau)) return fail(CALIBATT_ERR_INVALID_ARG, "tau is NaN");
+    cudaError_t e = calibatt::launch_select_blocks(energy, n_rows, nk, tau, mask, count_accum, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "select launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32_t n_prompts, float rho,
                                          uint8_t* mask, void* stream) {
-  if (n < 0 || n_prompts < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0 and n_prompts >= 1");
-  if (n > 0 && (!counts || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "counts and mask must be non-NULL");
-  if (!(rho == rho)) return fail(CALIBATT_ERR_INVALID_ARG, "rho is NaN");
-  cudaError_t e = calibatt::launch_aggregate(counts, n, n_prompts, rho, mask, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "aggregate launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n < 0 || n_prompts < 1) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0 and n_prompts >= 1");
+    if (n > 0 && (!counts || !mask)) return fail(CALIBATT_ERR_INVALID_ARG, "counts and mask must be non-NULL");
+    if (!(rho == rho)) return fail(CALIBATT_ERR_INVALID_ARG, "rho is NaN");
+    cudaError_t e = calibatt::launch_aggregate(counts, n, n_prompts, rho, mask, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "aggregate launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
-  if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
-  if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
-  cudaError_t e = calibatt::launch_exp2_fma(x, y, n, false, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
+    if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
+    cudaError_t e = calibatt::launch_exp2_fma(x, y, n, false, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_debug_exp2_fma_quintic(const float* x, float* y, int64_t n, void* stream) {
-  if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
-  if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
-  cudaError_t e = calibatt::launch_exp2_fma(x, y, n, true, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (n < 0) return fail(CALIBATT_ERR_INVALID_ARG, "n must be >= 0");
+    if (n > 0 && (!x || !y)) return fail(CALIBATT_ERR_INVALID_ARG, "x and y must be non-NULL");
+    cudaError_t e = calibatt::launch_exp2_fma(x, y, n, true, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "exp2 launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_debug_bounded_wait(void* stream) {
-  int32_t* p = status_word_ptr();
-  if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
-  cudaError_t e = calibatt::launch_bounded_wait(p, g_timeout_ns.load(), static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "bounded wait launch");
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    int32_t* p = status_word_ptr();
+    if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+    cudaError_t e = calibatt::launch_bounded_wait(p, g_timeout_ns.load(), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "bounded wait launch");
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear) {
-  if (!code) return fail(CALIBATT_ERR_INVALID_ARG, "code is NULL");
-  int32_t* p = status_word_ptr();
-  if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  e = cudaMemcpy(code, p, sizeof(int32_t), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "status read");
-  if (clear) {
-    e = cudaMemset(p, 0, sizeof(int32_t));
-    if (e != cudaSuccess) return cuda_fail(e, "status clear");
-  }
-  if (*code != 0) {
-    if ((*code & 0xFF) == CALIBATT_ERR_INVALID_ARG)
-      return fail(CALIBATT_ERR_INVALID_ARG, "a kernel met a key-block index outside the key range (code 0x%x)",
-                  *code);
-    return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
-  }
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!code) return fail(CALIBATT_ERR_INVALID_ARG, "code is NULL");
+    int32_t* p = status_word_ptr();
+    if (!p) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    e = cudaMemcpy(code, p, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (clear) {
+      e = cudaMemset(p, 0, sizeof(int32_t));
+      if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    }
+    if (*code != 0) {
+      if ((*code & 0xFF) == CALIBATT_ERR_INVALID_ARG)
+        return fail(CALIBATT_ERR_INVALID_ARG, "a kernel met a key-block index outside the key range (code 0x%x)",
+                    *code);
+      return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
+    }
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_set_wait_timeout_ms(int32_t ms) {
-  if (ms < 1) return fail(CALIBATT_ERR_INVALID_ARG, "timeout must be >= 1 ms");
-  g_timeout_ns.store(static_cast<unsigned long long>(ms) * 1000000ull);
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (ms < 1) return fail(CALIBATT_ERR_INVALID_ARG, "timeout must be >= 1 ms");
+    g_timeout_ns.store(static_cast<unsigned long long>(ms) * 1000000ull);
+    return CALIBATT_OK;
+  });
 }
 
 calibatt_status calibatt_device_sm_count(int32_t* out) {
-  if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
-  const int n = device_sm_count();
-  if (n < 1) {
-    cudaGetLastError();
-    return fail(CALIBATT_ERR_CUDA, "no CUDA device");
-  }
-  *out = n;
-  return CALIBATT_OK;
+  return guarded([&]() -> calibatt_status {
+    if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+    const int n = device_sm_count();
+    if (n < 1) {
+      cudaGetLastError();
+      return fail(CALIBATT_ERR_CUDA, "no CUDA device");
+    }
+    *out = n;
+    return CALIBATT_OK;
+  });
 }
 
 }  // extern "C"
