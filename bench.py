@@ -109,16 +109,18 @@ class ClockSampler:
 def measured_traffic(tiles):
     """DRAM bytes per launch of the sparse kernel from the committed ncu capture
     (profiles/tc_attn_sparse_720p_traffic.json), scaled by retained tiles; None
-    when the kernel source changed since the capture."""
+    when a source of the kernel (the kernel file and the headers it includes)
+    changed since the capture."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "tc_attn_sparse_720p_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
-    src = os.path.join(ROOT, t["kernel_source"])
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != t["kernel_source_sha256"]:
-        return None
+    for src, sha in t["kernel_sources_sha256"].items():
+        with open(os.path.join(ROOT, src), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != sha:
+                return None
     return t["dram_bytes_per_retained_tile"] * tiles
 
 
