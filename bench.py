@@ -106,13 +106,13 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def measured_traffic(tiles):
+def measured_traffic(tiles, path=None):
     """DRAM bytes per launch of the sparse kernel from the committed ncu capture
     (profiles/tc_attn_sparse_720p_traffic.json), scaled by retained tiles; None
     when a source of the kernel (the kernel file and the headers it includes)
     changed since the capture."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "tc_attn_sparse_720p_traffic.json")
+    path = path or os.path.join(ROOT, "profiles", "tc_attn_sparse_720p_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:

@@ -91,3 +91,27 @@ def test_sweep_recipe_small():
     d0 = [W.sweep_record_density(0, 0, h) for h in range(20)]
     d49 = [W.sweep_record_density(49, 0, h) for h in range(20)]
     assert all(0.57 <= d <= 0.63 for d in d0) and all(0.17 <= d <= 0.23 for d in d49)
+
+
+def test_traffic_record_is_tied_to_the_kernel_sources(tmp_path):
+    """bench.py reports the captured DRAM traffic only while every device
+    source of the kernel hashes as it did at the capture."""
+    import json
+    import os
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+
+    rec = json.load(open(os.path.join(root, "profiles", "tc_attn_sparse_720p_traffic.json")))
+    assert all(os.path.exists(os.path.join(root, f)) for f in rec["kernel_sources_sha256"])
+    per_tile = rec["dram_bytes_per_retained_tile"]
+    assert per_tile == (rec["dram_read_bytes"] + rec["dram_write_bytes"]) / rec["retained_tiles"]
+    tampered = dict(rec, kernel_sources_sha256=dict(rec["kernel_sources_sha256"]))
+    first = next(iter(tampered["kernel_sources_sha256"]))
+    tampered["kernel_sources_sha256"][first] = "0" * 64
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(tampered))
+    assert bench.measured_traffic(1000, str(path)) is None
+    assert bench.measured_traffic(1000, str(tmp_path / "missing.json")) is None
