@@ -952,6 +952,50 @@ def test_host_buffer_entry_point(C):
     assert torch.equal(dq, q)
 
 
+def test_calls_replay_in_a_cuda_graph(C):
+    """The block-sparse and the fused dual-path calls enqueue only kernels on
+    the caller's stream (no host sync, no allocation after the first call),
+    so they capture into a CUDA graph; replays compute on whatever the input
+    buffers hold, bitwise equal to direct calls."""
+    frames, rows, cols, anchors = 3, 10, 100, (2, 7)
+    n, h, d, block = frames * rows * cols, 3, 128, 128
+    nb = O.num_blocks(n, block)
+    q, k, v = W.make_qkv(61, 1, n, h, d, "bf16", 1.0, "cuda")
+    q2, k2, v2 = W.make_qkv(62, 1, n, h, d, "bf16", 1.0, "cuda")
+    masks = _random_masks(63, h, nb, 0.4)
+    rp, ci, rep = C.masks_to_layer_csr([masks[0], None, masks[2]], h, nb)
+    with C.MaskDictionary(1, 1, h, nb, nb, block, ci.size) as dct:
+        dct.set_anchor_geometry(frames, rows, cols, anchors)
+        dct.set_layer(0, 0, rp, ci, rep)
+        o_sparse, o_dual = torch.zeros_like(q), torch.zeros_like(q)
+
+        def step():
+            C.calibatt_block_sparse_attn(q, k, v, o_sparse, dct, 0, 0, block)
+            C.calibatt_dual_path_attn(q, k, v, o_dual, dct, 0, 0, frames, rows, cols, anchors, block)
+
+        step()                                          # warm-up outside the capture
+        torch.cuda.synchronize()
+        direct = (o_sparse.clone(), o_dual.clone())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        o_sparse.zero_()
+        o_dual.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o_sparse, direct[0]) and torch.equal(o_dual, direct[1])
+        for dst, src in ((q, q2), (k, k2), (v, v2)):     # new inputs in the captured buffers
+            dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        got = (o_sparse.clone(), o_dual.clone())
+        step()
+        _check_status(C)
+        assert torch.equal(got[0], o_sparse) and torch.equal(got[1], o_dual)
+        assert not torch.equal(got[1], direct[1])
+        del graph
+
+
 def test_bounded_wait_runs_out_and_context_survives(C):
     """A wait that nothing satisfies ends after the configured limit with the
     timeout status (wait point 15), no fault and no hang; the status clears
