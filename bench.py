@@ -291,6 +291,33 @@ def run_anchor_case(args, torch, C, pk):
         "output_bytes": len(rep_heads) * wd.seq_len * wd.head_dim * 2}}), flush=True)
 
 
+def run_dual_case(args, torch, C, pk):
+    """The dual-path 720p layer alone (28 block-sparse heads and 12 anchor heads
+    in ONE fused launch over the dictionary's joint schedule), timed with CUDA
+    events; a case of its own for profiling the fused kernel."""
+    wd = W.WORKLOADS["720p_dual"]
+    dmasks, rep_heads = W.workload_masks(wd)
+    geom = (wd.frames, wd.rows, wd.cols, wd.anchors)
+    q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
+    o = torch.empty_like(q)
+    d = build_dict(C, [dmasks[h] for h in range(wd.heads)], wd.heads, wd.num_blocks, wd.block, geom)
+    tiles = d.layer_info(0, 0)["retained_tiles"] + \
+        len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128) * wd.num_blocks
+    stream = torch.cuda.current_stream()
+    per_call = time_calls(torch, lambda: C.calibatt_dual_path_attn(q, k, v, o, d, 0, 0, wd.frames, wd.rows,
+                                                                   wd.cols, wd.anchors, wd.block, stream=stream),
+                          args.steps, args.warmup, stream)
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the dual-path case")
+    d.close()
+    ms = statistics.mean(per_call)
+    tf = tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12
+    print(json.dumps({"dual_case": {
+        "sparse_heads": wd.heads - len(rep_heads), "anchor_heads": len(rep_heads), "launches_per_call": 1,
+        "tiles": tiles, "ms_per_call": ms, "effective_tflops": tf, "frac_of_burst_peak": tf / pk["bf16_tflops"]}}),
+        flush=True)
+
+
 def run_epilogue_probe(torch, B, C):
     """Store rate of the anchor broadcast epilogue (the 12 repetitive heads of
     the dual-path 720p layer).  The measurement build records, per CTA, the
@@ -458,6 +485,8 @@ def main():
     ap.add_argument("--epilogue-probe", action="store_true",
                     help="time the anchor broadcast epilogue with the library's measurement build "
                          "(-DCALIBATT_TRACE) and print its store rate")
+    ap.add_argument("--dual-case", action="store_true",
+                    help="time the dual-path 720p layer alone (one fused launch of both paths)")
     ap.add_argument("--anchor-case", action="store_true",
                     help="time the anchor path alone (the 12 repetitive heads of the dual-path 720p layer)")
     ap.add_argument("--dense-sample", type=int, default=50,
@@ -495,6 +524,9 @@ def main():
         return
     if args.anchor_case:
         run_anchor_case(args, torch, C, pk)
+        return
+    if args.dual_case:
+        run_dual_case(args, torch, C, pk)
         return
     if args.workload == "sweep":
         if world > 1:
