@@ -107,8 +107,9 @@ class ClockSampler:
 
 
 def measured_traffic(tiles, path=None):
-    """DRAM bytes per launch of the sparse kernel from the committed ncu capture
-    (profiles/tc_attn_sparse_720p_traffic.json), scaled by retained tiles; None
+    """DRAM bytes per launch of the sparse kernel from the committed ncu counters
+    of the bench launch itself (profiles/tc_attn_sparse_720p_traffic.json), per
+    retained tile times the tiles of this launch; None
     when a source of the kernel (the kernel file and the headers it includes)
     changed since the capture."""
     import hashlib
@@ -300,7 +301,10 @@ def run_dual_case(args, torch, C, pk):
     geom = (wd.frames, wd.rows, wd.cols, wd.anchors)
     q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
     o = torch.empty_like(q)
-    d = build_dict(C, [dmasks[h] for h in range(wd.heads)], wd.heads, wd.num_blocks, wd.block, geom)
+    # one launch over the joint schedule, or (--dual-launches 2) the block-sparse
+    # and anchor launches of a dictionary without the anchor geometry
+    d = build_dict(C, [dmasks[h] for h in range(wd.heads)], wd.heads, wd.num_blocks, wd.block,
+                   geom if args.dual_launches == 1 else None)
     tiles = d.layer_info(0, 0)["retained_tiles"] + \
         len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128) * wd.num_blocks
     stream = torch.cuda.current_stream()
@@ -313,7 +317,8 @@ def run_dual_case(args, torch, C, pk):
     ms = statistics.mean(per_call)
     tf = tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12
     print(json.dumps({"dual_case": {
-        "sparse_heads": wd.heads - len(rep_heads), "anchor_heads": len(rep_heads), "launches_per_call": 1,
+        "sparse_heads": wd.heads - len(rep_heads), "anchor_heads": len(rep_heads),
+        "launches_per_call": args.dual_launches,
         "tiles": tiles, "ms_per_call": ms, "effective_tflops": tf, "frac_of_burst_peak": tf / pk["bf16_tflops"]}}),
         flush=True)
 
@@ -487,6 +492,8 @@ def main():
                          "(-DCALIBATT_TRACE) and print its store rate")
     ap.add_argument("--dual-case", action="store_true",
                     help="time the dual-path 720p layer alone (one fused launch of both paths)")
+    ap.add_argument("--dual-launches", type=int, default=1, choices=[1, 2],
+                    help="--dual-case as one fused launch (1) or block-sparse + anchor launches (2)")
     ap.add_argument("--anchor-case", action="store_true",
                     help="time the anchor path alone (the 12 repetitive heads of the dual-path 720p layer)")
     ap.add_argument("--dense-sample", type=int, default=50,
