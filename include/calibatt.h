@@ -80,13 +80,16 @@ typedef struct calibatt_dict calibatt_dict;
 
 /* ---------------------------------------------------------------- status */
 
-/* Static text for a status code. */
+/* Static text for a status code.
+ * Diagnostics; no counterpart in the paper note. */
 const char* calibatt_status_string(calibatt_status status);
 
-/* Message describing the last failure on the calling thread ("" if none). */
+/* Message describing the last failure on the calling thread ("" if none).
+ * Diagnostics; no counterpart in the paper note. */
 const char* calibatt_last_error(void);
 
-/* ABI version of this header (incremented on incompatible change). */
+/* ABI version of this header (incremented on incompatible change).
+ * No counterpart in the paper note. */
 int32_t calibatt_abi_version(void);
 
 /* ------------------------------------------------- host-only utilities */
@@ -129,7 +132,8 @@ calibatt_status calibatt_lpt_schedule(int32_t n_items, const int64_t* cost, int3
  * for up to nnz_capacity retained blocks in total (2 bytes each) plus
  * per-record offsets and schedules is allocated now, on the current device.
  * num_ctas <= 0 selects the device's SM count (the persistent grid size the
- * schedules are built for).  CALIBATT_ERR_OOM if the allocation fails. */
+ * schedules are built for).  CALIBATT_ERR_OOM if the allocation fails.
+ * Key Designs 4: the calibrated masks become read-only skip lists, loaded onto the GPU before generation. */
 calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk,
                                      int32_t block, int64_t nnz_capacity, int32_t num_ctas,
                                      calibatt_dict** out);
@@ -142,7 +146,9 @@ calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq
  * kept blocks in shared memory; results equal those of the list format.
  * Bitmap dictionaries serve the tensor-core path only (bf16, block 128;
  * otherwise the attention calls return CALIBATT_ERR_UNSUPPORTED) and hold
- * nq <= 2048.  All other dictionary functions apply unchanged. */
+ * nq <= 2048.  All other dictionary functions apply unchanged.
+ * Limitations & Future Work of the paper note: the 21.5 GB of mask memory
+ * at Wan 720p, reducible to 3.6 GB, and compacting the skip lists. */
 calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int32_t nq,
                                             int32_t nk, int32_t block, int32_t num_ctas,
                                             calibatt_dict** out);
@@ -181,17 +187,20 @@ calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* dict, int32_t f
                                                   int32_t cols, const int32_t* anchor_rows,
                                                   int32_t n_anchors);
 
-/* Totals: device bytes held, retained blocks stored, persistent grid size. */
+/* Totals: device bytes held, retained blocks stored, persistent grid size.
+ * Bookkeeping; no counterpart in the paper note. */
 calibatt_status calibatt_dict_info(const calibatt_dict* dict, int64_t* device_bytes,
                                    int64_t* nnz_total, int32_t* num_ctas);
 
 /* Per-layer counts: heads on each path and retained (query, key) block tiles
- * of its sparse heads.  CALIBATT_ERR_INVALID_ARG if the layer is not set. */
+ * of its sparse heads.  CALIBATT_ERR_INVALID_ARG if the layer is not set.
+ * Bookkeeping; no counterpart in the paper note. */
 calibatt_status calibatt_dict_layer_info(const calibatt_dict* dict, int32_t t, int32_t l,
                                          int32_t* n_sparse_heads, int32_t* n_repetitive_heads,
                                          int64_t* retained_tiles);
 
-/* Frees the dictionary's device and host memory (synchronises the device). */
+/* Frees the dictionary's device and host memory (synchronises the device).
+ * Bookkeeping; no counterpart in the paper note. */
 calibatt_status calibatt_dict_destroy(calibatt_dict* dict);
 
 /* Checkpoint of the calibration output (the dictionary is the method's only
@@ -251,7 +260,8 @@ calibatt_status calibatt_block_sparse_attn(const void* q, const void* k, const v
  * the copies to be asynchronous (they are then ordered on `stream` only);
  * callers may alternate streams and device buffer sets so that the copies of
  * one call overlap the attention of another.  Other arguments and errors as
- * calibatt_block_sparse_attn; a copy failure returns CALIBATT_ERR_CUDA. */
+ * calibatt_block_sparse_attn; a copy failure returns CALIBATT_ERR_CUDA.
+ * Key Designs 4 (the operation of calibatt_block_sparse_attn). */
 calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* k_host,
                                                 const void* v_host, void* o_host, void* q,
                                                 void* k, void* v, void* o,
@@ -269,7 +279,8 @@ calibatt_status calibatt_block_sparse_attn_host(const void* q_host, const void* 
  *   items: host uint32[n_heads * nq]; cta_ptr: host int32[grid + 1], the
  *     items of CTA c are items[cta_ptr[c] .. cta_ptr[c+1]).
  * nq <= 65535, heads <= 65535.  CALIBATT_ERR_INVALID_ARG on a bad argument
- * or a decreasing row_ptr; column indices are not read. */
+ * or a decreasing row_ptr; column indices are not read.
+ * No counterpart in the paper note: host scheduling for the persistent kernel. */
 calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* row_ptr,
                                       const int32_t* head_ids, int32_t n_heads, int32_t grid,
                                       uint32_t* items, int32_t* cta_ptr);
@@ -296,7 +307,8 @@ calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* 
  *     with block 128, which runs `grid` persistent CTAs; the CUDA-core
  *     kernel walks head_ids and ignores them, and they may then be NULL).
  * All device arrays are caller-owned and must stay valid until the call's
- * work on `stream` completes.  n_heads == 0 is a no-op. */
+ * work on `stream` completes.  n_heads == 0 is a no-op.
+ * Key Designs 4 (the operation of calibatt_block_sparse_attn). */
 calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, const void* v, void* o,
                                                const calibatt_shape* shape, int32_t block,
                                                const int32_t* row_ptr, const uint16_t* col_idx,
@@ -338,7 +350,8 @@ calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void
 
 /* ------------------------------------------------ offline calibration */
 
-/* Device scratch bytes calibatt_block_energy needs for `shape`. */
+/* Device scratch bytes calibatt_block_energy needs for `shape`.
+ * Key Designs 1, Eq. (5): the workspace of calibatt_block_energy. */
 calibatt_status calibatt_block_energy_workspace_size(const calibatt_shape* shape,
                                                      size_t* bytes);
 
@@ -437,7 +450,8 @@ calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_pro
  * (CALIBATT_ERR_INVALID_ARG in the low byte; 23: the device-side check that
  * calibatt_block_sparse_attn_csr runs before its attention kernel; 22: the
  * CUDA-core kernel met a block index >= nq and skipped that block).  Returns
- * the low byte's status when the word is non-zero. */
+ * the low byte's status when the word is non-zero.
+ * Diagnostics; no counterpart in the paper note. */
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);
 
 /* Failure-path check of the bounded waits: launches one warp that waits on
@@ -445,7 +459,8 @@ calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clea
  * use, with the current calibatt_set_wait_timeout_ms limit.  When the limit
  * passes it sets the status word (CALIBATT_ERR_TIMEOUT, wait point 15 in the
  * byte above it) and returns; no fault, no hang, the context stays usable.
- * Read the result with calibatt_device_status. */
+ * Read the result with calibatt_device_status.
+ * Diagnostics; no counterpart in the paper note. */
 calibatt_status calibatt_debug_bounded_wait(void* stream);
 
 /* Evaluates, on the device, the FMA-pipe base-2 exponential that the
@@ -458,14 +473,17 @@ calibatt_status calibatt_debug_exp2_fma(const float* x, float* y, int64_t n, voi
 /* The same for the quintic FMA-pipe exponential that the offline energy
  * passes use for a quarter of their exponentials: relative error below 3e-7
  * (the fit's 7.5e-8 plus float32 evaluation) for -125 <= x <= 126, about
- * 2^-125 for smaller x.  x, y: device float32[n]. */
+ * 2^-125 for smaller x.  x, y: device float32[n].
+ * No counterpart in the paper note (exposed so its error bound can be tested). */
 calibatt_status calibatt_debug_exp2_fma_quintic(const float* x, float* y, int64_t n, void* stream);
 
 /* Time limit of every in-kernel barrier wait, in milliseconds (default 4000;
- * applies to launches made after the call). */
+ * applies to launches made after the call).
+ * Diagnostics; no counterpart in the paper note. */
 calibatt_status calibatt_set_wait_timeout_ms(int32_t ms);
 
-/* Number of SMs of the current device (the default persistent grid size). */
+/* Number of SMs of the current device (the default persistent grid size).
+ * No counterpart in the paper note. */
 calibatt_status calibatt_device_sm_count(int32_t* out);
 
 #ifdef __cplusplus
