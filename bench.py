@@ -492,6 +492,9 @@ def main():
                          "(-DCALIBATT_TRACE) and print its store rate")
     ap.add_argument("--dual-case", action="store_true",
                     help="time the dual-path 720p layer alone (one fused launch of both paths)")
+    ap.add_argument("--layout", default="bnhd", choices=["bnhd", "bhnd"],
+                    help="storage of Q, K, V, O for the 720p call: token-major [B, N, H, D] (default) or "
+                         "head-major [B, H, N, D] (the same logical tensors, other strides)")
     ap.add_argument("--dual-launches", type=int, default=1, choices=[1, 2],
                     help="--dual-case as one fused launch (1) or block-sparse + anchor launches (2)")
     ap.add_argument("--anchor-case", action="store_true",
@@ -545,6 +548,10 @@ def main():
     masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])
     q, k, v = W.make_qkv(rank_seed(wl.seed, rank), 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std,
                          "cuda")
+    if args.layout == "bhnd":
+        # the same [batch, N, heads, head_dim] tensors stored head-major: a head's
+        # rows are contiguous (stride_n = head_dim) instead of heads*head_dim apart
+        q, k, v = (t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3) for t in (q, k, v))
     o = torch.empty_like(q)
     d_sparse = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block)
     tiles = d_sparse.layer_info(0, 0)["retained_tiles"]
@@ -650,8 +657,16 @@ def main():
     e2e = None
     if not args.no_extras:
         n_sets = 3
-        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-        hos = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(n_sets)]
+        if args.layout == "bnhd":
+            hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+            hos = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(n_sets)]
+        else:
+            # pinned host tensors with the device tensors' strides (the host call
+            # copies each tensor's byte extent as it lies)
+            def pinned(t):
+                return torch.empty_strided(t.size(), t.stride(), dtype=t.dtype, pin_memory=True)
+            hq, hk, hv = (pinned(t).copy_(t) for t in (q, k, v))
+            hos = [pinned(o) for _ in range(n_sets)]
         dsets = [[torch.empty_like(q) for _ in range(4)] for _ in range(n_sets)]
         streams = [torch.cuda.Stream() for _ in range(n_sets)]
         e2e_steps = max(6, args.steps // 2)
@@ -701,7 +716,9 @@ def main():
                        "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
                        "heads": wl.heads, "head_dim": wl.head_dim, "seq_len": wl.seq_len, "block": wl.block,
                        "density": round(density, 4), "retained_tiles": tiles,
-                       "l2": "inputs 2.32 GB > 126 MB L2, no flush", "parallelism": f"replicas x{world}"},
+                       "l2": "inputs 2.32 GB > 126 MB L2, no flush", "parallelism": f"replicas x{world}",
+                       "storage": "[batch, N, heads, head_dim]" if args.layout == "bnhd"
+                       else "[batch, heads, N, head_dim] (head-major)"},
             "pct_of_peak": achieved / pk["bf16_tflops"],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"], "traffic": measured_traffic(tiles),
