@@ -115,3 +115,31 @@ def test_traffic_record_is_tied_to_the_kernel_sources(tmp_path):
     path.write_text(json.dumps(tampered))
     assert bench.measured_traffic(1000, str(path)) is None
     assert bench.measured_traffic(1000, str(tmp_path / "missing.json")) is None
+
+
+def test_cpu_baseline_leg_reports_parity_of_the_given_output():
+    """bench.py's CPU-baseline leg times the oracle on sampled query blocks and,
+    given the library's output of the same call, reports its error on those
+    rows: zero-ish for the oracle's own output, large for a wrong one."""
+    import os
+    import sys
+
+    import torch
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    from oracle import calibatt_oracle as O
+
+    wl = W.WORKLOADS["tiny"]
+    q, k, v = W.make_qkv(wl.seed, 1, wl.seq_len, wl.heads, wl.head_dim, "fp32", wl.input_std, "cpu")
+    nb = wl.num_blocks
+    masks = {0: np.ones((nb, nb), bool), 1: np.eye(nb, dtype=bool)}
+    ref, _ = O.block_sparse_attention_bnhd(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                           [masks[0], masks[1]], wl.block)
+    base, par = bench.cpu_baseline(wl, masks, q, k, v, torch.from_numpy(ref).float(), budget_s=0.3)
+    assert base["kind"] == "oracle" and base["cores"] >= 1 and base["value"] > 0
+    assert par["within_tolerance"] and par["max_abs"] < 1e-6
+    _, bad = bench.cpu_baseline(wl, masks, q, k, v, torch.from_numpy(ref).float() + 0.1, budget_s=0.3)
+    assert not bad["within_tolerance"] and abs(bad["max_abs"] - 0.1) < 1e-3
+    assert isinstance(bench.cpu_baseline(wl, masks, q, k, v, budget_s=0.1), dict)   # no output: baseline only
