@@ -721,7 +721,9 @@ def main():
                        else "[batch, heads, N, head_dim] (head-major)"},
             "pct_of_peak": achieved / pk["bf16_tflops"],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"], "traffic": measured_traffic(tiles),
+                         "frac": achieved / pk["bf16_tflops"],
+                         # counters were taken on the default (token-major) storage
+                         "traffic": measured_traffic(tiles) if args.layout == "bnhd" else None,
                          "traffic_unit": "bytes per launch (DRAM read + write)",
                          "algorithmic_bytes": 4 * q.numel() * q.element_size(),
                          "peak_source": f"{pk['source']} burst bf16",
