@@ -38,6 +38,11 @@ Pins (tests/test_oracle_pins.py, run with ``-m "not gpu"``):
       one query over two keys == the two-term softmax closed form;
       empty row == zeros and LSE = -inf.
   attention_probabilities: rows sum to one.
+  block_sparse_attention_bnhd, anchor_attention_bnhd, block_energy_bnhd:
+      every (batch, head) slice equals the one-head function on explicitly
+      sliced inputs whose heads and batches differ in scale; the anchor and
+      energy wrappers also equal torch's batched SDPA / softmax over
+      [batch, heads, N, D] (gathered or block-summed outside the oracle).
   anchor_attention / nearest_anchor_rows:
       nearest-anchor tables of the tiny and 720p layouts
       (tests/golden/nearest_anchor_tables.json);

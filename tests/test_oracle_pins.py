@@ -139,6 +139,72 @@ def test_bnhd_wrapper_indexes_heads_and_batches():
             np.testing.assert_array_equal(out[bi, :, hi], ref)
 
 
+def _distinct_heads(seed, b, n, h, d):
+    """[b, n, h, d] draws whose heads and batches differ in scale as well as in
+    values, so that an exchanged (batch, head) slice changes every result."""
+    x = _rand(seed, b, n, h, d)
+    for bi in range(b):
+        for hi in range(h):
+            x[bi, :, hi] *= 0.5 + 0.6 * hi + 0.25 * bi
+    return x
+
+
+def test_anchor_bnhd_wrapper_indexes_heads_and_batches():
+    """anchor_attention_bnhd on batch 2, 3 heads, a head subset in reverse
+    order and a row subset, against (1) the one-head function on explicitly
+    sliced inputs and (2) torch's batched SDPA over [batch, heads, N, D]
+    followed by a gather of each token's nearest-anchor row written out by
+    loops (Key Designs 3: same frame, same column, nearest anchor row)."""
+    b, frames, rows, cols, h, d = 2, 2, 6, 3, 3, 8
+    n = frames * rows * cols
+    anchors = [1, 4]
+    q, k, v = (_distinct_heads(s, b, n, h, d) for s in (40, 41, 42))
+    heads = [2, 0]
+    sel = np.array([0, 5, 7, 17, 18, 26, 35])
+    out = O.anchor_attention_bnhd(q, k, v, frames, rows, cols, anchors, heads=heads, rows=sel)
+    assert out.shape == (b, len(sel), len(heads), d)
+    for bi in range(b):
+        for hi, hh in enumerate(heads):
+            ref, _ = O.anchor_attention(q[bi, :, hh], k[bi, :, hh], v[bi, :, hh],
+                                        frames, rows, cols, anchors, rows=sel)
+            np.testing.assert_array_equal(out[bi, :, hi], ref)
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)      # [b, h, n, d]
+    dense = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v)).numpy()
+    near = {0: 1, 1: 1, 2: 1, 3: 4, 4: 4, 5: 4}                  # row 2: |2-1| < |2-4|
+    for bi in range(b):
+        for hi, hh in enumerate(heads):
+            for si, tok in enumerate(sel):
+                f, rho, w = tok // (rows * cols), (tok // cols) % rows, tok % cols
+                src = (f * rows + near[rho]) * cols + w
+                np.testing.assert_allclose(out[bi, si, hi], dense[bi, hh, src], rtol=0, atol=1e-12)
+
+
+def test_energy_bnhd_wrapper_indexes_heads_and_batches():
+    """block_energy_bnhd on batch 2, 3 heads and a ragged length, against (1)
+    the one-head function on explicitly sliced inputs and (2) Eq. (5) computed
+    by torch over [batch, heads, N, N] at once: a batched softmax, block sums
+    by reshaping the zero-padded probabilities, divided by each query block's
+    valid row count."""
+    b, n, h, d, block = 2, 29, 3, 4, 8                           # 4 blocks, the last holds 5 tokens
+    q, k = (_distinct_heads(s, b, n + 3, h, d) for s in (43, 44))
+    q[:, n:] = np.nan                                             # padding rows are never read
+    k[:, n:] = np.nan
+    e = O.block_energy_bnhd(q, k, block, seq_len=n)
+    assert e.shape == (b, h, 4, 4)
+    for bi in range(b):
+        for hh in range(h):
+            np.testing.assert_array_equal(
+                e[bi, hh], O.block_energy(q[bi, :, hh], k[bi, :, hh], block, seq_len=n))
+    qt = torch.from_numpy(q[:, :n]).permute(0, 2, 1, 3)
+    kt = torch.from_numpy(k[:, :n]).permute(0, 2, 1, 3)
+    p = torch.softmax(qt @ kt.transpose(-1, -2) / math.sqrt(d), dim=-1)   # [b, h, n, n]
+    pad = torch.zeros(b, h, 32, 32, dtype=torch.float64)
+    pad[:, :, :n, :n] = p
+    sums = pad.reshape(b, h, 4, block, 4, block).sum(dim=(3, 5))
+    valid = torch.tensor([8.0, 8.0, 8.0, 5.0], dtype=torch.float64)
+    np.testing.assert_allclose(e, (sums / valid[:, None]).numpy(), rtol=0, atol=1e-14)
+
+
 # ---------------------------------------------------------------- anchors
 
 def test_nearest_anchor_tables():
