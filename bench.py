@@ -53,7 +53,8 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.mkdtemp(prefix="calibatt_clocks_"), f"clocks_rank{index}.csv")
         # nvidia-smi numbers GPUs physically, CUDA by CUDA_VISIBLE_DEVICES:
         # name the device by its UUID so that each rank samples its own GPU
         self.smi_id = str(index)
@@ -65,7 +66,6 @@ class ClockSampler:
             pass
 
     def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(

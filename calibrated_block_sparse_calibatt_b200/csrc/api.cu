@@ -340,7 +340,7 @@ struct calibatt_dict {
 
   LayerSchedule schedule(int t, int l) const {
     const int64_t ly = layer(t, l);
-    LayerSchedule s;
+    LayerSchedule s{};
     s.row_ptr = d_row_ptr + ly * H * (nq + 1);
     s.col_base = d_col_base + ly * H;
     s.col = d_col;
@@ -349,6 +349,7 @@ struct calibatt_dict {
     s.nq = nq;
     s.bitmap = bitmap ? d_bitmap + ly * H * nq * static_cast<int64_t>(words) : nullptr;
     s.words = words;
+    s.csr_gate = 0;  // lists validated on the host when the layer was set
     return s;
   }
 
@@ -1444,6 +1445,11 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
     for (int i = 0; i < n_heads; ++i) chk.head_ids[i] = heads[i];
     chk.status = status_word_ptr();
     if (!chk.status) return fail(CALIBATT_ERR_CUDA, "status word unavailable");
+    if (tc) {
+      chk.items = items;
+      chk.cta_ptr = cta_ptr;
+      chk.grid = grid;
+    }
     cudaError_t e = calibatt::launch_csr_check(chk, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "skip-list check launch");
     LayerSchedule sch;
@@ -1454,6 +1460,7 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
     sch.items = items;
     sch.cta_ptr = cta_ptr;
     sch.nq = nq;
+    sch.csr_gate = 1;
     return run_sparse(q, k, v, o, *shape, block, sch, tc ? grid : 1, heads, softmax_scale, lse,
                       static_cast<cudaStream_t>(stream));
   });
@@ -1751,9 +1758,14 @@ calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clea
       if (e != cudaSuccess) return cuda_fail(e, "status clear");
     }
     if (*code != 0) {
+      if ((*code & 0xFF) == CALIBATT_ERR_INVALID_ARG && ((*code >> 8) & 0xFF) == calibatt::kCodeScheduleViolation)
+        return fail(CALIBATT_ERR_INVALID_ARG,
+                    "a direct-CSR call's device schedule names an unlisted head or a query block >= nq, or its "
+                    "CTA offsets are not 0 .. n_heads*nq non-decreasing (code 0x%x)", *code);
       if ((*code & 0xFF) == CALIBATT_ERR_INVALID_ARG)
-        return fail(CALIBATT_ERR_INVALID_ARG, "a kernel met a key-block index outside the key range (code 0x%x)",
-                    *code);
+        return fail(CALIBATT_ERR_INVALID_ARG,
+                    "a kernel met a key-block index outside the key range, or a direct-CSR call's row pointers "
+                    "or list order were invalid (code 0x%x)", *code);
       return fail(CALIBATT_ERR_TIMEOUT, "device wait gave up (code 0x%x)", *code);
     }
     return CALIBATT_OK;

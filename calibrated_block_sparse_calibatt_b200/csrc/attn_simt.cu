@@ -31,6 +31,13 @@ __global__ void __launch_bounds__(2 * BLK) simt_attn_kernel(const __grid_constan
   const int tid = threadIdx.x;
   const int row = tid >> 1, half = tid & 1;
   constexpr int kE = HD / 2;
+  if (!ANCHOR && p.sched.csr_gate) {
+    // caller-held lists that the check before this launch found invalid
+    __shared__ int skip;
+    if (tid == 0) skip = p.status != nullptr && csr_violation_recorded(p.status);
+    __syncthreads();
+    if (skip) return;
+  }
 
   // ---- which tile
   int b, h, tile, n;

@@ -915,6 +915,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  if (MODE == kModeSparse && p.sched.csr_gate) {
+    // Caller-held lists: skip the whole CTA if the check that ran before
+    // this launch recorded a violation (one read, shared by the CTA, before
+    // any barrier or tensor memory is set up).
+    __shared__ int skip;
+    if (threadIdx.x == 0) skip = csr_violation_recorded(p.status);
+    __syncthreads();
+    if (skip) return;
+  }
 #ifdef CALIBATT_TRACE
   if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x] = globaltimer();
 #endif

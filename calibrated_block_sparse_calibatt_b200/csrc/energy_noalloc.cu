@@ -39,29 +39,30 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_energy_scratch[kMaxRows];
 
-struct DeviceScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-DeviceScratch g_scratch[kMaxDevices];
+// Per-device address of the array, looked up on the first call that runs on
+// that device.  Only a successful lookup is kept: a failed one (a sticky error
+// left by earlier work, or a call made during stream capture) is retried on
+// the next call instead of failing every later call on that device.
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up once
-// per device), or an error.  In host code the array's name is only a host-side
-// stand-in; a kernel must be given this address instead.
+// Device address of the scratch array on the current device, or an error.  In
+// host code the array's name is only a host-side stand-in; a kernel must be
+// given this address instead.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  DeviceScratch& s = g_scratch[dev];
-  std::call_once(s.once, [&s] {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    s.err = cudaGetSymbolAddress(&p, g_energy_scratch);
-    s.ptr = (s.err == cudaSuccess) ? p : nullptr;
-  });
-  *out = s.ptr;
-  return s.err;
+    e = cudaGetSymbolAddress(&p, g_energy_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -24,7 +24,22 @@ struct LayerSchedule {
   // kept, words 32-bit words per row, [H][nq][words]; row_ptr/col unused.
   const uint32_t* bitmap;
   int32_t words;
+  // Nonzero when the lists and schedule come from the caller's device memory
+  // (direct-CSR call): the kernels then do nothing if the status word holds a
+  // skip-list or schedule violation (codes 23, 24) recorded by the check that
+  // runs before them on the same stream.
+  int32_t csr_gate;
 };
+// Status-word codes (bits 8-15) of the direct-CSR checks.
+constexpr int kCodeListViolation = 23;
+constexpr int kCodeScheduleViolation = 24;
+
+// True when the status word holds a violation of caller-held lists or
+// schedule; read once per CTA by one thread (the caller shares the answer).
+__device__ __forceinline__ bool csr_violation_recorded(const int32_t* status) {
+  const int code = (*reinterpret_cast<const volatile int32_t*>(status) >> 8) & 0xFF;
+  return code == kCodeListViolation || code == kCodeScheduleViolation;
+}
 // Longest skip list a bitmap dictionary may hold per row (the producers decode
 // each row into a shared-memory list of this many 16-bit indices).
 constexpr int kMaxBitmapBlocks = 2048;
@@ -143,6 +158,11 @@ struct CsrCheckParams {
   int32_t n_heads;
   int16_t head_ids[kMaxHeadsPerCall];
   int32_t* status;
+  // persistent schedule of the tensor-core kernel (nullable): items
+  // [n_heads * nq], cta_ptr [grid + 1]
+  const uint32_t* items;
+  const int32_t* cta_ptr;
+  int32_t grid;
 };
 cudaError_t launch_csr_check(const CsrCheckParams& p, cudaStream_t s);
 

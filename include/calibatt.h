@@ -292,20 +292,26 @@ calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* 
  *   row_ptr: device int32[shape->heads][nq + 1], nq = ceil(seq_len / block),
  *     each head's offsets starting at 0;
  *   col_idx: device uint16, head h's list at col_idx + col_base[h], each row
- *     strictly ascending in [0, nq) (the rules calibatt_csr_validate checks;
- *     the call does not read device lists on the host: a small kernel checks
- *     them on `stream` before the attention and records the first violation
- *     in the device status word (calibatt_device_status); the attention
- *     kernels never read outside Q, K, V for a block index >= nq (the
- *     tensor-core kernel's copies are bounded by its tensor maps, the
- *     CUDA-core kernel skips the block), but that call's output is then
- *     meaningless);
+ *     strictly ascending in [0, nq) (the rules calibatt_csr_validate checks);
  *   col_base: device int64[shape->heads];
+ *     the caller guarantees that every listed head's lists lie inside the
+ *     col_idx allocation (col_base[h] + row_ptr[h][nq] entries), which the
+ *     library cannot see;
  *   head_ids: host int32[n_heads], distinct, in [0, heads), n_heads <= 128;
  *   items, cta_ptr, grid: the device copy of a calibatt_csr_schedule result
  *     for the same row_ptr and head_ids (used by the tensor-core kernel, BF16
  *     with block 128, which runs `grid` persistent CTAs; the CUDA-core
  *     kernel walks head_ids and ignores them, and they may then be NULL).
+ * Device checks: the call does not read device arrays on the host.  Small
+ * kernels check them on `stream` before the attention: row pointers start at
+ * 0, do not decrease and hold at most nq blocks per row, block indices are
+ * strictly ascending in [0, nq) (status code 23); every schedule item names a
+ * listed head and a query block < nq, and cta_ptr runs from 0 to
+ * n_heads * nq without decreasing (code 24).  The first violation is
+ * recorded in the device status word (calibatt_device_status, low byte
+ * CALIBATT_ERR_INVALID_ARG), and the attention kernels then return before
+ * reading any list or writing any output -- in that call and in every later
+ * direct-CSR call until the status word is read and cleared.
  * All device arrays are caller-owned and must stay valid until the call's
  * work on `stream` completes.  n_heads == 0 is a no-op.
  * Key Designs 4 (the operation of calibatt_block_sparse_attn). */
@@ -447,9 +453,10 @@ calibatt_status calibatt_repetition_flags(const float* similarity, int32_t n_pro
  * clears it.  The kernels set it (first event wins) when a bounded wait runs
  * out (CALIBATT_ERR_TIMEOUT in the low byte, the waiting role and barrier
  * above it) or when a skip list the host never read breaks the list rules
- * (CALIBATT_ERR_INVALID_ARG in the low byte; 23: the device-side check that
- * calibatt_block_sparse_attn_csr runs before its attention kernel; 22: the
- * CUDA-core kernel met a block index >= nq and skipped that block).  Returns
+ * (CALIBATT_ERR_INVALID_ARG in the low byte; 23 and 24: the device-side
+ * checks of lists and schedule that calibatt_block_sparse_attn_csr runs
+ * before its attention kernel, which then skips its work; 22: the CUDA-core
+ * kernel met a block index >= nq and skipped that block).  Returns
  * the low byte's status when the word is non-zero.
  * Diagnostics; no counterpart in the paper note. */
 calibatt_status calibatt_device_status(void* stream, int32_t* code, int32_t clear);

@@ -278,6 +278,85 @@ def test_csr_call_flags_block_index_out_of_range(C, dtype, block, d):
     assert code & 0xFF == C.ERR_INVALID_ARG and code >> 8 == 23, hex(code)
 
 
+def _padded_col(col_d, nb):
+    """The device list with nb + 64 zero entries after its end, so that even a
+    row pointer run past the lists stays inside the allocation."""
+    return torch.cat([col_d, torch.zeros(nb + 64, dtype=col_d.dtype, device=col_d.device)])
+
+
+@pytest.mark.parametrize("dtype,block,d", [("bf16", 128, 128), ("fp32", 64, 64)])
+def test_csr_call_with_invalid_row_pointers_writes_nothing(C, dtype, block, d):
+    """A row longer than nq (row pointers of head 0 shifted from row 4 on, so
+    they still increase) is flagged by the device check (code 23), and the
+    attention of that call then returns before reading any list: no output
+    is written.  The flag holds for later direct-CSR calls until the status
+    word is read and cleared; then the same call with valid lists runs."""
+    b, n, h = 1, 1000, 2
+    q, k, v = W.make_qkv(34, b, n, h, d, dtype, 1.0, "cuda")
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(12, h, nb, 0.5)
+    rp_d, col_d, base_d, rp = _device_csr(C, masks, h, nb)
+    col_d = _padded_col(col_d, nb)
+    delta = nb + 1 - int(rp[0, 4] - rp[0, 3])            # row 3 now holds nb + 1 blocks
+    bad_rp = rp_d.clone()
+    bad_rp[0, 4:] += delta
+    sched = None
+    if block == 128 and dtype == "bf16":
+        items, cta_ptr = C.csr_schedule(rp, [0, 1], 7)
+        sched = (torch.from_numpy(items.view(np.int32)).cuda(), torch.from_numpy(cta_ptr).cuda(), 7)
+    out = torch.full_like(q, float("nan"))
+    kw = dict(block=block)
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, bad_rp, col_d, base_d, [0, 1], *(sched or ()), **kw)
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [0, 1], *(sched or ()), **kw)
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all(), "the attention ran on lists the check had flagged"
+    code = C.device_status()
+    assert code & 0xFF == C.ERR_INVALID_ARG and code >> 8 == 23, hex(code)
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [0, 1], *(sched or ()), **kw)
+    _check_status(C)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block)
+    _assert_close(_np(out), ref, dtype)
+
+
+def test_csr_call_with_invalid_schedule_writes_nothing(C):
+    """The tensor-core kernel's device schedule is checked before it runs
+    (code 24): an item naming a head that is not listed, a last CTA offset
+    that is not n_heads * nq, and decreasing CTA offsets are each flagged,
+    and the call writes no output."""
+    b, n, h, block, grid = 1, 1000, 2, 128, 6
+    q, k, v = W.make_qkv(35, b, n, h, 128, "bf16", 1.0, "cuda")
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(13, h, nb, 0.5)
+    rp_d, col_d, base_d, rp = _device_csr(C, masks, h, nb)
+    items, cta_ptr = C.csr_schedule(rp, [0], grid)                     # head 0 only
+    unlisted = items.copy()
+    unlisted[3] = (1 << 16) | (int(items[3]) & 0xFFFF)                # head 1 is not listed
+    short_end = cta_ptr.copy()
+    short_end[grid] -= 1
+    decreasing = cta_ptr.copy()
+    c = int(np.argmax(np.diff(cta_ptr) > 0))                          # a CTA with work
+    decreasing[c + 1] = decreasing[c] - 1 if decreasing[c] > 0 else 0
+    decreasing[c] = max(decreasing[c], 1)
+    for it, cp in ((unlisted, cta_ptr), (items, short_end), (items, decreasing)):
+        out = torch.full_like(q, float("nan"))
+        C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [0],
+                                         torch.from_numpy(it.view(np.int32)).cuda(),
+                                         torch.from_numpy(cp).cuda(), grid, block=block)
+        torch.cuda.synchronize()
+        assert torch.isnan(out).all(), "the attention ran on a schedule the check had flagged"
+        code = C.device_status()
+        assert code & 0xFF == C.ERR_INVALID_ARG and code >> 8 == 24, hex(code)
+        assert "schedule" in C.last_error()
+    out = torch.full_like(q, float("nan"))
+    C.calibatt_block_sparse_attn_csr(q, k, v, out, rp_d, col_d, base_d, [0],
+                                     torch.from_numpy(items.view(np.int32)).cuda(),
+                                     torch.from_numpy(cta_ptr).cuda(), grid, block=block)
+    _check_status(C)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q)[:, :, :1], _np(k)[:, :, :1], _np(v)[:, :, :1], masks[:1], block)
+    _assert_close(_np(out)[:, :, :1], ref, "bf16")
+    assert torch.isnan(out[:, :, 1]).all()
+
+
 def test_csr_call_cuda_core_paths(C):
     for dtype, block, d in (("fp32", 64, 64), ("bf16", 64, 128), ("fp32", 128, 128)):
         b, n, h = 1, 700, 3
