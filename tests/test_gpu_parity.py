@@ -5,6 +5,8 @@ inputs max-abs <= 1e-4; bf16 inputs max-abs <= 2e-2 and mean-abs <= 2e-3;
 selected block sets bit-exact.
 """
 
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -540,34 +542,97 @@ def _margin_ok(e_ref, tau, margin=1e-5):
     return np.array(ok)
 
 
+def _check_selection(got, e_ref, tau, margin=1e-5):
+    """Every row of the GPU selection `got` (bool [rows, nk]) is checked
+    against the float64 energies `e_ref` (Key Designs 1: the shortest
+    energy-descending prefix whose cumulative mass reaches tau).
+
+    Rows decided with a margin above `margin` (no energy gap and no partial
+    mass within `margin` of tau) must equal the oracle's set bit for bit.  In
+    the other rows several sets are correct; the GPU set must be one of them:
+    its size is the oracle's k* (or, where the mass at the GPU's size is within
+    `margin` of tau, one of the sizes the rounding allows); its float64 mass
+    reaches tau - margin; it is a prefix of the energy order up to ties within
+    `margin` (no excluded block outweighs a kept one by more than that); and
+    dropping its lightest block leaves a mass below tau + margin.
+    Returns (rows checked bit for bit, rows checked for validity, rows whose
+    size differs from k* within the rounding margin)."""
+    ref = O.select_blocks(e_ref, tau)
+    ok = _margin_ok(e_ref, tau, margin)
+    assert (got[ok] == ref[ok]).all(), "a decided row differs from the oracle"
+    boundary = 0
+    for r in np.flatnonzero(~ok):
+        e, sel = e_ref[r], got[r]
+        kstar = int(ref[r].sum())
+        size = int(sel.sum())
+        mass = math.fsum(e[sel])
+        assert size >= 1, f"row {r}: empty selection"
+        if size != kstar:
+            cum = np.add.accumulate(np.sort(e)[::-1])
+            assert abs(cum[size - 1] - tau) <= margin or abs(cum[kstar - 1] - tau) <= margin, \
+                f"row {r}: size {size} != k* {kstar} away from the tau boundary"
+            boundary += 1
+        assert mass >= tau - margin or size == len(e), f"row {r}: mass {mass} < tau {tau}"
+        kept_min = e[sel].min()
+        excl = e[~sel]
+        assert excl.size == 0 or excl.max() <= kept_min + margin, f"row {r}: not an energy-descending prefix"
+        assert mass - kept_min < tau + margin, f"row {r}: a smaller prefix already reaches tau"
+    return int(ok.sum()), int((~ok).sum()), boundary
+
+
 @pytest.mark.parametrize("std,tau", [(1.0, 0.99), (4.0, 0.5), (4.0, 0.9)])
 def test_energy_select_union_tiny(C, std, tau):
-    """Tiny configuration: 4 seeded Q/K draws, selection at tau, masks unioned (rho = 1/4)."""
+    """Tiny configuration: 4 seeded Q/K draws, selection at tau, masks unioned
+    (rho = 1/4), on the CUDA-core energies (float32, 64-token blocks).  Every
+    row is checked (_check_selection); the union equals the OR of the draws'
+    GPU selections everywhere and the oracle's union on rows every draw
+    decided with a margin."""
     wl = W.WORKLOADS["tiny"]
-    nb = wl.num_blocks
-    cnt = torch.zeros((wl.batch * wl.heads * nb, nb), dtype=torch.int32, device="cuda")
-    ref_masks = []
-    decided = []
-    for s in (10, 11, 12, 13):
-        q, k, _ = W.make_qkv(s, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "fp32", std, "cuda")
-        e = _energy(C, q, k, wl.block)
-        mask = torch.zeros((wl.batch * wl.heads * nb, nb), dtype=torch.uint8, device="cuda")
+    _select_and_union(C, [W.make_qkv(s, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "fp32", std, "cuda")[:2]
+                          for s in (10, 11, 12, 13)], wl.block, tau)
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.9])
+def test_energy_select_union_tensor_core(C, tau):
+    """The same energy -> selection -> union chain on the tensor-core energies
+    (bf16, 128-token blocks): 2 heads, N = 2000 (15 full blocks and one of 80
+    tokens), peaked logits (std 4), 3 seeded draws, rho = 1/3."""
+    draws = [W.make_qkv(s, 1, 2000, 2, 128, "bf16", 4.0, "cuda")[:2] for s in (40, 41, 42)]
+    _select_and_union(C, draws, 128, tau)
+
+
+def _select_and_union(C, draws, block, tau):
+    q0 = draws[0][0]
+    b, n, h, _ = q0.shape
+    nb = O.num_blocks(n, block)
+    rows = b * h * nb
+    cnt = torch.zeros((rows, nb), dtype=torch.int32, device="cuda")
+    tau64 = float(np.float32(tau))
+    gpu_masks, ref_masks, decided = [], [], []
+    exact = checked = boundary = 0
+    for q, k in draws:
+        e = _energy(C, q, k, block)
+        mask = torch.zeros((rows, nb), dtype=torch.uint8, device="cuda")
         C.calibatt_select_blocks(e.view(-1, nb), tau, mask, cnt)
-        e_ref = O.block_energy_bnhd(_np(q), _np(k), wl.block).reshape(-1, nb)
-        tau64 = float(np.float32(tau))
-        ref = O.select_blocks(e_ref, tau64)
-        ok = _margin_ok(e_ref, tau64)
-        decided.append(ok)
+        _check_status(C)
+        e_ref = O.block_energy_bnhd(_np(q), _np(k), block).reshape(-1, nb)
         got = mask.cpu().numpy().astype(bool)
-        assert (got[ok] == ref[ok]).all()
-        ref_masks.append(ref)
+        x, c, bd = _check_selection(got, e_ref, tau64)
+        exact, checked, boundary = exact + x, checked + c, boundary + bd
+        gpu_masks.append(got)
+        ref_masks.append(O.select_blocks(e_ref, tau64))
+        decided.append(_margin_ok(e_ref, tau64))
+    assert (cnt.cpu().numpy() == np.sum(gpu_masks, axis=0)).all(), "selection counts"
     union = torch.zeros_like(cnt, dtype=torch.uint8)
-    C.calibatt_aggregate_masks(cnt, 4, 0.25, union)
+    C.calibatt_aggregate_masks(cnt, len(draws), 1.0 / len(draws), union)
     _check_status(C)
+    union = union.cpu().numpy().astype(bool)
+    assert (union == np.logical_or.reduce(gpu_masks)).all(), "union of the GPU selections"
     all_ok = np.logical_and.reduce(decided)
-    ref_union = O.aggregate_masks(np.stack(ref_masks), 4, 0.25)
-    assert (union.cpu().numpy().astype(bool)[all_ok] == ref_union[all_ok]).all()
-    assert all_ok.mean() > 0.5
+    ref_union = O.aggregate_masks(np.stack(ref_masks), len(draws), 1.0 / len(draws))
+    assert (union[all_ok] == ref_union[all_ok]).all(), \
+        f"{exact} rows bit-exact, {checked} margin rows checked for validity ({boundary} at the tau boundary)"
+    print(f"selection: {exact} rows bit-exact, {checked} margin rows valid, {boundary} at the tau boundary")
 
 
 def test_fma_exp2_error_bound(C):
