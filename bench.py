@@ -146,6 +146,24 @@ def aggregate_tflops(flop_per_rank, world, ms):
     return world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
+def head_partition(heads, rank, world):
+    """Heads of one attention call that rank `rank` of `world` computes under
+    --partition heads: heads[rank::world] (every head on exactly one rank;
+    heads are independent, so no exchange follows)."""
+    return list(range(heads))[rank::world]
+
+
+# MUFU exp2 issue rate of one SM per clock (4 per SM sub-partition), the
+# bound of the offline energy passes (16,384 exp2 per 128x128 tile against
+# 512 tensor-core cycles for its one Q K^T)
+EX2_PER_CLK_PER_SM = 16
+
+
+def mufu_exp2_peak(sm_count, sm_mhz):
+    """exp2 results per second of the whole GPU at a clock."""
+    return EX2_PER_CLK_PER_SM * sm_count * sm_mhz * 1e6
+
+
 DICT_BITMAP = False  # --dict-format bitmap
 
 
@@ -470,6 +488,169 @@ def run_sweep(args, C, torch, stream, pk):
     dct.close()
 
 
+def device_csr(C, torch, masks, heads, nb):
+    """Device row_ptr / 16-bit col_idx / col_base of per-head bool masks and
+    the host row_ptr (the direct-CSR call's inputs)."""
+    rp, ci, _ = C.masks_to_layer_csr(masks, heads, nb)
+    base = np.zeros(heads, np.int64)
+    base[1:] = np.cumsum(rp[:, -1].astype(np.int64))[:-1]
+    col = ci.astype(np.uint16).view(np.int16) if ci.size else np.zeros(1, np.int16)
+    return (torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(), torch.from_numpy(base).cuda(), rp)
+
+
+def run_480p_leg(args, torch, C, stream, pk):
+    """The 480p block-sparse layer (21 x 30 x 52 = 32,760 tokens, 40 heads),
+    timed like the headline call: ms per call, effective TFLOP/s and the
+    fraction of the tensor peak."""
+    wl = W.WORKLOADS["480p"]
+    masks, _ = W.workload_masks(wl)
+    q, k, v = W.make_qkv(wl.seed, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    o = torch.empty_like(q)
+    d = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block)
+    tiles = d.layer_info(0, 0)["retained_tiles"]
+    per_call = time_calls(torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block, stream=stream),
+                          max(5, args.steps), 3, stream)
+    d.close()
+    ms = statistics.mean(per_call)
+    tf = tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12
+    return {"workload": "wan2.1-14b-480p self-attention, block-sparse path", "seq_len": wl.seq_len,
+            "heads": wl.heads, "retained_tiles": tiles, "density": round(tiles / (wl.heads * wl.num_blocks ** 2), 4),
+            "ms_per_call": ms, "effective_tflops": tf, "frac_of_burst_peak": tf / pk["bf16_tflops"],
+            "l2": "inputs 1.0 GB > 126 MB L2, no flush"}
+
+
+def run_tiny_leg(torch, C):
+    """The tiny configuration in full, on the GPU and on the oracle: head 0
+    block-sparse, head 1 on the anchor path (anchors 0 and 4), float32, block
+    64; then block energies of 4 seeded Q/K draws, selection at tau = 0.99 and
+    their union.  Oracle wall time of the whole configuration, GPU device time
+    of the same calls, and the largest output difference."""
+    from oracle import calibatt_oracle as O
+
+    wl = W.WORKLOADS["tiny"]
+    masks, rep = W.workload_masks(wl)
+    nb = wl.num_blocks
+    q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "fp32", wl.input_std, "cuda")
+    draws = [W.make_qkv(s, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "fp32", wl.input_std, "cuda")[:2]
+             for s in (10, 11, 12, 13)]
+    o = torch.empty_like(q)
+    d = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, nb, wl.block)
+    e = torch.empty((wl.batch, wl.heads, nb, nb), device="cuda")
+    ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, device="cuda")
+    sel = torch.empty((wl.batch * wl.heads * nb, nb), dtype=torch.uint8, device="cuda")
+    cnt = torch.zeros((wl.batch * wl.heads * nb, nb), dtype=torch.int32, device="cuda")
+    union = torch.empty_like(sel)
+
+    def gpu_call():
+        C.calibatt_dual_path_attn(q, k, v, o, d, 0, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block)
+        cnt.zero_()
+        for dq, dk in draws:
+            C.calibatt_block_energy(dq, dk, e, ws, wl.block)
+            C.calibatt_select_blocks(e.view(-1, nb), 0.99, sel, cnt)
+        C.calibatt_aggregate_masks(cnt, 4, 0.25, union)
+
+    gpu_ms = statistics.median(time_calls(torch, gpu_call, 20, 3, torch.cuda.current_stream()))
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the tiny configuration")
+    d.close()
+    f64 = lambda t: t.detach().float().cpu().numpy().astype(np.float64)  # noqa: E731
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    dn = [(f64(a), f64(b)) for a, b in draws]
+    t0 = time.perf_counter()
+    sparse_heads = [h for h in range(wl.heads) if masks[h] is not None]
+    ref_s, _ = O.block_sparse_attention_bnhd(qn, kn, vn, masks, wl.block, heads=sparse_heads)
+    ref_a = O.anchor_attention_bnhd(qn, kn, vn, wl.frames, wl.rows, wl.cols, wl.anchors, heads=list(rep))
+    ref_sel = [O.select_blocks(O.block_energy_bnhd(a, b, wl.block).reshape(-1, nb), float(np.float32(0.99)))
+               for a, b in dn]
+    ref_union = O.aggregate_masks(np.stack(ref_sel), 4, 0.25)
+    oracle_s = time.perf_counter() - t0
+    out = f64(o)
+    err = max(float(np.abs(out[:, :, sparse_heads] - ref_s).max()),
+              float(np.abs(out[:, :, list(rep)] - ref_a).max()))
+    return {"workload": "tiny: 2 frames x 8 rows x 16 cols, 2 heads (block-sparse + anchor), head_dim 64, "
+                        "fp32, block 64; energy of 4 draws, tau 0.99, union",
+            "gpu_ms": gpu_ms, "oracle_ms": oracle_s * 1e3, "oracle_cores": os.cpu_count(),
+            "max_abs_err": err, "tolerance": 1e-4, "within_tolerance": err <= 1e-4,
+            "union_equal": bool((union.cpu().numpy().astype(bool) == ref_union).all())}
+
+
+SWEEP_SAMPLE_CALLS = 100
+SWEEP_SAMPLE_DENSE = 10
+
+
+def sweep_sample_picks(n_calls, steps=W.SWEEP_STEPS, layers=W.SWEEP_LAYERS):
+    """(timestep, layer) calls of a sample of the schedule sweep: the same
+    number of calls at every timestep (so the density ramp is sampled evenly),
+    layers spread over the schedule."""
+    per_t = max(1, n_calls // steps)
+    return [(t, (7 * t + j * layers // per_t) % layers) for t in range(steps) for j in range(per_t)][:n_calls]
+
+
+def run_sweep_sample(torch, C, stream, pk, n_calls=SWEEP_SAMPLE_CALLS, n_dense=SWEEP_SAMPLE_DENSE):
+    """A sample of the schedule sweep (n_calls of its 2,000 dual-path 720p
+    calls, fresh seeded Q/K/V per call, masks and repetitive heads exactly as
+    the full sweep draws them), with the dense path timed on n_dense of the
+    calls.  The aggregate ratio over the schedule is estimated as (mean dense
+    ms) / (mean dual-path ms) of the sample."""
+    wl = W.WORKLOADS["720p_sweep"]
+    picks = sweep_sample_picks(n_calls)
+    H, nb = wl.heads, wl.num_blocks
+    nnz = sum(W.sweep_record_blocks(wl, t, l, h) for t, l in picks for h in range(H))
+    dct = C.MaskDictionary(len(picks), 1, H, nb, nb, wl.block, nnz)
+    dct.set_anchor_geometry(wl.frames, wl.rows, wl.cols, wl.anchors)
+    for i, (t, l) in enumerate(picks):
+        masks, rep = W.sweep_layer_masks(wl, t, l, "cuda")
+        rp, ci = W.layer_csr(masks)
+        rep_arr = np.zeros(H, np.uint8)
+        rep_arr[list(rep)] = 1
+        dct.set_layer(i, 0, rp, ci, rep_arr)
+    anchor_tiles_per_head = -(-wl.frames * len(wl.anchors) * wl.cols // 128) * nb
+    tiles = []
+    for i in range(len(picks)):
+        li = dct.layer_info(i, 0)
+        tiles.append(li["retained_tiles"] + li["repetitive_heads"] * anchor_tiles_per_head)
+    o = None
+    per_call = []
+    for i, (t, l) in enumerate(picks):
+        q, k, v = W.make_qkv(W.seed_for("sweep-qkv", t, l) % (1 << 62), 1, wl.seq_len, H, wl.head_dim, "bf16",
+                             wl.input_std, "cuda")
+        if o is None:
+            o = torch.empty_like(q)
+            for _ in range(3):
+                C.calibatt_dual_path_attn(q, k, v, o, dct, i, 0, wl.frames, wl.rows, wl.cols, wl.anchors, wl.block,
+                                          stream=stream)
+        per_call.append(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_dual_path_attn(q, k, v, o, dct, i, 0, wl.frames, wl.rows, wl.cols, wl.anchors,
+                                                     wl.block, stream=stream), 1, 0, stream)))
+        del q, k, v
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the sweep sample")
+    dct.close()
+    ones = [np.ones((nb, nb), bool)] * H
+    d_dense = build_dict(C, ones, H, nb, wl.block)
+    dense_tiles = d_dense.layer_info(0, 0)["retained_tiles"]
+    dense_ms = []
+    for t, l in picks[::max(1, len(picks) // n_dense)][:n_dense]:
+        q, k, v = W.make_qkv(W.seed_for("sweep-qkv", t, l) % (1 << 62), 1, wl.seq_len, H, wl.head_dim, "bf16",
+                             wl.input_std, "cuda")
+        dense_ms.append(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d_dense, 0, 0, wl.block, stream=stream),
+            1, 1, stream)))
+        del q, k, v
+    d_dense.close()
+    sparse_mean = statistics.mean(per_call)
+    dense_mean = statistics.mean(dense_ms)
+    calls = W.SWEEP_STEPS * W.SWEEP_LAYERS
+    return {"workload": f"wan2.1-14b-720p schedule sweep, sample of {len(picks)} of its {calls} dual-path calls "
+                        f"({len(picks) // W.SWEEP_STEPS} per timestep), dense path on {len(dense_ms)} of them",
+            "ms_per_call": sparse_mean, "dense_ms_per_call": dense_mean,
+            "speedup_vs_dense": dense_mean / sparse_mean,
+            "estimated_total_s": sparse_mean * calls / 1e3, "estimated_dense_total_s": dense_mean * calls / 1e3,
+            "effective_tflops": sum(tiles) * FLOP_PER_TILE / (sum(per_call) * 1e-3) / 1e12,
+            "dense_tiles_per_call": dense_tiles,
+            "min_ms_per_call": min(per_call), "max_ms_per_call": max(per_call)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -499,6 +680,10 @@ def main():
                     help="--dual-case as one fused launch (1) or block-sparse + anchor launches (2)")
     ap.add_argument("--anchor-case", action="store_true",
                     help="time the anchor path alone (the 12 repetitive heads of the dual-path 720p layer)")
+    ap.add_argument("--partition", default="replicas", choices=["replicas", "heads"],
+                    help="with N > 1 ranks: every rank times its own 720p layer (replicas, weak scaling), or "
+                         "the ranks split the 40 heads of ONE call, rank r taking heads r, r+N, ... (strong "
+                         "scaling, each rank reading only its heads' Q/K/V)")
     ap.add_argument("--dense-sample", type=int, default=50,
                     help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
@@ -546,8 +731,11 @@ def main():
     import dataclasses
     wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
     masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])
-    q, k, v = W.make_qkv(rank_seed(wl.seed, rank), 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std,
-                         "cuda")
+    by_heads = args.partition == "heads"
+    # under --partition heads every rank holds the same call's inputs and
+    # computes only its heads of it
+    q, k, v = W.make_qkv(wl.seed if by_heads else rank_seed(wl.seed, rank), 1, wl.seq_len, wl.heads, wl.head_dim,
+                         "bf16", wl.input_std, "cuda")
     if args.layout == "bhnd":
         # the same [batch, N, heads, head_dim] tensors stored head-major: a head's
         # rows are contiguous (stride_n = head_dim) instead of heads*head_dim apart
@@ -560,6 +748,21 @@ def main():
 
     def sparse_call():
         C.calibatt_block_sparse_attn(q, k, v, o, d_sparse, 0, 0, wl.block, stream=stream)
+
+    my_heads = head_partition(wl.heads, rank, world) if by_heads else list(range(wl.heads))
+    my_tiles = tiles
+    if by_heads:
+        # this rank's share of the call: the direct-CSR call over its heads
+        # (device lists of every head, a schedule of its heads only)
+        rp_d, col_d, base_d, rp_h = device_csr(C, torch, [masks[h] for h in range(wl.heads)], wl.heads,
+                                               wl.num_blocks)
+        items, cta_ptr = C.csr_schedule(rp_h, my_heads, C.device_sm_count())
+        part_args = (rp_d, col_d, base_d, my_heads, torch.from_numpy(items.view(np.int32)).cuda(),
+                     torch.from_numpy(cta_ptr).cuda(), cta_ptr.size - 1)
+        my_tiles = int(sum(int(rp_h[h, -1]) for h in my_heads))
+
+        def sparse_call():  # noqa: F811
+            C.calibatt_block_sparse_attn_csr(q, k, v, o, *part_args, block=wl.block, stream=stream)
 
     # ---------------------------------------------------------------- timed region
     for _ in range(args.warmup):
@@ -579,12 +782,16 @@ def main():
         raise RuntimeError("device wait timed out during the benchmark")
     total_ms = max_over_ranks(sum(per_call), dist, "cuda")
     ms = total_ms / args.steps
-    value = aggregate_tflops(flop, world, ms)
+    # replicas: every rank did a whole call; heads: the ranks together did one
+    value = flop / (ms * 1e-3) / 1e12 if by_heads else aggregate_tflops(flop, world, ms)
     avg_launch_ms = statistics.mean(per_call)
-    achieved = flop / (avg_launch_ms * 1e-3) / 1e12
+    achieved = my_tiles * FLOP_PER_TILE / (avg_launch_ms * 1e-3) / 1e12
 
     extras = {}
-    if not args.no_extras:
+    if by_heads:
+        extras["head_partition"] = {"heads_this_rank": my_heads, "tiles_this_rank": my_tiles,
+                                    "api": "calibatt_block_sparse_attn_csr with this rank's head_ids"}
+    if not args.no_extras and not by_heads:
         # dense path on the same inputs: all-ones skip lists held on the device,
         # through the direct-CSR call (no dictionary)
         nbk, hh = wl.num_blocks, wl.heads
@@ -639,12 +846,24 @@ def main():
             torch, lambda: C.calibatt_block_energy(q, k, e_out, e_ws, wl.block, stream=stream),
             3, 1, stream)), dist, "cuda")
         del e_out, e_ws
+        exp2_per_call = 2 * wl.seq_len ** 2 * wl.heads      # both passes exponentiate every score
+        sms = C.device_sm_count()
+        ex2_peak = mufu_exp2_peak(sms, 1965.0)
         extras["block_energy_720p"] = {
             "ms_per_call": energy_ms, "heads": wl.heads,
             "tflops_two_qk_passes": 2 * 2.0 * wl.seq_len ** 2 * wl.head_dim * wl.heads / (energy_ms * 1e-3) / 1e12,
-            "exp2_per_call": 2 * wl.seq_len ** 2 * wl.heads}
+            "exp2_per_call": exp2_per_call,
+            "roofline": {"bound": "mufu", "achieved": exp2_per_call / (energy_ms * 1e-3) / 1e9,
+                         "peak": ex2_peak / 1e9, "unit": "G exp2/s",
+                         "frac": exp2_per_call / (energy_ms * 1e-3) / ex2_peak,
+                         "peak_basis": f"{EX2_PER_CLK_PER_SM} exp2/clk/SM x {sms} SMs x 1965 MHz (max SM clock); "
+                                       "one exp2 pair in four runs on the FMA pipe and is counted all the same"}}
         if C.device_status() != 0:
             raise RuntimeError("device wait timed out during the extra legs")
+        if world == 1:
+            extras["cfg_480p"] = run_480p_leg(args, torch, C, stream, pk)
+            extras["cfg_tiny"] = run_tiny_leg(torch, C)
+            extras["sweep_sample"] = run_sweep_sample(torch, C, stream, pk)
 
     # -------------------------------------------------------- end to end (host buffers)
     # Every step is one calibatt_block_sparse_attn_host call: its Q, K, V are
@@ -655,7 +874,7 @@ def main():
     # and the next step's input copy never queues behind an output copy
     # (2.3% faster than two sets; the link then carries ~64 GB/s both ways).
     e2e = None
-    if not args.no_extras:
+    if not args.no_extras and not by_heads:
         n_sets = 3
         if args.layout == "bnhd":
             hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -700,7 +919,7 @@ def main():
         del hq, hk, hv, hos, dsets
 
     cpu = parity = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not by_heads:
         # the block-sparse output of this run's inputs (the extra legs reused o)
         C.calibatt_block_sparse_attn(q, k, v, o, d_sparse, 0, 0, wl.block, stream=stream)
         torch.cuda.synchronize()
@@ -710,20 +929,22 @@ def main():
         line = {
             "metric": "effective TFLOP/s (retained blocks) and ms/call, % of B200 BF16 tensor peak",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "strong" if by_heads else "weak",
+            "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "wan2.1-14b-720p self-attention, block-sparse path", "batch": 1,
                        "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
                        "heads": wl.heads, "head_dim": wl.head_dim, "seq_len": wl.seq_len, "block": wl.block,
                        "density": round(density, 4), "retained_tiles": tiles,
-                       "l2": "inputs 2.32 GB > 126 MB L2, no flush", "parallelism": f"replicas x{world}",
+                       "l2": "inputs 2.32 GB > 126 MB L2, no flush",
+                       "parallelism": f"heads split over {world} ranks" if by_heads else f"replicas x{world}",
                        "storage": "[batch, N, heads, head_dim]" if args.layout == "bnhd"
                        else "[batch, heads, N, head_dim] (head-major)"},
             "pct_of_peak": achieved / pk["bf16_tflops"],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16_tflops"],
                          # counters were taken on the default (token-major) storage
-                         "traffic": measured_traffic(tiles) if args.layout == "bnhd" else None,
+                         "traffic": measured_traffic(my_tiles) if args.layout == "bnhd" and not by_heads else None,
                          "traffic_unit": "bytes per launch (DRAM read + write)",
                          "algorithmic_bytes": 4 * q.numel() * q.element_size(),
                          "peak_source": f"{pk['source']} burst bf16",
@@ -734,7 +955,8 @@ def main():
                                                if pk["bf16_tflops_sustained"] else None)},
             "clocks": clk.summary(),
             "e2e": e2e,
-            "gpu_launches": args.steps,
+            # the direct-CSR call of --partition heads also launches its list and schedule checks
+            "gpu_launches": args.steps * (3 if by_heads else 1),
             "cpu_baseline": cpu,
             "parity": parity,
             **extras,

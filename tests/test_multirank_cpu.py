@@ -34,8 +34,11 @@ def _worker(rank, world, port, out):
         local_ms = 10.0 + 5.0 * rank                    # rank 1 is the slow one
         job_ms = bench.max_over_ranks(local_ms, dist)
         first = bench.max_over_ranks(-rank, dist)       # collectives stay in step across calls
+        mine = bench.head_partition(40, rank, world)   # --partition heads: this rank's heads of one call
+        parts = [None] * world
+        dist.all_gather_object(parts, mine)
         out.put((rank, job_ms, first, bench.rank_seed(2000, rank),
-                 bench.aggregate_tflops(2.0e12, world, job_ms)))
+                 bench.aggregate_tflops(2.0e12, world, job_ms), parts))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -57,6 +60,22 @@ def test_two_gloo_ranks_time_is_max_over_ranks():
     assert res[0][3] != res[1][3]                       # independent inputs per rank
     # whole-job throughput: both ranks' work over the slowest rank's time
     assert res[0][4] == pytest.approx(2 * 2.0e12 / 15e-3 / 1e12)
+    # --partition heads: the ranks' head lists cover the 40 heads of the call
+    # exactly once, and every rank sees the same partition
+    parts = res[0][5]
+    assert parts == res[1][5]
+    assert sorted(h for p in parts for h in p) == list(range(40))
+    assert all(len(p) == 20 for p in parts)
+
+
+@pytest.mark.parametrize("heads,world", [(40, 3), (40, 8), (12, 5), (3, 4)])
+def test_head_partition_covers_every_head_once(heads, world):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    parts = [bench.head_partition(heads, r, world) for r in range(world)]
+    assert sorted(h for p in parts for h in p) == list(range(heads))
+    assert max(map(len, parts)) - min(map(len, parts)) <= 1
 
 
 def test_single_process_and_reference_arm_off_rank_zero():

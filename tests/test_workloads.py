@@ -143,3 +143,23 @@ def test_cpu_baseline_leg_reports_parity_of_the_given_output():
     _, bad = bench.cpu_baseline(wl, masks, q, k, v, torch.from_numpy(ref).float() + 0.1, budget_s=0.3)
     assert not bad["within_tolerance"] and abs(bad["max_abs"] - 0.1) < 1e-3
     assert isinstance(bench.cpu_baseline(wl, masks, q, k, v, budget_s=0.1), dict)   # no output: baseline only
+
+
+def test_sweep_sample_spreads_over_the_schedule():
+    """The bench's sampled sweep: the same number of calls at every timestep
+    (the density ramp is sampled evenly), distinct calls, layers in range."""
+    import bench
+
+    picks = bench.sweep_sample_picks(100)
+    assert len(picks) == 100 == len(set(picks))
+    per_t = {}
+    for t, l in picks:
+        assert 0 <= t < W.SWEEP_STEPS and 0 <= l < W.SWEEP_LAYERS
+        per_t[t] = per_t.get(t, 0) + 1
+    assert sorted(per_t) == list(range(W.SWEEP_STEPS)) and set(per_t.values()) == {2}
+
+
+def test_mufu_peak_arithmetic():
+    import bench
+
+    assert bench.mufu_exp2_peak(148, 1965.0) == 16 * 148 * 1965e6
