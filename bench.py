@@ -164,14 +164,18 @@ def mufu_exp2_peak(sm_count, sm_mhz):
     return EX2_PER_CLK_PER_SM * sm_count * sm_mhz * 1e6
 
 
-DICT_BITMAP = False  # --dict-format bitmap
+DICT_FORMAT = "lists"  # --dict-format
 
 
-def build_dict(C, masks, heads, nb, block, geometry=None):
-    """One-layer dictionary; with geometry = (frames, rows, cols, anchors) the
-    dual path of the layer runs as one launch."""
+def build_dict(C, masks, heads, nb, block, geometry=None, fmt=None):
+    """One-layer dictionary (format `fmt`, default --dict-format); with
+    geometry = (frames, rows, cols, anchors) the dual path of the layer runs
+    as one launch."""
+    fmt = fmt or DICT_FORMAT
     rp, ci, rep_arr = C.masks_to_layer_csr(masks, heads, nb)
-    d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, ci.size), bitmap=DICT_BITMAP)
+    cap = C.count_intervals(rp, ci) if fmt == "intervals" else ci.size
+    d = C.MaskDictionary(1, 1, heads, nb, nb, block, max(1, cap), bitmap=fmt == "bitmap",
+                         intervals=fmt == "intervals")
     if geometry is not None:
         d.set_anchor_geometry(*geometry)
     d.set_layer(0, 0, rp, ci, rep_arr)
@@ -401,7 +405,9 @@ def run_sweep(args, C, torch, stream, pk):
     T, L, H, nb = args.sweep_steps, args.sweep_layers, wl.heads, wl.num_blocks
     t_build = time.time()
     nnz = sum(W.sweep_record_blocks(wl, t, l, h, T) for t in range(T) for l in range(L) for h in range(H))
-    dct = C.MaskDictionary(T, L, H, nb, nb, wl.block, nnz, bitmap=DICT_BITMAP)
+    if DICT_FORMAT == "intervals":
+        raise SystemExit("the full sweep builds its dictionary as index lists or bitmaps")
+    dct = C.MaskDictionary(T, L, H, nb, nb, wl.block, nnz, bitmap=DICT_FORMAT == "bitmap")
     dct.set_anchor_geometry(wl.frames, wl.rows, wl.cols, wl.anchors)
     for t in range(T):
         for l in range(L):
@@ -471,7 +477,7 @@ def run_sweep(args, C, torch, stream, pk):
         "config": {"workload": "wan2.1-14b-720p schedule sweep, dual path (block-sparse + anchor heads)",
                    "timesteps": T, "layers": L, "heads": H, "repetitive_heads_per_call": W.SWEEP_REPETITIVE,
                    "anchors": list(wl.anchors), "density": "0.60 -> 0.20 over the timesteps",
-                   "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
+                   "dictionary_format": DICT_FORMAT,
                    "inputs": "fresh seeded Q/K/V per call (2.32 GB > L2)", "parallelism": "replicas x1"},
         "pct_of_peak": value / pk["bf16_tflops"],
         "clocks": clk.summary(),
@@ -496,6 +502,36 @@ def device_csr(C, torch, masks, heads, nb):
     base[1:] = np.cumsum(rp[:, -1].astype(np.int64))[:-1]
     col = ci.astype(np.uint16).view(np.int16) if ci.size else np.zeros(1, np.int16)
     return (torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(), torch.from_numpy(base).cuda(), rp)
+
+
+def run_format_ab(torch, C, stream, wl, masks, q, k, v, o, tiles, rounds=6, calls=2):
+    """The headline call over the three dictionary formats of the same masks
+    (index lists, bitmap, intervals), interleaved round by round so that the
+    power-capped clock drifts alike for all three; median ms per format, the
+    dictionary's device bytes, and whether the outputs are bitwise equal."""
+    dicts = {f: build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block, fmt=f)
+             for f in ("lists", "bitmap", "intervals")}
+    outs = {}
+    for f, d in dicts.items():
+        C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block, stream=stream)
+        torch.cuda.synchronize()
+        outs[f] = o.clone()
+    same = all(torch.equal(outs["lists"], outs[f]) for f in outs)
+    del outs
+    ms = {f: [] for f in dicts}
+    for _ in range(rounds):
+        for f, d in dicts.items():
+            ms[f] += time_calls(torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block,
+                                                                            stream=stream), calls, 1, stream)
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the dictionary-format comparison")
+    res = {"interleaved": f"{rounds} rounds x {calls} calls per format", "outputs_bitwise_equal": same}
+    for f, d in dicts.items():
+        med = statistics.median(ms[f])
+        res[f] = {"ms_per_call": med, "effective_tflops": tiles * FLOP_PER_TILE / (med * 1e-3) / 1e12,
+                  "device_bytes": d.info()["device_bytes"]}
+        d.close()
+    return res
 
 
 def run_480p_leg(args, torch, C, stream, pk):
@@ -664,8 +700,9 @@ def main():
     ap.add_argument("--workload", default="720p", choices=["720p", "sweep"],
                     help="sweep: the mask-dictionary schedule sweep (one dual-path 720p call per "
                          "timestep and layer), reported as aggregate time against the dense path")
-    ap.add_argument("--dict-format", default="lists", choices=["lists", "bitmap"],
-                    help="mask dictionary storage: 2-byte index lists, or one bit per block pair")
+    ap.add_argument("--dict-format", default="lists", choices=["lists", "bitmap", "intervals"],
+                    help="mask dictionary storage: 2-byte index lists, one bit per block pair, or each "
+                         "row's contiguous key-block intervals")
     ap.add_argument("--sweep-steps", type=int, default=W.SWEEP_STEPS)
     ap.add_argument("--sweep-layers", type=int, default=W.SWEEP_LAYERS)
     ap.add_argument("--epilogue-probe", action="store_true",
@@ -688,8 +725,8 @@ def main():
                     help="sweep calls also timed on the dense path (its time does not depend on the masks)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    global DICT_BITMAP
-    DICT_BITMAP = args.dict_format == "bitmap"
+    global DICT_FORMAT
+    DICT_FORMAT = args.dict_format
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -861,6 +898,7 @@ def main():
         if C.device_status() != 0:
             raise RuntimeError("device wait timed out during the extra legs")
         if world == 1:
+            extras["dictionary_formats"] = run_format_ab(torch, C, stream, wl, masks, q, k, v, o, tiles)
             extras["cfg_480p"] = run_480p_leg(args, torch, C, stream, pk)
             extras["cfg_tiny"] = run_tiny_leg(torch, C)
             extras["sweep_sample"] = run_sweep_sample(torch, C, stream, pk)
@@ -933,7 +971,7 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "wan2.1-14b-720p self-attention, block-sparse path", "batch": 1,
-                       "dictionary_format": "bitmap" if DICT_BITMAP else "index lists",
+                       "dictionary_format": DICT_FORMAT,
                        "heads": wl.heads, "head_dim": wl.head_dim, "seq_len": wl.seq_len, "block": wl.block,
                        "density": round(density, 4), "retained_tiles": tiles,
                        "l2": "inputs 2.32 GB > 126 MB L2, no flush",

@@ -62,6 +62,7 @@ SIGNATURES = {
     "calibatt_dict_set_layer": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp]),
     "calibatt_debug_bounded_wait": (_i32, [_vp]),
     "calibatt_dict_create_bitmap": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _P(_vp)]),
+    "calibatt_dict_create_intervals": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i32, _P(_vp)]),
     "calibatt_dict_set_anchor_geometry": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32]),
     "calibatt_spatial_similarity": (_i32, [_vp, _vp, _P(Shape), _i32, _i32, _i32, _vp, _i32, _f32, _vp, _vp,
                                            ctypes.c_size_t, _vp]),
@@ -178,6 +179,27 @@ def csr_to_intervals(nq, row_ptr, col_idx):
     return ptr, start[:n.value], length[:n.value]
 
 
+def count_intervals(row_ptr, col_idx):
+    """Contiguous key-block intervals of a layer's CSR (row_ptr [H, nq + 1],
+    the heads' lists concatenated): the capacity an interval dictionary needs
+    for it.  Counted with numpy (argument preparation for
+    calibatt_dict_create_intervals)."""
+    rp = np.asarray(row_ptr, dtype=np.int64).reshape(-1, np.asarray(row_ptr).shape[-1])
+    ci = np.asarray(col_idx, dtype=np.int64).reshape(-1)
+    if ci.size == 0:
+        return 0
+    # a block starts an interval unless it follows its predecessor in the same row
+    head_off = np.concatenate([[0], np.cumsum(rp[:, -1])])
+    starts = np.zeros(ci.size, bool)
+    for h in range(rp.shape[0]):
+        s = rp[h, :-1] + head_off[h]
+        e = rp[h, 1:] + head_off[h]
+        first = s[e > s]
+        starts[first] = True
+    starts[1:] |= ci[1:] != ci[:-1] + 1
+    return int(starts.sum())
+
+
 def lpt_schedule(cost, n_bins):
     c = np.ascontiguousarray(np.asarray(cost, dtype=np.int64))
     bin_ptr = np.zeros(n_bins + 1, np.int32)
@@ -236,13 +258,18 @@ def device_status(stream=None, clear=True) -> int:
 class MaskDictionary:
     """Owns a calibatt_dict (per (t, l, h) skip lists and repetitive flags on the GPU)."""
 
-    def __init__(self, T, L, H, nq, nk, block, nnz_capacity=0, num_ctas=0, bitmap=False):
+    def __init__(self, T, L, H, nq, nk, block, nnz_capacity=0, num_ctas=0, bitmap=False, intervals=False):
         """bitmap=True stores one bit per (query block, key block) per record
-        (calibatt_dict_create_bitmap) instead of index lists."""
+        (calibatt_dict_create_bitmap) instead of index lists; intervals=True
+        stores each row's contiguous key-block intervals
+        (calibatt_dict_create_intervals), nnz_capacity then counting intervals."""
         self.T, self.L, self.H, self.nq, self.nk, self.block = T, L, H, nq, nk, block
         h = ctypes.c_void_p(None)
         if bitmap:
             check(LIB.calibatt_dict_create_bitmap(T, L, H, nq, nk, block, int(num_ctas), ctypes.byref(h)))
+        elif intervals:
+            check(LIB.calibatt_dict_create_intervals(T, L, H, nq, nk, block, int(nnz_capacity), int(num_ctas),
+                                                     ctypes.byref(h)))
         else:
             check(LIB.calibatt_dict_create(T, L, H, nq, nk, block, int(nnz_capacity), int(num_ctas),
                                            ctypes.byref(h)))

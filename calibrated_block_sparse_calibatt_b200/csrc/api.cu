@@ -327,6 +327,13 @@ struct calibatt_dict {
   int64_t f_stride = 0;              // item slots per layer
   uint32_t* d_fitems = nullptr;
   int32_t* d_fcta_ptr = nullptr;
+  // Interval format (calibatt_dict_create_intervals): per row, contiguous
+  // key-block runs (start | length << 16) instead of one index per block;
+  // nnz_cap / nnz_used then count runs and blocks_used the retained blocks.
+  bool intervals = false;
+  int32_t* d_run_ptr = nullptr;
+  uint32_t* d_runs = nullptr;
+  int64_t blocks_used = 0;
 
   int64_t layer(int t, int l) const { return static_cast<int64_t>(t) * L + l; }
 
@@ -349,6 +356,11 @@ struct calibatt_dict {
     s.nq = nq;
     s.bitmap = bitmap ? d_bitmap + ly * H * nq * static_cast<int64_t>(words) : nullptr;
     s.words = words;
+    if (intervals) {
+      s.col = nullptr;
+      s.run_ptr = d_run_ptr + ly * H * (nq + 1);
+      s.runs = d_runs;
+    }
     s.csr_gate = 0;  // lists validated on the host when the layer was set
     return s;
   }
@@ -362,6 +374,10 @@ struct calibatt_dict {
     cudaFree(d_fitems);
     cudaFree(d_fcta_ptr);
     cudaFree(d_bitmap);
+    cudaFree(d_run_ptr);
+    cudaFree(d_runs);
+    d_run_ptr = nullptr;
+    d_runs = nullptr;
     d_bitmap = nullptr;
     d_fitems = nullptr;
     d_fcta_ptr = nullptr;
@@ -416,8 +432,9 @@ calibatt_status run_sparse(const void* q, const void* k, const void* v, void* o,
     return CALIBATT_OK;
   }
   // CUDA-core path, heads in chunks of kMaxHeadsPerCall.
-  if (sch.bitmap)
-    return fail(CALIBATT_ERR_UNSUPPORTED, "bitmap dictionaries run on the tensor-core path only (bf16, block 128)");
+  if (sch.bitmap || sch.runs)
+    return fail(CALIBATT_ERR_UNSUPPORTED,
+                "bitmap and interval dictionaries run on the tensor-core path only (bf16, block 128)");
   for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
     SimtParams p;
     std::memset(&p, 0, sizeof(p));
@@ -820,6 +837,63 @@ calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int
   });
 }
 
+calibatt_status calibatt_dict_create_intervals(int32_t T, int32_t L, int32_t H, int32_t nq, int32_t nk,
+                                               int32_t block, int64_t run_capacity, int32_t num_ctas,
+                                               calibatt_dict** out) {
+  return guarded([&]() -> calibatt_status {
+    if (!out) return fail(CALIBATT_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (T < 1 || L < 1 || H < 1 || nq < 1 || nk < 1 || run_capacity < 0)
+      return fail(CALIBATT_ERR_INVALID_ARG, "T, L, H, nq, nk must be >= 1 and run_capacity >= 0");
+    if (nq != nk) return fail(CALIBATT_ERR_INVALID_ARG, "self-attention dictionary needs nq == nk");
+    if (nq > calibatt::kMaxBitmapBlocks)
+      return fail(CALIBATT_ERR_UNSUPPORTED, "interval dictionaries hold at most %d blocks per row",
+                  calibatt::kMaxBitmapBlocks);
+    if (H > 65535) return fail(CALIBATT_ERR_UNSUPPORTED, "H must be <= 65535");
+    calibatt_status st = check_block(block);
+    if (st != CALIBATT_OK) return st;
+    int G = num_ctas;
+    if (G <= 0) G = device_sm_count();
+    if (G <= 0) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    std::unique_ptr<calibatt_dict> holder(new calibatt_dict());
+    calibatt_dict* d = holder.get();
+    d->T = T;
+    d->L = L;
+    d->H = H;
+    d->nq = nq;
+    d->nk = nk;
+    d->block = block;
+    d->G = G;
+    d->intervals = true;
+    cudaGetDevice(&d->device);
+    d->nnz_cap = run_capacity;
+    const int64_t layers = static_cast<int64_t>(T) * L;
+    d->layer_set.assign(layers, 0);
+    d->rep.assign(layers * H, 0);
+    d->n_sparse.assign(layers, 0);
+    d->n_rep.assign(layers, 0);
+    d->retained.assign(layers, 0);
+    const size_t b_rp = sizeof(int32_t) * layers * H * (nq + 1);
+    const size_t b_cb = sizeof(int64_t) * layers * H;
+    const size_t b_runs = sizeof(uint32_t) * std::max<int64_t>(1, run_capacity);
+    const size_t b_it = sizeof(uint32_t) * layers * H * nq;
+    const size_t b_cta = sizeof(int32_t) * layers * (G + 1);
+    cudaError_t e = cudaMalloc(&d->d_row_ptr, b_rp);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_run_ptr, b_rp);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_col_base, b_cb);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_runs, b_runs);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e != cudaSuccess) {
+      d->release();
+      return cuda_fail(e, "interval dictionary allocation");
+    }
+    d->device_bytes = static_cast<int64_t>(2 * b_rp + b_cb + b_runs + b_it + b_cta);
+    *out = holder.release();
+    return CALIBATT_OK;
+  });
+}
+
 calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, const int32_t* row_ptr,
                                         const int32_t* col_idx, const uint8_t* repetitive) {
   return guarded([&]() -> calibatt_status {
@@ -842,10 +916,37 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
       head_off[h + 1] = head_off[h] + rp[nq];
     }
     const int64_t nnz = head_off[H];
-    if (!d->bitmap && d->nnz_used + nnz > d->nnz_cap)
-      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld)",
-                  (long long)d->nnz_used, (long long)nnz, (long long)d->nnz_cap);
-    std::vector<uint16_t> col16(d->bitmap ? 0 : nnz);
+    // Interval format: each row's contiguous runs, and per head its run
+    // pointers (counted from the head's first run) and its first run's offset.
+    std::vector<uint32_t> runs;
+    std::vector<int32_t> run_ptr;
+    std::vector<int64_t> run_head_off(H + 1, 0);
+    if (d->intervals) {
+      run_ptr.assign(static_cast<size_t>(H) * (nq + 1), 0);
+      for (int h = 0; h < H; ++h) {
+        const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
+        const int32_t* ci = col_idx ? col_idx + head_off[h] : nullptr;
+        int32_t* hp = run_ptr.data() + static_cast<size_t>(h) * (nq + 1);
+        const size_t head_start = runs.size();
+        for (int r = 0; r < nq; ++r) {
+          hp[r] = static_cast<int32_t>(runs.size() - head_start);
+          for (int32_t x = rp[r]; x < rp[r + 1]; ++x) {
+            if (x > rp[r] && ci[x] == ci[x - 1] + 1)
+              runs.back() += 1u << 16;                         // extends the current run
+            else
+              runs.push_back(static_cast<uint32_t>(ci[x]) | (1u << 16));
+          }
+        }
+        hp[nq] = static_cast<int32_t>(runs.size() - head_start);
+        run_head_off[h + 1] = static_cast<int64_t>(runs.size());
+      }
+    }
+    const int64_t units = d->intervals ? static_cast<int64_t>(runs.size()) : nnz;
+    if (!d->bitmap && d->nnz_used + units > d->nnz_cap)
+      return fail(CALIBATT_ERR_INVALID_ARG, "dictionary capacity exceeded (%lld + %lld > %lld %s)",
+                  (long long)d->nnz_used, (long long)units, (long long)d->nnz_cap,
+                  d->intervals ? "intervals" : "blocks");
+    std::vector<uint16_t> col16(d->bitmap || d->intervals ? 0 : nnz);
     for (size_t i = 0; i < col16.size(); ++i) col16[i] = static_cast<uint16_t>(col_idx[i]);
     std::vector<uint32_t> bits;
     if (d->bitmap) {
@@ -860,7 +961,7 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
       }
     }
     std::vector<int64_t> col_base(H);
-    for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + head_off[h];
+    for (int h = 0; h < H; ++h) col_base[h] = d->nnz_used + (d->intervals ? run_head_off[h] : head_off[h]);
     // Work items of the sparse heads and their LPT schedule over the grid.
     std::vector<uint32_t> items;
     std::vector<int64_t> cost;
@@ -936,6 +1037,17 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     if (d->bitmap) {
       e = cudaMemcpy(d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words), bits.data(),
                      sizeof(uint32_t) * bits.size(), cudaMemcpyHostToDevice);
+    } else if (d->intervals) {
+      if (!runs.empty())
+        e = cudaMemcpy(d->d_runs + d->nnz_used, runs.data(), runs.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(d->d_run_ptr + ly * H * (nq + 1), run_ptr.data(), sizeof(int32_t) * H * (nq + 1),
+                       cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(d->d_row_ptr + ly * H * (nq + 1), row_ptr, sizeof(int32_t) * H * (nq + 1),
+                       cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(d->d_col_base + ly * H, col_base.data(), sizeof(int64_t) * H, cudaMemcpyHostToDevice);
     } else {
       if (nnz > 0)
         e = cudaMemcpy(d->d_col + d->nnz_used, col16.data(), nnz * sizeof(uint16_t), cudaMemcpyHostToDevice);
@@ -957,7 +1069,8 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
                      cudaMemcpyHostToDevice);
     if (prev != d->device) cudaSetDevice(prev);
     if (e != cudaSuccess) return cuda_fail(e, "dictionary upload");
-    d->nnz_used += nnz;
+    d->nnz_used += d->bitmap ? nnz : units;
+    d->blocks_used += nnz;
     for (int h = 0; h < H; ++h) d->rep[ly * H + h] = (repetitive && repetitive[h]) ? 1 : 0;
     d->n_sparse[ly] = n_sparse;
     d->n_rep[ly] = n_rep;
@@ -1022,7 +1135,7 @@ calibatt_status calibatt_dict_info(const calibatt_dict* d, int64_t* device_bytes
   return guarded([&]() -> calibatt_status {
     if (!d) return fail(CALIBATT_ERR_INVALID_ARG, "dictionary is NULL");
     if (device_bytes) *device_bytes = d->device_bytes;
-    if (nnz_total) *nnz_total = d->nnz_used;
+    if (nnz_total) *nnz_total = d->blocks_used;
     if (num_ctas) *num_ctas = d->G;
     return CALIBATT_OK;
   });
@@ -1067,7 +1180,7 @@ constexpr uint32_t kDictFileVersion = 1;
 struct DictFileHeader {
   char magic[8];
   uint32_t version;
-  uint32_t format;  // 0 index lists, 1 bitmap
+  uint32_t format;  // 0 index lists, 1 bitmap, 2 intervals
   int32_t T, L, H, nq, nk, block;
   int32_t has_geom, frames, rows, cols, n_anchors;
   int32_t anchors[calibatt::kMaxAnchors];
@@ -1138,7 +1251,7 @@ calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
     std::memset(&hd, 0, sizeof(hd));
     std::memcpy(hd.magic, kDictMagic, 8);
     hd.version = kDictFileVersion;
-    hd.format = d->bitmap ? 1u : 0u;
+    hd.format = d->bitmap ? 1u : (d->intervals ? 2u : 0u);
     hd.T = d->T;
     hd.L = d->L;
     hd.H = H;
@@ -1168,10 +1281,27 @@ calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
     std::vector<int64_t> cb;
     std::vector<uint16_t> col;
     std::vector<uint32_t> bits;
+    std::vector<int32_t> run_ptr;
     for (int64_t ly = 0; ly < layers && w.ok && e == cudaSuccess; ++ly) {
       if (!d->layer_set[ly]) continue;
       DictFileRecord rec{static_cast<int32_t>(ly / d->L), static_cast<int32_t>(ly % d->L), 0};
-      if (d->bitmap) {
+      if (d->intervals) {
+        // the record's unit count is its number of runs
+        rp.resize(static_cast<size_t>(H) * (nq + 1));
+        run_ptr.resize(rp.size());
+        cb.resize(H);
+        e = cudaMemcpy(rp.data(), d->d_row_ptr + ly * H * (nq + 1), sizeof(int32_t) * rp.size(),
+                       cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+          e = cudaMemcpy(run_ptr.data(), d->d_run_ptr + ly * H * (nq + 1), sizeof(int32_t) * run_ptr.size(),
+                         cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+          e = cudaMemcpy(cb.data(), d->d_col_base + ly * H, sizeof(int64_t) * H, cudaMemcpyDeviceToHost);
+        for (int h = 0; h < H; ++h) rec.nnz += run_ptr[static_cast<size_t>(h) * (nq + 1) + nq];
+        bits.resize(rec.nnz);
+        if (e == cudaSuccess && rec.nnz > 0)
+          e = cudaMemcpy(bits.data(), d->d_runs + cb[0], sizeof(uint32_t) * rec.nnz, cudaMemcpyDeviceToHost);
+      } else if (d->bitmap) {
         bits.resize(static_cast<size_t>(H) * nq * d->words);
         e = cudaMemcpy(bits.data(), d->d_bitmap + ly * H * nq * static_cast<int64_t>(d->words),
                        sizeof(uint32_t) * bits.size(), cudaMemcpyDeviceToHost);
@@ -1192,7 +1322,11 @@ calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
       if (e != cudaSuccess) break;
       w.put(&rec, sizeof(rec));
       w.put(d->rep.data() + ly * H, H);
-      if (d->bitmap) {
+      if (d->intervals) {
+        w.put(rp.data(), sizeof(int32_t) * rp.size());
+        w.put(run_ptr.data(), sizeof(int32_t) * run_ptr.size());
+        w.put(bits.data(), sizeof(uint32_t) * bits.size());
+      } else if (d->bitmap) {
         w.put(bits.data(), sizeof(uint32_t) * bits.size());
       } else {
         w.put(rp.data(), sizeof(int32_t) * rp.size());
@@ -1244,7 +1378,39 @@ calibatt_status load_records(DictReader& r, const DictFileHeader& hd, calibatt_d
       return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) has %lld blocks", path, rec.t, rec.l, (long long)rec.nnz);
     nnz_seen += rec.nnz;
     if (!r.get(rep.data(), H)) return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
-    if (hd.format == 1) {
+    if (hd.format == 2) {
+      // rec.nnz runs: row pointers (blocks), run pointers, packed runs
+      std::vector<int32_t> run_ptr(rp.size());
+      bits.resize(rec.nnz);
+      if (!r.get(rp.data(), sizeof(int32_t) * rp.size()) ||
+          !r.get(run_ptr.data(), sizeof(int32_t) * run_ptr.size()) ||
+          !r.get(bits.data(), sizeof(uint32_t) * bits.size()))
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
+      // expand into per-head CSR; each row's runs must add up to its block count
+      col32.clear();
+      int64_t run_at = 0;
+      for (int h = 0; h < H; ++h) {
+        const int32_t* hp = rp.data() + static_cast<size_t>(h) * (nq + 1);
+        const int32_t* rr = run_ptr.data() + static_cast<size_t>(h) * (nq + 1);
+        if (rr[0] != 0) return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d run_ptr[0] != 0", path, rec.t, rec.l, h);
+        const size_t head_start = col32.size();
+        for (int q = 0; q < nq; ++q) {
+          if (rr[q + 1] < rr[q] || run_at + (rr[q + 1] - rr[q]) > rec.nnz || hp[q] != static_cast<int32_t>(col32.size() - head_start))
+            return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d runs do not match its rows", path, rec.t, rec.l, h);
+          for (int32_t x = rr[q]; x < rr[q + 1]; ++x) {
+            const uint32_t run = bits[run_at++];
+            const int64_t start = run & 0xFFFFu, len = run >> 16;
+            if (len < 1 || start + len > hd.nk || static_cast<int64_t>(col32.size() - head_start) + len > static_cast<int64_t>(nq) * (q + 1))
+              return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) has an invalid run", path, rec.t, rec.l);
+            for (int64_t c = start; c < start + len; ++c) col32.push_back(static_cast<int32_t>(c));
+          }
+        }
+        if (hp[nq] != static_cast<int32_t>(col32.size() - head_start))
+          return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d runs do not match its rows", path, rec.t, rec.l, h);
+      }
+      if (run_at != rec.nnz)
+        return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) run count mismatch", path, rec.t, rec.l);
+    } else if (hd.format == 1) {
       bits.resize(static_cast<size_t>(H) * nq * words);
       if (!r.get(bits.data(), sizeof(uint32_t) * bits.size()))
         return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) is cut short", path, rec.t, rec.l);
@@ -1285,7 +1451,9 @@ calibatt_status load_records(DictReader& r, const DictFileHeader& hd, calibatt_d
           return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) head %d row_ptr decreases", path, rec.t, rec.l, h);
       total += hp[nq];
     }
-    if (total != rec.nnz || static_cast<int64_t>(col32.size()) != rec.nnz)
+    if (hd.format != 2 && (total != rec.nnz || static_cast<int64_t>(col32.size()) != rec.nnz))
+      return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) block count mismatch", path, rec.t, rec.l);
+    if (hd.format == 2 && total != static_cast<int64_t>(col32.size()))
       return fail(CALIBATT_ERR_INVALID_ARG, "%s: record (%d, %d) block count mismatch", path, rec.t, rec.l);
     calibatt_status st = calibatt_dict_set_layer(d, rec.t, rec.l, rp.data(), col32.empty() ? nullptr : col32.data(), rep.data());
     if (st != CALIBATT_OK) return st;
@@ -1310,17 +1478,19 @@ calibatt_status calibatt_dict_load(const char* path, int32_t num_ctas, calibatt_
     DictFileHeader hd;
     if (!r.get(&hd, sizeof(hd)) || std::memcmp(hd.magic, kDictMagic, 8) != 0)
       return fail(CALIBATT_ERR_INVALID_ARG, "%s is not a dictionary file", path);
-    if (hd.version != kDictFileVersion || hd.format > 1 || hd.reserved != 0)
+    if (hd.version != kDictFileVersion || hd.format > 2 || hd.reserved != 0)
       return fail(CALIBATT_ERR_INVALID_ARG, "%s: unsupported version %u / format %u", path, hd.version, hd.format);
     if (hd.T < 1 || hd.L < 1 || hd.H < 1 || hd.nq < 1 || hd.nk != hd.nq || hd.H > 65535 || hd.nq > 65535 ||
         (hd.block != 64 && hd.block != 128) || hd.records < 0 || hd.records > static_cast<int64_t>(hd.T) * hd.L ||
-        hd.nnz_total < 0 || (hd.format == 1 && hd.nq > calibatt::kMaxBitmapBlocks) || hd.n_anchors < 0 ||
+        hd.nnz_total < 0 || (hd.format >= 1 && hd.nq > calibatt::kMaxBitmapBlocks) || hd.n_anchors < 0 ||
         hd.n_anchors > calibatt::kMaxAnchors || (hd.has_geom != 0 && hd.has_geom != 1))
       return fail(CALIBATT_ERR_INVALID_ARG, "%s: header fields out of range", path);
     calibatt_dict* d = nullptr;
-    calibatt_status st = hd.format == 1
-        ? calibatt_dict_create_bitmap(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, num_ctas, &d)
-        : calibatt_dict_create(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d);
+    calibatt_status st =
+        hd.format == 1 ? calibatt_dict_create_bitmap(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, num_ctas, &d)
+        : hd.format == 2
+            ? calibatt_dict_create_intervals(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d)
+            : calibatt_dict_create(hd.T, hd.L, hd.H, hd.nq, hd.nk, hd.block, hd.nnz_total, num_ctas, &d);
     if (st != CALIBATT_OK) return st;
     if (hd.has_geom) st = calibatt_dict_set_anchor_geometry(d, hd.frames, hd.rows, hd.cols, hd.anchors, hd.n_anchors);
     if (st == CALIBATT_OK) {

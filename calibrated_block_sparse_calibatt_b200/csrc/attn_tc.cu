@@ -259,8 +259,15 @@ struct Cursor {
             const int32_t* rp = p.sched.row_ptr + static_cast<int64_t>(it.h) * (p.sched.nq + 1);
             const int s0 = rp[it.tile];
             it.n = rp[it.tile + 1] - s0;
-            it.cols = p.sched.col + p.sched.col_base[it.h] + s0;
-            it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
+            if (p.sched.runs == nullptr) {
+              it.cols = p.sched.col + p.sched.col_base[it.h] + s0;
+              it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
+            } else {
+              // interval row: the producers decode its runs, and only the
+              // softmax warps need the last block (interval_ends_ragged)
+              it.cols = nullptr;
+              it.ragged_last = false;
+            }
           }
         }
         idx += step;
@@ -272,6 +279,16 @@ struct Cursor {
     return false;
   }
 };
+
+// Whether the last block of an interval row (head h, query block r) is the
+// partial key block: its last run ends at nb.
+__device__ __forceinline__ bool interval_ends_ragged(const TcParams& p, int h, int r) {
+  const int64_t ro = static_cast<int64_t>(h) * (p.sched.nq + 1) + r;
+  const int32_t last = p.sched.run_ptr[ro + 1] - 1;
+  if (last < p.sched.run_ptr[ro]) return false;  // empty row
+  const uint32_t run = p.sched.runs[p.sched.col_base[h] + last];
+  return static_cast<int>((run & 0xFFFFu) + (run >> 16)) == p.nb;
+}
 
 __device__ __forceinline__ void map_coords(const TcParams& p, int n0, int h, int b, int& c1,
                                            int& c2, int& c3) {
@@ -390,6 +407,27 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
           word &= word - 1u;
         }
         offset += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      __syncwarp();
+      cols = list;
+    } else if (p.sched.runs != nullptr && !it.anchor) {
+      // Interval row -> this producer's list of kept key blocks: runs are
+      // read 32 at a time, one per lane, then the warp writes each run's
+      // blocks lane-parallel in order.
+      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
+      const int64_t ro = static_cast<int64_t>(it.h) * (p.sched.nq + 1) + it.tile;
+      const int r0 = p.sched.run_ptr[ro], n_runs = p.sched.run_ptr[ro + 1] - r0;
+      const uint32_t* runs = p.sched.runs + p.sched.col_base[it.h] + r0;
+      int pos = 0;
+      for (int x0 = 0; x0 < n_runs; x0 += 32) {
+        const uint32_t mine = x0 + lane < n_runs ? runs[x0 + lane] : 0u;
+        const int cnt = min(32, n_runs - x0);
+        for (int x = 0; x < cnt; ++x) {
+          const uint32_t run = __shfl_sync(0xFFFFFFFFu, mine, x);
+          const int start = static_cast<int>(run & 0xFFFFu), len = static_cast<int>(run >> 16);
+          for (int i = lane; i < len; i += 32) list[pos + i] = static_cast<uint16_t>(start + i);
+          pos += len;
+        }
       }
       __syncwarp();
       cols = list;
@@ -569,6 +607,8 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   uint32_t t_me = 0, t_other = 0;  // key blocks of this / the other stream so far (global)
   bool ok = true;
   while (cur.next(p, it)) {
+    if (p.sched.runs != nullptr && !it.anchor && ragged_cols != 0)
+      it.ragged_last = interval_ends_ragged(p, it.h, it.tile);
     const int n_s = (it.n + 1 - s) / 2;  // blocks of this stream in the item
     const uint32_t t_other0 = t_other;
     float m_own = -INFINITY, l = 0.f;    // this stream's row sum, relative to m_own

@@ -24,6 +24,13 @@ struct LayerSchedule {
   // kept, words 32-bit words per row, [H][nq][words]; row_ptr/col unused.
   const uint32_t* bitmap;
   int32_t words;
+  // Interval dictionaries instead of index lists: each row is a list of
+  // contiguous key-block runs, packed start | (length << 16), ascending and
+  // disjoint.  Head h's runs of query block r are
+  // runs[col_base[h] + run_ptr[h][r] .. col_base[h] + run_ptr[h][r+1]);
+  // row_ptr still counts blocks (the row's block count is the difference).
+  const int32_t* run_ptr;  // [H][nq + 1]
+  const uint32_t* runs;
   // Nonzero when the lists and schedule come from the caller's device memory
   // (direct-CSR call): the kernels then do nothing if the status word holds a
   // skip-list or schedule violation (codes 23, 24) recorded by the check that
@@ -40,8 +47,9 @@ __device__ __forceinline__ bool csr_violation_recorded(const int32_t* status) {
   const int code = (*reinterpret_cast<const volatile int32_t*>(status) >> 8) & 0xFF;
   return code == kCodeListViolation || code == kCodeScheduleViolation;
 }
-// Longest skip list a bitmap dictionary may hold per row (the producers decode
-// each row into a shared-memory list of this many 16-bit indices).
+// Longest skip list a bitmap or interval dictionary may hold per row (the
+// producers decode each row into a shared-memory list of this many 16-bit
+// indices).
 constexpr int kMaxBitmapBlocks = 2048;
 
 // Frame geometry of the anchor path.  Token = (f * rows + row) * cols + col.

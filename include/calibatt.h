@@ -153,6 +153,27 @@ calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int
                                             int32_t nk, int32_t block, int32_t num_ctas,
                                             calibatt_dict** out);
 
+/* Like calibatt_dict_create, but each row's skip list is stored as its
+ * contiguous key-block intervals, the encoding the paper note describes (Key
+ * Designs 4: a read-only skip list of contiguous key-block intervals per
+ * query block): one 32-bit word per interval (start | length << 16), plus a
+ * second int32 [H][nq + 1] interval pointer per record.  run_capacity is the
+ * total number of intervals the dictionary can hold (count them with
+ * calibatt_csr_to_intervals).  The banded masks of calibration take a few
+ * intervals per row, so the records take a small fraction of the bytes of
+ * index lists.  The tensor-core producers expand each row's intervals into a
+ * list of kept blocks in shared memory; results equal those of the list
+ * format, bit for bit.  Interval dictionaries serve the tensor-core path only
+ * (bf16, block 128; otherwise the attention calls return
+ * CALIBATT_ERR_UNSUPPORTED) and hold nq <= 2048.  calibatt_dict_set_layer
+ * takes the same CSR input and encodes it; calibatt_dict_info reports
+ * retained blocks as for the other formats.
+ * Key Designs 4 (interval-encoded skip lists); Limitations & Future Work of
+ * the paper note (compacting the skip lists). */
+calibatt_status calibatt_dict_create_intervals(int32_t T, int32_t L, int32_t H, int32_t nq,
+                                               int32_t nk, int32_t block, int64_t run_capacity,
+                                               int32_t num_ctas, calibatt_dict** out);
+
 /* Fills the records of layer l at timestep t for all H heads (each layer
  * may be set once).  Host inputs:
  *   row_ptr int32[H][nq + 1]: each head's CSR row pointer, starting at 0;
@@ -207,13 +228,15 @@ calibatt_status calibatt_dict_destroy(calibatt_dict* dict);
  * persistent artefact, computed offline and loaded before generation, Key
  * Designs 4).  Writes to `path` (replaced atomically: written to a temporary
  * name, then renamed) a little-endian file:
- *   header: "CALIBDCT", version 1, format (0 index lists, 1 bitmap), T, L,
- *     H, nq, nk, block, the anchor geometry if set, records stored, total
- *     retained blocks (144 bytes);
- *   one entry per set record (t, l) in (t, l) order: t, l, retained blocks,
+ *   header: "CALIBDCT", version 1, format (0 index lists, 1 bitmap, 2
+ *     intervals), T, L, H, nq, nk, block, the anchor geometry if set,
+ *     records stored, total stored units (retained blocks; intervals for
+ *     format 2) (144 bytes);
+ *   one entry per set record (t, l) in (t, l) order: t, l, stored units,
  *     the H repetitive flags, then the H CSR row pointers and the 16-bit
- *     block indices (index lists) or the H*nq*ceil(nk/32) bitmap words, each
- *     part zero-padded to 8 bytes;
+ *     block indices (index lists), the H*nq*ceil(nk/32) bitmap words, or the
+ *     H CSR row pointers, the H interval pointers and the packed intervals,
+ *     each part zero-padded to 8 bytes;
  *   trailer: "CALIBEND" and a 64-bit FNV-1a hash of every 8-byte word before
  *     it.
  * Schedules are not stored.  Copies the records from the device

@@ -208,3 +208,24 @@ def test_dict_load_rejects_bad_files_before_touching_the_device(calibatt_lib, tm
         assert words in C.last_error(), (kw, C.last_error())
     bad.write_bytes(header()[:100])                                  # cut inside the header
     assert L.calibatt_dict_load(os.fsencode(bad), 4, ctypes.byref(h)) == C.ERR_INVALID_ARG
+
+
+def test_count_intervals_matches_the_library_encoding(calibatt_lib):
+    """The binding's interval count (capacity of an interval dictionary) equals
+    the library's own encoding of every head's CSR, on random masks with runs
+    that end at a row's end and start the next row."""
+    C = calibatt_lib
+    rng = np.random.default_rng(5)
+    nb, h = 37, 3
+    masks = [rng.random((nb, nb)) < p for p in (0.3, 0.7, 0.95)]
+    masks[1][4, :] = False                                  # an empty row
+    rp, ci, _ = C.masks_to_layer_csr(masks, h, nb)
+    total = 0
+    off = 0
+    for hh in range(h):
+        n = int(rp[hh, -1])
+        ptr, start, length = C.csr_to_intervals(nb, rp[hh], ci[off:off + n])
+        assert int(length.sum()) == n
+        total += len(start)
+        off += n
+    assert C.count_intervals(rp, ci) == total

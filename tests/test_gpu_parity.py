@@ -393,7 +393,8 @@ def _block_rows(blocks, seq_len):
 @pytest.mark.parametrize("name", ["480p", "720p"])
 def test_full_size_sparse_sampled(C, name):
     """Every head at full size, 8 sampled q-blocks each including the first and
-    the ragged last one, against the oracle (evaluated in spawned workers)."""
+    the ragged last one, against the oracle (evaluated in spawned workers); at
+    720p the interval dictionary's output equals the index lists' bitwise."""
     import _oracle_jobs as J
 
     wl = W.WORKLOADS[name]
@@ -401,6 +402,17 @@ def test_full_size_sparse_sampled(C, name):
     masks, _ = W.workload_masks(wl)
     masks = [masks[h] for h in range(wl.heads)]
     out, _ = _run_sparse(C, q, k, v, masks, wl.block)
+    if name == "720p":
+        # the interval dictionary (the pages' encoding) gives the same output bit for bit
+        rp, ci, rep = C.masks_to_layer_csr(masks, wl.heads, wl.num_blocks)
+        alt = torch.full_like(q, float("nan"))
+        with _dictionary(C, "intervals", 1, 1, wl.heads, wl.num_blocks, wl.block, rp, ci) as dct:
+            dct.set_layer(0, 0, rp, ci, rep)
+            C.calibatt_block_sparse_attn(q, k, v, alt, dct, 0, 0, wl.block)
+            _check_status(C)
+            assert dct.info()["device_bytes"] < 0.2 * (ci.size * 2)       # far below the 16-bit lists
+        assert torch.equal(alt, out)
+        del alt
     rng = np.random.default_rng(1)
     jobs, got = [], []
     for h in range(wl.heads):
@@ -596,7 +608,7 @@ def test_energy_select_union_tiny(C, std, tau):
 def test_energy_select_union_tensor_core(C, tau):
     """The same energy -> selection -> union chain on the tensor-core energies
     (bf16, 128-token blocks): 2 heads, N = 2000 (15 full blocks and one of 80
-    tokens), peaked logits (std 4), 3 seeded draws, rho = 1/3."""
+    tokens), peaked logits (std 4), 3 seeded draws, their union (rho = 0.25)."""
     draws = [W.make_qkv(s, 1, 2000, 2, 128, "bf16", 4.0, "cuda")[:2] for s in (40, 41, 42)]
     _select_and_union(C, draws, 128, tau)
 
@@ -624,12 +636,14 @@ def _select_and_union(C, draws, block, tau):
         decided.append(_margin_ok(e_ref, tau64))
     assert (cnt.cpu().numpy() == np.sum(gpu_masks, axis=0)).all(), "selection counts"
     union = torch.zeros_like(cnt, dtype=torch.uint8)
-    C.calibatt_aggregate_masks(cnt, len(draws), 1.0 / len(draws), union)
+    # rho = 0.25 is exact in float32 and keeps every block chosen at least
+    # once for 3 or 4 draws (a union); 1/3 would round up above 1/3
+    C.calibatt_aggregate_masks(cnt, len(draws), 0.25, union)
     _check_status(C)
     union = union.cpu().numpy().astype(bool)
     assert (union == np.logical_or.reduce(gpu_masks)).all(), "union of the GPU selections"
     all_ok = np.logical_and.reduce(decided)
-    ref_union = O.aggregate_masks(np.stack(ref_masks), len(draws), 1.0 / len(draws))
+    ref_union = O.aggregate_masks(np.stack(ref_masks), len(draws), 0.25)
     assert (union[all_ok] == ref_union[all_ok]).all(), \
         f"{exact} rows bit-exact, {checked} margin rows checked for validity ({boundary} at the tau boundary)"
     print(f"selection: {exact} rows bit-exact, {checked} margin rows valid, {boundary} at the tau boundary")
@@ -872,47 +886,66 @@ def test_spatial_similarity_720p_sampled_and_flags(C):
     assert ref_flags.any() and not ref_flags.all()
 
 
-# ------------------------------------------------------------ bitmap dictionaries
+# ------------------------------------------- bitmap and interval dictionaries
+
+FORMATS = ("lists", "bitmap", "intervals")
+
+
+def _dictionary(C, fmt, T, L, h, nb, block, rp, ci, extra_capacity=1):
+    """An empty dictionary of format `fmt` with room for `extra_capacity`
+    layers like (rp, ci): blocks for index lists, intervals for the interval
+    format, nothing for bitmaps."""
+    if fmt == "intervals":
+        return C.MaskDictionary(T, L, h, nb, nb, block, max(1, extra_capacity * C.count_intervals(rp, ci)),
+                                intervals=True)
+    return C.MaskDictionary(T, L, h, nb, nb, block, max(1, extra_capacity * ci.size), bitmap=fmt == "bitmap")
+
 
 @pytest.mark.parametrize("d,n,h", [(128, 1000, 3), (64, 4100, 2)])  # ragged; 33 blocks -> 2 words per row
-def test_bitmap_dictionary_matches_lists(C, d, n, h):
-    """A bitmap dictionary gives bitwise the results of the index-list one:
-    sparse call with LSE (an empty row included) and the fused dual path."""
+def test_compact_dictionaries_match_lists(C, d, n, h):
+    """Bitmap and interval dictionaries give bitwise the results of the
+    index-list one: sparse call with LSE (an empty row, a row keeping every
+    block, single-block runs and the ragged last key block included) and the
+    fused dual path."""
     q, k, v = W.make_qkv(61, 1, n, h, d, "bf16", 1.0, "cuda")
     nb = O.num_blocks(n, 128)
     masks = _random_masks(62, h, nb, 0.4, empty_row_head=1)
     masks[0][:, nb - 1] = True                                  # ragged last key block kept by every row
+    masks[0][2, :] = True                                       # one run over the whole row
+    masks[h - 1][3, :] = np.arange(nb) % 2 == 0                 # runs of one block each
     rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
     outs, lses = [], []
-    for bitmap in (False, True):
+    for fmt in FORMATS:
         out = torch.full_like(q, float("nan"))
         lse = torch.full((1, h, n), float("nan"), device="cuda")
-        with C.MaskDictionary(1, 1, h, nb, nb, 128, ci.size, bitmap=bitmap) as dct:
+        with _dictionary(C, fmt, 1, 1, h, nb, 128, rp, ci) as dct:
             dct.set_layer(0, 0, rp, ci, rep)
             C.calibatt_block_sparse_attn(q, k, v, out, dct, 0, 0, 128, lse=lse)
             _check_status(C)
             assert dct.layer_info(0, 0)["retained_tiles"] == sum(int(m.sum()) for m in masks)
+            assert dct.info()["nnz"] == ci.size
         outs.append(out)
         lses.append(lse)
-    assert torch.equal(outs[0], outs[1])
-    assert torch.equal(lses[0], lses[1])
+    for i in (1, 2):
+        assert torch.equal(outs[0], outs[i]), FORMATS[i]
+        assert torch.equal(lses[0], lses[i]), FORMATS[i]
     ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, 128, seq_len=n)
-    _assert_close(_np(outs[1]), ref, "bf16")
-    # fused dual path over a bitmap dictionary
+    _assert_close(_np(outs[2]), ref, "bf16")
+    # fused dual path over each format
     frames, rows, cols = (2, 5, n // 10) if n % 10 == 0 else (1, 41, 100)
     assert frames * rows * cols == n
     dmasks = [None if i == h - 1 else masks[i] for i in range(h)]
     rp2, ci2, rep2 = C.masks_to_layer_csr(dmasks, h, nb)
     res = []
-    for bitmap in (False, True):
+    for fmt in FORMATS:
         out = torch.full_like(q, float("nan"))
-        with C.MaskDictionary(1, 1, h, nb, nb, 128, max(1, ci2.size), bitmap=bitmap) as dct:
+        with _dictionary(C, fmt, 1, 1, h, nb, 128, rp2, ci2) as dct:
             dct.set_anchor_geometry(frames, rows, cols, (1, 3) if rows == 5 else (10, 30))
             dct.set_layer(0, 0, rp2, ci2, rep2)
             C.calibatt_dual_path_attn(q, k, v, out, dct, 0, 0, frames, rows, cols, (1, 3) if rows == 5 else (10, 30))
             _check_status(C)
         res.append(out)
-    assert torch.equal(res[0], res[1])
+    assert torch.equal(res[0], res[1]) and torch.equal(res[0], res[2])
 
 
 def _compact_reference(q, k, v, n, r, cols, block=128):
@@ -966,10 +999,10 @@ def test_longest_sequence_of_index_lists(C):
 
 
 def test_longest_bitmap_row(C):
-    """The largest bitmap dictionary row: 2,048 key blocks, N = 262,066 (ragged
-    last block of 50 tokens), one query block keeping every key block and others
-    keeping few; bitwise equal to the index-list dictionary and against the
-    oracle."""
+    """The largest bitmap and interval dictionary row: 2,048 key blocks, N =
+    262,066 (ragged last block of 50 tokens), one query block keeping every key
+    block and others keeping few; bitwise equal to the index-list dictionary
+    and against the oracle."""
     nb, block = 2048, 128
     n = (nb - 1) * block + 50
     q, k, v = W.make_qkv(42, 1, n, 1, 128, "bf16", 1.0, "cuda")
@@ -980,16 +1013,17 @@ def test_longest_bitmap_row(C):
     masks[5, :] = False                       # an empty row
     rp, ci, rep = C.masks_to_layer_csr([masks], 1, nb)
     outs, lses = [], []
-    for bitmap in (False, True):
+    for fmt in FORMATS:
         out = torch.full_like(q, float("nan"))
         lse = torch.full((1, 1, n), float("nan"), device="cuda")
-        with C.MaskDictionary(1, 1, 1, nb, nb, block, 0 if bitmap else ci.size, bitmap=bitmap) as dct:
+        with _dictionary(C, fmt, 1, 1, 1, nb, block, rp, ci) as dct:
             dct.set_layer(0, 0, rp, ci, rep)
             C.calibatt_block_sparse_attn(q, k, v, out, dct, 0, 0, block, lse=lse)
             _check_status(C)
         outs.append(out)
         lses.append(lse)
-    assert torch.equal(outs[0], outs[1]) and torch.equal(lses[0], lses[1])
+    for i in (1, 2):
+        assert torch.equal(outs[0], outs[i]) and torch.equal(lses[0], lses[i]), FORMATS[i]
     lists = [np.nonzero(masks[r])[0] for r in range(nb)]
     _check_rows(C, outs[1], lses[1], q, k, v, n, lists, [0, 777, 1500, nb - 1])
     assert (outs[1][0, 5 * 128:6 * 128].float() == 0).all() and torch.isneginf(lses[1][0, 0, 5 * 128:6 * 128]).all()
@@ -1017,8 +1051,33 @@ def test_bitmap_dictionary_size_and_rules(C):
         C.MaskDictionary(1, 1, 1, 4096, 4096, 128, bitmap=True)    # more than 2048 blocks per row
 
 
-@pytest.mark.parametrize("bitmap", [False, True])
-def test_dictionary_save_load_round_trip(C, tmp_path, bitmap):
+def test_interval_dictionary_size_and_rules(C):
+    """Device bytes of the interval format at the 720p layer against index
+    lists, its capacity counted in intervals, and its limits."""
+    wl = W.WORKLOADS["720p"]
+    nb = wl.num_blocks
+    masks, _ = W.workload_masks(wl, heads=range(4))
+    rp, ci, rep = C.masks_to_layer_csr([masks[i] for i in range(4)], 4, nb)
+    runs = C.count_intervals(rp, ci)
+    assert runs < ci.size / 20                                       # banded masks: few runs per row
+    with C.MaskDictionary(2, 2, 4, nb, nb, 128, 4 * ci.size) as dl, \
+            C.MaskDictionary(2, 2, 4, nb, nb, 128, 4 * runs, intervals=True) as di:
+        assert di.info()["device_bytes"] < dl.info()["device_bytes"] / 5
+        di.set_layer(1, 1, rp, ci, rep)
+        assert di.info()["nnz"] == ci.size
+        q = torch.zeros((1, wl.seq_len, 4, 128), dtype=torch.float32, device="cuda")
+        with pytest.raises(C.CalibattError):                         # the CUDA-core path reads lists only
+            C.calibatt_block_sparse_attn(q, q, q, q, di, 1, 1, 128)
+    with C.MaskDictionary(1, 1, 4, nb, nb, 128, runs - 1, intervals=True) as small:
+        with pytest.raises(C.CalibattError) as e:                    # capacity is counted in intervals
+            small.set_layer(0, 0, rp, ci, rep)
+        assert "intervals" in str(e.value)
+    with pytest.raises(C.CalibattError):
+        C.MaskDictionary(1, 1, 1, 4096, 4096, 128, 10, intervals=True)   # more than 2048 blocks per row
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_dictionary_save_load_round_trip(C, tmp_path, fmt):
     """calibatt_dict_save / calibatt_dict_load: a dictionary with the anchor
     geometry, three of its four records set (repetitive heads included), written
     and read back with another persistent grid; every record's counts match and
@@ -1030,7 +1089,8 @@ def test_dictionary_save_load_round_trip(C, tmp_path, bitmap):
     q, k, v = W.make_qkv(51, 1, n, h, d, "bf16", 1.0, "cuda")
     path = tmp_path / "masks.dict"
     records = {(0, 0): (0, 3), (0, 1): (), (1, 1): (1,)}           # (t, l) -> repetitive heads
-    with C.MaskDictionary(2, 2, h, nb, nb, block, 4 * h * nb * nb, bitmap=bitmap) as dct:
+    with C.MaskDictionary(2, 2, h, nb, nb, block, 4 * h * nb * nb, bitmap=fmt == "bitmap",
+                          intervals=fmt == "intervals") as dct:
         dct.set_anchor_geometry(frames, rows, cols, anchors)
         for i, ((t, l), rep) in enumerate(records.items()):
             masks = _random_masks(60 + i, h, nb, 0.4)
