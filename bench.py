@@ -895,6 +895,25 @@ def main():
                          "frac": exp2_per_call / (energy_ms * 1e-3) / ex2_peak,
                          "peak_basis": f"{EX2_PER_CLK_PER_SM} exp2/clk/SM x {sms} SMs x 1965 MHz (max SM clock); "
                                        "one exp2 pair in four runs on the FMA pipe and is counted all the same"}}
+        # offline calibration: spatial-repetition scores of every (frame, row) of the 720p layer
+        wd_ = W.WORKLOADS["720p_dual"]
+        sim_out = torch.empty((1, wl.heads, wd_.frames, wd_.rows), device="cuda")
+        sim_ws = torch.empty(C.calibatt_spatial_similarity_workspace_size(q) // 4, device="cuda")
+        sim_ms = max_over_ranks(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_spatial_similarity(q, k, sim_out, sim_ws, wd_.frames, wd_.rows, wd_.cols,
+                                                         wd_.anchors, stream=stream),
+            3, 1, stream)), dist, "cuda")
+        del sim_out, sim_ws
+        # the LSE pass exponentiates every score once, the pass of sums twice
+        # (each query's and its anchor-row partner's)
+        sim_exp2 = 3 * wl.seq_len ** 2 * wl.heads
+        extras["spatial_similarity_720p"] = {
+            "ms_per_call": sim_ms, "heads": wl.heads, "frames_x_rows": wd_.frames * wd_.rows,
+            "exp2_per_call": sim_exp2,
+            "tflops_three_qk_passes": 3 * 2.0 * wl.seq_len ** 2 * wl.head_dim * wl.heads / (sim_ms * 1e-3) / 1e12,
+            "roofline": {"bound": "mufu", "achieved": sim_exp2 / (sim_ms * 1e-3) / 1e9, "peak": ex2_peak / 1e9,
+                         "unit": "G exp2/s", "frac": sim_exp2 / (sim_ms * 1e-3) / ex2_peak,
+                         "peak_basis": f"{EX2_PER_CLK_PER_SM} exp2/clk/SM x {sms} SMs x 1965 MHz (max SM clock)"}}
         if C.device_status() != 0:
             raise RuntimeError("device wait timed out during the extra legs")
         if world == 1:

@@ -67,6 +67,7 @@ SIGNATURES = {
     "calibatt_spatial_similarity": (_i32, [_vp, _vp, _P(Shape), _i32, _i32, _i32, _vp, _i32, _f32, _vp, _vp,
                                            ctypes.c_size_t, _vp]),
     "calibatt_repetition_flags": (_i32, [_vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
+    "calibatt_spatial_similarity_workspace_size": (_i32, [_P(Shape), _P(ctypes.c_size_t)]),
     "calibatt_dict_info": (_i32, [_vp, _P(_i64), _P(_i64), _P(_i32)]),
     "calibatt_dict_layer_info": (_i32, [_vp, _i32, _i32, _P(_i32), _P(_i32), _P(_i64)]),
     "calibatt_dict_destroy": (_i32, [_vp]),
@@ -392,10 +393,18 @@ def calibatt_dual_path_attn(q, k, v, o, d: MaskDictionary, t, l, frames, rows, c
                                       _stream(stream)))
 
 
+def calibatt_spatial_similarity_workspace_size(q) -> int:
+    shape = shape_of(q)
+    n = ctypes.c_size_t(0)
+    check(LIB.calibatt_spatial_similarity_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
 def calibatt_spatial_similarity(q, k, sim, workspace, frames, rows, cols, anchor_rows, softmax_scale=0.0,
                                 stream=None):
     """Spatial-repetition score of every (batch, head, frame, row) into sim
-    (float32 [batch, heads, frames, rows]); workspace as calibatt_block_energy's."""
+    (float32 [batch, heads, frames, rows]); workspace of at least
+    calibatt_spatial_similarity_workspace_size(q) bytes."""
     shape = shape_of(q)
     a = _i32_array(anchor_rows)
     nbytes = workspace.numel() * workspace.element_size()

@@ -147,6 +147,24 @@ int32_t heads_per_group(int32_t nq) {
   return static_cast<int32_t>(std::max<int64_t>(1, (static_cast<int64_t>(CALIBATT_L2_GROUP_MB) << 20) / per_head));
 }
 
+// Schedule group of the work item (k-th sparse head of the layer, query block
+// r).  Heads go in L2 groups of heads_per_group; with waves on, each head
+// group is further cut into waves of `grid` consecutive query blocks (in head,
+// then query-block order), so that every CTA takes about one item per wave and
+// the grid sweeps each head in query-block order: the keys and values in use
+// at a time are the band around the current wave (plus the first frame's and
+// the scattered blocks) rather than the whole head's.
+#ifndef CALIBATT_WAVES
+#define CALIBATT_WAVES 1
+#endif
+int32_t schedule_group(int32_t k, int32_t r, int32_t nq, int32_t hpg, int32_t grid) {
+  if (!CALIBATT_WAVES) return k / hpg;
+  const int64_t per_group = static_cast<int64_t>(hpg) * nq;
+  const int64_t waves = (per_group + grid - 1) / grid;
+  const int64_t pos = static_cast<int64_t>(k % hpg) * nq + r;
+  return static_cast<int32_t>((k / hpg) * waves + pos / grid);
+}
+
 // ------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -724,7 +742,7 @@ calibatt_status calibatt_csr_schedule(int32_t heads, int32_t nq, const int32_t* 
       for (int r = 0; r < nq; ++r) {
         all.push_back((static_cast<uint32_t>(head_ids[i]) << 16) | static_cast<uint32_t>(r));
         cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
-        group.push_back(i / hpg);
+        group.push_back(schedule_group(i, r, nq, hpg, grid));
       }
     }
     std::vector<int32_t> order(all.size());
@@ -974,13 +992,12 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
         ++n_rep;
         continue;
       }
-      const int32_t g = n_sparse / hpg;
-      ++n_sparse;
+      const int32_t k = n_sparse++;
       const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
       for (int r = 0; r < nq; ++r) {
         items.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
         cost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);  // +2: Q load and epilogue
-        group.push_back(g);
+        group.push_back(schedule_group(k, r, nq, hpg, d->G));
         retained += rp[r + 1] - rp[r];
       }
     }
@@ -1014,12 +1031,12 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
             fgroup.push_back(0);
           }
         } else {
-          const int32_t g = 1 + sparse_rank++ / hpg;
+          const int32_t k = sparse_rank++;
           const int32_t* rp = row_ptr + static_cast<int64_t>(h) * (nq + 1);
           for (int r = 0; r < nq; ++r) {
             fitems.push_back((static_cast<uint32_t>(h) << 16) | static_cast<uint32_t>(r));
             fcost.push_back(static_cast<int64_t>(rp[r + 1] - rp[r]) + 2);
-            fgroup.push_back(g);
+            fgroup.push_back(1 + schedule_group(k, r, nq, hpg, d->G));
           }
         }
       }
@@ -1771,6 +1788,18 @@ calibatt_status calibatt_block_energy(const void* q, const void* k, const caliba
   });
 }
 
+calibatt_status calibatt_spatial_similarity_workspace_size(const calibatt_shape* shape, size_t* bytes) {
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if (!bytes) return fail(CALIBATT_ERR_INVALID_ARG, "bytes is NULL");
+    // per query: its log-sum-exp, and on the tensor-core path (bf16) its three sums
+    const size_t per_query = shape->dtype == CALIBATT_DTYPE_BF16 ? 4 : 1;
+    *bytes = sizeof(float) * per_query * static_cast<size_t>(shape->batch) * shape->heads * shape->seq_len;
+    return CALIBATT_OK;
+  });
+}
+
 calibatt_status calibatt_spatial_similarity(const void* q, const void* k, const calibatt_shape* shape, int32_t frames,
                                             int32_t rows, int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
                                             float softmax_scale, float* similarity, void* workspace,
@@ -1795,10 +1824,54 @@ calibatt_status calibatt_spatial_similarity(const void* q, const void* k, const 
         return fail(CALIBATT_ERR_INVALID_ARG, "anchor rows must be strictly ascending");
     }
     size_t need = 0;
-    calibatt_block_energy_workspace_size(shape, &need);
+    calibatt_spatial_similarity_workspace_size(shape, &need);
     if (workspace_bytes < need)
-      return fail(CALIBATT_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", workspace_bytes, need);
+      return fail(CALIBATT_ERR_INVALID_ARG,
+                  "workspace of %zu bytes < %zu needed (calibatt_spatial_similarity_workspace_size)",
+                  workspace_bytes, need);
     const float sl2 = scale_log2_of(softmax_scale, shape->head_dim);
+    if (shape->dtype == CALIBATT_DTYPE_BF16) {
+      if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16)
+        return fail(CALIBATT_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
+      // Tensor-core path: the LSE pass, the pass of per-query sums (two score
+      // tiles per key block: the queries and their anchor-row partners), and
+      // the rows' fixed-order reduction.
+      TcParams t;
+      std::memset(&t, 0, sizeof(t));
+      if ((st = encode_qkv_map(&t.tm_q, q, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+      if ((st = encode_qkv_map(&t.tm_k, k, *shape, &t.pos_n, &t.pos_h, &t.pos_b)) != CALIBATT_OK) return st;
+      t.tm_v = t.tm_k;  // no V in these modes
+      const int64_t plane = static_cast<int64_t>(shape->batch) * shape->heads * shape->seq_len;
+      t.q = static_cast<const uint16_t*>(q);
+      t.lse = static_cast<float*>(workspace);
+      t.energy = static_cast<float*>(workspace) + plane;  // three planes of per-query sums
+      t.sb = shape->stride_b;
+      t.sn = shape->stride_n;
+      t.sh = shape->stride_h;
+      t.batch = shape->batch;
+      t.seq_len = shape->seq_len;
+      t.heads = shape->heads;
+      t.nb = ceil_div(shape->seq_len, 128);
+      t.scale_log2 = sl2;
+      t.anc.frames = frames;
+      t.anc.rows = rows;
+      t.anc.cols = cols;
+      t.anc.n_anchors = n_anchors;
+      anchor_groups(rows, anchor_rows, n_anchors, t.anc);
+      t.status = status_word_ptr();
+      t.timeout_ns = g_timeout_ns.load();
+      const int sms = device_sm_count();
+      if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+      const int grid = static_cast<int>(std::min<int64_t>(sms, static_cast<int64_t>(shape->heads) * t.nb));
+      cudaStream_t cs = static_cast<cudaStream_t>(stream);
+      cudaError_t e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeLse, grid, cs);
+      if (e == cudaSuccess) e = calibatt::launch_tc_attn(t, shape->head_dim, calibatt::kModeSimilarity, grid, cs);
+      if (e == cudaSuccess)
+        e = calibatt::launch_similarity_from_sums(t.energy, plane, shape->batch * shape->heads, shape->seq_len,
+                                                  frames, rows, cols, similarity, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "tensor-core spatial similarity launch");
+      return CALIBATT_OK;
+    }
     calibatt::EnergyParams e;
     std::memset(&e, 0, sizeof(e));
     e.q = q;

@@ -174,6 +174,25 @@ struct Layout {
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
 };
 
+// Modes without V and P.V: the offline calibration passes.
+__host__ __device__ constexpr bool calibration_mode(int mode) {
+  return mode == kModeLse || mode == kModeEnergy || mode == kModeSimilarity;
+}
+
+// Token whose query partners token `i` in the spatial-similarity mode: the
+// same frame and column in the nearest anchor row (Key Designs 3); the anchor
+// geometry's groups hold each anchor's rows.
+__device__ __forceinline__ int64_t partner_token(const AnchorGeom& g, int64_t i) {
+  const int64_t per_frame = static_cast<int64_t>(g.rows) * g.cols;
+  const int64_t f = i / per_frame;
+  const int rem = static_cast<int>(i - f * per_frame);
+  const int rho = rem / g.cols, w = rem - rho * g.cols;
+  int a = 0;
+  for (int x = 1; x < g.n_anchors; ++x)
+    if (rho >= g.group_lo[x]) a = x;
+  return (f * g.rows + g.anchor_row[a]) * g.cols + w;
+}
+
 struct Item {
   int b, h, tile;            // batch, head, query block (sparse) or anchor tile
   int n;                     // key blocks to visit
@@ -198,7 +217,7 @@ struct Cursor {
       begin = blockIdx.x;
       end = p.anc.n_heads * p.anc.tiles_per_head;
       step = gridDim.x;
-    } else if (MODE == kModeLse || MODE == kModeEnergy) {
+    } else if (calibration_mode(MODE)) {
       begin = blockIdx.x;
       end = p.heads * p.nb;
       step = gridDim.x;
@@ -214,7 +233,7 @@ struct Cursor {
       if (idx < end) {
         it.b = b;
         uint32_t w = 0;
-        if (MODE == kModeLse || MODE == kModeEnergy) {
+        if (calibration_mode(MODE)) {
           // every key block of query block (idx mod nb) of head (idx / nb)
           it.anchor = false;
           it.h = idx / p.nb;
@@ -327,7 +346,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
   constexpr int kEmpty = V ? L::bVEmpty : L::bKEmpty;
   constexpr int kRing = V ? L::kV : L::kK;
   const CUtensorMap* map = V ? &p.tm_v : &p.tm_k;
-  if (V && (MODE == kModeLse || MODE == kModeEnergy)) return;  // no P.V in the calibration modes
+  if (V && calibration_mode(MODE)) return;  // no P.V in the calibration modes
   Cursor<MODE> cur;
   cur.init(p);
   Item it;
@@ -377,6 +396,26 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::bQFull));
       } else {
+        if (MODE == kModeSimilarity) {
+          // The partner queries (nearest anchor row, same frame and column) of
+          // the tile's 128 queries, gathered into the swizzled layout in the
+          // V ring's space (no V in this mode), before the tile's own Q is
+          // requested: q_full then completes only after both are in place.
+          constexpr int kUnits = HD / 8;
+          const uint16_t* qb = p.q + static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
+          for (int idx = lane; idx < 128 * kUnits; idx += 32) {
+            const int r = idx / kUnits, u = idx % kUnits;
+            const int64_t tok = static_cast<int64_t>(it.tile) * 128 + r;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (tok < p.seq_len) val = __ldg(reinterpret_cast<const uint4*>(qb + partner_token(p.anc, tok) * p.sn + u * 8));
+            const uint32_t dst = base + L::kV + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val.x), "r"(val.y), "r"(val.z),
+                         "r"(val.w)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
         if (lane == 0) {
           mbar_arrive_expect_tx(bar(L::bQFull), L::kTile);
           tma_tile<HD>(base + L::kQ, &p.tm_q, bar(L::bQFull), p, it.tile * 128, it.h, it.b);
@@ -496,13 +535,22 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
       CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 3, g);
       if (lane == 0) {
         const uint32_t k_base = base + L::kK + ks * L::kTile;
-        const uint32_t d = tmem + kColS + s * 128;
+        // similarity mode: stream s has its two score tiles at 256 s and 256 s + 128
+        const uint32_t d = tmem + kColS + s * (MODE == kModeSimilarity ? 256 : 128);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           // K-major operands: 16 columns = 32 bytes per step inside a 64-column chunk.
           const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
           mma_ss(d, sw128_desc(base + L::kQ + off, 16, 1024), sw128_desc(k_base + off, 16, 1024), kIdescS,
                  k > 0 ? 1u : 0u);
+        }
+        if (MODE == kModeSimilarity) {
+#pragma unroll
+          for (int k = 0; k < HD / 16; ++k) {
+            const uint32_t off = (k >> 2) * kChunkBytes + (k & 3) * 32;
+            mma_ss(d + 128, sw128_desc(base + L::kV + off, 16, 1024), sw128_desc(k_base + off, 16, 1024), kIdescS,
+                   k > 0 ? 1u : 0u);
+          }
         }
         mma_commit(bar(L::bKEmpty + ks));
         mma_commit(bar(L::bSFull + s));
@@ -526,7 +574,7 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, HD, 1);
-  if (MODE == kModeLse || MODE == kModeEnergy) {
+  if (calibration_mode(MODE)) {
     // No P.V: only this thread's share of the drain barrier.
     if (lane == 0) mma_commit(bar(L::bDrain));
     __syncwarp();
@@ -944,6 +992,104 @@ __device__ void softmax_energy_role(const TcParams& p, uint32_t base, uint8_t* g
   }
 }
 
+// Spatial-repetition sums (Key Designs 3) on the tensor-core pipeline.  Per
+// key block, thread t of stream s reads row t of its two score tiles: its
+// query i = tile * 128 + t and the partner query i' (same frame and column,
+// nearest anchor row).  With P_ij = 2^(s_ij log2e scale - lse2_i) from the
+// LSE pass, it accumulates sum_j P_ij P_i'j, sum_j P_ij^2 and sum_j P_i'j^2
+// (four partial sums each, combined in a fixed order); the two streams'
+// sums are added in the epilogue and written per query, three planes of
+// [batch * heads * seq_len] floats.  The rows' cosine similarities come from
+// those per-query sums in a separate fixed-order reduction.
+template <int HD>
+__device__ void softmax_similarity_role(const TcParams& p, uint32_t base, uint8_t* gbase, uint32_t tmem,
+                                        const Waiter& W, int warp, int lane) {
+  using L = Layout<HD>;
+  constexpr int MODE = kModeSimilarity;
+  auto bar = [&](int i) { return base + L::kBar + 8u * i; };
+  const int quarter = warp & 3, s = warp >> 2;
+  const int row = quarter * 32 + lane;
+  const int pair_bar = 1 + quarter;
+  float* xchg = reinterpret_cast<float*>(gbase + L::kXchg);  // [2 item parity][3 sums][128 rows]
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tA = tmem + lane_off + kColS + s * 256;  // own queries
+  const uint32_t tB = tA + 128;                           // partner queries
+  const int ragged_cols = p.seq_len % 128;
+  const float sl2 = p.scale_log2;
+  const int64_t plane = static_cast<int64_t>(p.batch) * p.heads * p.seq_len;
+  Cursor<MODE> cur;
+  cur.init(p);
+  Item it;
+  uint32_t item = 0, t_me = 0;
+  bool ok = true;
+  while (cur.next(p, it)) {
+    const int n_s = (it.n + 1 - s) / 2;
+    const int64_t token = static_cast<int64_t>(it.tile) * 128 + row;
+    const bool valid = token < p.seq_len;
+    const int64_t bh = static_cast<int64_t>(it.b) * p.heads + it.h;
+    float la = 0.f, lb = 0.f;  // log2-sum-exp of the own and the partner query
+    if (valid) {
+      la = p.lse[bh * p.seq_len + token];
+      lb = p.lse[bh * p.seq_len + partner_token(p.anc, token)];
+    }
+    float ab[4] = {0.f, 0.f, 0.f, 0.f}, aa[4] = {0.f, 0.f, 0.f, 0.f}, bb[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < n_s; ++k) {
+      const int j = 2 * k + s;
+      ok = ok && W.wait(bar(L::bSFull + s), t_me & 1, 10);
+      if (ok) tc_fence_after();
+      const bool ragged = j == it.n - 1 && it.ragged_last;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t ra[64], rb[64];
+        tmem_ld_x64(tA + hh * 64, ra);
+        tmem_ld_x64(tB + hh * 64, rb);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float x0, x1, y0, y1;
+          fma2(x0, x1, __uint_as_float(ra[2 * c]), __uint_as_float(ra[2 * c + 1]), sl2, sl2, -la, -la);
+          fma2(y0, y1, __uint_as_float(rb[2 * c]), __uint_as_float(rb[2 * c + 1]), sl2, sl2, -lb, -lb);
+          float p0, p1, q0, q1;
+          if (kEnergyPolyEvery > 0 && (c % kEnergyPolyEvery) == kEnergyPolyEvery - 1) {
+            exp2_fma2_quintic(p0, p1, x0, x1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          q0 = fast_exp2(y0);
+          q1 = fast_exp2(y1);
+          if (ragged) {
+            const int col = hh * 64 + 2 * c;
+            if (col >= ragged_cols) p0 = q0 = 0.f;
+            if (col + 1 >= ragged_cols) p1 = q1 = 0.f;
+          }
+          const int acc = c & 3;
+          ab[acc] = fmaf(p0, q0, fmaf(p1, q1, ab[acc]));
+          aa[acc] = fmaf(p0, p0, fmaf(p1, p1, aa[acc]));
+          bb[acc] = fmaf(q0, q0, fmaf(q1, q1, bb[acc]));
+        }
+      }
+      // both score tiles are in registers: the stream's next S may overwrite them
+      tc_fence_before();
+      if (ok) mbar_arrive(bar(L::bSFree + s));
+      ++t_me;
+    }
+    // the two streams' sums of every row meet in shared memory; group 0 writes them
+    const float sums[3] = {(ab[0] + ab[1]) + (ab[2] + ab[3]), (aa[0] + aa[1]) + (aa[2] + aa[3]),
+                           (bb[0] + bb[1]) + (bb[2] + bb[3])};
+    float* xb = xchg + (item & 1) * 384;
+    if (s == 1) {
+#pragma unroll
+      for (int q = 0; q < 3; ++q) xb[q * 128 + row] = sums[q];
+    }
+    if (bar_red_or(pair_bar, 64, !ok)) { ok = false; break; }
+    if (s == 0 && valid) {
+#pragma unroll
+      for (int q = 0; q < 3; ++q) p.energy[q * plane + bh * p.seq_len + token] = sums[q] + xb[q * 128 + row];
+    }
+    ++item;
+  }
+}
+
 template <int HD, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams p) {
   using L = Layout<HD>;
@@ -1031,7 +1177,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 #endif
   } else {
     reg_alloc<kSoftmaxRegs>();
-    if (MODE == kModeLse || MODE == kModeEnergy)
+    if (MODE == kModeSimilarity)
+      softmax_similarity_role<HD>(p, base, gbase, tmem, W, warp, lane);
+    else if (MODE == kModeLse || MODE == kModeEnergy)
       softmax_energy_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
     else
       softmax_role<HD, MODE>(p, base, gbase, tmem, W, warp, lane);
@@ -1127,6 +1275,7 @@ cudaError_t launch_tc_attn(const TcParams& p, int head_dim, int mode, int grid, 
     if (mode == kModeFused) return launch_one<128, kModeFused>(p, grid, s);
     if (mode == kModeLse) return launch_one<128, kModeLse>(p, grid, s);
     if (mode == kModeEnergy) return launch_one<128, kModeEnergy>(p, grid, s);
+    if (mode == kModeSimilarity) return launch_one<128, kModeSimilarity>(p, grid, s);
   }
   if (head_dim == 64) {
     if (mode == kModeSparse) return launch_one<64, kModeSparse>(p, grid, s);
@@ -1134,6 +1283,7 @@ cudaError_t launch_tc_attn(const TcParams& p, int head_dim, int mode, int grid, 
     if (mode == kModeFused) return launch_one<64, kModeFused>(p, grid, s);
     if (mode == kModeLse) return launch_one<64, kModeLse>(p, grid, s);
     if (mode == kModeEnergy) return launch_one<64, kModeEnergy>(p, grid, s);
+    if (mode == kModeSimilarity) return launch_one<64, kModeSimilarity>(p, grid, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -123,6 +123,12 @@ constexpr int kModeFused = 2;
 // log-sum-exp, the energy mode the block energies from it.
 constexpr int kModeLse = 3;
 constexpr int kModeEnergy = 4;
+// Spatial-repetition score on the same pipeline (no V, no P.V): every (head,
+// query tile) visits all key blocks with two score tiles per block, its own
+// 128 queries and their partner queries in the nearest anchor row (same
+// frame and column, gathered); each query's sums of p p', p^2 and p'^2 over
+// all keys are written to `energy` as three planes [3][batch * heads * seq_len].
+constexpr int kModeSimilarity = 5;
 // Work-item word of the dictionary schedules: bit 31 marks an anchor tile
 // (fused schedules only), bits 16-30 the head, bits 0-15 the query block or
 // anchor tile.
@@ -149,6 +155,8 @@ struct RepetitionParams {
 };
 constexpr int kMaxRepetitionRows = 256;
 cudaError_t launch_spatial_similarity(const RepetitionParams& p, int head_dim, int dtype, cudaStream_t s);
+cudaError_t launch_similarity_from_sums(const float* sums, int64_t plane, int32_t bh_count, int32_t seq_len,
+                                        int32_t frames, int32_t rows, int32_t cols, float* sim, cudaStream_t s);
 cudaError_t launch_repetition_flags(const float* sim, int32_t n_prompts, int32_t n_heads, int32_t per_head,
                                     float threshold, float* mean, uint8_t* flags, cudaStream_t s);
 

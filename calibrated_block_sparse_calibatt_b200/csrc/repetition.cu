@@ -9,7 +9,9 @@
 // Pass 1 (energy.cu, row_lse_kernel) gives each query's log2-sum-exp, so
 // P_ij = 2^(s_ij log2 e - lse2_i) is available key by key without storing P.
 // Calibration work on CUDA cores in float32, fixed reduction orders: repeated
-// calls give bitwise identical scores.
+// calls give bitwise identical scores.  (bf16 inputs take the tensor-core
+// pass of attn_tc.cu instead, which leaves per-query sums for
+// similarity_from_sums_kernel below.)
 #include "internal.h"
 
 #include <cuda_bf16.h>
@@ -130,7 +132,38 @@ __global__ void __launch_bounds__(kFlagThreads) repetition_flags_kernel(const fl
   }
 }
 
+// The rows' similarities from the tensor-core pass's per-query sums: one
+// thread per (batch, head, frame, row) adds its cols queries' three sums in
+// column order.
+__global__ void similarity_from_sums_kernel(const float* __restrict__ sums, int64_t plane, int32_t bh_count,
+                                            int32_t seq_len, int32_t frames, int32_t rows, int32_t cols,
+                                            float* __restrict__ sim) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(bh_count) * frames * rows;
+  if (idx >= total) return;
+  const int64_t bh = idx / (static_cast<int64_t>(frames) * rows);
+  const int64_t fr = idx % (static_cast<int64_t>(frames) * rows);
+  const float* ab = sums + bh * seq_len + fr * cols;
+  float dot = 0.f, na = 0.f, nb = 0.f;
+  for (int w = 0; w < cols; ++w) {
+    dot += ab[w];
+    na += ab[plane + w];
+    nb += ab[2 * plane + w];
+  }
+  const float den = sqrtf(na) * sqrtf(nb);
+  sim[idx] = den > 0.f ? dot / den : 0.f;
+}
+
 }  // namespace
+
+cudaError_t launch_similarity_from_sums(const float* sums, int64_t plane, int32_t bh_count, int32_t seq_len,
+                                        int32_t frames, int32_t rows, int32_t cols, float* sim, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(bh_count) * frames * rows;
+  if (total == 0) return cudaSuccess;
+  similarity_from_sums_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
+      sums, plane, bh_count, seq_len, frames, rows, cols, sim);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_spatial_similarity(const RepetitionParams& p, int head_dim, int dtype, cudaStream_t s) {
   dim3 g(p.frames * p.rows, p.heads, p.batch);

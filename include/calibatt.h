@@ -447,10 +447,22 @@ calibatt_status calibatt_aggregate_masks(const int32_t* counts, int64_t n, int32
  *                       / sqrt(sum_w |P[(f,rho,w)]|^2 * sum_w |P[(f,a,w)]|^2)
  * with P the dense, unmasked softmax of scale * q.k.  Anchor rows score one.
  * similarity: device float32 [batch, heads, frames, rows].  workspace:
- * caller-owned device scratch of at least calibatt_block_energy_workspace_size
- * bytes (each query's log-sum-exp).  anchor_rows: host int32, strictly
- * ascending in [0, rows), 1..16 of them; rows <= 256.  Computed on CUDA cores
- * in float32 with fixed summation orders (bitwise repeatable). */
+ * caller-owned device scratch of at least
+ * calibatt_spatial_similarity_workspace_size bytes.  anchor_rows: host int32,
+ * strictly ascending in [0, rows), 1..16 of them; rows <= 256.  BF16 inputs
+ * run on the tensor cores (q and k 16-byte aligned): a pass of each query's
+ * log-sum-exp, then a pass that pairs every 128-query tile with the gathered
+ * tile of its partner queries in the nearest anchor row and accumulates, key
+ * block by key block, each query's sums of P P', P^2 and P'^2 (float32), then
+ * a fixed-order sum over each row's cols queries.  FP32 inputs run on CUDA
+ * cores in float32.  Both use fixed summation orders (bitwise repeatable). */
+/* Device scratch bytes calibatt_spatial_similarity needs for `shape`: one
+ * float per query (its log-sum-exp), four on the tensor-core path (BF16: the
+ * log-sum-exp and three per-query sums).
+ * Key Designs 3: the workspace of calibatt_spatial_similarity. */
+calibatt_status calibatt_spatial_similarity_workspace_size(const calibatt_shape* shape,
+                                                           size_t* bytes);
+
 calibatt_status calibatt_spatial_similarity(const void* q, const void* k,
                                             const calibatt_shape* shape, int32_t frames,
                                             int32_t rows, int32_t cols,

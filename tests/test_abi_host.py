@@ -132,7 +132,7 @@ def test_hot_path_rejects_bad_arguments_before_any_gpu_work(calibatt_lib):
     assert L.calibatt_set_wait_timeout_ms(0) == C.ERR_INVALID_ARG
 
 
-def test_csr_schedule_covers_listed_heads_in_l2_groups(calibatt_lib):
+def test_csr_schedule_covers_listed_heads_in_l2_groups_and_waves(calibatt_lib):
     C = calibatt_lib
     rng = np.random.default_rng(3)
     heads, nq, grid = 6, 1300, 7       # keys and values of one head (85 MB) fill an L2 group
@@ -145,12 +145,14 @@ def test_csr_schedule_covers_listed_heads_in_l2_groups(calibatt_lib):
     want = sorted((h << 16) | r for h in head_ids for r in range(nq))
     assert sorted(items.tolist()) == want
     rank = {h: i for i, h in enumerate(head_ids)}
+    # one head per L2 group here, cut into waves of `grid` consecutive query
+    # blocks: wave (head rank, r // grid)
     for c in range(grid):
         mine = items[cta_ptr[c]:cta_ptr[c + 1]]
-        groups = [rank[int(x) >> 16] for x in mine]
-        assert groups == sorted(groups)      # each CTA walks the heads in list order
-        for g in set(groups):                 # inside a group, costs do not increase
-            cost = [lengths[head_ids[g], int(x) & 0xFFFF] for x in mine if rank[int(x) >> 16] == g]
+        waves = [(rank[int(x) >> 16], (int(x) & 0xFFFF) // grid) for x in mine]
+        assert waves == sorted(waves)        # each CTA walks the heads in list order, waves in order
+        for wv in set(waves):                 # inside a wave, costs do not increase
+            cost = [lengths[head_ids[wv[0]], int(x) & 0xFFFF] for x, w in zip(mine, waves) if w == wv]
             assert (np.diff(cost) <= 0).all()
     # rejected: a head listed twice, a head out of range, a decreasing row_ptr
     for hid, rp in (([1, 1], row_ptr), ([6], row_ptr), ([0], row_ptr[:, ::-1].copy())):
