@@ -947,15 +947,17 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
         int32_t* hp = run_ptr.data() + static_cast<size_t>(h) * (nq + 1);
         const size_t head_start = runs.size();
         for (int r = 0; r < nq; ++r) {
-          hp[r] = static_cast<int32_t>(runs.size() - head_start);
+          hp[r] |= static_cast<int32_t>(runs.size() - head_start);  // keeps row r - 1's end flag
           for (int32_t x = rp[r]; x < rp[r + 1]; ++x) {
             if (x > rp[r] && ci[x] == ci[x - 1] + 1)
               runs.back() += 1u << 16;                         // extends the current run
             else
               runs.push_back(static_cast<uint32_t>(ci[x]) | (1u << 16));
           }
+          // bit 31 of the row's end entry: the row keeps the last key block
+          if (rp[r + 1] > rp[r] && ci[rp[r + 1] - 1] == nq - 1) hp[r + 1] = INT32_MIN;
         }
-        hp[nq] = static_cast<int32_t>(runs.size() - head_start);
+        hp[nq] |= static_cast<int32_t>(runs.size() - head_start);
         run_head_off[h + 1] = static_cast<int64_t>(runs.size());
       }
     }
@@ -1314,6 +1316,7 @@ calibatt_status calibatt_dict_save(const calibatt_dict* d, const char* path) {
                          cudaMemcpyDeviceToHost);
         if (e == cudaSuccess)
           e = cudaMemcpy(cb.data(), d->d_col_base + ly * H, sizeof(int64_t) * H, cudaMemcpyDeviceToHost);
+        for (int32_t& x : run_ptr) x &= 0x7FFFFFFF;  // the file stores plain offsets (end flags are rebuilt)
         for (int h = 0; h < H; ++h) rec.nnz += run_ptr[static_cast<size_t>(h) * (nq + 1) + nq];
         bits.resize(rec.nnz);
         if (e == cudaSuccess && rec.nnz > 0)

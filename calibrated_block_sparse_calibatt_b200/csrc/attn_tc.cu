@@ -283,7 +283,7 @@ struct Cursor {
               it.ragged_last = it.n > 0 && (p.seq_len % 128) != 0 && it.cols[it.n - 1] == p.nb - 1;
             } else {
               // interval row: the producers decode its runs, and only the
-              // softmax warps need the last block (interval_ends_ragged)
+              // softmax warps need the last block (a flag in run_ptr)
               it.cols = nullptr;
               it.ragged_last = false;
             }
@@ -298,16 +298,6 @@ struct Cursor {
     return false;
   }
 };
-
-// Whether the last block of an interval row (head h, query block r) is the
-// partial key block: its last run ends at nb.
-__device__ __forceinline__ bool interval_ends_ragged(const TcParams& p, int h, int r) {
-  const int64_t ro = static_cast<int64_t>(h) * (p.sched.nq + 1) + r;
-  const int32_t last = p.sched.run_ptr[ro + 1] - 1;
-  if (last < p.sched.run_ptr[ro]) return false;  // empty row
-  const uint32_t run = p.sched.runs[p.sched.col_base[h] + last];
-  return static_cast<int>((run & 0xFFFFu) + (run >> 16)) == p.nb;
-}
 
 __device__ __forceinline__ void map_coords(const TcParams& p, int n0, int h, int b, int& c1,
                                            int& c2, int& c3) {
@@ -455,7 +445,7 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
       // blocks lane-parallel in order.
       uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
       const int64_t ro = static_cast<int64_t>(it.h) * (p.sched.nq + 1) + it.tile;
-      const int r0 = p.sched.run_ptr[ro], n_runs = p.sched.run_ptr[ro + 1] - r0;
+      const int r0 = p.sched.run_ptr[ro] & 0x7FFFFFFF, n_runs = (p.sched.run_ptr[ro + 1] & 0x7FFFFFFF) - r0;
       const uint32_t* runs = p.sched.runs + p.sched.col_base[it.h] + r0;
       int pos = 0;
       for (int x0 = 0; x0 < n_runs; x0 += 32) {
@@ -655,8 +645,10 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   uint32_t t_me = 0, t_other = 0;  // key blocks of this / the other stream so far (global)
   bool ok = true;
   while (cur.next(p, it)) {
-    if (p.sched.runs != nullptr && !it.anchor && ragged_cols != 0)
-      it.ragged_last = interval_ends_ragged(p, it.h, it.tile);
+    // Interval rows: bit 31 of the row's end entry in run_ptr says that the
+    // row keeps the last key block.  Loaded here, used only at the last block.
+    const int32_t run_end =
+        (p.sched.runs != nullptr && !it.anchor) ? p.sched.run_ptr[static_cast<int64_t>(it.h) * (p.sched.nq + 1) + it.tile + 1] : 0;
     const int n_s = (it.n + 1 - s) / 2;  // blocks of this stream in the item
     const uint32_t t_other0 = t_other;
     float m_own = -INFINITY, l = 0.f;    // this stream's row sum, relative to m_own
@@ -675,7 +667,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       float sc[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sc[c] = __uint_as_float(sr[c]);
-      if (j == it.n - 1 && it.ragged_last) {
+      if (j == it.n - 1 && (it.ragged_last || (run_end < 0 && ragged_cols != 0))) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= ragged_cols) sc[c] = -INFINITY;

@@ -29,6 +29,8 @@ struct LayerSchedule {
   // disjoint.  Head h's runs of query block r are
   // runs[col_base[h] + run_ptr[h][r] .. col_base[h] + run_ptr[h][r+1]);
   // row_ptr still counts blocks (the row's block count is the difference).
+  // Bit 31 of run_ptr[h][r + 1] is set when row r keeps the last key block
+  // (nq - 1); offsets are the low 31 bits.
   const int32_t* run_ptr;  // [H][nq + 1]
   const uint32_t* runs;
   // Nonzero when the lists and schedule come from the caller's device memory
