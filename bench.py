@@ -396,6 +396,81 @@ def run_epilogue_probe(torch, B, C):
         "peak_hbm_gbs": peaks()["hbm_gbs"]}}), flush=True)
 
 
+def softmax_phase_breakdown(recs, first=100, last=3900):
+    """Per-block phases of the two softmax streams from trace records
+    (event, key-block iteration, SM clock) of CTA 0: for each block a stream
+    owns, the cycles from the end of its previous block to the scores being
+    ready, the tensor-memory load, the row maximum, the spin on the other
+    stream's reference, the publish, the wait for the P buffer, the
+    exponential chain and the hand-off.  Event numbers follow the kernel's
+    trace points (32/36 scores ready, 40/44 loaded, 12-17 reference, 56/60 P
+    buffer free, 48/52 exponentials done, 20/24 P handed over)."""
+    import collections
+    ev = collections.defaultdict(dict)
+    for e, i, t in recs:
+        ev[e][i] = t
+    names = ["wait_s_full", "tmem_ld", "row_max", "spin_ref", "publish", "wait_p_free", "exp_chain",
+             "rescale_p_full"]
+    out = {}
+    for s in (0, 1):
+        w = 4 * s
+        seq = [(32 + w), (40 + w), (12 + s), (14 + s), (16 + s), (56 + w), (48 + w), (20 + w)]
+        ph = collections.defaultdict(list)
+        prev = None
+        for g in sorted(ev[32 + w]):
+            if first <= g < last and prev is not None and prev in ev[20 + w] and all(g in ev[e] for e in seq):
+                t = [ev[20 + w][prev]] + [ev[e][g] for e in seq]
+                for k, name in enumerate(names):
+                    ph[name].append(t[k + 1] - t[k])
+                ph["total"].append(t[-1] - t[0])
+            prev = g
+        tot = sum(ph["total"]) or 1
+        out[f"stream{s}"] = {k: {"median_cycles": statistics.median(v), "share": round(sum(v) / tot, 4)}
+                             for k, v in ph.items() if v}
+        out[f"stream{s}"]["blocks"] = len(ph["total"])
+    return out
+
+
+def run_softmax_phases(args, torch, B, C):
+    """The measurement build (-DCALIBATT_TRACE) on the 720p layer with
+    --heads heads: one traced call after three warm-up calls, and the phase
+    breakdown of CTA 0's two softmax streams."""
+    import ctypes
+    import dataclasses
+    lib = ctypes.CDLL(B.build(trace=True))
+    for name, (res, argt) in C.SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, argt
+    lib.calibatt_trace_read.restype = ctypes.c_int
+    lib.calibatt_trace_read.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    C.LIB = lib
+    wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
+    masks, _ = W.workload_masks(wl, seed_base=W.MASK_SEED_BASE["720p"])
+    q, k, v = W.make_qkv(wl.seed, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    o = torch.empty_like(q)
+    d = build_dict(C, [masks[h] for h in range(wl.heads)], wl.heads, wl.num_blocks, wl.block)
+    for _ in range(3):
+        C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block)
+    torch.cuda.synchronize()
+    lib.calibatt_trace_reset()
+    C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block)
+    torch.cuda.synchronize()
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the traced call")
+    n_ev, n_it = 64, 4096
+    buf = (ctypes.c_ulonglong * (n_ev * n_it))()
+    n = lib.calibatt_trace_read(buf, n_ev * n_it)
+    recs = [(i // n_it, i % n_it, buf[i]) for i in range(n) if buf[i] != 0]
+    ms = statistics.mean(time_calls(torch, lambda: C.calibatt_block_sparse_attn(q, k, v, o, d, 0, 0, wl.block),
+                                    5, 1, torch.cuda.current_stream()))
+    tiles = d.layer_info(0, 0)["retained_tiles"]
+    d.close()
+    print(json.dumps({"softmax_phases": {
+        "workload": f"720p layer, {wl.heads} heads, measurement build, CTA 0",
+        "ms_per_call_measurement_build": ms, "effective_tflops": tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12,
+        **softmax_phase_breakdown(recs)}}), flush=True)
+
+
 def run_sweep(args, C, torch, stream, pk):
     """Schedule sweep: a dictionary holding every (timestep, layer) record of
     the schedule, then one dual-path call per (t, l) on fresh seeded inputs,
@@ -708,6 +783,9 @@ def main():
     ap.add_argument("--epilogue-probe", action="store_true",
                     help="time the anchor broadcast epilogue with the library's measurement build "
                          "(-DCALIBATT_TRACE) and print its store rate")
+    ap.add_argument("--softmax-phases", action="store_true",
+                    help="trace the softmax streams of the block-sparse kernel with the library's measurement "
+                         "build (-DCALIBATT_TRACE) and print their per-block phase breakdown")
     ap.add_argument("--dual-case", action="store_true",
                     help="time the dual-path 720p layer alone (one fused launch of both paths)")
     ap.add_argument("--layout", default="bnhd", choices=["bnhd", "bhnd"],
@@ -753,6 +831,9 @@ def main():
     stream = torch.cuda.current_stream()
     if args.epilogue_probe:
         run_epilogue_probe(torch, B, C)
+        return
+    if args.softmax_phases:
+        run_softmax_phases(args, torch, B, C)
         return
     if args.anchor_case:
         run_anchor_case(args, torch, C, pk)
