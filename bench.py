@@ -314,6 +314,30 @@ def run_anchor_case(args, torch, C, pk):
         "output_bytes": len(rep_heads) * wd.seq_len * wd.head_dim * 2}}), flush=True)
 
 
+def run_similarity_case(args, torch, C, pk):
+    """The spatial-similarity pass alone on the 720p geometry with --heads
+    heads (LSE pass, pass of per-query sums, row reduction), timed with CUDA
+    events; a case of its own for profiling the tensor-core similarity mode."""
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["720p_dual"], heads=args.heads)
+    q, k, _ = W.make_qkv(wl.seed, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    sim = torch.empty((1, wl.heads, wl.frames, wl.rows), device="cuda")
+    ws = torch.empty(C.calibatt_spatial_similarity_workspace_size(q) // 4, device="cuda")
+    stream = torch.cuda.current_stream()
+    per_call = time_calls(torch, lambda: C.calibatt_spatial_similarity(q, k, sim, ws, wl.frames, wl.rows, wl.cols,
+                                                                       wl.anchors, stream=stream),
+                          args.steps, args.warmup, stream)
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the similarity case")
+    ms = statistics.mean(per_call)
+    exp2 = 3 * wl.seq_len ** 2 * wl.heads
+    print(json.dumps({"similarity_case": {
+        "heads": wl.heads, "ms_per_call": ms, "exp2_per_call": exp2,
+        "g_exp2_per_s": exp2 / (ms * 1e-3) / 1e9,
+        "frac_of_mufu_peak_at_max_clock": exp2 / (ms * 1e-3) / mufu_exp2_peak(C.device_sm_count(), 1965.0)}}),
+        flush=True)
+
+
 def run_dual_case(args, torch, C, pk):
     """The dual-path 720p layer alone (28 block-sparse heads and 12 anchor heads
     in ONE fused launch over the dictionary's joint schedule), timed with CUDA
@@ -786,6 +810,8 @@ def main():
     ap.add_argument("--softmax-phases", action="store_true",
                     help="trace the softmax streams of the block-sparse kernel with the library's measurement "
                          "build (-DCALIBATT_TRACE) and print their per-block phase breakdown")
+    ap.add_argument("--similarity-case", action="store_true",
+                    help="time the spatial-similarity pass alone (720p geometry, --heads heads)")
     ap.add_argument("--dual-case", action="store_true",
                     help="time the dual-path 720p layer alone (one fused launch of both paths)")
     ap.add_argument("--layout", default="bnhd", choices=["bnhd", "bhnd"],
@@ -840,6 +866,9 @@ def main():
         return
     if args.dual_case:
         run_dual_case(args, torch, C, pk)
+        return
+    if args.similarity_case:
+        run_similarity_case(args, torch, C, pk)
         return
     if args.workload == "sweep":
         if world > 1:
