@@ -110,8 +110,9 @@ def measured_traffic(tiles, path=None):
     """DRAM bytes per launch of the sparse kernel from the committed ncu counters
     of the bench launch itself (profiles/tc_attn_sparse_720p_traffic.json), per
     retained tile times the tiles of this launch; None
-    when a source of the kernel (the kernel file and the headers it includes)
-    changed since the capture."""
+    when a source the traffic depends on (the kernel file, the headers it
+    includes, and the host file that builds the schedule) changed since the
+    capture."""
     import hashlib
     path = path or os.path.join(ROOT, "profiles", "tc_attn_sparse_720p_traffic.json")
     if not os.path.exists(path):
