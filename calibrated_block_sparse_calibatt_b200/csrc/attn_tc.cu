@@ -168,7 +168,12 @@ struct Layout {
   // uint16 lists of kept key blocks decoded from bitmap rows, one per producer
   static constexpr int kListBytes = kMaxBitmapBlocks * 2;
   static constexpr int kList = kMSlot + 2 * 128 * 8;
-  static constexpr int kUsed = kList + 2 * kListBytes;
+  // per softmax warp: 8 output rows' halves (HD bytes each) staged for the
+  // anchor broadcast
+  static constexpr int kStageRowBytes = HD;
+  static constexpr int kStageBytes = 8 * kStageRowBytes;
+  static constexpr int kStage = (kList + 2 * kListBytes + 127) & ~127;
+  static constexpr int kUsed = kStage + 8 * kStageBytes;
   // +1024 for aligning the base; at least 120 KB so only one CTA fits per SM
   // (each CTA holds all 512 tensor-memory columns).
   static constexpr int kBytes = (kUsed + 1024) > 120 * 1024 ? (kUsed + 1024) : 120 * 1024;
@@ -812,6 +817,68 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
 #ifdef CALIBATT_TRACE
     const unsigned long long t_epi = globaltimer();
 #endif
+    if (MODE != kModeSparse && it.anchor) {
+      // Anchor broadcast through shared memory: the warp stages 8 of its rows
+      // at a time (each row's HD/2 output columns, HD bytes), then every
+      // destination row is written by HD/16 lanes storing its contiguous
+      // bytes, so one warp-wide store covers 32*16/HD rows instead of 32
+      // rows 16 bytes each.
+      uint4 pk[HD / 64][4];
+#pragma unroll
+      for (int ch = 0; ch < HD / 64; ++ch) {
+        uint32_t o[32];
+        if (it.n > 0) {
+          tmem_ld_x32(tO + s * (HD / 2) + ch * 32, o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[8 * g + e]) * inv_l;
+          pk[ch][g].x = pack_bf16x2(v[0], v[1]);
+          pk[ch][g].y = pack_bf16x2(v[2], v[3]);
+          pk[ch][g].z = pack_bf16x2(v[4], v[5]);
+          pk[ch][g].w = pack_bf16x2(v[6], v[7]);
+        }
+      }
+      constexpr int kUnits = HD / 16;            // 16-byte units of a staged row
+      constexpr int kRowsPerStore = 32 / kUnits;  // rows one warp-wide store covers
+      uint8_t* stg = gbase + L::kStage + warp * L::kStageBytes;
+      const int u = lane % kUnits;
+#pragma unroll 1
+      for (int pass = 0; pass < 4; ++pass) {
+        if ((lane >> 3) == pass) {
+          // unit g of staged row r sits at position g ^ r (no bank conflicts
+          // between the 8 rows written at once)
+          const int r = lane & 7;
+          uint4* sp = reinterpret_cast<uint4*>(stg + r * L::kStageRowBytes);
+#pragma unroll
+          for (int ch = 0; ch < HD / 64; ++ch)
+#pragma unroll
+            for (int g = 0; g < 4; ++g) sp[((ch * 4 + g) ^ r) & (kUnits - 1)] = pk[ch][g];
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8 / kRowsPerStore; ++i) {
+          const int r = lane / kUnits + kRowsPerStore * i;  // staged row 0..7
+          const int src = pass * 8 + r;                     // lane that owns it
+          const int nd = __shfl_sync(0xFFFFFFFFu, n_dst, src);
+          const int f = __shfl_sync(0xFFFFFFFFu, anchor_f, src);
+          const int w = __shfl_sync(0xFFFFFFFFu, anchor_w, src);
+          const int l0 = __shfl_sync(0xFFFFFFFFu, lo, src);
+          const uint4 val = reinterpret_cast<const uint4*>(stg + r * L::kStageRowBytes)[(u ^ r) & (kUnits - 1)];
+#pragma unroll 1
+          for (int d = 0; d < nd; ++d) {
+            const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + l0 + d) * p.anc.cols + w;
+            reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + s * (HD / 2))[u] = val;
+          }
+        }
+        __syncwarp();
+      }
+    } else {
 #pragma unroll 1
     for (int ch = 0; ch < HD / 64; ++ch) {
       const int col = s * (HD / 2) + ch * 32;  // this group's output columns
@@ -842,6 +909,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
 #pragma unroll
         for (int g = 0; g < 4; ++g) dst[g] = pkd[g];
       }
+    }
     }
 #ifdef CALIBATT_TRACE
     if (it.anchor && warp == 0 && lane == 0 && blockIdx.x < 1024) {
