@@ -848,6 +848,12 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       constexpr int kRowsPerStore = 32 / kUnits;  // rows one warp-wide store covers
       uint8_t* stg = gbase + L::kStage + warp * L::kStageBytes;
       const int u = lane % kUnits;
+      // this thread's first destination (in 16-byte units from O) and the step
+      // between the rows its anchor serves (same column, next spatial row)
+      const int64_t first = (bh_off + ((static_cast<int64_t>(anchor_f) * p.anc.rows + lo) * p.anc.cols + anchor_w) * p.sn +
+                             s * (HD / 2)) / 8;
+      const int64_t step = static_cast<int64_t>(p.anc.cols) * p.sn / 8;
+      uint4* const o16 = reinterpret_cast<uint4*>(p.o);
 #pragma unroll 1
       for (int pass = 0; pass < 4; ++pass) {
         if ((lane >> 3) == pass) {
@@ -866,15 +872,10 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
           const int r = lane / kUnits + kRowsPerStore * i;  // staged row 0..7
           const int src = pass * 8 + r;                     // lane that owns it
           const int nd = __shfl_sync(0xFFFFFFFFu, n_dst, src);
-          const int f = __shfl_sync(0xFFFFFFFFu, anchor_f, src);
-          const int w = __shfl_sync(0xFFFFFFFFu, anchor_w, src);
-          const int l0 = __shfl_sync(0xFFFFFFFFu, lo, src);
+          uint4* dst = o16 + __shfl_sync(0xFFFFFFFFu, first, src) + u;
           const uint4 val = reinterpret_cast<const uint4*>(stg + r * L::kStageRowBytes)[(u ^ r) & (kUnits - 1)];
 #pragma unroll 1
-          for (int d = 0; d < nd; ++d) {
-            const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + l0 + d) * p.anc.cols + w;
-            reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + s * (HD / 2))[u] = val;
-          }
+          for (int d = 0; d < nd; ++d, dst += step) *dst = val;
         }
         __syncwarp();
       }
