@@ -370,9 +370,10 @@ def run_dual_case(args, torch, C, pk):
         flush=True)
 
 
-def run_epilogue_probe(torch, B, C):
+def run_epilogue_probe(torch, B, C, fused=False):
     """Store rate of the anchor broadcast epilogue (the 12 repetitive heads of
-    the dual-path 720p layer).  The measurement build records, per CTA, the
+    the dual-path 720p layer), in the anchor-only launch or (fused=True) in
+    the fused dual-path launch.  The measurement build records, per CTA, the
     nanoseconds its epilogues spend issuing the output stores of anchor tiles;
     every output row of those heads is written once (N x D x 2 bytes per
     head), so the aggregate rate while in the epilogue is bytes / (mean
@@ -390,8 +391,15 @@ def run_epilogue_probe(torch, B, C):
     q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
     o = torch.empty_like(q)
 
+    dmasks, _ = W.workload_masks(wd)
+    d = build_dict(C, [dmasks[h] for h in range(wd.heads)], wd.heads, wd.num_blocks, wd.block,
+                   (wd.frames, wd.rows, wd.cols, wd.anchors)) if fused else None
+
     def call():
-        C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors, list(rep_heads))
+        if fused:
+            C.calibatt_dual_path_attn(q, k, v, o, d, 0, 0, wd.frames, wd.rows, wd.cols, wd.anchors, wd.block)
+        else:
+            C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors, list(rep_heads))
 
     call()
     torch.cuda.synchronize()
@@ -410,14 +418,18 @@ def run_epilogue_probe(torch, B, C):
     total_bytes = len(rep_heads) * wd.seq_len * wd.head_dim * 2
     mean_ns = sum(t for t, _ in used) / len(used)
     n_items = sum(n for _, n in used)
+    if d is not None:
+        d.close()
     print(json.dumps({"epilogue_probe": {
-        "workload": "dual-path 720p layer, anchor path of its 12 repetitive heads",
+        "workload": "dual-path 720p layer, anchor tiles of its 12 repetitive heads, " +
+                    ("fused launch (staged stores)" if fused else "anchor-only launch (per-thread stores)"),
         "anchor_tiles": n_items, "ctas": len(used), "output_bytes": total_bytes,
         "epilogue_ns_per_tile": sum(t for t, _ in used) / n_items,
         "bytes_per_tile": total_bytes / n_items,
         "aggregate_gbs_in_epilogue": total_bytes / mean_ns,
         "call_ms_measurement_build": a.elapsed_time(b),
         "epilogue_share_of_call": mean_ns / (a.elapsed_time(b) * 1e6),
+        "call": "calibatt_dual_path_attn (one fused launch)" if fused else "calibatt_anchor_attn",
         "peak_hbm_gbs": peaks()["hbm_gbs"]}}), flush=True)
 
 
@@ -808,6 +820,8 @@ def main():
     ap.add_argument("--epilogue-probe", action="store_true",
                     help="time the anchor broadcast epilogue with the library's measurement build "
                          "(-DCALIBATT_TRACE) and print its store rate")
+    ap.add_argument("--epilogue-fused", action="store_true",
+                    help="with --epilogue-probe: the anchor tiles of the fused dual-path launch")
     ap.add_argument("--softmax-phases", action="store_true",
                     help="trace the softmax streams of the block-sparse kernel with the library's measurement "
                          "build (-DCALIBATT_TRACE) and print their per-block phase breakdown")
@@ -857,7 +871,7 @@ def main():
     pk = peaks()
     stream = torch.cuda.current_stream()
     if args.epilogue_probe:
-        run_epilogue_probe(torch, B, C)
+        run_epilogue_probe(torch, B, C, fused=args.epilogue_fused)
         return
     if args.softmax_phases:
         run_softmax_phases(args, torch, B, C)
