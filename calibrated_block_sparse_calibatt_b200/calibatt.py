@@ -183,22 +183,22 @@ def csr_to_intervals(nq, row_ptr, col_idx):
 def count_intervals(row_ptr, col_idx):
     """Contiguous key-block intervals of a layer's CSR (row_ptr [H, nq + 1],
     the heads' lists concatenated): the capacity an interval dictionary needs
-    for it.  Counted with numpy (argument preparation for
-    calibatt_dict_create_intervals)."""
-    rp = np.asarray(row_ptr, dtype=np.int64).reshape(-1, np.asarray(row_ptr).shape[-1])
-    ci = np.asarray(col_idx, dtype=np.int64).reshape(-1)
-    if ci.size == 0:
-        return 0
-    # a block starts an interval unless it follows its predecessor in the same row
-    head_off = np.concatenate([[0], np.cumsum(rp[:, -1])])
-    starts = np.zeros(ci.size, bool)
+    for it, as the library encodes each head (calibatt_csr_to_intervals)."""
+    rp = _i32_array(row_ptr).reshape(-1, np.asarray(row_ptr).shape[-1])
+    ci = _i32_array(col_idx).reshape(-1)
+    nq = rp.shape[1] - 1
+    total, off = 0, 0
+    ptr = np.zeros(nq + 1, np.int32)
     for h in range(rp.shape[0]):
-        s = rp[h, :-1] + head_off[h]
-        e = rp[h, 1:] + head_off[h]
-        first = s[e > s]
-        starts[first] = True
-    starts[1:] |= ci[1:] != ci[:-1] + 1
-    return int(starts.sum())
+        n = int(rp[h, -1])
+        head = np.ascontiguousarray(ci[off:off + n])
+        cnt = ctypes.c_int64(0)
+        # capacity 0: the library only counts (and reports the shortfall)
+        LIB.calibatt_csr_to_intervals(nq, _ptr(np.ascontiguousarray(rp[h])), _ptr(head) if n else None, _ptr(ptr),
+                                      None, None, 0, ctypes.byref(cnt))
+        total += cnt.value
+        off += n
+    return total
 
 
 def lpt_schedule(cost, n_bins):
