@@ -147,6 +147,25 @@ int32_t heads_per_group(int32_t nq) {
   return static_cast<int32_t>(std::max<int64_t>(1, (static_cast<int64_t>(CALIBATT_L2_GROUP_MB) << 20) / per_head));
 }
 
+// Items in the order the CTAs take them under dynamic assignment: group by
+// group, cost descending inside a group (ties by position) -- the order in
+// which the LPT lists are dealt out.
+std::vector<int32_t> consumption_order(const std::vector<int64_t>& cost, const std::vector<int32_t>& group) {
+  std::vector<int32_t> idx(cost.size());
+  std::iota(idx.begin(), idx.end(), 0);
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) {
+    return group[a] != group[b] ? group[a] < group[b] : cost[a] > cost[b];
+  });
+  return idx;
+}
+
+// Dictionary calls assign work dynamically (a ticket counter per call) unless
+// built with CALIBATT_DYNAMIC=0 (static per-CTA lists, as the direct-CSR call).
+#ifndef CALIBATT_DYNAMIC
+#define CALIBATT_DYNAMIC 1
+#endif
+constexpr int kTicketSlots = 64;
+
 // Schedule group of the work item (k-th sparse head of the layer, query block
 // r).  Heads go in L2 groups of heads_per_group; with waves on, each head
 // group is further cut into waves of `grid` consecutive query blocks (in head,
@@ -352,6 +371,15 @@ struct calibatt_dict {
   int32_t* d_run_ptr = nullptr;
   uint32_t* d_runs = nullptr;
   int64_t blocks_used = 0;
+  // Dynamic assignment: per layer, the items in consumption order (sparse
+  // schedule and joint schedule), their counts, and a pool of ticket counters
+  // taken round-robin by the calls, so that calls in flight together on
+  // different streams use different counters.
+  uint32_t* d_order = nullptr;   // [layers][H * nq]
+  uint32_t* d_forder = nullptr;  // [layers][f_stride]
+  std::vector<int32_t> n_order, n_forder;
+  uint32_t* d_tickets = nullptr;  // [kTicketSlots]
+  mutable std::atomic<uint32_t> next_ticket{0};
 
   int64_t layer(int t, int l) const { return static_cast<int64_t>(t) * L + l; }
 
@@ -361,6 +389,20 @@ struct calibatt_dict {
     s.items = d_fitems + ly * f_stride;
     s.cta_ptr = d_fcta_ptr + ly * (G + 1);
     return s;
+  }
+
+  // Dynamic assignment for one call on `stream`: a ticket counter from the
+  // pool (round-robin), zeroed on the stream ahead of the launch, and the
+  // layer's consumption order.  Returns false if the counter cannot be set.
+  bool take_ticket(LayerSchedule& s, int t, int l, bool fused, cudaStream_t stream) const {
+    if (!CALIBATT_DYNAMIC) return true;
+    const int64_t ly = layer(t, l);
+    const uint32_t slot = next_ticket.fetch_add(1u) % kTicketSlots;
+    if (cudaMemsetAsync(d_tickets + slot, 0, sizeof(uint32_t), stream) != cudaSuccess) return false;
+    s.ticket = d_tickets + slot;
+    s.order = fused ? d_forder + ly * f_stride : d_order + ly * H * nq;
+    s.n_order = fused ? n_forder[ly] : n_order[ly];
+    return true;
   }
 
   LayerSchedule schedule(int t, int l) const {
@@ -384,6 +426,10 @@ struct calibatt_dict {
   }
 
   void release() {
+    cudaFree(d_order);
+    cudaFree(d_forder);
+    cudaFree(d_tickets);
+    d_order = d_forder = d_tickets = nullptr;
     cudaFree(d_row_ptr);
     cudaFree(d_col_base);
     cudaFree(d_col);
@@ -489,7 +535,12 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
   std::vector<int16_t> heads;
   for (int h = 0; h < d->H; ++h)
     if (!d->rep[ly * d->H + h]) heads.push_back(static_cast<int16_t>(h));
-  return run_sparse(q, k, v, o, s, block, d->schedule(t, l), d->G, heads, softmax_scale, lse, stream);
+  LayerSchedule sch = d->schedule(t, l);
+  if (s.dtype == CALIBATT_DTYPE_BF16 && block == 128 && !d->take_ticket(sch, t, l, false, stream)) {
+    cudaGetLastError();
+    return fail(CALIBATT_ERR_CUDA, "work-ticket reset failed");
+  }
+  return run_sparse(q, k, v, o, s, block, sch, d->G, heads, softmax_scale, lse, stream);
 }
 
 calibatt_status launch_anchor(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
@@ -613,6 +664,10 @@ calibatt_status launch_fused(const void* q, const void* k, const void* v, void* 
   p.nb = ceil_div(s.seq_len, 128);
   p.scale_log2 = scale_log2_of(softmax_scale, s.head_dim);
   p.sched = d->fused_schedule(t, l);
+  if (!d->take_ticket(p.sched, t, l, true, stream)) {
+    cudaGetLastError();
+    return fail(CALIBATT_ERR_CUDA, "work-ticket reset failed");
+  }
   p.anc = g;
   p.status = status_word_ptr();
   p.timeout_ns = g_timeout_ns.load();
@@ -795,11 +850,15 @@ calibatt_status calibatt_dict_create(int32_t T, int32_t L, int32_t H, int32_t nq
     if (e == cudaSuccess) e = cudaMalloc(&d->d_col, b_col);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_order, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_tickets, sizeof(uint32_t) * kTicketSlots);
     if (e != cudaSuccess) {
       d->release();
       return cuda_fail(e, "dictionary allocation");
     }
-    d->device_bytes = static_cast<int64_t>(b_rp + b_cb + b_col + b_it + b_cta);
+    d->n_order.assign(layers, 0);
+    d->n_forder.assign(layers, 0);
+    d->device_bytes = static_cast<int64_t>(b_rp + b_cb + b_col + 2 * b_it + b_cta + sizeof(uint32_t) * kTicketSlots);
     *out = holder.release();
     return CALIBATT_OK;
   });
@@ -845,11 +904,15 @@ calibatt_status calibatt_dict_create_bitmap(int32_t T, int32_t L, int32_t H, int
     cudaError_t e = cudaMalloc(&d->d_bitmap, b_bm);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_order, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_tickets, sizeof(uint32_t) * kTicketSlots);
     if (e != cudaSuccess) {
       d->release();
       return cuda_fail(e, "bitmap dictionary allocation");
     }
-    d->device_bytes = static_cast<int64_t>(b_bm + b_it + b_cta);
+    d->n_order.assign(layers, 0);
+    d->n_forder.assign(layers, 0);
+    d->device_bytes = static_cast<int64_t>(b_bm + 2 * b_it + b_cta + sizeof(uint32_t) * kTicketSlots);
     *out = holder.release();
     return CALIBATT_OK;
   });
@@ -902,11 +965,15 @@ calibatt_status calibatt_dict_create_intervals(int32_t T, int32_t L, int32_t H, 
     if (e == cudaSuccess) e = cudaMalloc(&d->d_runs, b_runs);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_items, b_it);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_cta_ptr, b_cta);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_order, b_it);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_tickets, sizeof(uint32_t) * kTicketSlots);
     if (e != cudaSuccess) {
       d->release();
       return cuda_fail(e, "interval dictionary allocation");
     }
-    d->device_bytes = static_cast<int64_t>(2 * b_rp + b_cb + b_runs + b_it + b_cta);
+    d->n_order.assign(layers, 0);
+    d->n_forder.assign(layers, 0);
+    d->device_bytes = static_cast<int64_t>(2 * b_rp + b_cb + b_runs + 2 * b_it + b_cta + sizeof(uint32_t) * kTicketSlots);
     *out = holder.release();
     return CALIBATT_OK;
   });
@@ -1007,6 +1074,12 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     lpt_grouped(static_cast<int32_t>(items.size()), cost.data(), group.data(), d->G, cta_ptr.data(), order.data());
     std::vector<uint32_t> sched(items.size());
     for (size_t i = 0; i < items.size(); ++i) sched[i] = items[order[i]];
+    // the same items in consumption order, for dynamic assignment
+    std::vector<uint32_t> dyn(items.size());
+    {
+      const std::vector<int32_t> co = consumption_order(cost, group);
+      for (size_t i = 0; i < items.size(); ++i) dyn[i] = items[co[i]];
+    }
     // Joint schedule of the dual path.  All anchor tiles of the repetitive
     // heads come first, as one group in head order (a tile visits all nq key
     // blocks; its epilogue writes about rows / n_anchors output rows per query,
@@ -1017,7 +1090,7 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     // in head-order groups let CTAs drift several groups apart behind the large
     // anchor tiles, and the keys and values of the heads in flight no longer
     // fitted in L2.)
-    std::vector<uint32_t> fsched;
+    std::vector<uint32_t> fsched, fdyn;
     std::vector<int32_t> fcta_ptr;
     if (d->has_geom) {
       std::vector<uint32_t> fitems;
@@ -1048,6 +1121,9 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
                   forder.data());
       fsched.resize(fitems.size());
       for (size_t i = 0; i < fitems.size(); ++i) fsched[i] = fitems[forder[i]];
+      const std::vector<int32_t> co = consumption_order(fcost, fgroup);
+      fdyn.resize(fitems.size());
+      for (size_t i = 0; i < fitems.size(); ++i) fdyn[i] = fitems[co[i]];
     }
     int prev = 0;
     cudaGetDevice(&prev);
@@ -1078,6 +1154,11 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     }
     if (e == cudaSuccess && !sched.empty())
       e = cudaMemcpy(d->d_items + ly * H * nq, sched.data(), sizeof(uint32_t) * sched.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !dyn.empty())
+      e = cudaMemcpy(d->d_order + ly * H * nq, dyn.data(), sizeof(uint32_t) * dyn.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && d->has_geom && !fdyn.empty())
+      e = cudaMemcpy(d->d_forder + ly * d->f_stride, fdyn.data(), sizeof(uint32_t) * fdyn.size(),
+                     cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
       e = cudaMemcpy(d->d_cta_ptr + ly * (d->G + 1), cta_ptr.data(), sizeof(int32_t) * (d->G + 1), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && d->has_geom && !fsched.empty())
@@ -1093,6 +1174,8 @@ calibatt_status calibatt_dict_set_layer(calibatt_dict* d, int32_t t, int32_t l, 
     for (int h = 0; h < H; ++h) d->rep[ly * H + h] = (repetitive && repetitive[h]) ? 1 : 0;
     d->n_sparse[ly] = n_sparse;
     d->n_rep[ly] = n_rep;
+    d->n_order[ly] = static_cast<int32_t>(dyn.size());
+    d->n_forder[ly] = static_cast<int32_t>(fdyn.size());
     d->retained[ly] = retained;
     d->layer_set[ly] = 1;
     return CALIBATT_OK;
@@ -1128,6 +1211,7 @@ calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* d, int32_t fram
     cudaGetDevice(&prev);
     if (prev != d->device) cudaSetDevice(d->device);
     cudaError_t e = cudaMalloc(&d->d_fitems, sizeof(uint32_t) * layers * stride);
+    if (e == cudaSuccess) e = cudaMalloc(&d->d_forder, sizeof(uint32_t) * layers * stride);
     if (e == cudaSuccess) e = cudaMalloc(&d->d_fcta_ptr, sizeof(int32_t) * layers * (d->G + 1));
     if (prev != d->device) cudaSetDevice(prev);
     if (e != cudaSuccess) {
@@ -1137,7 +1221,7 @@ calibatt_status calibatt_dict_set_anchor_geometry(calibatt_dict* d, int32_t fram
       d->d_fcta_ptr = nullptr;
       return cuda_fail(e, "joint schedule allocation");
     }
-    d->device_bytes += static_cast<int64_t>(sizeof(uint32_t) * layers * stride + sizeof(int32_t) * layers * (d->G + 1));
+    d->device_bytes += static_cast<int64_t>(2 * sizeof(uint32_t) * layers * stride + sizeof(int32_t) * layers * (d->G + 1));
     d->f_stride = stride;
     d->g_frames = frames;
     d->g_rows = rows;

@@ -63,6 +63,11 @@ __device__ unsigned long long g_cta_span[2 * 1024];
 // number of such tiles (warp 0, lane 0 times its warp's stores).
 __device__ unsigned long long g_epi_ns[1024];
 __device__ unsigned long long g_epi_items[1024];
+// Start (globaltimer, ns) and work-item word of the first kItemTrace items
+// of every CTA, recorded by the Q/K producer.
+constexpr int kItemTrace = 256;
+__device__ unsigned long long g_item_t[1024 * kItemTrace];
+__device__ unsigned int g_item_w[1024 * kItemTrace];
 #ifndef CALIBATT_TRACE_OFFSET
 #define CALIBATT_TRACE_OFFSET 0
 #endif
@@ -140,6 +145,10 @@ constexpr int kPolyEvery = CALIBATT_POLY_EVERY;
 constexpr int kEnergyPolyEvery = CALIBATT_ENERGY_POLY_EVERY;
 
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
+// Dynamic assignment: the Q/K producer takes each ticket and hands it to the
+// other eleven warps through a ring of kItemRing slots in shared memory.
+constexpr int kItemRing = 4;
+constexpr int kItemReaders = 11;  // softmax warps 0-7, S issuer, V producer, P.V issuer
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 template <int HD>
@@ -160,9 +169,12 @@ struct Layout {
   static constexpr int bOFull = bPFree + 2;          // every P.V of the item finished
   static constexpr int bOFree = bOFull + 1;          // epilogue has read O
   static constexpr int bDrain = bOFree + 1;
-  static constexpr int kNumBars = bDrain + 1;
-  static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag
-  static constexpr int kXchg = kMisc + 16;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
+  static constexpr int bItemFull = bDrain + 1;              // [kItemRing] ticket published
+  static constexpr int bItemEmpty = bItemFull + kItemRing;  // [kItemRing] every other role has read it
+  static constexpr int kNumBars = bItemEmpty + kItemRing;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // u32 tmem base, i32 abort flag, u32 tickets [kItemRing]
+  static constexpr int kRing = kMisc + 8;
+  static constexpr int kXchg = kMisc + 8 + 4 * kItemRing;  // float [2 item parity][2 streams][2 (m, l)][128 rows]
   // {m bits, stream ordinal + 1} [2 streams][128 rows], 8-byte slots
   static constexpr int kMSlot = kXchg + 2 * 2 * 2 * 128 * 4;
   // uint16 lists of kept key blocks decoded from bitmap rows, one per producer
@@ -213,10 +225,20 @@ __device__ __forceinline__ const uint32_t* bitmap_row(const TcParams& p, int h, 
 }
 
 // Walks this CTA's work items in the same order in every role.
-template <int MODE>
+template <int HD, int MODE>
 struct Cursor {
   int b, idx, begin, end, step;
-  __device__ void init(const TcParams& p) {
+  uint32_t ring = 0;  // dynamic assignment: shared-memory base of the ring
+  uint32_t seq = 0;   // tickets taken from the ring so far
+  bool fetcher = false;
+  __device__ bool dynamic(const TcParams& p) const {
+    return (MODE == kModeSparse || MODE == kModeFused) && p.sched.ticket != nullptr;
+  }
+  // base: the CTA's 1024-aligned shared-memory base; is_fetcher: this warp
+  // takes the tickets (the Q/K producer) and the others read them.
+  __device__ void init(const TcParams& p, uint32_t base, bool is_fetcher) {
+    ring = base;
+    fetcher = is_fetcher;
     b = 0;
     if (MODE == kModeAnchor) {
       begin = blockIdx.x;
@@ -227,15 +249,51 @@ struct Cursor {
       end = p.heads * p.nb;
       step = gridDim.x;
     } else {
-      begin = p.sched.cta_ptr[blockIdx.x];
-      end = p.sched.cta_ptr[blockIdx.x + 1];
+      begin = dynamic(p) ? 0 : p.sched.cta_ptr[blockIdx.x];
+      end = dynamic(p) ? 0 : p.sched.cta_ptr[blockIdx.x + 1];
       step = 1;
     }
     idx = begin;
   }
-  __device__ bool next(const TcParams& p, Item& it) {
+  // Dynamic assignment: the next ticket, through the ring.  The fetcher waits
+  // until all readers are done with the slot's previous ticket, takes a ticket
+  // (atomicAdd) and publishes it; a reader waits for the slot, reads it and
+  // frees it.  Returns false past the last ticket or when a wait gives up.
+  __device__ bool take_ticket(const TcParams& p, const Waiter& W, uint32_t& t) {
+    using L = Layout<HD>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t slot = seq % kItemRing, use = seq / kItemRing;
+    const uint32_t full = ring + L::kBar + 8u * (L::bItemFull + slot);
+    const uint32_t empty = ring + L::kBar + 8u * (L::bItemEmpty + slot);
+    const uint32_t cell = ring + L::kRing + 4u * slot;
+    t = 0;
+    if (fetcher) {
+      if (use > 0 && !W.wait(empty, (use - 1) & 1, 16)) return false;
+      if (lane == 0) {
+        t = atomicAdd(p.sched.ticket, 1u);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(cell), "r"(t) : "memory");
+        mbar_arrive(full);
+      }
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+    } else {
+      if (!W.wait(full, use & 1, 17)) return false;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(t) : "r"(cell) : "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty);
+    }
+    ++seq;
+    return t < static_cast<uint32_t>(p.batch) * static_cast<uint32_t>(p.sched.n_order);
+  }
+  __device__ bool next(const TcParams& p, Item& it, const Waiter& W) {
     while (b < p.batch) {
-      if (idx < end) {
+      uint32_t t_dyn = 0;
+      const bool dyn = dynamic(p);
+      if (dyn) {
+        if (!take_ticket(p, W, t_dyn)) return false;
+        b = static_cast<int>(t_dyn / static_cast<uint32_t>(p.sched.n_order));
+        idx = static_cast<int>(t_dyn % static_cast<uint32_t>(p.sched.n_order));
+      }
+      if (dyn || idx < end) {
         it.b = b;
         uint32_t w = 0;
         if (calibration_mode(MODE)) {
@@ -249,7 +307,7 @@ struct Cursor {
           idx += step;
           return true;
         }
-        if (MODE != kModeAnchor) w = p.sched.items[idx];
+        if (MODE != kModeAnchor) w = dyn ? p.sched.order[idx] : p.sched.items[idx];
         if (MODE == kModeAnchor || (MODE == kModeFused && (w & kItemAnchorBit))) {
           it.anchor = true;
           if (MODE == kModeAnchor) {
@@ -342,15 +400,22 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
   constexpr int kRing = V ? L::kV : L::kK;
   const CUtensorMap* map = V ? &p.tm_v : &p.tm_k;
   if (V && calibration_mode(MODE)) return;  // no P.V in the calibration modes
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, !V);  // the Q/K producer takes the tickets
   Item it;
   uint32_t kv = 0, item = 0, issued = 0, q_items = 0;
   bool ok = true;
-  while (ok && cur.next(p, it)) {
+  while (ok && cur.next(p, it, W)) {
     if (!V) {
       if (item > 0 && !W.wait(bar(L::bQEmpty), (item - 1) & 1, 1)) break;
       CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 9, item + CALIBATT_TRACE_OFFSET);
+#ifdef CALIBATT_TRACE
+      if (lane == 0 && blockIdx.x < 1024 && item < static_cast<uint32_t>(kItemTrace)) {
+        g_item_t[blockIdx.x * kItemTrace + item] = globaltimer();
+        g_item_w[blockIdx.x * kItemTrace + item] =
+            (it.anchor ? 0x80000000u : 0u) | (static_cast<uint32_t>(it.h) << 16) | static_cast<uint32_t>(it.tile);
+      }
+#endif
       if (it.anchor) {
         // Gather this tile's 128 anchor-row queries into the 128-byte swizzled
         // K-major layout the MMA expects (16-byte unit u of row r lands at
@@ -507,13 +572,13 @@ __device__ void mma_s_role(const TcParams& p, uint32_t base, uint32_t tmem, cons
   using L = Layout<HD>;
   auto bar = [&](int i) { return base + L::kBar + 8u * i; };
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0);
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, false);
   Item it;
   uint32_t g = 0, item = 0;      // global key-block iteration, item counter
   uint32_t t0 = 0, t1 = 0;       // blocks issued per stream
   bool ok = true;
-  while (ok && cur.next(p, it)) {
+  while (ok && cur.next(p, it, W)) {
     if (!W.wait(bar(L::bQFull), item & 1, 4)) break;
     tc_fence_after();
     CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 8, item + CALIBATT_TRACE_OFFSET);
@@ -575,13 +640,13 @@ __device__ void mma_pv_role(const TcParams& p, uint32_t base, uint32_t tmem, con
     __syncwarp();
     return;
   }
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, false);
   Item it;
   uint32_t g = 0, item = 0;
   uint32_t t0 = 0, t1 = 0;
   bool ok = true;
-  while (ok && cur.next(p, it)) {
+  while (ok && cur.next(p, it, W)) {
     // The epilogue of the previous item has read O (waited for every item,
     // empty ones included, so each phase of o_free is consumed in order).
     if (item > 0 && !W.wait(bar(L::bOFree), (item - 1) & 1, 9)) break;
@@ -643,13 +708,13 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
   const uint32_t tO = tmem + lane_off + kColO;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, false);
   Item it;
   uint32_t kv = 0, item = 0;
   uint32_t t_me = 0, t_other = 0;  // key blocks of this / the other stream so far (global)
   bool ok = true;
-  while (cur.next(p, it)) {
+  while (cur.next(p, it, W)) {
     // Interval rows: bit 31 of the row's end entry in run_ptr says that the
     // row keeps the last key block.  Loaded here, used only at the last block.
     const int32_t run_end =
@@ -959,12 +1024,12 @@ __device__ void softmax_energy_role(const TcParams& p, uint32_t base, uint8_t* g
   const uint32_t tS = tmem + lane_off + kColS + s * 128;
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, false);
   Item it;
   uint32_t item = 0, t_me = 0;
   bool ok = true;
-  while (cur.next(p, it)) {
+  while (cur.next(p, it, W)) {
     const int n_s = (it.n + 1 - s) / 2;
     const int token = it.tile * 128 + row;
     const bool valid = token < p.seq_len;
@@ -1083,12 +1148,12 @@ __device__ void softmax_similarity_role(const TcParams& p, uint32_t base, uint8_
   const int ragged_cols = p.seq_len % 128;
   const float sl2 = p.scale_log2;
   const int64_t plane = static_cast<int64_t>(p.batch) * p.heads * p.seq_len;
-  Cursor<MODE> cur;
-  cur.init(p);
+  Cursor<HD, MODE> cur;
+  cur.init(p, base, false);
   Item it;
   uint32_t item = 0, t_me = 0;
   bool ok = true;
-  while (cur.next(p, it)) {
+  while (cur.next(p, it, W)) {
     const int n_s = (it.n + 1 - s) / 2;
     const int64_t token = static_cast<int64_t>(it.tile) * 128 + row;
     const bool valid = token < p.seq_len;
@@ -1200,6 +1265,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     mbar_init(bar(L::bOFull), 1);
     mbar_init(bar(L::bOFree), kSoftmaxThreads);
     mbar_init(bar(L::bDrain), 2);  // one commit from each MMA-issuing thread
+    for (int r = 0; r < kItemRing; ++r) {
+      mbar_init(bar(L::bItemFull + r), 1);
+      mbar_init(bar(L::bItemEmpty + r), kItemReaders);
+    }
     for (int i = 0; i < 256; ++i) st_shared_v2(base + L::kMSlot + i * 8, 0u, 0u);  // tag 0: no m yet
     *abort_flag = 0;
     fence_mbar_init();
@@ -1309,6 +1378,12 @@ extern "C" int calibatt_epilogue_probe_read(unsigned long long* ns, unsigned lon
   cudaMemcpyFromSymbol(items, g_epi_items, sizeof(unsigned long long) * n);
   return n;
 }
+extern "C" int calibatt_item_trace_read(unsigned long long* t, unsigned int* w, int max_records) {
+  const int n = 1024 * kItemTrace < max_records ? 1024 * kItemTrace : max_records;
+  cudaMemcpyFromSymbol(t, g_item_t, sizeof(unsigned long long) * n);
+  cudaMemcpyFromSymbol(w, g_item_w, sizeof(unsigned int) * n);
+  return n;
+}
 extern "C" void calibatt_trace_reset() {
   static unsigned long long zeros_cta[1024];
   cudaMemcpyToSymbol(g_epi_ns, zeros_cta, sizeof(zeros_cta));
@@ -1316,6 +1391,8 @@ extern "C" void calibatt_trace_reset() {
   cudaMemset(nullptr, 0, 0);
   static unsigned long long zeros[kTraceEvents * kTraceIters];
   cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros));
+  static unsigned long long zeros_items[1024 * kItemTrace];
+  cudaMemcpyToSymbol(g_item_t, zeros_items, sizeof(zeros_items));
 }
 #endif
 

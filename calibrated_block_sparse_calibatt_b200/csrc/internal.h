@@ -33,6 +33,14 @@ struct LayerSchedule {
   // (nq - 1); offsets are the low 31 bits.
   const int32_t* run_ptr;  // [H][nq + 1]
   const uint32_t* runs;
+  // Dynamic assignment (dictionary calls): instead of the per-CTA lists in
+  // items/cta_ptr, the CTAs take tickets 0, 1, ... from *ticket (zeroed before
+  // the launch); ticket t is item order[t % n_order] of batch t / n_order.
+  // order lists the layer's items in consumption order (L2 group, wave, cost
+  // descending).  nullptr = static lists.
+  uint32_t* ticket;
+  const uint32_t* order;
+  int32_t n_order;
   // Nonzero when the lists and schedule come from the caller's device memory
   // (direct-CSR call): the kernels then do nothing if the status word holds a
   // skip-list or schedule violation (codes 23, 24) recorded by the check that

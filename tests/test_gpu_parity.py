@@ -1041,7 +1041,9 @@ def test_bitmap_dictionary_size_and_rules(C):
     with C.MaskDictionary(2, 2, 4, nb, nb, 128, 4 * ci.size) as dl, \
             C.MaskDictionary(2, 2, 4, nb, nb, 128, bitmap=True) as db:
         bl, bb = dl.info()["device_bytes"], db.info()["device_bytes"]
-        assert bb == 4 * 4 * nb * ((nb + 31) // 32) * 4 + 4 * 4 * nb * 4 + 4 * (db.info()["num_ctas"] + 1) * 4
+        # bitmap words, the work items and their consumption order, CTA offsets, the ticket counters
+        assert bb == (4 * 4 * nb * ((nb + 31) // 32) * 4 + 2 * 4 * 4 * nb * 4 + 4 * (db.info()["num_ctas"] + 1) * 4
+                      + 64 * 4)
         db.set_layer(1, 1, rp, ci, rep)
         assert db.info()["nnz"] == ci.size
         assert bb < bl
