@@ -21,6 +21,13 @@
  *   - GPU work is enqueued asynchronously on the caller's stream (a
  *     cudaStream_t passed as void*; NULL is the legacy default stream).
  *     Nothing is synchronised except where a function says so.
+ *   - Attention calls on a dictionary (bf16, block 128) hand out their work
+ *     dynamically: each call zeroes one of the dictionary's 64 work counters
+ *     on its stream (taken round-robin, call by call) and the persistent CTAs
+ *     take work items from it.  Up to 64 calls on one dictionary may be in
+ *     flight on the GPU at once; a call captured in a CUDA graph keeps its
+ *     counter, so a replay must not overlap the 64th call after it on
+ *     another stream.
  *   - Activations are [batch, N_alloc, heads, head_dim] with the last dimension
  *     contiguous; strides are in elements.  Tokens are ordered frame-major,
  *     then spatial row, then column: token = f*R*C + row*C + col.  Only the
