@@ -1225,3 +1225,34 @@ def test_bounded_wait_runs_out_and_context_survives(C):
     out, _ = _run_sparse(C, q, k, v, masks, 128)
     ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, 128)
     _assert_close(_np(out), ref, "bf16")
+
+
+def test_dictionary_calls_in_flight_on_several_streams(C):
+    """Dictionary calls hand out work through per-call counters (64 per
+    dictionary, taken round-robin): calls on one dictionary issued on three
+    streams at once, 72 of them in all (the pool wraps), each give bitwise the
+    output of a call made alone; block-sparse and fused dual-path calls."""
+    frames, rows, cols, anchors = 2, 10, 64, (2, 7)
+    n, h, d, block = frames * rows * cols, 4, 128, 128
+    nb = O.num_blocks(n, block)
+    masks = _random_masks(81, h, nb, 0.5)
+    masks[1] = None                                              # one head on the anchor path
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    q, k, v = W.make_qkv(82, 1, n, h, d, "bf16", 1.0, "cuda")
+    with C.MaskDictionary(1, 1, h, nb, nb, block, ci.size) as dct:
+        dct.set_anchor_geometry(frames, rows, cols, anchors)
+        dct.set_layer(0, 0, rp, ci, rep)
+        ref_s, ref_d = torch.zeros_like(q), torch.zeros_like(q)
+        C.calibatt_block_sparse_attn(q, k, v, ref_s, dct, 0, 0, block)
+        C.calibatt_dual_path_attn(q, k, v, ref_d, dct, 0, 0, frames, rows, cols, anchors, block)
+        _check_status(C)
+        streams = [torch.cuda.Stream() for _ in range(3)]
+        outs = [[torch.zeros_like(q), torch.zeros_like(q)] for _ in streams]
+        for rnd in range(12):                                   # 12 rounds x 3 streams x 2 calls = 72
+            for st, (os_, od) in zip(streams, outs):
+                C.calibatt_block_sparse_attn(q, k, v, os_, dct, 0, 0, block, stream=st)
+                C.calibatt_dual_path_attn(q, k, v, od, dct, 0, 0, frames, rows, cols, anchors, block, stream=st)
+        torch.cuda.synchronize()
+        _check_status(C)
+    for os_, od in outs:
+        assert torch.equal(os_, ref_s) and torch.equal(od, ref_d)
