@@ -194,8 +194,10 @@ def count_intervals(row_ptr, col_idx):
         head = np.ascontiguousarray(ci[off:off + n])
         cnt = ctypes.c_int64(0)
         # capacity 0: the library only counts (and reports the shortfall)
-        LIB.calibatt_csr_to_intervals(nq, _ptr(np.ascontiguousarray(rp[h])), _ptr(head) if n else None, _ptr(ptr),
-                                      None, None, 0, ctypes.byref(cnt))
+        st = LIB.calibatt_csr_to_intervals(nq, _ptr(np.ascontiguousarray(rp[h])), _ptr(head) if n else None,
+                                           _ptr(ptr), None, None, 0, ctypes.byref(cnt))
+        if st != OK and cnt.value == 0:
+            raise CalibattError(st, last_error())
         total += cnt.value
         off += n
     return total
