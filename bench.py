@@ -296,8 +296,12 @@ def run_anchor_case(args, torch, C, pk):
     layer (anchor rows attend to all keys, the output is broadcast to every
     row), timed with CUDA events; a case of its own for profiling the anchor
     kernel.  Prints effective TFLOP/s (8.39 MFLOP per anchor tile x key block)."""
+    import dataclasses
     wd = W.WORKLOADS["720p_dual"]
     _, rep_heads = W.workload_masks(wd)
+    # --heads: the layer's first heads only (a smaller case for profiling)
+    wd = dataclasses.replace(wd, heads=min(args.heads, wd.heads))
+    rep_heads = tuple(h for h in rep_heads if h < wd.heads)
     q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
     o = torch.empty_like(q)
     stream = torch.cuda.current_stream()
@@ -343,8 +347,12 @@ def run_dual_case(args, torch, C, pk):
     """The dual-path 720p layer alone (28 block-sparse heads and 12 anchor heads
     in ONE fused launch over the dictionary's joint schedule), timed with CUDA
     events; a case of its own for profiling the fused kernel."""
+    import dataclasses
     wd = W.WORKLOADS["720p_dual"]
     dmasks, rep_heads = W.workload_masks(wd)
+    # --heads: the layer's first heads only (a smaller case for profiling)
+    wd = dataclasses.replace(wd, heads=min(args.heads, wd.heads))
+    rep_heads = tuple(h for h in rep_heads if h < wd.heads)
     geom = (wd.frames, wd.rows, wd.cols, wd.anchors)
     q, k, v = W.make_qkv(wd.seed, 1, wd.seq_len, wd.heads, wd.head_dim, "bf16", wd.input_std, "cuda")
     o = torch.empty_like(q)
@@ -808,7 +816,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the dense / dual-path / e2e legs")
     ap.add_argument("--heads", type=int, default=40,
-                    help="heads of the 720p layer (fewer heads = smaller case for profiling)")
+                    help="heads of the 720p layer (fewer heads = smaller case for profiling); with --dual-case "
+                         "and --anchor-case the dual-path layer's first heads")
     ap.add_argument("--workload", default="720p", choices=["720p", "sweep"],
                     help="sweep: the mask-dictionary schedule sweep (one dual-path 720p call per "
                          "timestep and layer), reported as aggregate time against the dense path")
