@@ -306,17 +306,29 @@ def run_anchor_case(args, torch, C, pk):
     o = torch.empty_like(q)
     stream = torch.cuda.current_stream()
     tiles = len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128) * wd.num_blocks
+    ws = anchor_workspace(torch, C, q, wd, len(rep_heads))
     per_call = time_calls(torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols,
-                                                                wd.anchors, list(rep_heads), stream=stream),
+                                                                wd.anchors, list(rep_heads), workspace=ws,
+                                                                stream=stream),
                           args.steps, args.warmup, stream)
     if C.device_status() != 0:
         raise RuntimeError("device wait timed out in the anchor case")
     ms = statistics.mean(per_call)
     tf = tiles * FLOP_PER_TILE / (ms * 1e-3) / 1e12
+    n_tiles = len(rep_heads) * -(-wd.frames * len(wd.anchors) * wd.cols // 128)
+    first, parts = C.anchor_split_plan(n_tiles, C.device_sm_count(), wd.num_blocks)
     print(json.dumps({"anchor_case": {
         "heads": len(rep_heads), "anchor_tiles_x_key_blocks": tiles, "ms_per_call": ms,
         "effective_tflops": tf, "frac_of_burst_peak": tf / pk["bf16_tflops"],
+        "split_tiles": n_tiles - first, "parts_per_split_tile": parts,
         "output_bytes": len(rep_heads) * wd.seq_len * wd.head_dim * 2}}), flush=True)
+
+
+def anchor_workspace(torch, C, q, wd, n_heads):
+    """The anchor call's workspace (its last partial wave of tiles split over
+    key ranges), or None when the call would not split."""
+    nbytes = C.calibatt_anchor_attn_workspace_size(q, wd.frames, wd.rows, wd.cols, len(wd.anchors), n_heads)
+    return torch.empty(nbytes // 4, dtype=torch.float32, device="cuda") if nbytes else None
 
 
 def run_similarity_case(args, torch, C, pk):
@@ -998,18 +1010,27 @@ def main():
                                                      wd.anchors, wd.block, stream=stream),
             max(3, args.steps // 4), 2, stream)), dist, "cuda")
         d_two.close()
+        # the anchor path alone, with the workspace that splits its last wave
+        # of tiles and, for comparison, every tile whole
+        a_ws = anchor_workspace(torch, C, q, wd, len(rep_heads))
         anchor_ms = max_over_ranks(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
+                                                  list(rep_heads), workspace=a_ws, stream=stream),
+            max(3, args.steps // 4), 2, stream)), dist, "cuda")
+        anchor_whole_ms = max_over_ranks(statistics.mean(time_calls(
             torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
                                                   list(rep_heads), stream=stream),
             max(3, args.steps // 4), 2, stream)), dist, "cuda")
+        del a_ws
         d_dual.close()
         bcast_bytes = len(rep_heads) * wd.seq_len * wd.head_dim * 2
+        anchor_tf = anchor_tiles * FLOP_PER_TILE / (anchor_ms * 1e-3) / 1e12
         extras["dual_path_720p"] = {
             "ms_per_call": dual_ms, "launches": 1, "two_launch_ms_per_call": two_ms,
             "effective_tflops": (dual_tiles + anchor_tiles) * FLOP_PER_TILE / (dual_ms * 1e-3) / 1e12,
             "anchor_heads": len(rep_heads), "anchor_ms": anchor_ms,
-            "anchor_effective_tflops": anchor_tiles * FLOP_PER_TILE / (anchor_ms * 1e-3) / 1e12,
-            "anchor_output_bytes": bcast_bytes}
+            "anchor_effective_tflops": anchor_tf, "anchor_frac_of_burst_peak": anchor_tf / pk["bf16_tflops"],
+            "anchor_whole_tiles_ms": anchor_whole_ms, "anchor_output_bytes": bcast_bytes}
         # offline calibration: block energies of the dense attention (two Q K^T passes on the tensor cores)
         e_out = torch.empty((1, wl.heads, wl.num_blocks, wl.num_blocks), device="cuda")
         e_ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, device="cuda")

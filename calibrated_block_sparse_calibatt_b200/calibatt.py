@@ -80,7 +80,10 @@ SIGNATURES = {
     "calibatt_block_sparse_attn_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32,
                                                _i32, _f32, _vp, _vp]),
     "calibatt_anchor_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _i32, _i32, _i32, _vp, _i32, _vp,
-                                    _i32, _f32, _vp]),
+                                    _i32, _f32, _vp, ctypes.c_size_t, _vp]),
+    "calibatt_anchor_attn_workspace_size": (_i32, [_P(Shape), _i32, _i32, _i32, _i32, _i32,
+                                                   _P(ctypes.c_size_t)]),
+    "calibatt_anchor_split_plan": (_i32, [_i64, _i32, _i32, _P(_i64), _P(_i32)]),
     "calibatt_dual_path_attn": (_i32, [_vp, _vp, _vp, _vp, _P(Shape), _i32, _vp, _i32, _i32, _i32, _i32, _i32,
                                        _vp, _i32, _f32, _vp, _vp]),
     "calibatt_block_energy_workspace_size": (_i32, [_P(Shape), _P(ctypes.c_size_t)]),
@@ -377,13 +380,34 @@ def calibatt_block_sparse_attn_csr(q, k, v, o, row_ptr, col_idx, col_base, head_
 
 
 def calibatt_anchor_attn(q, k, v, o, frames, rows, cols, anchor_rows, head_ids, block=128, softmax_scale=0.0,
-                         stream=None):
+                         workspace=None, stream=None):
+    """Anchor-row attention with broadcast for head_ids; workspace (a device
+    tensor of at least calibatt_anchor_attn_workspace_size bytes) lets the
+    call split its last partial wave of tiles over key ranges."""
     shape = shape_of(q)
     a = _i32_array(anchor_rows)
     h = _i32_array(head_ids)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     check(LIB.calibatt_anchor_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shape), block, frames, rows,
                                    cols, _ptr(a), a.size, _ptr(h) if h.size else None, h.size,
-                                   float(softmax_scale), _stream(stream)))
+                                   float(softmax_scale), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def calibatt_anchor_attn_workspace_size(q, frames, rows, cols, n_anchors, n_heads) -> int:
+    shape = shape_of(q)
+    n = ctypes.c_size_t(0)
+    check(LIB.calibatt_anchor_attn_workspace_size(ctypes.byref(shape), frames, rows, cols, n_anchors, n_heads,
+                                                  ctypes.byref(n)))
+    return n.value
+
+
+def anchor_split_plan(tiles, grid, key_blocks):
+    """(first, parts): the anchor call's split of its last wave of tiles."""
+    first = ctypes.c_int64(0)
+    parts = ctypes.c_int32(0)
+    check(LIB.calibatt_anchor_split_plan(int(tiles), int(grid), int(key_blocks), ctypes.byref(first),
+                                         ctypes.byref(parts)))
+    return first.value, parts.value
 
 
 def calibatt_dual_path_attn(q, k, v, o, d: MaskDictionary, t, l, frames, rows, cols, anchor_rows, block=128,

@@ -543,10 +543,55 @@ calibatt_status launch_sparse(const void* q, const void* k, const void* v, void*
   return run_sparse(q, k, v, o, s, block, sch, d->G, heads, softmax_scale, lse, stream);
 }
 
+// Split plan of the anchor-only launch: `tiles` equal anchor tiles on `grid`
+// persistent CTAs leave a last partial wave of r = tiles mod grid tiles (all
+// of them when tiles < grid).  Cut into s key ranges each, that wave takes
+// ceil(r s / grid) / s of a tile's time instead of a whole tile's.  s runs
+// over 1..4, each part keeping at least two key blocks; the smallest s with
+// the shortest wave wins.  The split tiles are the last r of the sequence.
+void anchor_split_plan(int64_t tiles, int64_t grid, int32_t nb, int64_t& first, int32_t& parts) {
+  parts = 1;
+  first = tiles;
+  if (grid <= 0 || tiles <= 0) return;
+  const int64_t r = tiles % grid;
+  if (r == 0) return;
+  int64_t best_num = 1, best_den = 1;  // the wave as it is: one tile's time
+  for (int32_t sp = 2; sp <= 4 && nb >= 2 * sp; ++sp) {
+    const int64_t num = (r * sp + grid - 1) / grid;
+    if (num * best_den < best_num * sp) {
+      best_num = num;
+      best_den = sp;
+      parts = sp;
+    }
+  }
+  if (parts > 1) first = tiles - r;
+}
+
+// Byte layout of the anchor split workspace: partial outputs, (m, l) pairs and
+// counters, each region 256-byte aligned.
+struct SplitLayout {
+  size_t o_bytes, ml_bytes, cnt_bytes, total;
+};
+SplitLayout split_layout(int64_t slots, int32_t parts, int32_t head_dim) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  SplitLayout L;
+  L.o_bytes = up(static_cast<size_t>(slots) * parts * 8 * (head_dim / 2) * 32 * sizeof(float));
+  L.ml_bytes = up(static_cast<size_t>(slots) * parts * 8 * 32 * 2 * sizeof(float));
+  L.cnt_bytes = up(static_cast<size_t>(slots) * 8 * sizeof(uint32_t));
+  L.total = slots > 0 && parts > 1 ? L.o_bytes + L.ml_bytes + L.cnt_bytes : 0;
+  return L;
+}
+
+// Tiles of one anchor-only call (batch x heads x tiles per head).
+int64_t anchor_call_tiles(const calibatt_shape& s, int32_t frames, int32_t cols, int32_t n_anchors, int32_t n_heads) {
+  const int64_t per_head = (static_cast<int64_t>(frames) * n_anchors * cols + 127) / 128;
+  return static_cast<int64_t>(s.batch) * n_heads * per_head;
+}
+
 calibatt_status launch_anchor(const void* q, const void* k, const void* v, void* o, const calibatt_shape& s,
                               int32_t block, int32_t frames, int32_t rows, int32_t cols, const int32_t* anchors,
                               int32_t n_anchors, const int32_t* head_ids, int32_t n_heads, float softmax_scale,
-                              cudaStream_t stream) {
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (frames < 1 || rows < 1 || cols < 1)
     return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows and cols must be >= 1");
   if (static_cast<int64_t>(frames) * rows * cols != s.seq_len)
@@ -603,7 +648,31 @@ calibatt_status launch_anchor(const void* q, const void* k, const void* v, void*
     p.timeout_ns = g_timeout_ns.load();
     const int sms = device_sm_count();
     if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
-    const int64_t items = static_cast<int64_t>(n_heads) * g.tiles_per_head;
+    const int64_t tiles = anchor_call_tiles(s, frames, cols, n_anchors, n_heads);
+    if (tiles > (int64_t{1} << 28)) return fail(CALIBATT_ERR_UNSUPPORTED, "more than 2^28 anchor tiles in one call");
+    int64_t first = tiles;
+    int32_t parts = 1;
+    if (workspace != nullptr) anchor_split_plan(tiles, sms, p.nb, first, parts);
+    const SplitLayout sl = split_layout(tiles - first, parts, s.head_dim);
+    p.split.first = static_cast<int32_t>(first);
+    p.split.parts = parts;
+    p.split.n_tiles = static_cast<int32_t>(tiles);
+    if (parts > 1) {
+      if (reinterpret_cast<uintptr_t>(workspace) % 256)
+        return fail(CALIBATT_ERR_INVALID_ARG, "the anchor workspace must be 256-byte aligned");
+      if (workspace_bytes < sl.total)
+        return fail(CALIBATT_ERR_INVALID_ARG, "anchor workspace of %zu bytes, this call needs %zu", workspace_bytes,
+                    sl.total);
+      uint8_t* w = static_cast<uint8_t*>(workspace);
+      p.split.o = reinterpret_cast<float*>(w);
+      p.split.ml = reinterpret_cast<float2*>(w + sl.o_bytes);
+      p.split.cnt = reinterpret_cast<uint32_t*>(w + sl.o_bytes + sl.ml_bytes);
+      if (cudaMemsetAsync(p.split.cnt, 0, sl.cnt_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(CALIBATT_ERR_CUDA, "anchor split counter reset failed");
+      }
+    }
+    const int64_t items = first + (tiles - first) * parts;
     const int grid = static_cast<int>(std::min<int64_t>(sms, items));
     cudaError_t e = calibatt::launch_tc_attn(p, s.head_dim, calibatt::kModeAnchor, grid, stream);
     if (e != cudaSuccess) return cuda_fail(e, "anchor tensor-core launch");
@@ -1743,14 +1812,48 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
 calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
                                      const calibatt_shape* shape, int32_t block, int32_t frames, int32_t rows,
                                      int32_t cols, const int32_t* anchor_rows, int32_t n_anchors,
-                                     const int32_t* head_ids, int32_t n_heads, float softmax_scale, void* stream) {
+                                     const int32_t* head_ids, int32_t n_heads, float softmax_scale,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
   return guarded([&]() -> calibatt_status {
     calibatt_status st;
     if ((st = check_shape(shape)) != CALIBATT_OK) return st;
     if ((st = check_ptrs(q, k, v, o)) != CALIBATT_OK) return st;
     if ((st = check_block(block)) != CALIBATT_OK) return st;
     return launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, head_ids, n_heads,
-                         softmax_scale, static_cast<cudaStream_t>(stream));
+                         softmax_scale, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  });
+}
+
+calibatt_status calibatt_anchor_attn_workspace_size(const calibatt_shape* shape, int32_t frames, int32_t rows,
+                                                    int32_t cols, int32_t n_anchors, int32_t n_heads, size_t* bytes) {
+  return guarded([&]() -> calibatt_status {
+    calibatt_status st;
+    if ((st = check_shape(shape)) != CALIBATT_OK) return st;
+    if (!bytes) return fail(CALIBATT_ERR_INVALID_ARG, "bytes is NULL");
+    if (frames < 1 || rows < 1 || cols < 1 || n_anchors < 1 || n_anchors > calibatt::kMaxAnchors || n_heads < 0 ||
+        n_heads > calibatt::kMaxHeadsPerCall)
+      return fail(CALIBATT_ERR_INVALID_ARG, "frames, rows, cols, n_anchors or n_heads out of range");
+    *bytes = 0;
+    if (shape->dtype != CALIBATT_DTYPE_BF16 || n_heads == 0) return CALIBATT_OK;
+    const int sms = device_sm_count();
+    if (sms < 1) return fail(CALIBATT_ERR_CUDA, "cannot query the SM count");
+    int64_t first = 0;
+    int32_t parts = 1;
+    const int64_t tiles = anchor_call_tiles(*shape, frames, cols, n_anchors, n_heads);
+    anchor_split_plan(tiles, sms, ceil_div(shape->seq_len, 128), first, parts);
+    *bytes = split_layout(tiles - first, parts, shape->head_dim).total;
+    return CALIBATT_OK;
+  });
+}
+
+calibatt_status calibatt_anchor_split_plan(int64_t tiles, int32_t grid, int32_t key_blocks, int64_t* first,
+                                           int32_t* parts) {
+  return guarded([&]() -> calibatt_status {
+    if (!first || !parts) return fail(CALIBATT_ERR_INVALID_ARG, "first and parts must be non-NULL");
+    if (tiles < 0 || grid < 1 || key_blocks < 1)
+      return fail(CALIBATT_ERR_INVALID_ARG, "tiles >= 0, grid >= 1 and key_blocks >= 1 are required");
+    anchor_split_plan(tiles, grid, key_blocks, *first, *parts);
+    return CALIBATT_OK;
   });
 }
 
@@ -1794,7 +1897,7 @@ calibatt_status calibatt_dual_path_attn(const void* q, const void* k, const void
     for (size_t h0 = 0; h0 < heads.size(); h0 += calibatt::kMaxHeadsPerCall) {
       const int32_t nh = static_cast<int32_t>(std::min<size_t>(calibatt::kMaxHeadsPerCall, heads.size() - h0));
       st = launch_anchor(q, k, v, o, *shape, block, frames, rows, cols, anchor_rows, n_anchors, heads.data() + h0, nh,
-                         softmax_scale, static_cast<cudaStream_t>(stream));
+                         softmax_scale, nullptr, 0, static_cast<cudaStream_t>(stream));
       if (st != CALIBATT_OK) return st;
     }
     return CALIBATT_OK;

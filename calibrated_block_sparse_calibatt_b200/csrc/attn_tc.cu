@@ -216,7 +216,19 @@ struct Item {
   const uint16_t* cols;      // retained key blocks (index lists), nullptr = bitmap row or 0..n-1
   bool ragged_last;          // last visited key block is the partial one
   bool anchor;               // anchor-row tile (gathered queries, broadcast epilogue)
+  int part;                  // key-range part of a split anchor tile: slot * 4 + part; -1 = whole
 };
+
+// Key-block indices 0, 1, ..., 65535, built at compile time: a key-range part
+// of a split anchor tile visits blocks k0 .. k1 - 1 as the list starting at
+// entry k0, so the producers walk it like any retained-block list.
+struct KeyIdentity {
+  uint16_t v[65536];
+  constexpr KeyIdentity() : v() {
+    for (int i = 0; i < 65536; ++i) v[i] = static_cast<uint16_t>(i);
+  }
+};
+__device__ const KeyIdentity g_key_identity;
 
 
 // Row (head h, query block r) of a bitmap dictionary layer.
@@ -241,8 +253,9 @@ struct Cursor {
     fetcher = is_fetcher;
     b = 0;
     if (MODE == kModeAnchor) {
+      // one item sequence over batch x heads x tiles, the split parts last
       begin = blockIdx.x;
-      end = p.anc.n_heads * p.anc.tiles_per_head;
+      end = p.split.first + (p.split.n_tiles - p.split.first) * p.split.parts;
       step = gridDim.x;
     } else if (calibration_mode(MODE)) {
       begin = blockIdx.x;
@@ -285,6 +298,36 @@ struct Cursor {
     return t < static_cast<uint32_t>(p.batch) * static_cast<uint32_t>(p.sched.n_order);
   }
   __device__ bool next(const TcParams& p, Item& it, const Waiter& W) {
+    if (MODE == kModeAnchor) {
+      if (idx >= end) return false;
+      int t = idx, part = -1, slot = 0;
+      if (idx >= p.split.first) {
+        slot = (idx - p.split.first) / p.split.parts;
+        part = (idx - p.split.first) % p.split.parts;
+        t = p.split.first + slot;
+      }
+      const int per_b = p.anc.n_heads * p.anc.tiles_per_head;
+      it.b = t / per_b;
+      const int r = t % per_b;
+      it.h = p.anc.head_ids[r / p.anc.tiles_per_head];
+      it.tile = r % p.anc.tiles_per_head;
+      it.anchor = true;
+      if (part < 0) {
+        it.n = p.nb;
+        it.cols = nullptr;
+        it.ragged_last = (p.seq_len % 128) != 0;
+        it.part = -1;
+      } else {
+        const int k0 = p.nb * part / p.split.parts, k1 = p.nb * (part + 1) / p.split.parts;
+        it.n = k1 - k0;
+        it.cols = g_key_identity.v + k0;
+        it.ragged_last = k1 == p.nb && (p.seq_len % 128) != 0;
+        it.part = slot * 4 + part;
+      }
+      idx += step;
+      return true;
+    }
+    it.part = -1;
     while (b < p.batch) {
       uint32_t t_dyn = 0;
       const bool dyn = dynamic(p);
@@ -307,16 +350,11 @@ struct Cursor {
           idx += step;
           return true;
         }
-        if (MODE != kModeAnchor) w = dyn ? p.sched.order[idx] : p.sched.items[idx];
-        if (MODE == kModeAnchor || (MODE == kModeFused && (w & kItemAnchorBit))) {
+        w = dyn ? p.sched.order[idx] : p.sched.items[idx];
+        if (MODE == kModeFused && (w & kItemAnchorBit)) {
           it.anchor = true;
-          if (MODE == kModeAnchor) {
-            it.h = p.anc.head_ids[idx / p.anc.tiles_per_head];
-            it.tile = idx % p.anc.tiles_per_head;
-          } else {
-            it.h = static_cast<int>((w >> 16) & 0x7FFFu);
-            it.tile = static_cast<int>(w & 0xFFFFu);
-          }
+          it.h = static_cast<int>((w >> 16) & 0x7FFFu);
+          it.tile = static_cast<int>(w & 0xFFFFu);
           it.n = p.nb;
           it.cols = nullptr;
           it.ragged_last = (p.seq_len % 128) != 0;
@@ -856,7 +894,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
     const float m = fmaxf(m_own, m_o);
     const float l_row = (m_own == -INFINITY ? 0.f : l * fast_exp2(m_own - m)) +
                         (m_o == -INFINITY ? 0.f : l_o * fast_exp2(m_o - m));
-    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+    float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
     const int64_t bh_off = static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
     // Destination rows of this thread's output.
     int64_t dst_token = -1;
@@ -877,6 +915,62 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       if (token < p.seq_len) {
         dst_token = token;
         n_dst = 1;
+      }
+    }
+    // A key-range part of a split anchor tile (anchor-only launch): this
+    // warp's 32 rows x HD/2 columns of O and the rows' (m, l) go to the
+    // workspace, float32, coalesced (column-major over the warp's rows);
+    // after a fence the warp counts itself in.  The warp that completes the
+    // (tile, rows, half) merges every part in part order -- so the result does
+    // not depend on which part ends last -- and writes the output below; the
+    // others write nothing.  No warp ever waits for another CTA.
+    [[maybe_unused]] bool merge = false;
+    [[maybe_unused]] float w_part[4] = {0.f, 0.f, 0.f, 0.f};
+    [[maybe_unused]] int64_t rec0 = 0;
+    if (MODE == kModeAnchor && it.part >= 0) {
+      const int parts = p.split.parts, slot = it.part >> 2, part = it.part & 3;
+      const int qs = quarter * 2 + s;  // this warp's rows (quarter) and column half (stream)
+      rec0 = static_cast<int64_t>(slot) * parts * 8 + qs;  // record of part i: rec0 + 8 * i
+      const int64_t rec = rec0 + 8 * part;
+      float* po = p.split.o + rec * (HD / 2) * 32 + lane;
+#pragma unroll 1
+      for (int ch = 0; ch < HD / 64; ++ch) {
+        uint32_t o[32];
+        tmem_ld_x32(tO + s * (HD / 2) + ch * 32, o);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) po[(ch * 32 + c) * 32] = __uint_as_float(o[c]);
+      }
+      p.split.ml[rec * 32 + lane] = make_float2(m, l_row);
+      __threadfence();
+      __syncwarp();
+      uint32_t arrived = 0;
+      if (lane == 0) arrived = atomicAdd(p.split.cnt + static_cast<int64_t>(slot) * 8 + qs, 1u);
+      arrived = __shfl_sync(0xFFFFFFFFu, arrived, 0);
+      merge = arrived == static_cast<uint32_t>(parts - 1);
+      if (!merge) {
+        n_dst = 0;
+      } else {
+        __threadfence();
+        float mi[4], li[4];
+        float mm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mi[i] = -INFINITY;
+          li[i] = 0.f;
+          if (i < parts) {
+            const float2 v = i == part ? make_float2(m, l_row) : __ldcg(p.split.ml + (rec0 + 8 * i) * 32 + lane);
+            mi[i] = v.x;
+            li[i] = v.y;
+            mm = fmaxf(mm, v.x);
+          }
+        }
+        float lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          w_part[i] = (i < parts && mi[i] != -INFINITY) ? fast_exp2(mi[i] - mm) : 0.f;
+          lsum = fmaf(w_part[i], li[i], lsum);
+        }
+        inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
       }
     }
 #ifdef CALIBATT_TRACE
@@ -959,6 +1053,27 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0u;
+      }
+      if (MODE == kModeAnchor && merge) {
+        // sum over the parts in part order (this part's values from tensor
+        // memory are the ones it wrote)
+        const int parts = p.split.parts, part = it.part & 3;
+        float acc[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i < parts) {
+            const float* src = p.split.o + (rec0 + 8 * i) * (HD / 2) * 32 + (ch * 32) * 32 + lane;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float x = i == part ? __uint_as_float(o[c]) : __ldcg(src + c * 32);
+              acc[c] = fmaf(w_part[i], x, acc[c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(acc[c]);
       }
       uint4 pkd[4];
 #pragma unroll

@@ -77,6 +77,23 @@ struct AnchorGeom {
   int16_t head_ids[kMaxHeadsPerCall];
 };
 
+// Anchor-only launch: the last tiles of the item sequence split into key
+// ranges, so that the persistent grid ends together.  Items [0, first) are
+// whole tiles; item first + e is part e % parts of tile first + e / parts
+// (keys [nb * part / parts, nb * (part + 1) / parts)).  Each softmax warp of a
+// part writes its rows x column half of O (float32, relative to its maximum)
+// and (maximum, row sum) to the workspace, then counts itself in; the warp
+// that completes a (tile, rows, half) merges the parts in part order and
+// writes the output.  parts == 1: no split (first == n_tiles).
+struct AnchorSplit {
+  int32_t first;    // whole tiles before the split ones
+  int32_t parts;    // key ranges per split tile, 1..4
+  int32_t n_tiles;  // tiles over batch x heads x tiles per head
+  float* o;         // [slot][part][8 warps][HD / 2 columns][32 rows]
+  float2* ml;       // [slot][part][8 warps][32 rows] (maximum, row sum), exp2 domain
+  uint32_t* cnt;    // [slot][8 warps] parts counted in, zeroed before the launch
+};
+
 // Tensor-core (tcgen05) attention kernel parameters, passed as __grid_constant__.
 struct TcParams {
   CUtensorMap tm_q;  // bf16 Q/K/V, dims {D, x1, x2, x3}, box {64, 1|128, ...}
@@ -92,6 +109,7 @@ struct TcParams {
   float scale_log2;             // softmax_scale * log2(e)
   LayerSchedule sched;
   AnchorGeom anc;
+  AnchorSplit split;  // anchor-only mode
   int32_t* status;
   unsigned long long timeout_ns;
 };

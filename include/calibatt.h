@@ -361,13 +361,48 @@ calibatt_status calibatt_block_sparse_attn_csr(const void* q, const void* k, con
  *   anchor_rows: host int32[n_anchors], strictly ascending in [0, rows),
  *     1 <= n_anchors <= 16;
  *   head_ids: host int32[n_heads], distinct heads in [0, heads), n_heads <= 128.
+ *   workspace: NULL, or caller-owned device scratch of at least
+ *     calibatt_anchor_attn_workspace_size() bytes, 256-byte aligned.  With it
+ *     (bf16) the last, partial wave of anchor tiles on the persistent grid is
+ *     cut into key ranges that run on different SMs and are merged exactly
+ *     (per-range maximum and row sum, float32 partial outputs, summed in
+ *     range order by whichever SM finishes a tile's last range), so the grid
+ *     ends together; the result is deterministic, and differs from the
+ *     unsplit tiles' only by float32 rounding.  Without it every tile runs
+ *     whole.  The call zeroes the workspace's counters on `stream`; calls in
+ *     flight together need workspaces of their own.  A workspace smaller
+ *     than this call's need is CALIBATT_ERR_INVALID_ARG.
  * Every token of the listed heads is written. */
 calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v, void* o,
                                      const calibatt_shape* shape, int32_t block,
                                      int32_t frames, int32_t rows, int32_t cols,
                                      const int32_t* anchor_rows, int32_t n_anchors,
                                      const int32_t* head_ids, int32_t n_heads,
-                                     float softmax_scale, void* stream);
+                                     float softmax_scale, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Device scratch bytes calibatt_anchor_attn uses to split its last wave of
+ * tiles, for `shape` and n_heads listed heads on the current device (its SM
+ * count sizes the persistent grid); 0 when the call would not split (no
+ * partial wave, fewer than four key blocks, or float32 inputs).  The
+ * workspace holds, per split tile and key range, 128 x head_dim float32
+ * partial outputs and 128 (maximum, row sum) pairs, and 8 counters per
+ * split tile.  No counterpart in the pages: a scheduling device of this
+ * implementation (Key Designs 3 defines the operation). */
+calibatt_status calibatt_anchor_attn_workspace_size(const calibatt_shape* shape, int32_t frames,
+                                                    int32_t rows, int32_t cols, int32_t n_anchors,
+                                                    int32_t n_heads, size_t* bytes);
+
+/* The split plan calibatt_anchor_attn follows (host only, no device):
+ * `tiles` equal anchor tiles on `grid` persistent CTAs leave r = tiles mod
+ * grid tiles in a last partial wave; each is cut into `parts` key ranges,
+ * parts in 1..4 minimising ceil(r * parts / grid) / parts (the smallest on
+ * ties, each range at least two of the key_blocks blocks).  The split tiles
+ * are the last r of the call's sequence (batch, then listed head, then
+ * tile): *first = tiles - r, or *first = tiles and *parts = 1 when nothing is
+ * split.  No counterpart in the pages. */
+calibatt_status calibatt_anchor_split_plan(int64_t tiles, int32_t grid, int32_t key_blocks,
+                                           int64_t* first, int32_t* parts);
 
 /* Both paths of record (t, l): the dictionary's repetitive heads through the
  * anchor path and the rest through the block-sparse path, enqueued on one

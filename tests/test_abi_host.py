@@ -102,29 +102,32 @@ def test_hot_path_rejects_bad_arguments_before_any_gpu_work(calibatt_lib):
     assert st == C.ERR_INVALID_ARG and "dictionary" in C.last_error()
     # unsupported head_dim
     bad = C.Shape(1, 256, 2, 96, 256 * 2 * 96, 2 * 96, 96, C.DTYPE_FP32, 0)
-    st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(bad), 64, 2, 8, 16, None, 0, None, 0, 0.0, None)
+    st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(bad), 64, 2, 8, 16, None, 0, None, 0, 0.0,
+                                None, 0, None)
     assert st == C.ERR_UNSUPPORTED
     # unsupported block
-    st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(shape), 32, 2, 8, 16, None, 0, None, 0, 0.0, None)
+    st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(shape), 32, 2, 8, 16, None, 0, None, 0, 0.0,
+                                None, 0, None)
     assert st == C.ERR_UNSUPPORTED
     # null q
-    st = L.calibatt_anchor_attn(None, buf, buf, buf, ctypes.byref(shape), 64, 2, 8, 16, None, 0, None, 0, 0.0, None)
+    st = L.calibatt_anchor_attn(None, buf, buf, buf, ctypes.byref(shape), 64, 2, 8, 16, None, 0, None, 0, 0.0,
+                                None, 0, None)
     assert st == C.ERR_INVALID_ARG
     # frames*rows*cols != seq_len
     anchors = (ctypes.c_int32 * 2)(0, 4)
     heads = (ctypes.c_int32 * 1)(1)
     st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(shape), 64, 2, 8, 15, anchors, 2, heads, 1, 0.0,
-                                None)
+                                None, 0, None)
     assert st == C.ERR_INVALID_ARG and "seq_len" in C.last_error()
     # anchors not ascending
     anchors_bad = (ctypes.c_int32 * 2)(4, 0)
     st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(shape), 64, 2, 8, 16, anchors_bad, 2, heads, 1,
-                                0.0, None)
+                                0.0, None, 0, None)
     assert st == C.ERR_INVALID_ARG
     # misaligned bf16 stride
     s2 = C.Shape(1, 256, 2, 64, 256 * 2 * 64, 2 * 64 + 4, 64, C.DTYPE_BF16, 0)
     st = L.calibatt_anchor_attn(buf, buf, buf, buf, ctypes.byref(s2), 128, 2, 8, 16, anchors, 2, heads, 1, 0.0,
-                                None)
+                                None, 0, None)
     assert st == C.ERR_INVALID_ARG
     # select / aggregate argument checks
     assert L.calibatt_select_blocks(buf, 1, 5000, ctypes.c_float(0.9), buf, None, None) == C.ERR_UNSUPPORTED
@@ -231,3 +234,29 @@ def test_count_intervals_matches_the_library_encoding(calibatt_lib):
         total += len(start)
         off += n
     assert C.count_intervals(rp, ci) == total
+
+
+def test_anchor_split_plan_shortens_the_last_wave(calibatt_lib):
+    """The anchor call's split of its last partial wave: against every choice
+    of 1..4 key ranges (brute force), the plan's last wave is the shortest
+    one, the smallest such count wins, each range keeps two key blocks, and
+    the split tiles are the last tiles % grid of the sequence."""
+    C = calibatt_lib
+    for tiles in (1, 5, 74, 75, 147, 148, 149, 200, 222, 230, 260, 295, 296, 330, 792, 2640, 10 ** 6 + 3):
+        for grid in (1, 7, 148):
+            for nb in (1, 3, 4, 6, 7, 8, 591):
+                first, parts = C.anchor_split_plan(tiles, grid, nb)
+                r = tiles % grid
+                wave = {s: -(-r * s // grid) / s for s in range(1, 5) if s == 1 or nb >= 2 * s}
+                best = min(wave.values()) if r else 1.0
+                if r == 0 or wave[1] == best:
+                    assert (first, parts) == (tiles, 1), (tiles, grid, nb)
+                    continue
+                assert parts == min(s for s, w in wave.items() if w == best), (tiles, grid, nb)
+                assert first == tiles - r and nb >= 2 * parts
+    # the dual-path 720p layer's 12 anchor heads: 792 tiles on 148 SMs -> the
+    # last 52 tiles in halves (a wave of half a tile instead of a whole one)
+    assert C.anchor_split_plan(792, 148, 591) == (740, 2)
+    assert C.anchor_split_plan(10, 148, 591) == (0, 4)     # fewer tiles than SMs: quarters
+    with pytest.raises(C.CalibattError):
+        C.anchor_split_plan(10, 0, 591)

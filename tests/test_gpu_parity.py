@@ -182,6 +182,63 @@ def test_tc_anchor_broadcast(C):
         assert torch.equal(o[:, :, rho, :, [0, 2]], o[:, :, near[rho], :, [0, 2]])
 
 
+@pytest.mark.parametrize("batch,heads,d", [(1, 22, 128), (1, 33, 128), (2, 11, 64)])
+def test_tc_anchor_split_last_wave(C, batch, heads, d):
+    """With a workspace the anchor call cuts its last partial wave of tiles
+    into key ranges and merges them exactly: every listed head matches the
+    oracle; whole tiles are bitwise those of the call without a workspace and
+    split tiles agree with them to rounding; a repeated call is bitwise equal
+    (the merge sums the ranges in range order, whichever ends last); broadcast
+    rows are bitwise copies of their anchors; the workspace's counters are
+    reset by the call (it starts as NaN bytes).  N = 3600: 29 key blocks, the
+    last of 16 tokens; 7 anchor tiles per head, the last of 32 queries."""
+    frames, rows, cols, anchors = 4, 9, 100, (2, 6)
+    n = frames * rows * cols
+    nb, tph = O.num_blocks(n, 128), -(-frames * len(anchors) * cols // 128)
+    q, k, v = W.make_qkv(71 + heads, batch, n, heads, d, "bf16", 1.0, "cuda")
+    head_ids = list(np.random.default_rng(heads).permutation(heads))
+    tiles = batch * heads * tph
+    first, parts = C.anchor_split_plan(tiles, C.device_sm_count(), nb)
+    assert parts > 1 and first < tiles, "this case must split its last wave"
+    nbytes = C.calibatt_anchor_attn_workspace_size(q, frames, rows, cols, len(anchors), heads)
+    assert nbytes > 0
+    ws = torch.full((nbytes // 4,), float("nan"), device="cuda")
+    with pytest.raises(C.CalibattError):          # too small
+        C.calibatt_anchor_attn(q, k, v, torch.empty_like(q), frames, rows, cols, anchors, head_ids,
+                               workspace=ws[:-64])
+    with pytest.raises(C.CalibattError):          # not 256-byte aligned
+        C.calibatt_anchor_attn(q, k, v, torch.empty_like(q), frames, rows, cols, anchors, head_ids,
+                               workspace=ws[1:])
+    split = torch.full_like(q, float("nan"))
+    whole = torch.full_like(q, float("nan"))
+    C.calibatt_anchor_attn(q, k, v, split, frames, rows, cols, anchors, head_ids, workspace=ws)
+    C.calibatt_anchor_attn(q, k, v, whole, frames, rows, cols, anchors, head_ids)
+    again = torch.full_like(q, float("nan"))
+    C.calibatt_anchor_attn(q, k, v, again, frames, rows, cols, anchors, head_ids, workspace=ws)
+    _check_status(C)
+    assert not torch.isnan(split).any()
+    assert torch.equal(split, again)
+    ref = O.anchor_attention_bnhd(_np(q), _np(k), _np(v), frames, rows, cols, anchors)
+    _assert_close(_np(split), ref, "bf16")
+    # the tokens of the split tiles: item t = (batch, listed head, tile) for t >= first
+    near = O.nearest_anchor_rows(rows, anchors)
+    a_of_row = np.array([list(anchors).index(near[r]) for r in range(rows)])
+    f, rho, w = np.meshgrid(np.arange(frames), np.arange(rows), np.arange(cols), indexing="ij")
+    tile_of_token = torch.as_tensor(((f * len(anchors) + a_of_row[rho]) * cols + w).reshape(-1) // 128)
+    in_split = torch.zeros((batch, n, heads), dtype=torch.bool)
+    for t in range(first, tiles):
+        b, r = divmod(t, heads * tph)
+        in_split[b, :, head_ids[r // tph]] |= tile_of_token == r % tph
+    in_split = in_split.cuda()
+    assert in_split.any() and not in_split.all()
+    assert torch.equal(split[~in_split], whole[~in_split])
+    diff = (split[in_split].float() - whole[in_split].float()).abs().max().item()
+    assert diff <= 1e-2, diff
+    o = split.view(batch, frames, rows, cols, heads, d)
+    for r in range(rows):
+        assert torch.equal(o[:, :, r], o[:, :, near[r]])
+
+
 def test_simt_anchor_fp32(C):
     frames, rows, cols, h, d = 2, 9, 16, 2, 64
     n = frames * rows * cols
