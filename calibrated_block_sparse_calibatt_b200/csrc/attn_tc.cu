@@ -458,38 +458,28 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
         // Gather this tile's 128 anchor-row queries into the 128-byte swizzled
         // K-major layout the MMA expects (16-byte unit u of row r lands at
         // chunk u/8, row r, position (u%8) ^ (r%8)).
+        // Every copy is an asynchronous 16-byte global -> shared copy, all of
+        // them in flight at once (no registers hold the data; the producer
+        // warpgroup has 40 per thread); queries past the anchor tokens are
+        // zero-filled.
         constexpr int kUnits = HD / 8;
         const int per_frame = p.anc.n_anchors * p.anc.cols;
         const uint16_t* qb = p.q + static_cast<int64_t>(it.b) * p.sb + static_cast<int64_t>(it.h) * p.sh;
-        // Two 16-byte loads in flight per lane before their stores (the
-        // producer warpgroup has 40 registers per thread).
-        constexpr int kBatch = 2;
-        static_assert((128 * kUnits) % (32 * kBatch) == 0, "gather batches");
-        for (int i0 = lane; i0 < 128 * kUnits; i0 += 32 * kBatch) {
-          uint4 val[kBatch];
-#pragma unroll
-          for (int e = 0; e < kBatch; ++e) {
-            const int idx = i0 + 32 * e;
-            const int r = idx / kUnits, u = idx % kUnits;
-            const int pq = it.tile * 128 + r;
-            val[e] = make_uint4(0u, 0u, 0u, 0u);
-            if (pq < p.anc.anchor_tokens) {
-              const int f = pq / per_frame, rem = pq % per_frame;
-              const int a = rem / p.anc.cols, w = rem % p.anc.cols;
-              const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + p.anc.anchor_row[a]) * p.anc.cols + w;
-              val[e] = __ldg(reinterpret_cast<const uint4*>(qb + token * p.sn + u * 8));
-            }
+        for (int idx = lane; idx < 128 * kUnits; idx += 32) {
+          const int r = idx / kUnits, u = idx % kUnits;
+          const int pq = it.tile * 128 + r;
+          const uint16_t* src = qb;
+          uint32_t bytes = 0;
+          if (pq < p.anc.anchor_tokens) {
+            const int f = pq / per_frame, rem = pq % per_frame;
+            const int a = rem / p.anc.cols, w = rem % p.anc.cols;
+            const int64_t token = (static_cast<int64_t>(f) * p.anc.rows + p.anc.anchor_row[a]) * p.anc.cols + w;
+            src = qb + token * p.sn + u * 8;
+            bytes = 16;
           }
-#pragma unroll
-          for (int e = 0; e < kBatch; ++e) {
-            const int idx = i0 + 32 * e;
-            const int r = idx / kUnits, u = idx % kUnits;
-            const uint32_t dst = base + L::kQ + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val[e].x), "r"(val[e].y),
-                         "r"(val[e].z), "r"(val[e].w)
-                         : "memory");
-          }
+          cp_async_16(base + L::kQ + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4), src, bytes);
         }
+        cp_async_wait_all();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::bQFull));
@@ -504,13 +494,11 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
           for (int idx = lane; idx < 128 * kUnits; idx += 32) {
             const int r = idx / kUnits, u = idx % kUnits;
             const int64_t tok = static_cast<int64_t>(it.tile) * 128 + r;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (tok < p.seq_len) val = __ldg(reinterpret_cast<const uint4*>(qb + partner_token(p.anc, tok) * p.sn + u * 8));
-            const uint32_t dst = base + L::kV + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(val.x), "r"(val.y), "r"(val.z),
-                         "r"(val.w)
-                         : "memory");
+            const bool in = tok < p.seq_len;
+            cp_async_16(base + L::kV + (u >> 3) * kChunkBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4),
+                        in ? qb + partner_token(p.anc, tok) * p.sn + u * 8 : qb, in ? 16u : 0u);
           }
+          cp_async_wait_all();
           fence_proxy_async_smem();
           __syncwarp();
         }

@@ -177,6 +177,13 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
+// 16-byte asynchronous copy global -> shared (LDGSTS); src_bytes 0 fills the
+// 16 bytes with zeros without reading.  Completion: cp_async_wait_all().
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
