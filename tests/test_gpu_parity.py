@@ -182,17 +182,20 @@ def test_tc_anchor_broadcast(C):
         assert torch.equal(o[:, :, rho, :, [0, 2]], o[:, :, near[rho], :, [0, 2]])
 
 
-@pytest.mark.parametrize("batch,heads,d", [(1, 22, 128), (1, 33, 128), (2, 11, 64)])
-def test_tc_anchor_split_last_wave(C, batch, heads, d):
+@pytest.mark.parametrize("batch,heads,d,frames,rows,cols,anchors", [
+    (1, 22, 128, 4, 9, 100, (2, 6)),    # N = 3600: 29 key blocks (last of 16 tokens), 7 tiles per head
+    (1, 33, 128, 4, 9, 100, (2, 6)),    # 231 tiles: the last 83 in 3 ranges
+    (2, 11, 64, 4, 9, 100, (2, 6)),     # two batches, head_dim 64
+    (1, 50, 128, 5, 10, 10, (2, 7)),    # N = 500: 4 key blocks (last of 116 tokens), 1 tile per head, all
+])                                      # 50 tiles split in 2 ranges of 2 blocks
+def test_tc_anchor_split_last_wave(C, batch, heads, d, frames, rows, cols, anchors):
     """With a workspace the anchor call cuts its last partial wave of tiles
     into key ranges and merges them exactly: every listed head matches the
     oracle; whole tiles are bitwise those of the call without a workspace and
     split tiles agree with them to rounding; a repeated call is bitwise equal
     (the merge sums the ranges in range order, whichever ends last); broadcast
     rows are bitwise copies of their anchors; the workspace's counters are
-    reset by the call (it starts as NaN bytes).  N = 3600: 29 key blocks, the
-    last of 16 tokens; 7 anchor tiles per head, the last of 32 queries."""
-    frames, rows, cols, anchors = 4, 9, 100, (2, 6)
+    reset by the call (it starts as NaN bytes)."""
     n = frames * rows * cols
     nb, tph = O.num_blocks(n, 128), -(-frames * len(anchors) * cols // 128)
     q, k, v = W.make_qkv(71 + heads, batch, n, heads, d, "bf16", 1.0, "cuda")
@@ -230,7 +233,7 @@ def test_tc_anchor_split_last_wave(C, batch, heads, d):
         b, r = divmod(t, heads * tph)
         in_split[b, :, head_ids[r // tph]] |= tile_of_token == r % tph
     in_split = in_split.cuda()
-    assert in_split.any() and not in_split.all()
+    assert in_split.any()
     assert torch.equal(split[~in_split], whole[~in_split])
     diff = (split[in_split].float() - whole[in_split].float()).abs().max().item()
     assert diff <= 1e-2, diff
