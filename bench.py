@@ -1011,16 +1011,20 @@ def main():
             max(3, args.steps // 4), 2, stream)), dist, "cuda")
         d_two.close()
         # the anchor path alone, with the workspace that splits its last wave
-        # of tiles and, for comparison, every tile whole
+        # of tiles and, for comparison, every tile whole: interleaved, the
+        # order alternating round by round, so the power-capped clock drifts
+        # alike for both
         a_ws = anchor_workspace(torch, C, q, wd, len(rep_heads))
-        anchor_ms = max_over_ranks(statistics.mean(time_calls(
-            torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
-                                                  list(rep_heads), workspace=a_ws, stream=stream),
-            max(3, args.steps // 4), 2, stream)), dist, "cuda")
-        anchor_whole_ms = max_over_ranks(statistics.mean(time_calls(
-            torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
-                                                  list(rep_heads), stream=stream),
-            max(3, args.steps // 4), 2, stream)), dist, "cuda")
+        a_ms = {True: [], False: []}
+        for rnd in range(6):
+            for split in ((True, False) if rnd % 2 == 0 else (False, True)):
+                a_ms[split] += time_calls(
+                    torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wd.frames, wd.rows, wd.cols, wd.anchors,
+                                                          list(rep_heads), workspace=a_ws if split else None,
+                                                          stream=stream),
+                    2, 1, stream)
+        anchor_ms = max_over_ranks(statistics.median(a_ms[True]), dist, "cuda")
+        anchor_whole_ms = max_over_ranks(statistics.median(a_ms[False]), dist, "cuda")
         del a_ws
         d_dual.close()
         bcast_bytes = len(rep_heads) * wd.seq_len * wd.head_dim * 2

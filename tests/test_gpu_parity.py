@@ -1221,10 +1221,11 @@ def test_host_buffer_entry_point(C):
 
 
 def test_calls_replay_in_a_cuda_graph(C):
-    """The block-sparse and the fused dual-path calls enqueue only kernels on
-    the caller's stream (no host sync, no allocation after the first call),
-    so they capture into a CUDA graph; replays compute on whatever the input
-    buffers hold, bitwise equal to direct calls."""
+    """The block-sparse, the fused dual-path and the anchor call with its
+    split workspace enqueue only kernels and memsets on the caller's stream
+    (no host sync, no allocation after the first call), so they capture into
+    a CUDA graph; replays compute on whatever the input buffers hold, bitwise
+    equal to direct calls."""
     frames, rows, cols, anchors = 3, 10, 100, (2, 7)
     n, h, d, block = frames * rows * cols, 3, 128, 128
     nb = O.num_blocks(n, block)
@@ -1235,32 +1236,37 @@ def test_calls_replay_in_a_cuda_graph(C):
     with C.MaskDictionary(1, 1, h, nb, nb, block, ci.size) as dct:
         dct.set_anchor_geometry(frames, rows, cols, anchors)
         dct.set_layer(0, 0, rp, ci, rep)
-        o_sparse, o_dual = torch.zeros_like(q), torch.zeros_like(q)
+        o_sparse, o_dual, o_anchor = torch.zeros_like(q), torch.zeros_like(q), torch.zeros_like(q)
+        a_ws = torch.empty(C.calibatt_anchor_attn_workspace_size(q, frames, rows, cols, len(anchors), 1) // 4,
+                           device="cuda")
+        assert a_ws.numel() > 0                         # 5 tiles on the SMs: split in key ranges
 
         def step():
             C.calibatt_block_sparse_attn(q, k, v, o_sparse, dct, 0, 0, block)
             C.calibatt_dual_path_attn(q, k, v, o_dual, dct, 0, 0, frames, rows, cols, anchors, block)
+            C.calibatt_anchor_attn(q, k, v, o_anchor, frames, rows, cols, anchors, [1], workspace=a_ws)
 
         step()                                          # warm-up outside the capture
         torch.cuda.synchronize()
-        direct = (o_sparse.clone(), o_dual.clone())
+        outs = (o_sparse, o_dual, o_anchor)
+        direct = tuple(o.clone() for o in outs)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step()
-        o_sparse.zero_()
-        o_dual.zero_()
+        for o in outs:
+            o.zero_()
         graph.replay()
         torch.cuda.synchronize()
-        assert torch.equal(o_sparse, direct[0]) and torch.equal(o_dual, direct[1])
+        assert all(torch.equal(o, r) for o, r in zip(outs, direct))
         for dst, src in ((q, q2), (k, k2), (v, v2)):     # new inputs in the captured buffers
             dst.copy_(src)
         graph.replay()
         torch.cuda.synchronize()
-        got = (o_sparse.clone(), o_dual.clone())
+        got = tuple(o.clone() for o in outs)
         step()
         _check_status(C)
-        assert torch.equal(got[0], o_sparse) and torch.equal(got[1], o_dual)
-        assert not torch.equal(got[1], direct[1])
+        assert all(torch.equal(g, o) for g, o in zip(got, outs))
+        assert not torch.equal(got[1], direct[1]) and not torch.equal(got[2], direct[2])
         del graph
 
 
@@ -1285,6 +1291,33 @@ def test_bounded_wait_runs_out_and_context_survives(C):
     out, _ = _run_sparse(C, q, k, v, masks, 128)
     ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, 128)
     _assert_close(_np(out), ref, "bf16")
+
+
+def test_anchor_calls_in_flight_with_their_own_workspaces(C):
+    """Anchor calls with split workspaces issued on three streams at once,
+    each stream with its own workspace, 8 rounds: every output is bitwise the
+    one of a call made alone (no counter or partial output is shared)."""
+    frames, rows, cols, anchors, h, d = 4, 9, 100, (2, 6), 22, 128
+    n = frames * rows * cols
+    q, k, v = W.make_qkv(83, 1, n, h, d, "bf16", 1.0, "cuda")
+    heads = list(range(h))
+    nbytes = C.calibatt_anchor_attn_workspace_size(q, frames, rows, cols, len(anchors), h)
+    assert nbytes > 0
+    ref = torch.zeros_like(q)
+    ws0 = torch.empty(nbytes // 4, device="cuda")
+    C.calibatt_anchor_attn(q, k, v, ref, frames, rows, cols, anchors, heads, workspace=ws0)
+    _check_status(C)
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    wss = [torch.empty(nbytes // 4, device="cuda") for _ in streams]
+    outs = [torch.zeros_like(q) for _ in streams]
+    torch.cuda.synchronize()
+    for _ in range(8):
+        for st, ws, o in zip(streams, wss, outs):
+            C.calibatt_anchor_attn(q, k, v, o, frames, rows, cols, anchors, heads, workspace=ws, stream=st)
+    torch.cuda.synchronize()
+    _check_status(C)
+    for o in outs:
+        assert torch.equal(o, ref)
 
 
 def test_dictionary_calls_in_flight_on_several_streams(C):
