@@ -442,7 +442,7 @@ def run_epilogue_probe(torch, B, C, fused=False):
         d.close()
     print(json.dumps({"epilogue_probe": {
         "workload": "dual-path 720p layer, anchor tiles of its 12 repetitive heads, " +
-                    ("fused launch (staged stores)" if fused else "anchor-only launch (per-thread stores)"),
+                    ("fused launch" if fused else "anchor-only launch, whole tiles") + " (staged stores)",
         "anchor_tiles": n_items, "ctas": len(used), "output_bytes": total_bytes,
         "epilogue_ns_per_tile": sum(t for t, _ in used) / n_items,
         "bytes_per_tile": total_bytes / n_items,

@@ -964,17 +964,13 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
 #ifdef CALIBATT_TRACE
     const unsigned long long t_epi = globaltimer();
 #endif
-    if (MODE == kModeFused && it.anchor) {
+    if ((MODE == kModeFused || MODE == kModeAnchor) && it.anchor) {
       // Anchor broadcast through shared memory: the warp stages 8 of its rows
       // at a time (each row's HD/2 output columns, HD bytes), then every
       // destination row is written by HD/16 lanes storing its contiguous
       // bytes, so one warp-wide store covers 32*16/HD rows instead of 32
-      // rows 16 bytes each (a third of the L2 write sectors; the stores issue
-      // at HBM rate).  Used in the fused launch, where anchor tiles end at
-      // scattered times; in the anchor-only launch every CTA ends its equal
-      // tiles together, and there the per-thread stores below measured 3.6%
-      // faster end to end (a synchronized burst of full-line writes competes
-      // with the next tiles' key/value reads).
+      // rows 16 bytes each (half the L2 write sectors; the stores issue at
+      // HBM rate).
       uint4 pk[HD / 64][4];
 #pragma unroll
       for (int ch = 0; ch < HD / 64; ++ch) {
@@ -984,6 +980,27 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        if (MODE == kModeAnchor && merge) {
+          // sum over the parts in part order (this part's values from tensor
+          // memory are the ones it wrote)
+          const int parts = p.split.parts, part = it.part & 3;
+          float acc[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (i < parts) {
+              const float* src = p.split.o + (rec0 + 8 * i) * (HD / 2) * 32 + (ch * 32) * 32 + lane;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const float x = i == part ? __uint_as_float(o[c]) : __ldcg(src + c * 32);
+                acc[c] = fmaf(w_part[i], x, acc[c]);
+              }
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(acc[c]);
         }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -1032,6 +1049,7 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         __syncwarp();
       }
     } else {
+    // block-sparse item: this thread's row, its HD/2 output columns
 #pragma unroll 1
     for (int ch = 0; ch < HD / 64; ++ch) {
       const int col = s * (HD / 2) + ch * 32;  // this group's output columns
@@ -1041,27 +1059,6 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0u;
-      }
-      if (MODE == kModeAnchor && merge) {
-        // sum over the parts in part order (this part's values from tensor
-        // memory are the ones it wrote)
-        const int parts = p.split.parts, part = it.part & 3;
-        float acc[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (i < parts) {
-            const float* src = p.split.o + (rec0 + 8 * i) * (HD / 2) * 32 + (ch * 32) * 32 + lane;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float x = i == part ? __uint_as_float(o[c]) : __ldcg(src + c * 32);
-              acc[c] = fmaf(w_part[i], x, acc[c]);
-            }
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(acc[c]);
       }
       uint4 pkd[4];
 #pragma unroll
@@ -1074,12 +1071,8 @@ __device__ void softmax_role(const TcParams& p, uint32_t base, uint8_t* gbase, u
         pkd[g].z = pack_bf16x2(v[4], v[5]);
         pkd[g].w = pack_bf16x2(v[6], v[7]);
       }
-#pragma unroll 1
-      for (int d = 0; d < n_dst; ++d) {
-        const int64_t token = it.anchor
-            ? (static_cast<int64_t>(anchor_f) * p.anc.rows + lo + d) * p.anc.cols + anchor_w
-            : dst_token;
-        uint4* dst = reinterpret_cast<uint4*>(p.o + bh_off + token * p.sn + col);
+      if (n_dst > 0) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + bh_off + static_cast<int64_t>(dst_token) * p.sn + col);
 #pragma unroll
         for (int g = 0; g < 4; ++g) dst[g] = pkd[g];
       }
