@@ -975,6 +975,23 @@ def main():
         extras["head_partition"] = {"heads_this_rank": my_heads, "tiles_this_rank": my_tiles,
                                     "api": "calibatt_block_sparse_attn_csr with this rank's head_ids"}
     if not args.no_extras and not by_heads:
+        # the anchor path alone: the dual-path layer's 12 repetitive heads on
+        # the same inputs, with the workspace that splits its last wave of
+        # tiles, timed like the headline call (steps calls back to back)
+        wa = W.WORKLOADS["720p_dual"]
+        _, a_heads = W.workload_masks(wa)
+        a_ws = anchor_workspace(torch, C, q, wa, len(a_heads))
+        a_ms = max_over_ranks(statistics.mean(time_calls(
+            torch, lambda: C.calibatt_anchor_attn(q, k, v, o, wa.frames, wa.rows, wa.cols, wa.anchors,
+                                                  list(a_heads), workspace=a_ws, stream=stream),
+            args.steps, args.warmup, stream)), dist, "cuda")
+        a_tiles = len(a_heads) * -(-wa.frames * len(wa.anchors) * wa.cols // 128) * wa.num_blocks
+        a_tf = a_tiles * FLOP_PER_TILE / (a_ms * 1e-3) / 1e12
+        del a_ws
+        extras["anchor_720p"] = {"heads": len(a_heads), "anchor_tiles_x_key_blocks": a_tiles, "ms_per_call": a_ms,
+                                 "effective_tflops": a_tf, "frac_of_burst_peak": a_tf / pk["bf16_tflops"],
+                                 "timing": f"{args.steps} calls back to back after {args.warmup} warm-up calls",
+                                 "api": "calibatt_anchor_attn with its split workspace"}
         # dense path on the same inputs: all-ones skip lists held on the device,
         # through the direct-CSR call (no dictionary)
         nbk, hh = wl.num_blocks, wl.heads
