@@ -260,3 +260,23 @@ def test_anchor_split_plan_shortens_the_last_wave(calibatt_lib):
     assert C.anchor_split_plan(10, 148, 591) == (0, 4)     # fewer tiles than SMs: quarters
     with pytest.raises(C.CalibattError):
         C.anchor_split_plan(10, 0, 591)
+
+
+def test_anchor_workspace_size_checks_arguments_on_the_host(calibatt_lib):
+    """calibatt_anchor_attn_workspace_size validates its arguments before it
+    asks the device anything, and float32 calls (the CUDA-core anchor path,
+    which never splits) need no workspace."""
+    C = calibatt_lib
+    L = C.LIB
+    n = ctypes.c_size_t(123)
+    f32 = C.Shape(1, 3600, 4, 128, 3600 * 4 * 128, 4 * 128, 128, C.DTYPE_FP32, 0)
+    assert L.calibatt_anchor_attn_workspace_size(ctypes.byref(f32), 4, 9, 100, 2, 4, ctypes.byref(n)) == C.OK
+    assert n.value == 0
+    assert L.calibatt_anchor_attn_workspace_size(ctypes.byref(f32), 4, 9, 100, 2, 4, None) == C.ERR_INVALID_ARG
+    for frames, rows, cols, na, nh in ((0, 9, 100, 2, 4), (4, 9, 100, 0, 4), (4, 9, 100, 17, 4),
+                                       (4, 9, 100, 2, -1), (4, 9, 100, 2, 129)):
+        st = L.calibatt_anchor_attn_workspace_size(ctypes.byref(f32), frames, rows, cols, na, nh, ctypes.byref(n))
+        assert st == C.ERR_INVALID_ARG, (frames, rows, cols, na, nh)
+    bad = C.Shape(1, 3600, 4, 96, 3600 * 4 * 96, 4 * 96, 96, C.DTYPE_BF16, 0)
+    assert L.calibatt_anchor_attn_workspace_size(ctypes.byref(bad), 4, 9, 100, 2, 4, ctypes.byref(n)) == \
+        C.ERR_UNSUPPORTED
