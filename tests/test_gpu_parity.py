@@ -242,6 +242,39 @@ def test_tc_anchor_split_last_wave(C, batch, heads, d, frames, rows, cols, ancho
         assert torch.equal(o[:, :, r], o[:, :, near[r]])
 
 
+@pytest.mark.parametrize("rows,anchors", [(16, tuple(range(16))), (9, (5,))])
+def test_tc_anchor_degenerate_geometries(C, rows, anchors):
+    """The anchor path's degenerate cases, with and without the split
+    workspace: every spatial row an anchor (16 anchors, the most a call
+    takes) makes every query attend densely and serve only itself, so the
+    output is dense attention (the oracle's block-sparse attention with
+    all-ones masks); a single anchor row serves every row of its frame, so
+    all rows of a frame and column are bitwise equal."""
+    frames, cols, h, d = 2, 64, 3, 128
+    n = frames * rows * cols
+    q, k, v = W.make_qkv(91 + rows, 1, n, h, d, "bf16", 1.0, "cuda")
+    nbytes = C.calibatt_anchor_attn_workspace_size(q, frames, rows, cols, len(anchors), h)
+    ws = torch.empty(max(1, nbytes // 4), device="cuda")
+    outs = []
+    for w in (None, ws if nbytes else None):
+        out = torch.full_like(q, float("nan"))
+        C.calibatt_anchor_attn(q, k, v, out, frames, rows, cols, anchors, list(range(h)), workspace=w)
+        outs.append(out)
+    _check_status(C)
+    ref = O.anchor_attention_bnhd(_np(q), _np(k), _np(v), frames, rows, cols, anchors)
+    for out in outs:
+        _assert_close(_np(out), ref, "bf16")
+    o = outs[0].view(1, frames, rows, cols, h, d)
+    if len(anchors) == rows:
+        nb = O.num_blocks(n, 128)
+        dense, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), [np.ones((nb, nb), bool)] * h, 128)
+        np.testing.assert_allclose(ref, dense, rtol=0, atol=1e-12)
+        _assert_close(_np(outs[0]), dense, "bf16")
+    else:
+        for r in range(rows):
+            assert torch.equal(o[:, :, r], o[:, :, anchors[0]])
+
+
 def test_simt_anchor_fp32(C):
     frames, rows, cols, h, d = 2, 9, 16, 2, 64
     n = frames * rows * cols
