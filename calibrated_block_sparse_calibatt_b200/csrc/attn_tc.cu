@@ -444,6 +444,57 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
   uint32_t kv = 0, item = 0, issued = 0, q_items = 0;
   bool ok = true;
   while (ok && cur.next(p, it, W)) {
+    // The row's list first (bitmap and interval rows are expanded into this
+    // producer's shared-memory list), so that the Q/K producer does it while
+    // the previous item's last score MMAs still hold the Q buffer.
+    const uint16_t* cols = it.cols;
+    if (p.sched.bitmap != nullptr && !it.anchor) {
+      // Bitmap row -> this producer's list of kept key blocks, ascending:
+      // lane x takes word x of each 32-word stretch, a prefix sum of the
+      // words' bit counts places its indices.
+      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
+      int offset = 0;
+      for (int w0 = 0; w0 < p.sched.words; w0 += 32) {
+        const int x = w0 + lane;
+        uint32_t word = x < p.sched.words ? bitmap_row(p, it.h, it.tile)[x] : 0u;
+        const int c = __popc(word);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        int pos = offset + incl - c;
+        while (word) {
+          list[pos++] = static_cast<uint16_t>(x * 32 + __ffs(word) - 1);
+          word &= word - 1u;
+        }
+        offset += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      __syncwarp();
+      cols = list;
+    } else if (p.sched.runs != nullptr && !it.anchor) {
+      // Interval row -> this producer's list of kept key blocks: runs are
+      // read 32 at a time, one per lane, then the warp writes each run's
+      // blocks lane-parallel in order.
+      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
+      const int64_t ro = static_cast<int64_t>(it.h) * (p.sched.nq + 1) + it.tile;
+      const int r0 = p.sched.run_ptr[ro] & 0x7FFFFFFF, n_runs = (p.sched.run_ptr[ro + 1] & 0x7FFFFFFF) - r0;
+      const uint32_t* runs = p.sched.runs + p.sched.col_base[it.h] + r0;
+      int pos = 0;
+      for (int x0 = 0; x0 < n_runs; x0 += 32) {
+        const uint32_t mine = x0 + lane < n_runs ? runs[x0 + lane] : 0u;
+        const int cnt = min(32, n_runs - x0);
+        for (int x = 0; x < cnt; ++x) {
+          const uint32_t run = __shfl_sync(0xFFFFFFFFu, mine, x);
+          const int start = static_cast<int>(run & 0xFFFFu), len = static_cast<int>(run >> 16);
+          for (int i = lane; i < len; i += 32) list[pos + i] = static_cast<uint16_t>(start + i);
+          pos += len;
+        }
+      }
+      __syncwarp();
+      cols = list;
+    }
     if (!V) {
       if (item > 0 && !W.wait(bar(L::bQEmpty), (item - 1) & 1, 1)) break;
       CALIBATT_TRACE_EVENT(kTraceMma && lane == 0, 9, item + CALIBATT_TRACE_OFFSET);
@@ -508,54 +559,6 @@ __device__ void producer_role(const TcParams& p, uint32_t base, uint8_t* gbase, 
         }
       }
       ++q_items;  // every item completes one phase of q_full, whichever way its Q came
-    }
-    const uint16_t* cols = it.cols;
-    if (p.sched.bitmap != nullptr && !it.anchor) {
-      // Bitmap row -> this producer's list of kept key blocks, ascending:
-      // lane x takes word x of each 32-word stretch, a prefix sum of the
-      // words' bit counts places its indices.
-      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
-      int offset = 0;
-      for (int w0 = 0; w0 < p.sched.words; w0 += 32) {
-        const int x = w0 + lane;
-        uint32_t word = x < p.sched.words ? bitmap_row(p, it.h, it.tile)[x] : 0u;
-        const int c = __popc(word);
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        int pos = offset + incl - c;
-        while (word) {
-          list[pos++] = static_cast<uint16_t>(x * 32 + __ffs(word) - 1);
-          word &= word - 1u;
-        }
-        offset += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-      __syncwarp();
-      cols = list;
-    } else if (p.sched.runs != nullptr && !it.anchor) {
-      // Interval row -> this producer's list of kept key blocks: runs are
-      // read 32 at a time, one per lane, then the warp writes each run's
-      // blocks lane-parallel in order.
-      uint16_t* list = reinterpret_cast<uint16_t*>(gbase + L::kList + (V ? 1 : 0) * L::kListBytes);
-      const int64_t ro = static_cast<int64_t>(it.h) * (p.sched.nq + 1) + it.tile;
-      const int r0 = p.sched.run_ptr[ro] & 0x7FFFFFFF, n_runs = (p.sched.run_ptr[ro + 1] & 0x7FFFFFFF) - r0;
-      const uint32_t* runs = p.sched.runs + p.sched.col_base[it.h] + r0;
-      int pos = 0;
-      for (int x0 = 0; x0 < n_runs; x0 += 32) {
-        const uint32_t mine = x0 + lane < n_runs ? runs[x0 + lane] : 0u;
-        const int cnt = min(32, n_runs - x0);
-        for (int x = 0; x < cnt; ++x) {
-          const uint32_t run = __shfl_sync(0xFFFFFFFFu, mine, x);
-          const int start = static_cast<int>(run & 0xFFFFu), len = static_cast<int>(run >> 16);
-          for (int i = lane; i < len; i += 32) list[pos + i] = static_cast<uint16_t>(start + i);
-          pos += len;
-        }
-      }
-      __syncwarp();
-      cols = list;
     }
     uint32_t my_col = 0;
     for (int j = 0; j < it.n; ++j) {
