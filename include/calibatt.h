@@ -386,8 +386,8 @@ calibatt_status calibatt_anchor_attn(const void* q, const void* k, const void* v
  * count sizes the persistent grid); 0 when the call would not split (no
  * partial wave, fewer than four key blocks, or float32 inputs).  The
  * workspace holds, per split tile and key range, 128 x head_dim float32
- * partial outputs and 128 (maximum, row sum) pairs, and 8 counters per
- * split tile.  No counterpart in the pages: a scheduling device of this
+ * partial outputs and 256 (maximum, row sum) pairs (one per row and output
+ * column half), and 8 counters per split tile.  No counterpart in the pages: a scheduling device of this
  * implementation (Key Designs 3 defines the operation). */
 calibatt_status calibatt_anchor_attn_workspace_size(const calibatt_shape* shape, int32_t frames,
                                                     int32_t rows, int32_t cols, int32_t n_anchors,
