@@ -572,6 +572,60 @@ def test_full_size_dual_path_sampled(C):
         assert torch.equal(o[:, :, rho], o[:, :, near[rho]])
 
 
+def test_full_size_anchor_split_sampled(C):
+    """The anchor path alone at the dual-path 720p layer's size (12
+    repetitive heads, 792 tiles on the grid) with its split workspace: the
+    split tiles' rows match the oracle on a sample, every other row is
+    bitwise the call's output without a workspace, repeated calls are
+    bitwise equal, and broadcast rows are bitwise copies of their anchors."""
+    import _oracle_jobs as J
+
+    wl = W.WORKLOADS["720p_dual"]
+    q, k, v = W.make_qkv(wl.seed, wl.batch, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    _, rep_heads = W.workload_masks(wl)
+    heads = list(rep_heads)
+    tph = -(-wl.frames * len(wl.anchors) * wl.cols // 128)
+    first, parts = C.anchor_split_plan(len(heads) * tph, C.device_sm_count(), wl.num_blocks)
+    assert parts > 1
+    ws = torch.empty(C.calibatt_anchor_attn_workspace_size(q, wl.frames, wl.rows, wl.cols, len(wl.anchors),
+                                                           len(heads)) // 4, device="cuda")
+    split = torch.full_like(q, float("nan"))
+    again = torch.full_like(q, float("nan"))
+    whole = torch.full_like(q, float("nan"))
+    C.calibatt_anchor_attn(q, k, v, split, wl.frames, wl.rows, wl.cols, wl.anchors, heads, workspace=ws)
+    C.calibatt_anchor_attn(q, k, v, again, wl.frames, wl.rows, wl.cols, wl.anchors, heads, workspace=ws)
+    C.calibatt_anchor_attn(q, k, v, whole, wl.frames, wl.rows, wl.cols, wl.anchors, heads)
+    _check_status(C)
+    assert torch.equal(split, again)
+    del again
+    # tokens of the split tiles: item t >= first is tile t % tph of listed head t // tph
+    near = O.nearest_anchor_rows(wl.rows, wl.anchors)
+    a_of_row = np.array([list(wl.anchors).index(near[r]) for r in range(wl.rows)])
+    f, rho, w = np.meshgrid(np.arange(wl.frames), np.arange(wl.rows), np.arange(wl.cols), indexing="ij")
+    tile_of_token = ((f * len(wl.anchors) + a_of_row[rho]) * wl.cols + w).reshape(-1) // 128
+    split_tokens = {}
+    for t in range(first, len(heads) * tph):
+        split_tokens.setdefault(heads[t // tph], set()).add(t % tph)
+    for h in heads:
+        sel = np.isin(tile_of_token, sorted(split_tokens.get(h, ())))
+        idx = torch.as_tensor(np.nonzero(~sel)[0], device=q.device)
+        assert torch.equal(split[0, idx, h], whole[0, idx, h])
+    del whole
+    rng = np.random.default_rng(5)
+    jobs, checks = [], []
+    for h, tiles in sorted(split_tokens.items()):
+        toks = np.nonzero(np.isin(tile_of_token, sorted(tiles)))[0]
+        sample = np.sort(rng.choice(toks, min(300, len(toks)), replace=False))
+        jobs.append((_f32(q[0, :wl.seq_len, h]), _f32(k[0, :wl.seq_len, h]), _f32(v[0, :wl.seq_len, h]),
+                     wl.frames, wl.rows, wl.cols, wl.anchors, sample))
+        checks.append((h, sample))
+    for (h, sample), ref in zip(checks, J.anchor_rows_many(jobs)):
+        _assert_close(_np(split[0, torch.as_tensor(sample, device=q.device), h]), ref, "bf16")
+    o = split.view(1, wl.frames, wl.rows, wl.cols, wl.heads, wl.head_dim)[..., heads, :]
+    for r in range(wl.rows):
+        assert torch.equal(o[:, :, r], o[:, :, near[r]])
+
+
 # --------------------------------------------------------- offline calibration
 
 def _energy(C, q, k, block):
