@@ -331,6 +331,29 @@ def anchor_workspace(torch, C, q, wd, n_heads):
     return torch.empty(nbytes // 4, dtype=torch.float32, device="cuda") if nbytes else None
 
 
+def run_energy_case(args, torch, C, pk):
+    """The block energy alone on the 720p geometry with --heads heads (LSE
+    pass, energy pass), timed with CUDA events; a case of its own for
+    profiling the tensor-core energy modes."""
+    import dataclasses
+    wl = dataclasses.replace(W.WORKLOADS["720p"], heads=args.heads)
+    q, k, _ = W.make_qkv(wl.seed, 1, wl.seq_len, wl.heads, wl.head_dim, "bf16", wl.input_std, "cuda")
+    e = torch.empty((1, wl.heads, wl.num_blocks, wl.num_blocks), device="cuda")
+    ws = torch.empty(C.calibatt_block_energy_workspace_size(q) // 4, device="cuda")
+    stream = torch.cuda.current_stream()
+    per_call = time_calls(torch, lambda: C.calibatt_block_energy(q, k, e, ws, wl.block, stream=stream),
+                          args.steps, args.warmup, stream)
+    if C.device_status() != 0:
+        raise RuntimeError("device wait timed out in the energy case")
+    ms = statistics.mean(per_call)
+    exp2 = 2 * wl.seq_len ** 2 * wl.heads      # both passes exponentiate every score
+    print(json.dumps({"energy_case": {
+        "heads": wl.heads, "ms_per_call": ms, "exp2_per_call": exp2,
+        "g_exp2_per_s": exp2 / (ms * 1e-3) / 1e9,
+        "frac_of_mufu_peak_at_max_clock": exp2 / (ms * 1e-3) / mufu_exp2_peak(C.device_sm_count(), 1965.0)}}),
+        flush=True)
+
+
 def run_similarity_case(args, torch, C, pk):
     """The spatial-similarity pass alone on the 720p geometry with --heads
     heads (LSE pass, pass of per-query sums, row reduction), timed with CUDA
@@ -848,6 +871,8 @@ def main():
                          "build (-DCALIBATT_TRACE) and print their per-block phase breakdown")
     ap.add_argument("--similarity-case", action="store_true",
                     help="time the spatial-similarity pass alone (720p geometry, --heads heads)")
+    ap.add_argument("--energy-case", action="store_true",
+                    help="time the block energy alone (720p geometry, --heads heads)")
     ap.add_argument("--dual-case", action="store_true",
                     help="time the dual-path 720p layer alone (one fused launch of both paths)")
     ap.add_argument("--layout", default="bnhd", choices=["bnhd", "bhnd"],
@@ -905,6 +930,9 @@ def main():
         return
     if args.similarity_case:
         run_similarity_case(args, torch, C, pk)
+        return
+    if args.energy_case:
+        run_energy_case(args, torch, C, pk)
         return
     if args.workload == "sweep":
         if world > 1:
