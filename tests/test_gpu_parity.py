@@ -1308,6 +1308,53 @@ def test_host_buffer_entry_point(C):
     assert torch.equal(dq, q)
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_head_major_storage_matches_token_major(C, batch):
+    """The calls take any strides: the same logical [batch, N, heads, D]
+    tensors stored head-major ([batch, heads, N, D] in memory) give bitwise
+    the outputs of token-major storage -- block-sparse and fused dual-path
+    dictionary calls, the anchor call with its split workspace, and the block
+    energy."""
+    frames, rows, cols, anchors = 3, 10, 100, (2, 7)
+    n, h, d, block = frames * rows * cols, 4, 128, 128
+    nb = O.num_blocks(n, block)
+    q, k, v = W.make_qkv(95 + batch, batch, n, h, d, "bf16", 1.0, "cuda")
+
+    def head_major(t):
+        return t.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+
+    qh, kh, vh = head_major(q), head_major(k), head_major(v)
+    assert qh.stride(2) == n * d and qh.stride(1) == d and torch.equal(qh, q)
+    masks = _random_masks(96, h, nb, 0.45)
+    masks[1] = None
+    rp, ci, rep = C.masks_to_layer_csr(masks, h, nb)
+    nbytes = C.calibatt_anchor_attn_workspace_size(q, frames, rows, cols, len(anchors), h)
+    ws = torch.empty(max(1, nbytes // 4), device="cuda")
+    outs = {}
+    with C.MaskDictionary(1, 1, h, nb, nb, block, ci.size) as dct:
+        dct.set_anchor_geometry(frames, rows, cols, anchors)
+        dct.set_layer(0, 0, rp, ci, rep)
+        for name, (a, b_, c_) in (("token", (q, k, v)), ("head", (qh, kh, vh))):
+            o_s, o_d, o_a = (torch.full_like(a, float("nan")) for _ in range(3))
+            C.calibatt_block_sparse_attn(a, b_, c_, o_s, dct, 0, 0, block)
+            C.calibatt_dual_path_attn(a, b_, c_, o_d, dct, 0, 0, frames, rows, cols, anchors, block)
+            C.calibatt_anchor_attn(a, b_, c_, o_a, frames, rows, cols, anchors, list(range(h)),
+                                   workspace=ws if nbytes else None)
+            e = torch.full((batch, h, nb, nb), float("nan"), device="cuda")
+            e_ws = torch.empty(C.calibatt_block_energy_workspace_size(a) // 4, device="cuda")
+            C.calibatt_block_energy(a, b_, e, e_ws, block)
+            _check_status(C)
+            assert o_a.stride() == a.stride()
+            outs[name] = (o_s, o_d, o_a, e)
+    sparse = [i for i in range(h) if i != 1]
+    ts, td, ta, te = outs["token"]
+    hs, hd, ha, he = outs["head"]
+    assert torch.equal(ts[:, :, sparse], hs[:, :, sparse])     # head 1 (repetitive) is not written there
+    assert torch.equal(td, hd) and torch.equal(ta, ha) and torch.equal(te, he)
+    ref, _ = O.block_sparse_attention_bnhd(_np(q), _np(k), _np(v), masks, block, heads=sparse)
+    _assert_close(_np(hs)[:, :, sparse], ref, "bf16")
+
+
 def test_calls_replay_in_a_cuda_graph(C):
     """The block-sparse, the fused dual-path and the anchor call with its
     split workspace enqueue only kernels and memsets on the caller's stream
